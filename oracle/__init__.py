@@ -1,0 +1,184 @@
+"""CPU oracle for the balancer's hot path (TEST INFRASTRUCTURE ONLY).
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never imports, links or calls it, and it shares no code
+with them.  The arithmetic lives in ``ue_oracle.c`` (plain single-threaded C);
+this module only marshals numpy arrays into it.
+
+Pinning status (what fixes each function other than itself; the tests under
+``tests/test_oracle_*.py`` check every item):
+  load          numpy.bincount of the ids; brute-force per-rank counting;
+                sum = T*K; balls-in-bins expectation of the busiest rank at s=0.
+  expert_load   brute-force counting of occurrences before each rank's tokens.
+  plan          hand-worked examples (tests/golden/plan_cases.json); invariants
+                (conservation, <= R replicas per rank, redundant quotas >= 1,
+                loads <= Q unless slots ran out); optimality max load = Q when
+                slots do not run out (Q is a lower bound for any plan); the
+                brute-force optimum over all replica placements with an
+                integer max-flow on tiny inputs.
+  reroute       numpy stable argsort + searchsorted; per-slot counts equal
+                quotas; every phys slot holds the token's expert.
+  sync          byte-map conservation: every byte of every filled redundant
+                slot comes from the right home byte exactly once, other slots
+                untouched.
+  grad_reduce   exact closed-form sums on dyadic values; zero gradients
+                leave the master unchanged; numpy float32 reference order.
+
+None of these pins comes from the UltraEP pages themselves, which print no
+worked example, table or value for any step: parity against the pages is
+"unpinned by the pages" for all five steps; the pins above are the
+mathematics and hand-worked cases of the stated rule.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ue_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libue_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+P_I32 = ctypes.POINTER(ctypes.c_int32)
+
+
+def build(force: bool = False) -> str:
+    """Compile ue_oracle.c into oracle/libue_oracle.so with gcc (no fast-math, no FMA)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+                               "-fno-fast-math", "-Wall", "-Wextra", "-o", tmp, _SRC])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _get():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            vp, i64, ci = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+            lib.ue_oracle_load.argtypes = [vp, i64, ci, ci, ci, vp, vp]
+            lib.ue_oracle_expert_load.argtypes = [vp, ci, ci, vp, vp]
+            lib.ue_oracle_plan.argtypes = [ci, ci, ci, vp] + [vp] * 9
+            lib.ue_oracle_reroute.argtypes = [vp, i64, ci, ci, vp, vp, vp, vp, vp]
+            lib.ue_oracle_sync.argtypes = [vp, i64, i64, ci, ci, ci, vp]
+            lib.ue_oracle_grad_reduce.argtypes = [vp, i64, vp, ci, i64, i64, ci, ci, ci, vp, vp]
+            for f in ("ue_oracle_load", "ue_oracle_expert_load", "ue_oracle_plan",
+                      "ue_oracle_reroute", "ue_oracle_sync", "ue_oracle_grad_reduce"):
+                getattr(lib, f).restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise OracleError(f"{what} failed with code {rc}")
+
+
+def _p(a: np.ndarray | None):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def load(ids: np.ndarray, E: int, N: int):
+    """Step 1: per-source-rank histogram counts[N][E] and per-rank bad-id counts."""
+    ids = _c(ids, np.int32)
+    T, K = ids.shape
+    counts = np.empty((N, E), np.int32)
+    bad = np.empty(N, np.int32)
+    _check(_get().ue_oracle_load(_p(ids), T, K, E, N, _p(counts), _p(bad)), "load")
+    return counts, bad
+
+
+def expert_load(counts: np.ndarray):
+    """load[e] = column sums of counts; rank_off[r][e] = exclusive column prefix."""
+    counts = _c(counts, np.int32)
+    N, E = counts.shape
+    ld = np.empty(E, np.int32)
+    off = np.empty((N, E), np.int32)
+    _check(_get().ue_oracle_expert_load(_p(counts), N, E, _p(ld), _p(off)), "expert_load")
+    return ld, off
+
+
+PLAN_FIELDS = ("slot_expert", "slot_quota", "rep_off", "rep_slot", "rep_cum", "rep_experts",
+               "rank_load_before", "rank_load_after", "info")
+
+
+def plan(load_e: np.ndarray, N: int, R: int) -> dict:
+    """Step 2: the quota-driven plan (see ue_oracle.c for the exact rule)."""
+    load_e = _c(load_e, np.int32)
+    E = load_e.shape[0]
+    if E % N:
+        raise OracleError("E must be a multiple of N")
+    H = E // N
+    S = N * (H + R)
+    out = {
+        "slot_expert": np.empty(S, np.int32), "slot_quota": np.empty(S, np.int32),
+        "rep_off": np.empty(E + 1, np.int32), "rep_slot": np.empty(E + N * R, np.int32),
+        "rep_cum": np.empty(E + N * R, np.int32), "rep_experts": np.empty(E, np.int32),
+        "rank_load_before": np.empty(N, np.int32), "rank_load_after": np.empty(N, np.int32),
+        "info": np.empty(8, np.int32),
+    }
+    rc = _get().ue_oracle_plan(E, N, R, _p(load_e), *[_p(out[f]) for f in PLAN_FIELDS])
+    _check(rc, "plan")
+    return out
+
+
+def reroute(ids: np.ndarray, E: int, pl: dict) -> np.ndarray:
+    """Step 3: physical slot of every (t, k)."""
+    ids = _c(ids, np.int32)
+    T, K = ids.shape
+    phys = np.empty_like(ids)
+    rc = _get().ue_oracle_reroute(_p(ids), T, K, E, _p(_c(pl["rep_off"], np.int32)),
+                                  _p(_c(pl["rep_slot"], np.int32)), _p(_c(pl["rep_cum"], np.int32)),
+                                  _p(_c(pl["slot_quota"], np.int32)), _p(phys))
+    _check(rc, "reroute")
+    return phys
+
+
+def sync(W: np.ndarray, nbytes: int, E: int, N: int, R: int, slot_expert: np.ndarray) -> None:
+    """Step 4, in place on W viewed as bytes [S][slot_stride]."""
+    if not (W.flags.c_contiguous and W.ndim == 2):
+        raise OracleError("W must be a C-contiguous [S][stride] array")
+    stride = W.shape[1] * W.itemsize
+    rc = _get().ue_oracle_sync(_p(W), stride, nbytes, E, N, R, _p(_c(slot_expert, np.int32)))
+    _check(rc, "sync")
+
+
+def grad_reduce(master: np.ndarray, grads: np.ndarray, n: int, E: int, N: int, R: int,
+                pl: dict) -> None:
+    """Step 5, in place on master (float32 [E][mstride]); grads float32 or bf16 bits (uint16)."""
+    if master.dtype != np.float32 or not master.flags.c_contiguous:
+        raise OracleError("master must be C-contiguous float32")
+    if not grads.flags.c_contiguous:
+        raise OracleError("grads must be C-contiguous")
+    is_bf16 = 1 if grads.dtype == np.uint16 else 0
+    if not is_bf16 and grads.dtype != np.float32:
+        raise OracleError("grads must be float32 or bf16 bits (uint16)")
+    rc = _get().ue_oracle_grad_reduce(_p(master), master.shape[1], _p(grads), is_bf16,
+                                      grads.shape[1], n, E, N, R,
+                                      _p(_c(pl["rep_off"], np.int32)), _p(_c(pl["rep_slot"], np.int32)))
+    _check(rc, "grad_reduce")
+
+
+def rebalance(ids: np.ndarray, E: int, N: int, R: int):
+    """Steps 1-3 chained: counts, expert loads, rank offsets, plan, phys."""
+    counts, bad = load(ids, E, N)
+    ld, off = expert_load(counts)
+    pl = plan(ld, N, R)
+    phys = reroute(ids, E, pl)
+    return {"counts": counts, "bad": bad, "load": ld, "rank_off": off, "plan": pl, "phys": phys}

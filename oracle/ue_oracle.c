@@ -1,0 +1,345 @@
+/*
+ * CPU oracle for the UltraEP balancer's per-layer, per-microbatch hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file; only the tests, the smoke check and the timed CPU baseline
+ * of the benchmark use it.  It shares no code, header, table or constant with
+ * the CUDA library: every step below is a plain, single-threaded restatement
+ * of what the step computes, written for a reader to check by eye.
+ *
+ * Sources.  "How dots-infra/ultraep works" (gitdiagram summary, component
+ * list "GPU operations" and its "Connections") names the five steps: load
+ * computation, placement planning, routing expansion, replica weight sync and
+ * replica gradient reduction.  The UltraEP news summary ("Comment fonctionne
+ * l'équilibrage en 300 microsecondes") calls the planner a quota-driven,
+ * exact-load scheduler that runs right after gating.  The exact plan rule
+ * taken here: Q = ceil(sum of loads / N); each expert's home rank takes
+ * min(load, Q - current); overflow goes greedily, largest overflow first, to
+ * the rank with the most spare capacity (ties to the lowest rank id), with at
+ * most R replicas per rank; the j-th occurrence of expert e in token-major
+ * (t, k) order goes to the replica whose cumulative quota covers j.
+ *
+ * Readings where the pages are silent (each is listed in the design notes):
+ *   - expert e lives on home rank e / H in local slot e % H, H = E / N;
+ *     physical slot id = r * (H + R) + s, redundant local slots s in [H, H+R);
+ *   - the home pass visits experts in increasing id;
+ *   - overflow order is fixed once after the home pass: overflow descending,
+ *     ties to the lower expert id; each expert is placed fully before the next;
+ *   - a rank is eligible while it has a free redundant slot and spare > 0;
+ *   - if no rank is eligible ("slots run out") the remaining overflow stays on
+ *     the expert's home slot, which then exceeds Q, and flag bit 0 is set;
+ *   - replica order for the cumulative quotas: home slot first, then the
+ *     redundant slots in allocation order; j is 0-based;
+ *   - the per-rank histogram partitions tokens by source rank t / (T / N);
+ *   - ids outside [0, E) are not counted and are rerouted to -1;
+ *   - gradient reduction adds replica gradients into the fp32 master in
+ *     replica order, widening bf16 exactly, one fp32 round-to-nearest add each.
+ *
+ * Every function returns 0 on success and a negative code on a violated
+ * precondition or a broken internal invariant.
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_OK 0
+#define ORC_BAD_ARG (-1)
+#define ORC_INVARIANT (-2)
+
+/* ---- step 1: load computation --------------------------------------------
+ * counts[r][e] = number of (t, k) with t in rank r's tokens and ids[t][k] = e.
+ * bad[r] = number of ids of rank r's tokens outside [0, E).
+ */
+int ue_oracle_load(const int32_t *ids, int64_t T, int K, int E, int N,
+                   int32_t *counts, int32_t *bad)
+{
+    if (T < 0 || K < 1 || E < 1 || N < 1 || T % N != 0) return ORC_BAD_ARG;
+    int64_t tokens_per_rank = T / N;
+    memset(counts, 0, sizeof(int32_t) * (size_t)N * (size_t)E);
+    if (bad) memset(bad, 0, sizeof(int32_t) * (size_t)N);
+    for (int64_t t = 0; t < T; ++t) {
+        int64_t r = t / tokens_per_rank;
+        for (int k = 0; k < K; ++k) {
+            int32_t e = ids[t * K + k];
+            if (e < 0 || e >= E) {
+                if (bad) bad[r] += 1;
+                continue;
+            }
+            counts[r * E + e] += 1;
+        }
+    }
+    return ORC_OK;
+}
+
+/* load[e] = sum over ranks of counts[r][e];
+ * rank_off[r][e] = sum over ranks r' < r of counts[r'][e], i.e. how many
+ * occurrences of e precede rank r's first token in token-major order. */
+int ue_oracle_expert_load(const int32_t *counts, int N, int E,
+                          int32_t *load, int32_t *rank_off)
+{
+    if (N < 1 || E < 1) return ORC_BAD_ARG;
+    for (int e = 0; e < E; ++e) {
+        int64_t run = 0;
+        for (int r = 0; r < N; ++r) {
+            if (rank_off) rank_off[(int64_t)r * E + e] = (int32_t)run;
+            run += counts[(int64_t)r * E + e];
+        }
+        if (run > INT32_MAX) return ORC_BAD_ARG;
+        load[e] = (int32_t)run;
+    }
+    return ORC_OK;
+}
+
+/* ---- step 2: quota-driven placement planning -----------------------------
+ * Outputs (all caller-allocated):
+ *   slot_expert[S], slot_quota[S]  S = N*(H+R); empty slots: -1 / 0
+ *   rep_off[E+1]                   replicas of e are entries rep_off[e] .. rep_off[e+1]-1
+ *   rep_slot[E+N*R], rep_cum[E+N*R] slot of each replica, exclusive prefix of quotas
+ *                                   (entries past rep_off[E] are set to -1)
+ *   rep_experts[E]                 experts holding >= 1 redundant replica, increasing id (-1 tail)
+ *   rank_load_before[N], rank_load_after[N]
+ *   info[8] = { Q, L, flags (bit 0: slots ran out), M = #rep_experts,
+ *               filled redundant slots, max rank load before, max after, 0 }
+ */
+typedef struct { int32_t ovf; int32_t e; } orc_ovf;
+
+static int orc_ovf_cmp(const void *a, const void *b)
+{
+    const orc_ovf *x = (const orc_ovf *)a, *y = (const orc_ovf *)b;
+    if (x->ovf != y->ovf) return x->ovf > y->ovf ? -1 : 1;   /* larger overflow first */
+    return x->e < y->e ? -1 : (x->e > y->e ? 1 : 0);         /* tie: lower expert id */
+}
+
+int ue_oracle_plan(int E, int N, int R, const int32_t *load,
+                   int32_t *slot_expert, int32_t *slot_quota,
+                   int32_t *rep_off, int32_t *rep_slot, int32_t *rep_cum,
+                   int32_t *rep_experts,
+                   int32_t *rank_load_before, int32_t *rank_load_after,
+                   int32_t *info)
+{
+    if (E < 1 || N < 1 || R < 0 || E % N != 0) return ORC_BAD_ARG;
+    const int H = E / N, HR = H + R, S = N * HR, NR = N * R;
+    int64_t L = 0;
+    for (int e = 0; e < E; ++e) {
+        if (load[e] < 0) return ORC_BAD_ARG;
+        L += load[e];
+    }
+    if (L > INT32_MAX) return ORC_BAD_ARG;
+    const int64_t Q = (L == 0) ? 0 : (L + N - 1) / N;        /* Q = ceil(L / N) */
+
+    int64_t *cur = calloc((size_t)N, sizeof(int64_t));        /* tokens taken by rank r */
+    int32_t *used = calloc((size_t)N, sizeof(int32_t));       /* redundant slots used on r */
+    int64_t *home_quota = calloc((size_t)E, sizeof(int64_t));
+    int64_t *ovf = calloc((size_t)E, sizeof(int64_t));
+    orc_ovf *order = calloc((size_t)E, sizeof(orc_ovf));
+    int32_t *asg_e = calloc((size_t)NR + 1, sizeof(int32_t)); /* assignments, allocation order */
+    int32_t *asg_s = calloc((size_t)NR + 1, sizeof(int32_t));
+    int64_t *asg_c = calloc((size_t)NR + 1, sizeof(int64_t));
+    int rc = ORC_OK;
+    if (!cur || !used || !home_quota || !ovf || !order || !asg_e || !asg_s || !asg_c) {
+        rc = ORC_BAD_ARG;
+        goto done;
+    }
+    int flags = 0, n_asg = 0;
+
+    /* Home pass: experts in increasing id; the home rank takes min(load, Q - cur). */
+    for (int e = 0; e < E; ++e) {
+        int h = e / H;
+        int64_t take = load[e] < Q - cur[h] ? load[e] : Q - cur[h];
+        cur[h] += take;
+        home_quota[e] = take;
+        ovf[e] = load[e] - take;
+    }
+
+    /* Overflow order, fixed once: largest overflow first, ties to lower id. */
+    int n_ovf = 0;
+    for (int e = 0; e < E; ++e)
+        if (ovf[e] > 0) { order[n_ovf].ovf = (int32_t)ovf[e]; order[n_ovf].e = e; ++n_ovf; }
+    qsort(order, (size_t)n_ovf, sizeof(orc_ovf), orc_ovf_cmp);
+
+    /* Greedy: each chunk goes to the eligible rank with most spare capacity. */
+    for (int m = 0; m < n_ovf; ++m) {
+        int e = order[m].e, h = e / H;
+        int64_t rem = ovf[e];
+        while (rem > 0) {
+            int best = -1;
+            for (int r = 0; r < N; ++r) {
+                if (used[r] >= R || Q - cur[r] <= 0) continue;   /* not eligible */
+                if (best < 0 || Q - cur[r] > Q - cur[best]) best = r;   /* ties keep lowest r */
+            }
+            if (best < 0) {               /* slots ran out: the rest stays home */
+                home_quota[e] += rem;
+                cur[h] += rem;
+                rem = 0;
+                flags |= 1;
+                break;
+            }
+            if (best == h) { rc = ORC_INVARIANT; goto done; }  /* home is full whenever ovf > 0 */
+            for (int a = 0; a < n_asg; ++a)                      /* one replica of e per rank */
+                if (asg_e[a] == e && asg_s[a] / HR == best) { rc = ORC_INVARIANT; goto done; }
+            int64_t spare = Q - cur[best];
+            int64_t c = rem < spare ? rem : spare;
+            asg_e[n_asg] = e;
+            asg_s[n_asg] = best * HR + H + used[best];
+            asg_c[n_asg] = c;
+            ++n_asg;
+            used[best] += 1;
+            cur[best] += c;
+            rem -= c;
+        }
+    }
+
+    /* Slot table. */
+    for (int s = 0; s < S; ++s) { slot_expert[s] = -1; slot_quota[s] = 0; }
+    for (int e = 0; e < E; ++e) {
+        int s = (e / H) * HR + (e % H);
+        slot_expert[s] = e;
+        slot_quota[s] = (int32_t)home_quota[e];
+    }
+    for (int a = 0; a < n_asg; ++a) {
+        slot_expert[asg_s[a]] = asg_e[a];
+        slot_quota[asg_s[a]] = (int32_t)asg_c[a];
+    }
+
+    /* Replica lists: home first, then redundant slots in allocation order;
+     * rep_cum is the exclusive prefix of the replicas' quotas. */
+    int pos = 0, M = 0;
+    for (int e = 0; e < E; ++e) {
+        rep_off[e] = pos;
+        rep_slot[pos] = (e / H) * HR + (e % H);
+        rep_cum[pos] = 0;
+        int64_t cum = home_quota[e];
+        ++pos;
+        int nred = 0;
+        for (int a = 0; a < n_asg; ++a) {
+            if (asg_e[a] != e) continue;
+            rep_slot[pos] = asg_s[a];
+            rep_cum[pos] = (int32_t)cum;
+            cum += asg_c[a];
+            ++pos;
+            ++nred;
+        }
+        if (cum != load[e]) { rc = ORC_INVARIANT; goto done; }   /* conservation */
+        if (nred > 0) rep_experts[M++] = e;
+    }
+    rep_off[E] = pos;
+    for (int p = pos; p < E + NR; ++p) { rep_slot[p] = -1; rep_cum[p] = -1; }
+    for (int m = M; m < E; ++m) rep_experts[m] = -1;
+
+    int64_t max_before = 0, max_after = 0;
+    for (int r = 0; r < N; ++r) {
+        int64_t before = 0;
+        for (int e = r * H; e < (r + 1) * H; ++e) before += load[e];
+        rank_load_before[r] = (int32_t)before;
+        rank_load_after[r] = (int32_t)cur[r];
+        if (before > max_before) max_before = before;
+        if (cur[r] > max_after) max_after = cur[r];
+    }
+    info[0] = (int32_t)Q;
+    info[1] = (int32_t)L;
+    info[2] = flags;
+    info[3] = M;
+    info[4] = n_asg;
+    info[5] = (int32_t)max_before;
+    info[6] = (int32_t)max_after;
+    info[7] = 0;
+
+done:
+    free(cur); free(used); free(home_quota); free(ovf); free(order);
+    free(asg_e); free(asg_s); free(asg_c);
+    return rc;
+}
+
+/* ---- step 3: routing expansion -------------------------------------------
+ * The j-th occurrence (0-based, token-major (t, k) order) of expert e goes to
+ * the replica i of e with rep_cum[i] <= j < rep_cum[i] + quota of replica i.
+ */
+int ue_oracle_reroute(const int32_t *ids, int64_t T, int K, int E,
+                      const int32_t *rep_off, const int32_t *rep_slot,
+                      const int32_t *rep_cum, const int32_t *slot_quota,
+                      int32_t *phys)
+{
+    if (T < 0 || K < 1 || E < 1) return ORC_BAD_ARG;
+    int64_t *occ = calloc((size_t)E, sizeof(int64_t));
+    if (!occ) return ORC_BAD_ARG;
+    int rc = ORC_OK;
+    for (int64_t t = 0; t < T; ++t) {
+        for (int k = 0; k < K; ++k) {
+            int64_t x = t * K + k;
+            int32_t e = ids[x];
+            if (e < 0 || e >= E) { phys[x] = -1; continue; }
+            int64_t j = occ[e]++;
+            int found = -1;
+            for (int i = rep_off[e]; i < rep_off[e + 1]; ++i) {
+                int64_t lo = rep_cum[i], q = slot_quota[rep_slot[i]];
+                if (lo <= j && j < lo + q) { found = i; break; }
+            }
+            if (found < 0) { rc = ORC_INVARIANT; phys[x] = -1; continue; }
+            phys[x] = rep_slot[found];
+        }
+    }
+    free(occ);
+    return rc;
+}
+
+/* ---- step 4: replica weight sync ------------------------------------------
+ * Every filled redundant slot s (slot_expert[s] = e >= 0, s % (H+R) >= H)
+ * receives a copy of e's home slot.  Slot s starts at byte s * slot_stride of
+ * W; the first nbytes bytes of each slot are copied (nbytes = the slot size
+ * for a full sync, less for a bounded sample).
+ */
+int ue_oracle_sync(uint8_t *W, int64_t slot_stride, int64_t nbytes,
+                   int E, int N, int R, const int32_t *slot_expert)
+{
+    if (E < 1 || N < 1 || R < 0 || E % N != 0 || nbytes > slot_stride || nbytes < 0) return ORC_BAD_ARG;
+    const int H = E / N, HR = H + R, S = N * HR;
+    for (int s = 0; s < S; ++s) {
+        int e = slot_expert[s];
+        if (s % HR < H || e < 0) continue;
+        if (e >= E) return ORC_BAD_ARG;
+        int64_t home = (int64_t)(e / H) * HR + (e % H);
+        memcpy(W + (int64_t)s * slot_stride, W + home * slot_stride, (size_t)nbytes);
+    }
+    return ORC_OK;
+}
+
+/* ---- step 5: replica gradient reduction -----------------------------------
+ * For each expert e with redundant replicas, in replica order i = 1, 2, ...:
+ *     master[e][x] = master[e][x] + float(grad[g(i)][x])
+ * where g(i) is the replica-gradient row of redundant slot rep_slot[i]:
+ * slot r*(H+R) + H + u  ->  row r*R + u.  master rows have stride `mstride`
+ * floats, gradient rows `gstride` elements; n elements of each are reduced.
+ */
+static float orc_bf16_to_f32(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+int ue_oracle_grad_reduce(float *master, int64_t mstride, const void *grads,
+                          int grad_is_bf16, int64_t gstride, int64_t n,
+                          int E, int N, int R,
+                          const int32_t *rep_off, const int32_t *rep_slot)
+{
+    if (E < 1 || N < 1 || R < 0 || E % N != 0 || n < 0) return ORC_BAD_ARG;
+    const int H = E / N, HR = H + R;
+    for (int e = 0; e < E; ++e) {
+        float *m = master + (int64_t)e * mstride;
+        for (int i = rep_off[e] + 1; i < rep_off[e + 1]; ++i) {
+            int s = rep_slot[i];
+            int r = s / HR, u = s % HR - H;
+            if (u < 0 || u >= R) return ORC_INVARIANT;
+            int64_t row = (int64_t)r * R + u;
+            if (grad_is_bf16) {
+                const uint16_t *g = (const uint16_t *)grads + row * gstride;
+                for (int64_t x = 0; x < n; ++x) m[x] = m[x] + orc_bf16_to_f32(g[x]);
+            } else {
+                const float *g = (const float *)grads + row * gstride;
+                for (int64_t x = 0; x < n; ++x) m[x] = m[x] + g[x];
+            }
+        }
+    }
+    return ORC_OK;
+}
