@@ -1,0 +1,169 @@
+/*
+ * ue.h - C ABI of libue.so, a B200 (sm_100a) implementation of the per-layer,
+ * per-microbatch hot path of UltraEP's real-time MoE expert balancer
+ * (arXiv 2606.04101, "UltraEP: Unleash MoE Training and Inference on
+ * Rack-Scale Nodes with Near-Optimal Load Balancing").
+ *
+ * The pipeline runs right after gating (UltraEP news summary, "Comment
+ * fonctionne l'équilibrage en 300 microsecondes"): load computation ->
+ * placement planning -> routing expansion -> replica weight sync, and, in the
+ * backward pass, replica gradient reduction ("How dots-infra/ultraep works",
+ * component list "GPU operations" and its "Connections").  All N
+ * expert-parallel (EP) ranks are simulated as partitions of one GPU's memory.
+ *
+ * Layout shared by every call (E experts, N ranks, H = E / N, R redundant
+ * slots per rank, S = N * (H + R) physical slots):
+ *   - expert e is homed on rank e / H in local slot e % H;
+ *   - physical slot id = r * (H + R) + s; local slots s in [H, H + R) are the
+ *     rank's redundant (replica) slots;
+ *   - token t belongs to source rank t / (T / N); ids are token-major [T][K].
+ *
+ * Conventions.
+ *   - Every array is caller-owned device memory unless stated; the library
+ *     allocates nothing per call.  `stream` is a cudaStream_t (NULL = legacy
+ *     default stream).  Calls are asynchronous and never synchronize the host.
+ *   - Host-detectable errors (null or misaligned pointers, sizes out of
+ *     range) return UE_ERR_INVALID_ARG before any launch; outputs are then
+ *     left untouched.  ue_last_error() gives a one-line reason.
+ *   - Device-detected bad input (an id outside [0, E)) never traps: the id is
+ *     not counted, its rerouted slot is -1, and ue_load reports it per rank.
+ *   - Limits: 1 <= E <= 1024, 1 <= N <= 1024, E % N == 0, 0 <= R,
+ *     N * R <= 4096, 1 <= K, T % N == 0, T * K <= 2^31 - 1.
+ */
+#ifndef UE_H
+#define UE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    UE_OK = 0,
+    UE_ERR_INVALID_ARG = 1,   /* rejected before launch; outputs untouched */
+    UE_ERR_CUDA = 2,          /* a CUDA runtime call or launch failed */
+    UE_ERR_UNSUPPORTED = 3,   /* device is not sm_100 or lacks a needed feature */
+    UE_ERR_DEVICE = 4         /* a kernel gave up a bounded wait (see ue_ctx_device_error) */
+} ue_status;
+
+/* Opaque per-device context: caches device properties and kernel attributes
+ * and owns one device status word for bounded-wait failures. */
+typedef struct ue_ctx ue_ctx;
+
+/* Problem shape.  H = E / N and S = N * (H + R) are derived. */
+typedef struct {
+    int32_t E;   /* experts */
+    int32_t N;   /* simulated EP ranks */
+    int32_t R;   /* redundant (replica) slots per rank */
+    int32_t K;   /* top-k experts per token */
+    int64_t T;   /* tokens in the microbatch (all ranks) */
+} ue_config;
+
+/* The placement plan: device arrays, caller-allocated with the sizes below
+ * (ue_plan_sizes), written by ue_plan and read by ue_reroute, ue_sync and
+ * ue_grad_reduce.  "Placement planning -> Native Manager: placement plan"
+ * ("How dots-infra/ultraep works", Connections). */
+typedef struct {
+    int32_t *slot_expert;       /* [S]    expert held by each physical slot, -1 = empty       */
+    int32_t *slot_quota;        /* [S]    tokens routed to each slot                          */
+    int32_t *rep_off;           /* [E+1]  replicas of e are entries rep_off[e] .. rep_off[e+1]-1 */
+    int32_t *rep_slot;          /* [E+N*R] slot of each replica: home first, then allocation order; -1 tail */
+    int32_t *rep_cum;           /* [E+N*R] exclusive prefix of the replicas' quotas; -1 tail   */
+    int32_t *rep_experts;       /* [E]    experts with >= 1 redundant replica, increasing id; -1 tail */
+    int32_t *load;              /* [E]    exact load: occurrences of e in the microbatch      */
+    int32_t *rank_off;          /* [N*E]  occurrences of e in the tokens of ranks < r          */
+    int32_t *rank_load_before;  /* [N]    tokens routed to rank r's home experts              */
+    int32_t *rank_load_after;   /* [N]    tokens rank r serves under the plan                 */
+    int32_t *info;              /* [8]    Q, L, flags (bit 0: slots ran out), M = #rep_experts,
+                                          filled redundant slots, max before, max after, 0    */
+} ue_plan_buffers;
+
+/* Element counts (int32 entries) of the 11 ue_plan_buffers arrays, in field
+ * order, for a configuration.  Host only. */
+ue_status ue_plan_sizes(const ue_config *cfg, int64_t sizes[11]);
+
+/* Create a context on CUDA device `device` (made current for the call). */
+ue_status ue_ctx_create(int device, ue_ctx **out);
+ue_status ue_ctx_destroy(ue_ctx *ctx);
+
+/* Copy the context's device status word to *host_word (synchronizes
+ * `stream`) and clear it.  Nonzero means a kernel gave up a bounded wait. */
+ue_status ue_ctx_device_error(ue_ctx *ctx, int32_t *host_word, void *stream);
+
+/* ---- step 1: load computation ----------------------------------------------
+ * "Load computation" (csrc/kernels/load_compute.cu in the component list of
+ * "How dots-infra/ultraep works"; "exact-load" in the arXiv abstract).
+ *   ids    [T][K] int32, 16-byte aligned: post-gating top-k expert ids.
+ *   counts [N][E] int32 out: counts[r][e] = #{(t,k): t in rank r, ids[t][k] = e}.
+ *   bad    [N] int32 out, may be NULL: ids of rank r's tokens outside [0, E).
+ * Every entry of counts (and bad) is overwritten; no pre-zeroing needed. */
+ue_status ue_load(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids,
+                  int32_t *counts, int32_t *bad, void *stream);
+
+/* ---- step 2: quota-driven placement planning ---------------------------------
+ * "Placement planning" (csrc/kernels/placement.cu); the quota-driven scheduler
+ * of the news summary.  From counts [N][E] (as written by ue_load):
+ *   load[e] = sum_r counts[r][e], L = sum_e load[e], Q = ceil(L / N);
+ *   home pass in increasing e: the home rank takes min(load, Q - current);
+ *   overflow experts, largest overflow first (ties: lower id), are placed
+ *   chunk by chunk on the rank with most spare capacity Q - current (ties:
+ *   lowest rank) among ranks with a free redundant slot and spare > 0, each
+ *   chunk min(remaining, spare); at most R replicas per rank; if no rank is
+ *   eligible the remainder stays on the home slot (flag bit 0).
+ * Writes every array of *plan (the buffers themselves are read from host
+ * memory; their contents are device memory). */
+ue_status ue_plan(ue_ctx *ctx, const ue_config *cfg, const int32_t *counts,
+                  const ue_plan_buffers *plan, void *stream);
+
+/* ---- step 3: routing expansion ---------------------------------------------
+ * "Routing expansion" (csrc/kernels/reroute.cu; "Routing expansion -> Token
+ * dispatch: physical routing").  The j-th occurrence (0-based, token-major
+ * (t, k) order) of expert e goes to replica i of e with
+ * rep_cum[i] <= j < rep_cum[i] + quota(i):  phys[t][k] = rep_slot[i].
+ *   ids  [T][K] int32, 16-byte aligned (the ids the plan was computed from).
+ *   phys [T][K] int32 out; -1 for ids outside [0, E). */
+ue_status ue_reroute(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids,
+                     const ue_plan_buffers *plan, int32_t *phys, void *stream);
+
+/* Steps 1-3 back to back on one stream (three launches). */
+ue_status ue_rebalance(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids,
+                       int32_t *counts, int32_t *bad, const ue_plan_buffers *plan,
+                       int32_t *phys, void *stream);
+
+/* ---- step 4: replica weight sync ---------------------------------------------
+ * "Replica weight sync" (csrc/kernels/weight_sync.cu; "persistent tile
+ * streaming" with a relay against fan-out overload in the news summary).
+ * For every filled redundant slot s holding expert e, slot s receives a byte
+ * copy of e's home slot.  Each home tile is read once and written to all of
+ * that expert's replicas.
+ *   weights     device base of S slots, slot s at byte s * slot_bytes,
+ *               16-byte aligned; home slots are read, filled redundant slots
+ *               written, empty slots untouched.
+ *   slot_bytes  bytes per slot (3 bf16 matrices: 6 * rows * cols), multiple of 16. */
+ue_status ue_sync(ue_ctx *ctx, const ue_config *cfg, void *weights, int64_t slot_bytes,
+                  const ue_plan_buffers *plan, void *stream);
+
+/* ---- step 5: replica gradient reduction ------------------------------------
+ * "Replica gradient reduction" (csrc/kernels/grad_reduce.cu; "Expert compute
+ * -> Replica gradient reduction: replica gradients", "-> MoE framework:
+ * master gradients").  For every expert e with redundant replicas, in replica
+ * order: master[e][x] = master[e][x] + float(grad[row(i)][x]) (one fp32
+ * round-to-nearest add per replica; bf16 widened exactly), where the replica
+ * gradient row of redundant slot r*(H+R) + H + u is r*R + u.
+ *   master     [E][P] fp32 in/out, 16-byte aligned (rows of unreplicated experts untouched).
+ *   grads      [N*R][P] fp32 (grad_dtype 0) or bf16 (grad_dtype 1), 16-byte aligned.
+ *   P          elements per expert, multiple of 8. */
+ue_status ue_grad_reduce(ue_ctx *ctx, const ue_config *cfg, float *master,
+                         const void *grads, int grad_dtype, int64_t P,
+                         const ue_plan_buffers *plan, void *stream);
+
+/* Status name, and the reason for the last non-OK status on this thread. */
+const char *ue_status_string(ue_status s);
+const char *ue_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* UE_H */

@@ -1,0 +1,344 @@
+// C ABI of libue.so: argument validation, per-device context and launches.
+// See include/ue.h for the contract of every entry point.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "ue_internal.cuh"
+
+namespace ue {
+cudaError_t set_load_attributes(size_t max_smem);
+cudaError_t set_reroute_attributes(size_t max_smem);
+cudaError_t set_plan_attributes(size_t max_smem);
+cudaError_t set_sync_attributes(size_t max_smem);
+int grad_blocks_per_sm(int grad_dtype);
+}  // namespace ue
+
+struct ue_ctx {
+    int device;
+    int sms;
+    int max_smem;          // opt-in dynamic shared memory per block
+    int grad_blocks[2];    // resident grad-reduce CTAs per SM (fp32, bf16)
+    int32_t *dev_err;      // device status word for bounded waits
+};
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+ue_status fail(ue_status s, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+ue_status cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(UE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Validates the shape; fills `sh`.  `need_tokens` adds the T/K checks.
+ue_status make_shape(const ue_config *cfg, bool need_tokens, ue::Shape *sh)
+{
+    if (!cfg) return fail(UE_ERR_INVALID_ARG, "config is NULL");
+    const ue_config c = *cfg;
+    if (c.E < 1 || c.E > ue::kMaxE) return fail(UE_ERR_INVALID_ARG, "E=%d outside [1, %d]", c.E, ue::kMaxE);
+    if (c.N < 1 || c.N > ue::kMaxN) return fail(UE_ERR_INVALID_ARG, "N=%d outside [1, %d]", c.N, ue::kMaxN);
+    if (c.E % c.N != 0) return fail(UE_ERR_INVALID_ARG, "E=%d is not a multiple of N=%d", c.E, c.N);
+    if (c.R < 0 || (int64_t)c.N * c.R > ue::kMaxNR)
+        return fail(UE_ERR_INVALID_ARG, "R=%d invalid (need 0 <= R and N*R <= %d)", c.R, ue::kMaxNR);
+    if (need_tokens) {
+        if (c.K < 1) return fail(UE_ERR_INVALID_ARG, "K=%d < 1", c.K);
+        if (c.T < 0 || c.T % c.N != 0)
+            return fail(UE_ERR_INVALID_ARG, "T=%lld must be >= 0 and a multiple of N=%d", (long long)c.T, c.N);
+        if (c.T * (int64_t)c.K > (int64_t)INT32_MAX)
+            return fail(UE_ERR_INVALID_ARG, "T*K=%lld exceeds 2^31-1", (long long)(c.T * c.K));
+    }
+    sh->E = c.E;
+    sh->N = c.N;
+    sh->R = c.R;
+    sh->K = c.K;
+    sh->H = c.E / c.N;
+    sh->HR = sh->H + c.R;
+    sh->S = c.N * sh->HR;
+    sh->NR = c.N * c.R;
+    sh->T = c.T;
+    sh->per_rank = need_tokens ? (c.T / c.N) * c.K : 0;
+    return UE_OK;
+}
+
+ue_status check_plan(const ue_plan_buffers *p)
+{
+    if (!p) return fail(UE_ERR_INVALID_ARG, "plan is NULL");
+    const int32_t *f[11] = {p->slot_expert, p->slot_quota, p->rep_off, p->rep_slot, p->rep_cum, p->rep_experts,
+                            p->load, p->rank_off, p->rank_load_before, p->rank_load_after, p->info};
+    for (int i = 0; i < 11; ++i)
+        if (!f[i]) return fail(UE_ERR_INVALID_ARG, "plan array %d is NULL", i);
+    return UE_OK;
+}
+
+ue_status check_ctx(const ue_ctx *ctx)
+{
+    if (!ctx) return fail(UE_ERR_INVALID_ARG, "context is NULL");
+    return UE_OK;
+}
+
+// Clusters of CTAs per simulated rank for load / reroute: enough CTAs to fill
+// the GPU about twice, each with at least 2048 ids.
+int choose_cluster(const ue::Shape &sh, int sms)
+{
+    int C = 1;
+    while (C < ue::kMaxCluster && (int64_t)sh.N * C < 2 * (int64_t)sms && sh.per_rank / (2 * C) >= 2048) C *= 2;
+    return C;
+}
+
+ue::Launch launch_of(const ue_ctx *ctx, const ue::Shape &sh)
+{
+    ue::Launch ln;
+    ln.sms = ctx->sms;
+    ln.cluster = choose_cluster(sh, ctx->sms);
+    return ln;
+}
+
+// Run fn with ctx's device current, restoring the caller's device.
+template <class F>
+ue_status on_device(const ue_ctx *ctx, F &&fn)
+{
+    int prev = -1;
+    cudaError_t e = cudaGetDevice(&prev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (prev != ctx->device && (e = cudaSetDevice(ctx->device)) != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+    ue_status s = fn();
+    if (prev != ctx->device) cudaSetDevice(prev);
+    return s;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *ue_status_string(ue_status s)
+{
+    switch (s) {
+    case UE_OK: return "UE_OK";
+    case UE_ERR_INVALID_ARG: return "UE_ERR_INVALID_ARG";
+    case UE_ERR_CUDA: return "UE_ERR_CUDA";
+    case UE_ERR_UNSUPPORTED: return "UE_ERR_UNSUPPORTED";
+    case UE_ERR_DEVICE: return "UE_ERR_DEVICE";
+    }
+    return "UE_ERR_UNKNOWN";
+}
+
+const char *ue_last_error(void) { return g_last_error; }
+
+ue_status ue_plan_sizes(const ue_config *cfg, int64_t sizes[11])
+{
+    ue::Shape sh{};
+    ue_status s = make_shape(cfg, false, &sh);
+    if (s != UE_OK) return s;
+    if (!sizes) return fail(UE_ERR_INVALID_ARG, "sizes is NULL");
+    const int64_t v[11] = {sh.S, sh.S, sh.E + 1, sh.E + sh.NR, sh.E + sh.NR, sh.E,
+                           sh.E, (int64_t)sh.N * sh.E, sh.N, sh.N, 8};
+    memcpy(sizes, v, sizeof v);
+    return UE_OK;
+}
+
+ue_status ue_ctx_create(int device, ue_ctx **out)
+{
+    if (!out) return fail(UE_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    int ndev = 0;
+    cudaError_t e = cudaGetDeviceCount(&ndev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceCount");
+    if (device < 0 || device >= ndev) return fail(UE_ERR_INVALID_ARG, "device %d not in [0, %d)", device, ndev);
+    cudaDeviceProp prop;
+    if ((e = cudaGetDeviceProperties(&prop, device)) != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+    if (prop.major != 10)
+        return fail(UE_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", device,
+                    prop.major, prop.minor);
+    ue_ctx tmp;
+    tmp.device = device;
+    tmp.sms = prop.multiProcessorCount;
+    tmp.max_smem = (int)prop.sharedMemPerBlockOptin;
+    tmp.dev_err = nullptr;
+    ue_status s = on_device(&tmp, [&]() -> ue_status {
+        cudaError_t err;
+        const size_t m = (size_t)tmp.max_smem;
+        if ((err = ue::set_load_attributes(m)) != cudaSuccess) return cuda_fail(err, "load attributes");
+        if ((err = ue::set_reroute_attributes(m)) != cudaSuccess) return cuda_fail(err, "reroute attributes");
+        if ((err = ue::set_plan_attributes(m)) != cudaSuccess) return cuda_fail(err, "plan attributes");
+        if ((err = ue::set_sync_attributes(m)) != cudaSuccess) return cuda_fail(err, "sync attributes");
+        tmp.grad_blocks[0] = ue::grad_blocks_per_sm(0);
+        tmp.grad_blocks[1] = ue::grad_blocks_per_sm(1);
+        if ((err = cudaMalloc(&tmp.dev_err, sizeof(int32_t))) != cudaSuccess) return cuda_fail(err, "cudaMalloc");
+        if ((err = cudaMemset(tmp.dev_err, 0, sizeof(int32_t))) != cudaSuccess) {
+            cudaFree(tmp.dev_err);
+            return cuda_fail(err, "cudaMemset");
+        }
+        return UE_OK;
+    });
+    if (s != UE_OK) return s;
+    ue_ctx *ctx = new (std::nothrow) ue_ctx(tmp);
+    if (!ctx) {
+        on_device(&tmp, [&]() { cudaFree(tmp.dev_err); return UE_OK; });
+        return fail(UE_ERR_INVALID_ARG, "out of host memory");
+    }
+    *out = ctx;
+    return UE_OK;
+}
+
+ue_status ue_ctx_destroy(ue_ctx *ctx)
+{
+    if (!ctx) return UE_OK;
+    ue_status s = on_device(ctx, [&]() -> ue_status {
+        cudaError_t e = cudaFree(ctx->dev_err);
+        return e == cudaSuccess ? UE_OK : cuda_fail(e, "cudaFree");
+    });
+    delete ctx;
+    return s;
+}
+
+ue_status ue_ctx_device_error(ue_ctx *ctx, int32_t *host_word, void *stream)
+{
+    ue_status s = check_ctx(ctx);
+    if (s != UE_OK) return s;
+    if (!host_word) return fail(UE_ERR_INVALID_ARG, "host_word is NULL");
+    return on_device(ctx, [&]() -> ue_status {
+        cudaStream_t st = static_cast<cudaStream_t>(stream);
+        cudaError_t e = cudaMemcpyAsync(host_word, ctx->dev_err, sizeof(int32_t), cudaMemcpyDeviceToHost, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(ctx->dev_err, 0, sizeof(int32_t), st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        return e == cudaSuccess ? UE_OK : cuda_fail(e, "device status word");
+    });
+}
+
+ue_status ue_load(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids, int32_t *counts, int32_t *bad,
+                  void *stream)
+{
+    ue::Shape sh{};
+    ue_status s = make_shape(cfg, true, &sh);
+    if (s != UE_OK) return s;
+    if (!counts) return fail(UE_ERR_INVALID_ARG, "counts is NULL");
+    if (sh.T > 0 && (!ids || !aligned16(ids))) return fail(UE_ERR_INVALID_ARG, "ids must be non-NULL and 16-byte aligned");
+    if ((s = check_ctx(ctx)) != UE_OK) return s;
+    return on_device(ctx, [&]() -> ue_status {
+        cudaError_t e = ue::launch_load(sh, launch_of(ctx, sh), ids, counts, bad, static_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? UE_OK : cuda_fail(e, "load launch");
+    });
+}
+
+ue_status ue_plan(ue_ctx *ctx, const ue_config *cfg, const int32_t *counts, const ue_plan_buffers *plan,
+                  void *stream)
+{
+    ue::Shape sh{};
+    ue_status s = make_shape(cfg, false, &sh);
+    if (s == UE_OK) s = check_plan(plan);
+    if (s != UE_OK) return s;
+    if (!counts) return fail(UE_ERR_INVALID_ARG, "counts is NULL");
+    if ((s = check_ctx(ctx)) != UE_OK) return s;
+    if (ue::plan_smem_bytes(sh) > (size_t)ctx->max_smem)
+        return fail(UE_ERR_INVALID_ARG, "plan needs %zu bytes of shared memory (> %d)", ue::plan_smem_bytes(sh),
+                    ctx->max_smem);
+    return on_device(ctx, [&]() -> ue_status {
+        cudaError_t e = ue::launch_plan(sh, counts, ue::to_dev(*plan), static_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? UE_OK : cuda_fail(e, "plan launch");
+    });
+}
+
+ue_status ue_reroute(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids, const ue_plan_buffers *plan,
+                     int32_t *phys, void *stream)
+{
+    ue::Shape sh{};
+    ue_status s = make_shape(cfg, true, &sh);
+    if (s == UE_OK) s = check_plan(plan);
+    if (s != UE_OK) return s;
+    if (sh.T > 0 && (!ids || !aligned16(ids))) return fail(UE_ERR_INVALID_ARG, "ids must be non-NULL and 16-byte aligned");
+    if (sh.T > 0 && !phys) return fail(UE_ERR_INVALID_ARG, "phys is NULL");
+    if ((s = check_ctx(ctx)) != UE_OK) return s;
+    if (ue::reroute_smem_bytes(sh) > (size_t)ctx->max_smem)
+        return fail(UE_ERR_INVALID_ARG, "reroute needs %zu bytes of shared memory (> %d)", ue::reroute_smem_bytes(sh),
+                    ctx->max_smem);
+    return on_device(ctx, [&]() -> ue_status {
+        cudaError_t e = ue::launch_reroute(sh, launch_of(ctx, sh), ids, ue::to_dev(*plan), phys,
+                                           static_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? UE_OK : cuda_fail(e, "reroute launch");
+    });
+}
+
+ue_status ue_rebalance(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids, int32_t *counts, int32_t *bad,
+                       const ue_plan_buffers *plan, int32_t *phys, void *stream)
+{
+    // Validate everything before the first launch so a refusal leaves all outputs untouched.
+    ue::Shape sh{};
+    ue_status s = make_shape(cfg, true, &sh);
+    if (s == UE_OK) s = check_plan(plan);
+    if (s != UE_OK) return s;
+    if (!counts) return fail(UE_ERR_INVALID_ARG, "counts is NULL");
+    if (sh.T > 0 && (!ids || !aligned16(ids))) return fail(UE_ERR_INVALID_ARG, "ids must be non-NULL and 16-byte aligned");
+    if (sh.T > 0 && !phys) return fail(UE_ERR_INVALID_ARG, "phys is NULL");
+    if ((s = check_ctx(ctx)) != UE_OK) return s;
+    if (ue::plan_smem_bytes(sh) > (size_t)ctx->max_smem || ue::reroute_smem_bytes(sh) > (size_t)ctx->max_smem)
+        return fail(UE_ERR_INVALID_ARG, "shape needs more shared memory than the device offers");
+    return on_device(ctx, [&]() -> ue_status {
+        const cudaStream_t st = static_cast<cudaStream_t>(stream);
+        const ue::Launch ln = launch_of(ctx, sh);
+        const ue::PlanDev pd = ue::to_dev(*plan);
+        cudaError_t e = ue::launch_load(sh, ln, ids, counts, bad, st);
+        if (e != cudaSuccess) return cuda_fail(e, "load launch");
+        if ((e = ue::launch_plan(sh, counts, pd, st)) != cudaSuccess) return cuda_fail(e, "plan launch");
+        if ((e = ue::launch_reroute(sh, ln, ids, pd, phys, st)) != cudaSuccess) return cuda_fail(e, "reroute launch");
+        return UE_OK;
+    });
+}
+
+ue_status ue_sync(ue_ctx *ctx, const ue_config *cfg, void *weights, int64_t slot_bytes, const ue_plan_buffers *plan,
+                  void *stream)
+{
+    ue::Shape sh{};
+    ue_status s = make_shape(cfg, false, &sh);
+    if (s == UE_OK) s = check_plan(plan);
+    if (s != UE_OK) return s;
+    if (!weights || !aligned16(weights)) return fail(UE_ERR_INVALID_ARG, "weights must be non-NULL and 16-byte aligned");
+    if (slot_bytes <= 0 || slot_bytes % 16 != 0)
+        return fail(UE_ERR_INVALID_ARG, "slot_bytes=%lld must be a positive multiple of 16", (long long)slot_bytes);
+    if ((s = check_ctx(ctx)) != UE_OK) return s;
+    if (ue::sync_smem_bytes(sh) > (size_t)ctx->max_smem)
+        return fail(UE_ERR_INVALID_ARG, "sync needs %zu bytes of shared memory (> %d)", ue::sync_smem_bytes(sh),
+                    ctx->max_smem);
+    return on_device(ctx, [&]() -> ue_status {
+        cudaError_t e = ue::launch_sync(sh, launch_of(ctx, sh), static_cast<uint8_t *>(weights), slot_bytes,
+                                        ue::to_dev(*plan), ctx->dev_err, static_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? UE_OK : cuda_fail(e, "sync launch");
+    });
+}
+
+ue_status ue_grad_reduce(ue_ctx *ctx, const ue_config *cfg, float *master, const void *grads, int grad_dtype,
+                         int64_t P, const ue_plan_buffers *plan, void *stream)
+{
+    ue::Shape sh{};
+    ue_status s = make_shape(cfg, false, &sh);
+    if (s == UE_OK) s = check_plan(plan);
+    if (s != UE_OK) return s;
+    if (grad_dtype != 0 && grad_dtype != 1) return fail(UE_ERR_INVALID_ARG, "grad_dtype=%d (0 = fp32, 1 = bf16)", grad_dtype);
+    if (P <= 0 || P % 8 != 0) return fail(UE_ERR_INVALID_ARG, "P=%lld must be a positive multiple of 8", (long long)P);
+    if (!master || !aligned16(master)) return fail(UE_ERR_INVALID_ARG, "master must be non-NULL and 16-byte aligned");
+    if (sh.NR > 0 && (!grads || !aligned16(grads)))
+        return fail(UE_ERR_INVALID_ARG, "grads must be non-NULL and 16-byte aligned");
+    if ((s = check_ctx(ctx)) != UE_OK) return s;
+    return on_device(ctx, [&]() -> ue_status {
+        ue::Launch ln = launch_of(ctx, sh);
+        ln.sms = ctx->sms * ctx->grad_blocks[grad_dtype];
+        cudaError_t e = ue::launch_grad_reduce(sh, ln, master, grads, grad_dtype, P, ue::to_dev(*plan),
+                                               static_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? UE_OK : cuda_fail(e, "grad-reduce launch");
+    });
+}
+
+}  // extern "C"

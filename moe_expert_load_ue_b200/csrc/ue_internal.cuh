@@ -1,0 +1,82 @@
+// Internal declarations shared by the kernels of libue.so (sm_100a only).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "ue.h"
+
+namespace ue {
+
+// Limits of the C ABI (also stated in ue.h).
+constexpr int kMaxE = 1024;
+constexpr int kMaxN = 1024;
+constexpr int kMaxNR = 4096;
+constexpr int kMaxCluster = 8;        // portable cluster size
+
+// Device-side view of the plan (same arrays as ue_plan_buffers).
+struct PlanDev {
+    int32_t *slot_expert, *slot_quota, *rep_off, *rep_slot, *rep_cum, *rep_experts;
+    int32_t *load, *rank_off, *rank_load_before, *rank_load_after, *info;
+};
+
+inline PlanDev to_dev(const ue_plan_buffers &p)
+{
+    return PlanDev{p.slot_expert, p.slot_quota, p.rep_off, p.rep_slot, p.rep_cum, p.rep_experts,
+                   p.load, p.rank_off, p.rank_load_before, p.rank_load_after, p.info};
+}
+
+// Shape derived from ue_config.
+struct Shape {
+    int E, N, R, K, H, HR, S, NR;
+    int64_t T, per_rank;   // per_rank = (T / N) * K ids of each source rank
+};
+
+// Per-launch choices made on the host.
+struct Launch {
+    int sms;               // SM count of the device
+    int cluster;           // CTAs per simulated rank for load / reroute
+};
+
+// Host launchers (one per kernel file).  Each returns cudaGetLastError().
+cudaError_t launch_load(const Shape &sh, const Launch &ln, const int32_t *ids, int32_t *counts,
+                        int32_t *bad, cudaStream_t st);
+size_t load_smem_bytes(const Shape &sh);
+
+cudaError_t launch_plan(const Shape &sh, const int32_t *counts, const PlanDev &plan, cudaStream_t st);
+size_t plan_smem_bytes(const Shape &sh);
+int plan_cluster(const Shape &sh);
+
+cudaError_t launch_reroute(const Shape &sh, const Launch &ln, const int32_t *ids, const PlanDev &plan,
+                           int32_t *phys, cudaStream_t st);
+size_t reroute_smem_bytes(const Shape &sh);
+
+cudaError_t launch_sync(const Shape &sh, const Launch &ln, uint8_t *weights, int64_t slot_bytes,
+                        const PlanDev &plan, int32_t *dev_err, cudaStream_t st);
+size_t sync_smem_bytes(const Shape &sh);
+
+cudaError_t launch_grad_reduce(const Shape &sh, const Launch &ln, float *master, const void *grads,
+                               int grad_dtype, int64_t P, const PlanDev &plan, cudaStream_t st);
+size_t grad_smem_bytes(const Shape &sh);
+
+// Kernel attribute set-up (dynamic shared memory opt-in), once per device.
+cudaError_t set_kernel_attributes();
+
+// ---- device helpers ---------------------------------------------------------
+
+__device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
+
+__device__ __forceinline__ unsigned lanemask_lt()
+{
+    unsigned m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+__device__ __forceinline__ int clampi(int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi : v); }
+
+// Split cluster barrier (release on arrive, acquire on wait).
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+
+}  // namespace ue

@@ -1,0 +1,195 @@
+// Step 4 - replica weight sync: home slot -> every redundant slot of the expert.
+//
+// "Replica weight sync" (csrc/kernels/weight_sync.cu in "How dots-infra/ultraep
+// works"; the news summary describes the transfers of expert states as
+// persistent tile streaming with a relay mechanism against fan-out overload).
+//
+// Design (sm_100a): a persistent grid, one CTA per SM.  Work items are
+// (replicated expert m, tile t) pairs, dealt round-robin to the CTAs.  One
+// elected thread per CTA streams them through a ring of shared-memory stages
+// with the Tensor Memory Accelerator's bulk copies (no tensor maps):
+//   cp.async.bulk global->shared  (completion on an mbarrier, expect_tx)
+//   cp.async.bulk shared->global  once per replica of the expert (bulk_group)
+// so each home tile is read from HBM once and fanned out to all of its
+// replicas - the one-GPU form of the pages' relay against fan-out overload.
+// Stage reuse waits on cp.async.bulk.wait_group.read.  No multicast anywhere.
+// Every mbarrier wait is bounded by the global timer; on timeout the kernel
+// records an error in the context's status word, drains its stores and exits.
+#include "ue_internal.cuh"
+
+namespace ue {
+namespace {
+
+constexpr int kSyncThreads = 128;
+constexpr int kSyncStages = 4;
+constexpr int kSyncTile = 48 * 1024;                       // bytes per stage
+constexpr unsigned long long kWaitLimitNs = 2000000000ull; // 2 s per wait
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ unsigned long long global_ns()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, unsigned count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, unsigned bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity)
+{
+    unsigned ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ void bulk_load(void *dst_smem, const void *src, unsigned bytes, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst_smem)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_store(void *dst, const void *src_smem, unsigned bytes)
+{
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+                 "r"(smem_addr(src_smem)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+struct SyncItem {
+    const uint8_t *src;
+    unsigned bytes;
+    int m;
+    int64_t offset;
+};
+
+__global__ void __launch_bounds__(kSyncThreads, 1)
+k_sync(uint8_t *__restrict__ W, int64_t slot_bytes, int E, int S, int cap,
+       const int32_t *__restrict__ rep_off, const int32_t *__restrict__ rep_slot,
+       const int32_t *__restrict__ rep_experts, const int32_t *__restrict__ info,
+       int32_t *__restrict__ dev_err)
+{
+    extern __shared__ __align__(128) uint8_t sm_sync[];
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm_sync);                 // [stages]
+    uint8_t *stage = sm_sync + 128;                                        // [stages][tile]
+    int32_t *x_home = reinterpret_cast<int32_t *>(stage + (size_t)kSyncStages * kSyncTile);  // [E]
+    int32_t *x_first = x_home + E;                                         // [E] first redundant entry
+    int32_t *x_cnt = x_first + E;                                          // [E] redundant replicas
+    int32_t *x_slot = x_cnt + E;                                           // [cap]
+
+    const int M = clampi(__ldg(info + 3), 0, E);
+    for (int m = threadIdx.x; m < M; m += blockDim.x) {
+        const int e = clampi(__ldg(rep_experts + m), 0, E - 1);
+        const int off = clampi(__ldg(rep_off + e), 0, cap - 1);
+        const int end = clampi(__ldg(rep_off + e + 1), off + 1, cap);
+        x_home[m] = clampi(__ldg(rep_slot + off), 0, S - 1);
+        x_first[m] = off + 1;
+        x_cnt[m] = end - off - 1;
+    }
+    for (int p = threadIdx.x; p < cap; p += blockDim.x) x_slot[p] = clampi(__ldg(rep_slot + p), 0, S - 1);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kSyncStages; ++i) mbar_init(&bar[i], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x != 0 || M == 0) return;
+
+    const int64_t ntiles = (slot_bytes + kSyncTile - 1) / kSyncTile;
+    const int64_t total = (int64_t)M * ntiles;
+    if ((int64_t)blockIdx.x >= total) return;
+    const int64_t nmy = (total - 1 - blockIdx.x) / gridDim.x + 1;
+
+    auto item = [&](int64_t k) {
+        const int64_t i = (int64_t)blockIdx.x + k * gridDim.x;
+        SyncItem it;
+        it.m = (int)(i % M);
+        const int64_t t = i / M;
+        it.offset = t * kSyncTile;
+        const int64_t left = slot_bytes - it.offset;
+        it.bytes = (unsigned)(left < kSyncTile ? left : kSyncTile);
+        it.src = W + (int64_t)x_home[it.m] * slot_bytes + it.offset;
+        return it;
+    };
+    auto issue_load = [&](int64_t k) {
+        const SyncItem it = item(k);
+        const int b = (int)(k % kSyncStages);
+        mbar_expect_tx(&bar[b], it.bytes);
+        bulk_load(stage + (size_t)b * kSyncTile, it.src, it.bytes, &bar[b]);
+    };
+
+    for (int64_t k = 0; k < nmy && k < kSyncStages; ++k) issue_load(k);
+    for (int64_t k = 0; k < nmy; ++k) {
+        const int b = (int)(k % kSyncStages);
+        const unsigned parity = (unsigned)((k / kSyncStages) & 1);
+        if (!mbar_try_wait(&bar[b], parity)) {
+            const unsigned long long t0 = global_ns();
+            while (!mbar_try_wait(&bar[b], parity)) {
+                if (global_ns() - t0 > kWaitLimitNs) {
+                    atomicOr(dev_err, 1);
+                    bulk_wait_all();
+                    return;
+                }
+            }
+        }
+        const SyncItem it = item(k);
+        const uint8_t *src = stage + (size_t)b * kSyncTile;
+        const int first = x_first[it.m], cnt = x_cnt[it.m];
+        for (int j = 0; j < cnt; ++j)
+            bulk_store(W + (int64_t)x_slot[first + j] * slot_bytes + it.offset, src, it.bytes);
+        bulk_commit();
+        // Refill the previous stage once its stores have read it.
+        if (k >= 1 && k - 1 + kSyncStages < nmy) {
+            bulk_wait_read_1();
+            issue_load(k - 1 + kSyncStages);
+        }
+    }
+    bulk_wait_all();
+}
+
+}  // namespace
+
+size_t sync_smem_bytes(const Shape &sh)
+{
+    return 128 + (size_t)kSyncStages * kSyncTile + (size_t)(3 * sh.E + sh.E + sh.NR) * sizeof(int32_t);
+}
+
+cudaError_t launch_sync(const Shape &sh, const Launch &ln, uint8_t *weights, int64_t slot_bytes,
+                        const PlanDev &plan, int32_t *dev_err, cudaStream_t st)
+{
+    k_sync<<<ln.sms, kSyncThreads, sync_smem_bytes(sh), st>>>(weights, slot_bytes, sh.E, sh.S, sh.E + sh.NR,
+                                                               plan.rep_off, plan.rep_slot, plan.rep_experts,
+                                                               plan.info, dev_err);
+    return cudaGetLastError();
+}
+
+cudaError_t set_sync_attributes(size_t max_smem)
+{
+    return cudaFuncSetAttribute(k_sync, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)max_smem);
+}
+
+}  // namespace ue

@@ -1,0 +1,227 @@
+"""Thin Python binding of libue.so (argument marshalling only).
+
+Every function here forwards torch CUDA tensors (device pointers), sizes and
+the current CUDA stream to the C ABI declared in include/ue.h; every step of
+the balancer runs in the library's sm_100a kernels.  There is no CPU path:
+if libue.so is missing or the device is not sm_100, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libue.so")
+
+UE_OK, UE_ERR_INVALID_ARG, UE_ERR_CUDA, UE_ERR_UNSUPPORTED, UE_ERR_DEVICE = range(5)
+
+PLAN_FIELDS = ("slot_expert", "slot_quota", "rep_off", "rep_slot", "rep_cum", "rep_experts",
+               "load", "rank_off", "rank_load_before", "rank_load_after", "info")
+
+# Entry points declared in include/ue.h (checked against the header by the tests).
+EXPORTS = ("ue_plan_sizes", "ue_ctx_create", "ue_ctx_destroy", "ue_ctx_device_error", "ue_load",
+           "ue_plan", "ue_reroute", "ue_rebalance", "ue_sync", "ue_grad_reduce",
+           "ue_status_string", "ue_last_error")
+
+
+class UeConfig(ctypes.Structure):
+    _fields_ = [("E", ctypes.c_int32), ("N", ctypes.c_int32), ("R", ctypes.c_int32),
+                ("K", ctypes.c_int32), ("T", ctypes.c_int64)]
+
+
+class UePlanBuffers(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_void_p) for f in PLAN_FIELDS]
+
+
+class UeError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        super().__init__(f"{where}: {_status_name(status)}: {detail}")
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib() -> ctypes.CDLL:
+    """Load libue.so (raises if it was not built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(f"{LIB_PATH} is missing: build it with "
+                                  "`python -m moe_expert_load_ue_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, i64, ci = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+            cfgp, planp = ctypes.POINTER(UeConfig), ctypes.POINTER(UePlanBuffers)
+            sig = {
+                "ue_plan_sizes": [cfgp, ctypes.POINTER(ctypes.c_int64)],
+                "ue_ctx_create": [ci, ctypes.POINTER(vp)],
+                "ue_ctx_destroy": [vp],
+                "ue_ctx_device_error": [vp, ctypes.POINTER(ctypes.c_int32), vp],
+                "ue_load": [vp, cfgp, vp, vp, vp, vp],
+                "ue_plan": [vp, cfgp, vp, planp, vp],
+                "ue_reroute": [vp, cfgp, vp, planp, vp, vp],
+                "ue_rebalance": [vp, cfgp, vp, vp, vp, planp, vp, vp],
+                "ue_sync": [vp, cfgp, vp, i64, planp, vp],
+                "ue_grad_reduce": [vp, cfgp, vp, vp, ci, i64, planp, vp],
+            }
+            for name, args in sig.items():
+                fn = getattr(L, name)
+                fn.argtypes = args
+                fn.restype = ci
+            L.ue_status_string.argtypes = [ci]
+            L.ue_status_string.restype = ctypes.c_char_p
+            L.ue_last_error.argtypes = []
+            L.ue_last_error.restype = ctypes.c_char_p
+            _lib = L
+    return _lib
+
+
+def _status_name(s: int) -> str:
+    try:
+        return lib().ue_status_string(s).decode()
+    except Exception:  # pragma: no cover
+        return str(s)
+
+
+def _check(status: int, where: str) -> None:
+    if status != UE_OK:
+        raise UeError(status, where, lib().ue_last_error().decode())
+
+
+@dataclasses.dataclass(frozen=True)
+class Config:
+    E: int
+    N: int
+    R: int
+    K: int = 8
+    T: int = 0
+
+    @property
+    def H(self) -> int:
+        return self.E // self.N
+
+    @property
+    def S(self) -> int:
+        return self.N * (self.H + self.R)
+
+    def c(self) -> UeConfig:
+        return UeConfig(self.E, self.N, self.R, self.K, self.T)
+
+
+def plan_sizes(cfg: Config) -> dict:
+    sizes = (ctypes.c_int64 * 11)()
+    _check(lib().ue_plan_sizes(ctypes.byref(cfg.c()), sizes), "ue_plan_sizes")
+    return dict(zip(PLAN_FIELDS, list(sizes)))
+
+
+class Plan:
+    """Device buffers of one placement plan (int32 torch tensors)."""
+
+    def __init__(self, cfg: Config, device="cuda"):
+        self.cfg = cfg
+        self.tensors = {f: torch.empty(n, dtype=torch.int32, device=device)
+                        for f, n in plan_sizes(cfg).items()}
+        self.tensors["rank_off"] = self.tensors["rank_off"].view(cfg.N, cfg.E)
+        self._c = UePlanBuffers(*[self.tensors[f].data_ptr() for f in PLAN_FIELDS])
+
+    def __getitem__(self, k):
+        return self.tensors[k]
+
+    def ref(self):
+        return ctypes.byref(self._c)
+
+    def to_host(self) -> dict:
+        return {k: v.cpu().numpy() for k, v in self.tensors.items()}
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * 4 for t in self.tensors.values())
+
+
+def _stream(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+class Context:
+    """ue_ctx for one CUDA device."""
+
+    def __init__(self, device: int | None = None):
+        if device is None:
+            device = torch.cuda.current_device()
+        self.device = device
+        h = ctypes.c_void_p()
+        _check(lib().ue_ctx_create(device, ctypes.byref(h)), "ue_ctx_create")
+        self._h = h
+
+    @property
+    def handle(self):
+        return self._h
+
+    def close(self):
+        if self._h:
+            _check(lib().ue_ctx_destroy(self._h), "ue_ctx_destroy")
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):  # pragma: no cover
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def device_error(self, stream=None) -> int:
+        w = ctypes.c_int32(0)
+        _check(lib().ue_ctx_device_error(self._h, ctypes.byref(w), _stream(stream)), "ue_ctx_device_error")
+        return w.value
+
+
+# ---- the five steps, under the C ABI's names ---------------------------------
+
+def ue_load(ctx: Context, cfg: Config, ids: torch.Tensor, counts: torch.Tensor,
+            bad: torch.Tensor | None = None, stream=None) -> None:
+    _check(lib().ue_load(ctx.handle, ctypes.byref(cfg.c()), _ptr(ids), _ptr(counts), _ptr(bad),
+                         _stream(stream)), "ue_load")
+
+
+def ue_plan(ctx: Context, cfg: Config, counts: torch.Tensor, plan: Plan, stream=None) -> None:
+    _check(lib().ue_plan(ctx.handle, ctypes.byref(cfg.c()), _ptr(counts), plan.ref(), _stream(stream)),
+           "ue_plan")
+
+
+def ue_reroute(ctx: Context, cfg: Config, ids: torch.Tensor, plan: Plan, phys: torch.Tensor,
+               stream=None) -> None:
+    _check(lib().ue_reroute(ctx.handle, ctypes.byref(cfg.c()), _ptr(ids), plan.ref(), _ptr(phys),
+                            _stream(stream)), "ue_reroute")
+
+
+def ue_rebalance(ctx: Context, cfg: Config, ids: torch.Tensor, counts: torch.Tensor,
+                 bad: torch.Tensor | None, plan: Plan, phys: torch.Tensor, stream=None) -> None:
+    _check(lib().ue_rebalance(ctx.handle, ctypes.byref(cfg.c()), _ptr(ids), _ptr(counts), _ptr(bad),
+                              plan.ref(), _ptr(phys), _stream(stream)), "ue_rebalance")
+
+
+def ue_sync(ctx: Context, cfg: Config, weights: torch.Tensor, slot_bytes: int, plan: Plan,
+            stream=None) -> None:
+    _check(lib().ue_sync(ctx.handle, ctypes.byref(cfg.c()), _ptr(weights), int(slot_bytes), plan.ref(),
+                         _stream(stream)), "ue_sync")
+
+
+def ue_grad_reduce(ctx: Context, cfg: Config, master: torch.Tensor, grads: torch.Tensor, P: int,
+                   plan: Plan, stream=None) -> None:
+    if grads.dtype == torch.bfloat16:
+        dt = 1
+    elif grads.dtype == torch.float32:
+        dt = 0
+    else:
+        raise TypeError("replica grads must be float32 or bfloat16")
+    _check(lib().ue_grad_reduce(ctx.handle, ctypes.byref(cfg.c()), _ptr(master), _ptr(grads), dt, int(P),
+                                plan.ref(), _stream(stream)), "ue_grad_reduce")
