@@ -1,0 +1,479 @@
+#!/usr/bin/env python
+"""Benchmark of the balancer's per-layer, per-microbatch hot path on B200.
+
+One step = one pass of the whole path over one microbatch: load -> plan ->
+reroute (the "rebalance") -> replica weight sync -> replica gradient
+reduction, all through the C ABI of libue.so, with every input resident in
+HBM.  The headline value is the rebalance latency in microseconds per
+layer-microbatch; weight-sync and grad-reduce bandwidths are reported beside
+it against the measured HBM copy peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the CPU oracle on the host cores
+
+Under torchrun (N > 1) every rank runs an independent replica of the
+workload on its own GPU (the path does not shard: no data-path collective);
+timings are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from moe_expert_load_ue_b200 import inputs  # noqa: E402
+
+METRIC = "rebalance µs/layer-microbatch (load+plan+reroute); sync & grad-reduce HBM GB/s"
+UNIT = "µs"
+FALLBACK_HBM_GBS = 6650.0
+# DRAM bytes per launch of the dominant kernel from the committed ncu capture
+# (profiles/), scaled to this workload; None until a capture of the current
+# kernel exists.
+TRAFFIC_BYTES = {}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="671B-class", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--microbatches", type=int, default=None,
+                    help="distinct resident microbatches cycled by the steps (default: the workload's)")
+    ap.add_argument("--expert-shape", default=None,
+                    help="override the expert matrices' rows x cols (e.g. 1024x512) for small profiling cases")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ---- distributed plumbing (barrier and max over ranks only) -----------------------
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend: str):
+        if self.world > 1:
+            import datetime
+
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+        return self
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, values, device=None):
+        """Element-wise max over ranks of a list of floats."""
+        if not self.pg:
+            return list(values)
+        import torch
+        t = torch.tensor(list(values), dtype=torch.float64, device=device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return t.tolist()
+
+    def sum(self, values, device=None):
+        if not self.pg:
+            return list(values)
+        import torch
+        t = torch.tensor(list(values), dtype=torch.float64, device=device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.SUM)
+        return t.tolist()
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# ---- clocks ---------------------------------------------------------------------
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str, period_ms: int = 100):
+        self.gpu_id, self.period_ms = gpu_id, period_ms
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", str(self.period_ms), "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, power, reasons = [], [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    smax.append(float(parts[1]))
+                    power.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[4:8]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
+
+
+def measured_peaks() -> tuple[float, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---- the GPU arm ------------------------------------------------------------------
+
+def run_ours(args, dist: Dist):
+    import torch
+
+    from moe_expert_load_ue_b200 import ue
+
+    torch.cuda.set_device(dist.local_rank)
+    dev = torch.device("cuda", dist.local_rank)
+    dist.init("nccl")
+    w = inputs.WORKLOADS[args.workload].with_(base_seed=dist.rank)
+    if args.expert_shape:
+        rows, cols = (int(x) for x in args.expert_shape.lower().split("x"))
+        w = w.with_(rows=rows, cols=cols)
+    n_mb = args.microbatches or w.microbatches
+    cfg = ue.Config(E=w.E, N=w.N, R=w.R, K=w.K, T=w.T)
+    ctx = ue.Context(dist.local_rank)
+    stream = torch.cuda.Stream(device=dev)
+
+    # Inputs: every microbatch's ids resident in HBM (and pinned on the host for the e2e leg).
+    ids_host = [inputs.topk_ids(w, mb) for mb in range(n_mb)]
+    ids_dev = torch.empty((n_mb, w.T, w.K), dtype=torch.int32, device=dev)
+    for mb in range(n_mb):
+        ids_dev[mb].copy_(torch.from_numpy(ids_host[mb]))
+    counts = torch.empty((w.N, w.E), dtype=torch.int32, device=dev)
+    bad = torch.empty(w.N, dtype=torch.int32, device=dev)
+    plan = ue.Plan(cfg, device=dev)
+    phys = torch.empty((w.T, w.K), dtype=torch.int32, device=dev)
+    P = w.P
+    slot_bytes = 2 * P
+    gen = torch.Generator(device=dev).manual_seed(1234 + dist.rank)
+    weights = torch.empty((w.S, P), dtype=torch.bfloat16, device=dev)
+    for s in range(w.S):
+        weights[s].normal_(0.0, 0.02, generator=gen)
+    gdt = torch.bfloat16 if w.grad_dtype == "bf16" else torch.float32
+    grads = torch.empty((w.N * w.R, P), dtype=gdt, device=dev)
+    for r in range(w.N * w.R):
+        grads[r].normal_(0.0, 1e-3, generator=gen)
+    master = torch.empty((w.E, P), dtype=torch.float32, device=dev)
+    for e in range(w.E):
+        master[e].normal_(0.0, 1e-3, generator=gen)
+    torch.cuda.synchronize(dev)
+
+    def step(mb, ev=None):
+        ids = ids_dev[mb]
+        if ev:
+            ev[0].record(stream)
+        ue.ue_load(ctx, cfg, ids, counts, bad, stream=stream)
+        if ev:
+            ev[1].record(stream)
+        ue.ue_plan(ctx, cfg, counts, plan, stream=stream)
+        if ev:
+            ev[2].record(stream)
+        ue.ue_reroute(ctx, cfg, ids, plan, phys, stream=stream)
+        if ev:
+            ev[3].record(stream)
+        ue.ue_sync(ctx, cfg, weights, slot_bytes, plan, stream=stream)
+        if ev:
+            ev[4].record(stream)
+        ue.ue_grad_reduce(ctx, cfg, master, grads, P, plan, stream=stream)
+        if ev:
+            ev[5].record(stream)
+
+    KERNELS_PER_STEP = 5
+    with torch.cuda.stream(stream):
+        for k in range(args.warmup):
+            step(k % n_mb)
+    stream.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    gpu_id = gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}"
+    clocks = ClockSampler(gpu_id).start()
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        for k in range(args.steps):
+            step(k % n_mb, evs[k])
+    stream.synchronize()
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    clk = clocks.stop()
+    err = ctx.device_error(stream)
+    if err:
+        raise RuntimeError(f"a kernel gave up a bounded wait (status word {err})")
+
+    seg = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(5)] for k in range(args.steps)]) * 1e3
+    total_ms = evs[0][0].elapsed_time(evs[-1][5])
+    rebalance_us = seg[:, 0:3].sum(axis=1)
+
+    # Plans per microbatch (recomputed after the timed region) for the byte accounting.
+    per_mb = []
+    with torch.cuda.stream(stream):
+        for mb in range(n_mb):
+            ue.ue_rebalance(ctx, cfg, ids_dev[mb], counts, bad, plan, phys, stream=stream)
+            stream.synchronize()
+            info = plan["info"].cpu().numpy()
+            per_mb.append({"Q": int(info[0]), "L": int(info[1]), "ran_out": int(info[2] & 1), "M": int(info[3]),
+                           "filled": int(info[4]), "max_before": int(info[5]), "max_after": int(info[6])})
+    gsize = 2 if w.grad_dtype == "bf16" else 4
+    sync_bytes = np.array([(p["M"] + p["filled"]) * slot_bytes for p in per_mb], dtype=np.float64)
+    grad_bytes = np.array([p["M"] * P * 8 + p["filled"] * P * gsize for p in per_mb], dtype=np.float64)
+    step_mb = np.array([k % n_mb for k in range(args.steps)])
+    sync_gbs = sync_bytes[step_mb].sum() / (seg[:, 3].sum() * 1e-6) / 1e9
+    grad_gbs = grad_bytes[step_mb].sum() / (seg[:, 4].sum() * 1e-6) / 1e9
+    rebalance_alg_bytes = 3.0 * w.L * 4
+
+    # Launch floor: one tiny kernel bracketed by events on the same stream.
+    tiny = torch.zeros(1, device=dev)
+    floor = []
+    with torch.cuda.stream(stream):
+        for _ in range(50):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            tiny.add_(1.0)
+            b.record(stream)
+            stream.synchronize()
+            floor.append(a.elapsed_time(b) * 1e3)
+    launch_floor_us = statistics.median(floor)
+
+    # Max over ranks (timings) / sums (work).
+    mean_reb = float(rebalance_us.mean())
+    vals = dist.max([mean_reb, total_ms, float(seg[:, 3].mean()), float(seg[:, 4].mean())], device=dev)
+    mean_reb_max, total_ms_max, sync_us_max, grad_us_max = vals
+
+    # End-to-end through the public API with host buffers: H2D ids, rebalance, D2H phys + plan.
+    e2e = None
+    if not args.no_e2e:
+        ids_pinned = [torch.from_numpy(x).pin_memory() for x in ids_host]
+        ids_buf = torch.empty((w.T, w.K), dtype=torch.int32, device=dev)
+        phys_h = torch.empty((w.T, w.K), dtype=torch.int32).pin_memory()
+        plan_h = {k: torch.empty(v.shape, dtype=torch.int32).pin_memory() for k, v in plan.tensors.items()}
+        n_e2e = max(8, min(args.steps, 64))
+        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_e2e)]
+        with torch.cuda.stream(stream):
+            for k in range(args.warmup + n_e2e):
+                mb = k % n_mb
+                e = ev2[k - args.warmup] if k >= args.warmup else None
+                if e:
+                    e[0].record(stream)
+                ids_buf.copy_(ids_pinned[mb], non_blocking=True)
+                ue.ue_rebalance(ctx, cfg, ids_buf, counts, bad, plan, phys, stream=stream)
+                phys_h.copy_(phys, non_blocking=True)
+                for kk, t in plan.tensors.items():
+                    plan_h[kk].copy_(t, non_blocking=True)
+                if e:
+                    e[1].record(stream)
+            stream.synchronize()
+        e2e_us = dist.max([statistics.mean(a.elapsed_time(b) * 1e3 for a, b in ev2)], device=dev)[0]
+        h2d = w.T * w.K * 4
+        d2h = w.T * w.K * 4 + plan.nbytes()
+        e2e = {"value": round(e2e_us, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "path": "pinned host ids -> ue_rebalance -> pinned host phys + plan, one stream"}
+
+    peak, peak_kind = measured_peaks()
+    dom = "grad_reduce" if seg[:, 4].sum() >= seg[:, 3].sum() else "sync"
+    if dom == "grad_reduce":
+        ach = grad_gbs
+        per_launch = float(grad_bytes[step_mb].mean())
+    else:
+        ach = sync_gbs
+        per_launch = float(sync_bytes[step_mb].mean())
+    roofline = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(ach / peak, 4), "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_kind == "measured" else "fallback 6650 GB/s",
+                "traffic": TRAFFIC_BYTES.get((dom, args.workload)),
+                "algorithmic_bytes_per_launch": per_launch}
+
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, ids_host, P, gsize)
+
+    result = {
+        "metric": METRIC, "value": round(mean_reb_max, 2), "unit": UNIT, "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms_max / args.steps, 4),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "int32",
+        "data": "synthetic: seeded Zipf-popularity Gumbel-top-k routing, random bf16 weights and replica grads",
+        "config": {"workload": w.name, "E": w.E, "N": w.N, "H": w.H, "R": w.R, "K": w.K, "T": w.T,
+                   "P": P, "slot_bytes": slot_bytes, "grad_dtype": w.grad_dtype, "zipf_s": w.s,
+                   "microbatches_cycled": n_mb, "parallelism": f"replicas x{dist.world}",
+                   "l2": "inputs larger than L2: every step streams > 1 GB (sync + grad reduce), "
+                         "so each rebalance reads its ids from HBM"},
+        "breakdown_us": {
+            "load": round(float(seg[:, 0].mean()), 2), "plan": round(float(seg[:, 1].mean()), 2),
+            "reroute": round(float(seg[:, 2].mean()), 2),
+            "rebalance_p10": round(float(np.percentile(rebalance_us, 10)), 2),
+            "rebalance_p50": round(float(np.percentile(rebalance_us, 50)), 2),
+            "rebalance_p90": round(float(np.percentile(rebalance_us, 90)), 2),
+            "sync": round(sync_us_max, 1), "grad_reduce": round(grad_us_max, 1),
+            "launch_floor": round(launch_floor_us, 2),
+        },
+        "rebalance_hbm_floor_us": round(rebalance_alg_bytes / (peak * 1e9) * 1e6, 2),
+        "sync_gbs": round(sync_gbs, 1), "sync_frac": round(sync_gbs / peak, 4),
+        "grad_reduce_gbs": round(grad_gbs, 1), "grad_reduce_frac": round(grad_gbs / peak, 4),
+        "frac_of_8000_gbs": {"sync": round(sync_gbs / 8000, 4), "grad_reduce": round(grad_gbs / 8000, 4)},
+        "imbalance": {
+            "before": round(float(np.mean([p["max_before"] / (p["L"] / w.N) for p in per_mb])), 4),
+            "after": round(float(np.mean([p["max_after"] / (p["L"] / w.N) for p in per_mb])), 4),
+            "slots_ran_out_frac": round(float(np.mean([p["ran_out"] for p in per_mb])), 4),
+            "replicated_experts_mean": round(float(np.mean([p["M"] for p in per_mb])), 2),
+            "filled_redundant_slots_mean": round(float(np.mean([p["filled"] for p in per_mb])), 2),
+        },
+        "context_pages": {"rebalance_us": 300, "imbalance_before": "1.30-4.01", "imbalance_after": "1.01-1.04",
+                          "hardware": "rack-scale NVL72 / Atlas 900 A3"},
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clk,
+        "job_microbatches_per_s": round(dist.world * args.steps / (total_ms_max * 1e-3), 2),
+    }
+    ctx.close()
+    dist.barrier()
+    dist.close()
+    return result
+
+
+# ---- the CPU oracle, timed on the host cores ------------------------------------
+
+def cpu_baseline(w, ids_host, P, gsize, budget_s: float = 10.0):
+    import oracle
+    n_mb = len(ids_host)
+    t_reb = []
+    t0 = time.perf_counter()
+    plans = []
+    while time.perf_counter() - t0 < 0.6 * budget_s or len(t_reb) < n_mb:
+        mb = len(t_reb) % n_mb
+        a = time.perf_counter()
+        out = oracle.rebalance(ids_host[mb], w.E, w.N, w.R)
+        t_reb.append(time.perf_counter() - a)
+        if len(plans) < n_mb:
+            plans.append(out["plan"])
+    # weight sync over a 1 MiB window of every slot; grad reduce over a 64 Ki-element window of every expert
+    win = 1 << 20
+    Wh = np.random.default_rng(0).integers(0, 256, size=(w.S, win), dtype=np.uint8)
+    nb, ts = 0, 0.0
+    gw = 1 << 16
+    mh = np.random.default_rng(1).standard_normal((w.E, gw), dtype=np.float32)
+    gh = (inputs.random_bf16_bits((w.N * w.R, gw), 1e-3, 2) if gsize == 2
+          else inputs.random_f32((w.N * w.R, gw), 1e-3, 2))
+    gb, tg = 0, 0.0
+    t1 = time.perf_counter()
+    i = 0
+    while time.perf_counter() - t1 < 0.4 * budget_s or i < n_mb:
+        pl = plans[i % n_mb]
+        a = time.perf_counter()
+        oracle.sync(Wh, win, w.E, w.N, w.R, pl["slot_expert"])
+        ts += time.perf_counter() - a
+        nb += (pl["info"][3] + pl["info"][4]) * win
+        a = time.perf_counter()
+        oracle.grad_reduce(mh, gh, gw, w.E, w.N, w.R, pl)
+        tg += time.perf_counter() - a
+        gb += pl["info"][3] * gw * 8 + pl["info"][4] * gw * gsize
+        i += 1
+    return {"value": round(statistics.mean(t_reb) * 1e6, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{len(t_reb)} full microbatches of the workload (load+plan+reroute); weight sync over a "
+                      f"1 MiB window of every slot and grad reduce over a 64 Ki-element window of every "
+                      f"expert, {i} plans",
+            "sync_gbs": round(nb / ts / 1e9, 2), "grad_reduce_gbs": round(gb / tg / 1e9, 2),
+            "threads": "single-threaded C (gcc -O2)", "nproc": os.cpu_count()}
+
+
+def run_reference(args, dist: Dist):
+    """The reference arm: the CPU oracle, timed as it stands on the host cores."""
+    if dist.rank != 0:
+        return None
+    import oracle
+    w = inputs.WORKLOADS[args.workload]
+    n_mb = args.microbatches or w.microbatches
+    ids_host = [inputs.topk_ids(w, mb) for mb in range(n_mb)]
+    for k in range(args.warmup):
+        oracle.rebalance(ids_host[k % n_mb], w.E, w.N, w.R)
+    times = []
+    for k in range(args.steps):
+        a = time.perf_counter()
+        oracle.rebalance(ids_host[k % n_mb], w.E, w.N, w.R)
+        times.append(time.perf_counter() - a)
+    v = round(statistics.mean(times) * 1e6, 1)
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(statistics.mean(times) * 1e3, 3),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "int32",
+        "data": "synthetic: seeded Zipf-popularity Gumbel-top-k routing",
+        "config": {"workload": w.name, "E": w.E, "N": w.N, "H": w.H, "R": w.R, "K": w.K, "T": w.T,
+                   "microbatches_cycled": n_mb},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"each step one full microbatch (load+plan+reroute), {args.steps} steps"},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    dist = Dist()
+    if args.impl == "reference":
+        res = run_reference(args, dist)
+    else:
+        res = run_ours(args, dist)
+    if res is not None and dist.rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -11,7 +11,9 @@ fonctionne l'équilibrage en 300 microsecondes") describe production routing
 that is skewed and non-stationary.  We stand in for those traces with a Zipf
 popularity over a seeded permutation of experts, p_e ∝ (pi(e) + 1)^-s, and
 draw each token's K distinct experts by Gumbel-top-k on log p_e (highest
-perturbed score first, so position k = 0 is the token's top choice).  The
+perturbed score first, so position k = 0 is the token's top choice).  Tokens
+are drawn in fixed chunks of 16384 with their own child seeds, so the ids do
+not depend on how many threads generate them.  The
 106B/671B workloads re-draw the permutation every microbatch (non-stationary
 load); the extreme-skew workload additionally forces one hot expert into 30 %
 of the tokens.
@@ -20,6 +22,8 @@ from __future__ import annotations
 
 import dataclasses
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 from typing import Iterator
 
 import numpy as np
@@ -108,47 +112,67 @@ def zipf_popularity(E: int, s: float, rng: np.random.Generator) -> np.ndarray:
     return p / p.sum()
 
 
-def _gumbel_topk(logp: np.ndarray, T: int, K: int, rng: np.random.Generator,
-                 chunk: int = 16384) -> np.ndarray:
+_CHUNK = 16384            # tokens per independently seeded chunk (fixed: keeps draws thread-count independent)
+
+
+def _topk_chunk(seed_seq: np.random.SeedSequence, n: int, inv_p: np.ndarray, K: int) -> np.ndarray:
+    """Gumbel-top-k for n tokens.  With G = -log(X), X ~ Exp(1), G is standard
+    Gumbel noise, and log p_e + G_e orders the experts exactly as X_e / p_e
+    does in reverse, so the K smallest X_e / p_e are the K largest perturbed
+    scores, in the same order (the exponential-race form of Gumbel-top-k)."""
+    rng = np.random.default_rng(seed_seq)
+    E = inv_p.shape[0]
+    x = rng.standard_exponential((n, E), dtype=np.float32)
+    x *= inv_p
+    if K < E:
+        part = np.argpartition(x, K - 1, axis=1)[:, :K]
+    else:
+        part = np.tile(np.arange(E), (n, 1))
+    sc = np.take_along_axis(x, part, axis=1)
+    order = np.argsort(sc, axis=1, kind="stable")
+    return np.take_along_axis(part, order, axis=1).astype(np.int32)
+
+
+def _gumbel_topk(p: np.ndarray, T: int, K: int, seed_seq: np.random.SeedSequence) -> np.ndarray:
     """K distinct experts per token, ordered by decreasing perturbed score."""
-    E = logp.shape[0]
+    with np.errstate(divide="ignore"):
+        inv_p = (1.0 / p).astype(np.float32)        # p_e = 0 -> never drawn
+    n_chunks = (T + _CHUNK - 1) // _CHUNK
+    kids = seed_seq.spawn(n_chunks)
+    sizes = [min(_CHUNK, T - i * _CHUNK) for i in range(n_chunks)]
     out = np.empty((T, K), dtype=np.int32)
-    lp = logp.astype(np.float32)
-    tiny = np.float32(np.finfo(np.float32).tiny)
-    for a in range(0, T, chunk):
-        b = min(T, a + chunk)
-        u = rng.random((b - a, E), dtype=np.float32)
-        np.maximum(u, tiny, out=u)
-        g = -np.log(-np.log(u))          # standard Gumbel noise
-        g += lp
-        if K < E:
-            part = np.argpartition(-g, K - 1, axis=1)[:, :K]
-        else:
-            part = np.tile(np.arange(E), (b - a, 1))
-        sc = np.take_along_axis(g, part, axis=1)
-        order = np.argsort(-sc, axis=1, kind="stable")
-        out[a:b] = np.take_along_axis(part, order, axis=1)
+    if n_chunks == 0:
+        return out
+    workers = max(1, min(8, os.cpu_count() or 1, n_chunks))
+    with ThreadPoolExecutor(workers) as ex:
+        parts = list(ex.map(lambda a: _topk_chunk(kids[a], sizes[a], inv_p, K), range(n_chunks)))
+    for i, part in enumerate(parts):
+        out[i * _CHUNK:i * _CHUNK + sizes[i]] = part
     return out
+
+
+def popularity(w: Workload, microbatch: int = 0) -> np.ndarray:
+    """Expert popularity p_e of a microbatch (re-permuted per microbatch unless stationary)."""
+    mb = microbatch if w.repermute else 0
+    ss_perm = np.random.SeedSequence(w.seed(mb)).spawn(3)[0]
+    return zipf_popularity(w.E, w.s, np.random.default_rng(ss_perm))
 
 
 def topk_ids(w: Workload, microbatch: int = 0) -> np.ndarray:
     """Post-gating top-K expert ids, int32 [T, K], row-major (token-major)."""
-    rng = np.random.default_rng(w.seed(microbatch))
-    if w.repermute or microbatch == 0:
-        p = zipf_popularity(w.E, w.s, rng)
-    else:  # stationary popularity: the permutation of microbatch 0
-        p = zipf_popularity(w.E, w.s, np.random.default_rng(w.seed(0)))
-    logp = np.log(p)
+    _, ss_hot, ss_draw = np.random.SeedSequence(w.seed(microbatch)).spawn(3)
+    p = popularity(w, microbatch)
     if w.hot_fraction <= 0.0:
-        return _gumbel_topk(logp, w.T, w.K, rng)
+        return _gumbel_topk(p, w.T, w.K, ss_draw)
     # One hot expert forced into floor(hot_fraction * T) tokens as their top
     # choice; every other draw excludes it so its count is exact.
-    hot = int(rng.integers(w.E))
+    rng_hot = np.random.default_rng(ss_hot)
+    hot = int(rng_hot.integers(w.E))
     n_hot = int(math.floor(w.hot_fraction * w.T))
-    hot_tokens = rng.choice(w.T, size=n_hot, replace=False)
-    logp_x = logp.copy()
-    logp_x[hot] = -np.inf
-    ids = _gumbel_topk(logp_x, w.T, w.K, rng)
+    hot_tokens = rng_hot.choice(w.T, size=n_hot, replace=False)
+    p_x = p.copy()
+    p_x[hot] = 0.0
+    ids = _gumbel_topk(p_x, w.T, w.K, ss_draw)
     ids[hot_tokens, 1:] = ids[hot_tokens, :-1]
     ids[hot_tokens, 0] = hot
     return ids
@@ -156,9 +180,8 @@ def topk_ids(w: Workload, microbatch: int = 0) -> np.ndarray:
 
 def hot_expert(w: Workload, microbatch: int = 0) -> int:
     """The forced hot expert of an extreme-skew microbatch (same draw as topk_ids)."""
-    rng = np.random.default_rng(w.seed(microbatch))
-    zipf_popularity(w.E, w.s, rng)
-    return int(rng.integers(w.E))
+    ss_hot = np.random.SeedSequence(w.seed(microbatch)).spawn(3)[1]
+    return int(np.random.default_rng(ss_hot).integers(w.E))
 
 
 def gates(ids: np.ndarray, w: Workload, microbatch: int = 0) -> np.ndarray:

@@ -20,7 +20,7 @@ def test_zipf_skew_orders_popularity():
     w = inputs.CLASS_106B.with_(tokens_per_rank=256)
     ids = inputs.topk_ids(w, 0)
     cnt = np.bincount(ids.ravel(), minlength=w.E)
-    p = inputs.zipf_popularity(w.E, w.s, np.random.default_rng(w.seed(0)))
+    p = inputs.popularity(w, 0)
     # the most popular expert by construction is among the most frequent
     assert cnt[np.argmax(p)] >= np.sort(cnt)[-3]
 

@@ -87,7 +87,7 @@ def test_balls_in_bins_imbalance_at_s0():
         draws = rng.multivariate_hypergeometric([w.H] * w.N, w.K, size=w.T).sum(axis=0)
         sims.append(draws.max() / (w.L / w.N))
     assert abs(np.mean(ours) - np.mean(sims)) < 0.04, (np.mean(ours), np.mean(sims))
-    assert np.mean(ours) > 1.1       # the max bin sits well above the mean
+    assert np.mean(ours) > 1.05      # the busiest rank sits well above the mean
 
 
 # ---- reroute ----------------------------------------------------------------
