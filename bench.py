@@ -219,29 +219,23 @@ def run_ours(args, dist: Dist):
         ids = ids_dev[mb]
         if ev:
             ev[0].record(stream)
-        ue.ue_load(ctx, cfg, ids, counts, bad, stream=stream)
+        ue.ue_rebalance(ctx, cfg, ids, counts, bad, plan, phys, stream=stream)   # load + plan + reroute
         if ev:
             ev[1].record(stream)
-        ue.ue_plan(ctx, cfg, counts, plan, stream=stream)
-        if ev:
-            ev[2].record(stream)
-        ue.ue_reroute(ctx, cfg, ids, plan, phys, stream=stream)
-        if ev:
-            ev[3].record(stream)
         ue.ue_sync(ctx, cfg, weights, slot_bytes, plan, stream=stream)
         if ev:
-            ev[4].record(stream)
+            ev[2].record(stream)
         ue.ue_grad_reduce(ctx, cfg, master, grads, P, plan, stream=stream)
         if ev:
-            ev[5].record(stream)
+            ev[3].record(stream)
 
-    KERNELS_PER_STEP = 5
+    KERNELS_PER_STEP = 5     # load, plan, reroute (one ue_rebalance call), sync, grad reduce
     with torch.cuda.stream(stream):
         for k in range(args.warmup):
             step(k % n_mb)
     stream.synchronize()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
     gpu_id = gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}"
     clocks = ClockSampler(gpu_id).start()
@@ -258,9 +252,27 @@ def run_ours(args, dist: Dist):
     if err:
         raise RuntimeError(f"a kernel gave up a bounded wait (status word {err})")
 
-    seg = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(5)] for k in range(args.steps)]) * 1e3
-    total_ms = evs[0][0].elapsed_time(evs[-1][5])
-    rebalance_us = seg[:, 0:3].sum(axis=1)
+    seg = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(3)] for k in range(args.steps)]) * 1e3
+    total_ms = evs[0][0].elapsed_time(evs[-1][3])
+    rebalance_us = seg[:, 0]
+
+    # Per-kernel breakdown of the rebalance: the three steps as separate calls
+    # with events between them (no launch overlap), after the timed region.
+    n_bd = max(8, min(args.steps, 64))
+    evb = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_bd)]
+    with torch.cuda.stream(stream):
+        for k in range(n_bd):
+            ids = ids_dev[k % n_mb]
+            evb[k][0].record(stream)
+            ue.ue_load(ctx, cfg, ids, counts, bad, stream=stream)
+            evb[k][1].record(stream)
+            ue.ue_plan(ctx, cfg, counts, plan, stream=stream)
+            evb[k][2].record(stream)
+            ue.ue_reroute(ctx, cfg, ids, plan, phys, stream=stream)
+            evb[k][3].record(stream)
+            ue.ue_sync(ctx, cfg, weights, slot_bytes, plan, stream=stream)   # keeps L2 cold as in the step
+    stream.synchronize()
+    bd = np.array([[evb[k][i].elapsed_time(evb[k][i + 1]) for i in range(3)] for k in range(n_bd)]) * 1e3
 
     # Plans per microbatch (recomputed after the timed region) for the byte accounting.
     per_mb = []
@@ -275,8 +287,8 @@ def run_ours(args, dist: Dist):
     sync_bytes = np.array([(p["M"] + p["filled"]) * slot_bytes for p in per_mb], dtype=np.float64)
     grad_bytes = np.array([p["M"] * P * 8 + p["filled"] * P * gsize for p in per_mb], dtype=np.float64)
     step_mb = np.array([k % n_mb for k in range(args.steps)])
-    sync_gbs = sync_bytes[step_mb].sum() / (seg[:, 3].sum() * 1e-6) / 1e9
-    grad_gbs = grad_bytes[step_mb].sum() / (seg[:, 4].sum() * 1e-6) / 1e9
+    sync_gbs = sync_bytes[step_mb].sum() / (seg[:, 1].sum() * 1e-6) / 1e9
+    grad_gbs = grad_bytes[step_mb].sum() / (seg[:, 2].sum() * 1e-6) / 1e9
     rebalance_alg_bytes = 3.0 * w.L * 4
 
     # Launch floor: one tiny kernel bracketed by events on the same stream.
@@ -294,7 +306,7 @@ def run_ours(args, dist: Dist):
 
     # Max over ranks (timings) / sums (work).
     mean_reb = float(rebalance_us.mean())
-    vals = dist.max([mean_reb, total_ms, float(seg[:, 3].mean()), float(seg[:, 4].mean())], device=dev)
+    vals = dist.max([mean_reb, total_ms, float(seg[:, 1].mean()), float(seg[:, 2].mean())], device=dev)
     mean_reb_max, total_ms_max, sync_us_max, grad_us_max = vals
 
     # End-to-end through the public API with host buffers: H2D ids, rebalance, D2H phys + plan.
@@ -327,7 +339,7 @@ def run_ours(args, dist: Dist):
                "path": "pinned host ids -> ue_rebalance -> pinned host phys + plan, one stream"}
 
     peak, peak_kind = measured_peaks()
-    dom = "grad_reduce" if seg[:, 4].sum() >= seg[:, 3].sum() else "sync"
+    dom = "grad_reduce" if seg[:, 2].sum() >= seg[:, 1].sum() else "sync"
     if dom == "grad_reduce":
         ach = grad_gbs
         per_launch = float(grad_bytes[step_mb].mean())
@@ -355,8 +367,9 @@ def run_ours(args, dist: Dist):
                    "l2": "inputs larger than L2: every step streams > 1 GB (sync + grad reduce), "
                          "so each rebalance reads its ids from HBM"},
         "breakdown_us": {
-            "load": round(float(seg[:, 0].mean()), 2), "plan": round(float(seg[:, 1].mean()), 2),
-            "reroute": round(float(seg[:, 2].mean()), 2),
+            "load": round(float(bd[:, 0].mean()), 2), "plan": round(float(bd[:, 1].mean()), 2),
+            "reroute": round(float(bd[:, 2].mean()), 2),
+            "rebalance_as_separate_calls": round(float(bd.sum(axis=1).mean()), 2),
             "rebalance_p10": round(float(np.percentile(rebalance_us, 10)), 2),
             "rebalance_p50": round(float(np.percentile(rebalance_us, 50)), 2),
             "rebalance_p90": round(float(np.percentile(rebalance_us, 90)), 2),
@@ -420,11 +433,11 @@ def cpu_baseline(w, ids_host, P, gsize, budget_s: float = 10.0):
         a = time.perf_counter()
         oracle.sync(Wh, win, w.E, w.N, w.R, pl["slot_expert"])
         ts += time.perf_counter() - a
-        nb += (pl["info"][3] + pl["info"][4]) * win
+        nb += (int(pl["info"][3]) + int(pl["info"][4])) * win
         a = time.perf_counter()
         oracle.grad_reduce(mh, gh, gw, w.E, w.N, w.R, pl)
         tg += time.perf_counter() - a
-        gb += pl["info"][3] * gw * 8 + pl["info"][4] * gw * gsize
+        gb += int(pl["info"][3]) * gw * 8 + int(pl["info"][4]) * gw * gsize
         i += 1
     return {"value": round(statistics.mean(t_reb) * 1e6, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"{len(t_reb)} full microbatches of the workload (load+plan+reroute); weight sync over a "

@@ -28,7 +28,7 @@
  *   - Device-detected bad input (an id outside [0, E)) never traps: the id is
  *     not counted, its rerouted slot is -1, and ue_load reports it per rank.
  *   - Limits: 1 <= E <= 1024, 1 <= N <= 1024, E % N == 0, 0 <= R,
- *     N * R <= 4096, 1 <= K, T % N == 0, T * K <= 2^31 - 1.
+ *     N * R <= 4096, 1 <= K, T % N == 0, T * K <= 2^30.
  */
 #ifndef UE_H
 #define UE_H

@@ -57,8 +57,8 @@ ue_status make_shape(const ue_config *cfg, bool need_tokens, ue::Shape *sh)
         if (c.K < 1) return fail(UE_ERR_INVALID_ARG, "K=%d < 1", c.K);
         if (c.T < 0 || c.T % c.N != 0)
             return fail(UE_ERR_INVALID_ARG, "T=%lld must be >= 0 and a multiple of N=%d", (long long)c.T, c.N);
-        if (c.T * (int64_t)c.K > (int64_t)INT32_MAX)
-            return fail(UE_ERR_INVALID_ARG, "T*K=%lld exceeds 2^31-1", (long long)(c.T * c.K));
+        if (c.T * (int64_t)c.K > ((int64_t)1 << 30))
+            return fail(UE_ERR_INVALID_ARG, "T*K=%lld exceeds 2^30", (long long)(c.T * c.K));
     }
     sh->E = c.E;
     sh->N = c.N;
@@ -89,12 +89,15 @@ ue_status check_ctx(const ue_ctx *ctx)
     return UE_OK;
 }
 
-// Clusters of CTAs per simulated rank for load / reroute: enough CTAs to fill
-// the GPU about twice, each with at least 2048 ids.
+// CTAs per simulated rank (one cluster per rank) for load / reroute: as many
+// as keep the grid within one wave of two 512-thread CTAs per SM, leaving
+// room for the planner's cluster that runs beside the reroute grid, with at
+// least 2048 ids per CTA.
 int choose_cluster(const ue::Shape &sh, int sms)
 {
+    const int64_t wave = 2 * (int64_t)sms - 2 * ue::kMaxCluster;
     int C = 1;
-    while (C < ue::kMaxCluster && (int64_t)sh.N * C < 2 * (int64_t)sms && sh.per_rank / (2 * C) >= 2048) C *= 2;
+    while (C < ue::kMaxCluster && (int64_t)sh.N * C * 2 <= wave && sh.per_rank / (2 * C) >= 2048) C *= 2;
     return C;
 }
 
@@ -247,7 +250,7 @@ ue_status ue_plan(ue_ctx *ctx, const ue_config *cfg, const int32_t *counts, cons
         return fail(UE_ERR_INVALID_ARG, "plan needs %zu bytes of shared memory (> %d)", ue::plan_smem_bytes(sh),
                     ctx->max_smem);
     return on_device(ctx, [&]() -> ue_status {
-        cudaError_t e = ue::launch_plan(sh, counts, ue::to_dev(*plan), static_cast<cudaStream_t>(stream));
+        cudaError_t e = ue::launch_plan(sh, counts, ue::to_dev(*plan), static_cast<cudaStream_t>(stream), false);
         return e == cudaSuccess ? UE_OK : cuda_fail(e, "plan launch");
     });
 }
@@ -267,7 +270,7 @@ ue_status ue_reroute(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids, cons
                     ctx->max_smem);
     return on_device(ctx, [&]() -> ue_status {
         cudaError_t e = ue::launch_reroute(sh, launch_of(ctx, sh), ids, ue::to_dev(*plan), phys,
-                                           static_cast<cudaStream_t>(stream));
+                                           static_cast<cudaStream_t>(stream), false);
         return e == cudaSuccess ? UE_OK : cuda_fail(e, "reroute launch");
     });
 }
@@ -292,8 +295,12 @@ ue_status ue_rebalance(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids, in
         const ue::PlanDev pd = ue::to_dev(*plan);
         cudaError_t e = ue::launch_load(sh, ln, ids, counts, bad, st);
         if (e != cudaSuccess) return cuda_fail(e, "load launch");
-        if ((e = ue::launch_plan(sh, counts, pd, st)) != cudaSuccess) return cuda_fail(e, "plan launch");
-        if ((e = ue::launch_reroute(sh, ln, ids, pd, phys, st)) != cudaSuccess) return cuda_fail(e, "reroute launch");
+        // The planner and the reroute kernel use programmatic dependent launch:
+        // each may start while its predecessor drains, and waits for it
+        // (griddepcontrol.wait) before reading what it wrote.
+        if ((e = ue::launch_plan(sh, counts, pd, st, true)) != cudaSuccess) return cuda_fail(e, "plan launch");
+        if ((e = ue::launch_reroute(sh, ln, ids, pd, phys, st, true)) != cudaSuccess)
+            return cuda_fail(e, "reroute launch");
         return UE_OK;
     });
 }

@@ -2,6 +2,8 @@
 #pragma once
 
 #include <cstdint>
+#include <utility>
+
 #include <cuda_runtime.h>
 
 #include "ue.h"
@@ -43,12 +45,13 @@ cudaError_t launch_load(const Shape &sh, const Launch &ln, const int32_t *ids, i
                         int32_t *bad, cudaStream_t st);
 size_t load_smem_bytes(const Shape &sh);
 
-cudaError_t launch_plan(const Shape &sh, const int32_t *counts, const PlanDev &plan, cudaStream_t st);
+cudaError_t launch_plan(const Shape &sh, const int32_t *counts, const PlanDev &plan, cudaStream_t st,
+                        bool pdl);
 size_t plan_smem_bytes(const Shape &sh);
 int plan_cluster(const Shape &sh);
 
 cudaError_t launch_reroute(const Shape &sh, const Launch &ln, const int32_t *ids, const PlanDev &plan,
-                           int32_t *phys, cudaStream_t st);
+                           int32_t *phys, cudaStream_t st, bool pdl);
 size_t reroute_smem_bytes(const Shape &sh);
 
 cudaError_t launch_sync(const Shape &sh, const Launch &ln, uint8_t *weights, int64_t slot_bytes,
@@ -59,8 +62,37 @@ cudaError_t launch_grad_reduce(const Shape &sh, const Launch &ln, float *master,
                                int grad_dtype, int64_t P, const PlanDev &plan, cudaStream_t st);
 size_t grad_smem_bytes(const Shape &sh);
 
-// Kernel attribute set-up (dynamic shared memory opt-in), once per device.
-cudaError_t set_kernel_attributes();
+// Launch with an optional thread-block cluster (cluster > 1) and optional
+// programmatic dependent launch (pdl: the kernel may start while the previous
+// kernel on the stream finishes; it must griddepcontrol.wait before reading
+// that kernel's outputs).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t st,
+                      unsigned cluster, bool pdl, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    unsigned n = 0;
+    if (cluster > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    if (pdl) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // ---- device helpers ---------------------------------------------------------
 
@@ -74,6 +106,11 @@ __device__ __forceinline__ unsigned lanemask_lt()
 }
 
 __device__ __forceinline__ int clampi(int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi : v); }
+
+// Programmatic dependent launch: wait for the previous grid on the stream to
+// complete (and its writes to be visible); allow the next grid to launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // Split cluster barrier (release on arrive, acquire on wait).
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }

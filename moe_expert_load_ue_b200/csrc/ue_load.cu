@@ -5,12 +5,12 @@
 // "exact-load" balancer).  counts[r][e] = #{(t, k) : t in rank r, ids[t][k] = e}.
 //
 // Design (sm_100a): one thread-block cluster per simulated rank.  Each CTA of
-// the cluster histograms a contiguous share of the rank's ids into shared
-// memory with 16-byte (int4) loads and warp-aggregated shared atomics
-// (__match_any_sync groups equal ids so each distinct id in a warp does one
-// atomic).  The cluster then reduces its CTA histograms over distributed
-// shared memory, each CTA summing a slice of the E columns, and writes its
-// rank's row of counts with plain stores: no global atomics, no pre-zeroing,
+// the cluster histograms a contiguous share of the rank's ids with 16-byte
+// (int4) loads into shared-memory histograms (8 copies, one per pair of
+// warps, so that shared atomics on a popular expert collide rarely), sums the
+// copies, and the cluster then reduces its CTA histograms over distributed
+// shared memory, each CTA summing a slice of the E columns.  The rank's row
+// of counts is written with plain stores: no global atomics, no pre-zeroing,
 // no workspace.
 #include <cooperative_groups.h>
 
@@ -22,21 +22,12 @@ namespace ue {
 namespace {
 
 constexpr int kLoadWarps = 16;
+constexpr int kCopies = 8;       // shared-memory histogram copies per CTA
 
-// One warp step: every lane offers `key` (-1 = nothing); each group of equal
-// keys adds its size to hist[key] once, from its lowest lane.
-__device__ __forceinline__ void warp_hist_add(int32_t *hist, int key)
+__device__ __forceinline__ void count_id(int32_t *h, int id, int E, int &nbad)
 {
-    const unsigned m = __match_any_sync(0xffffffffu, key);
-    if (key >= 0 && (lanemask_lt() & m) == 0) atomicAdd(&hist[key], __popc(m));
-}
-
-__device__ __forceinline__ int valid_key(int id, int E, bool in_range, int &nbad)
-{
-    if (!in_range) return -1;
-    if ((unsigned)id < (unsigned)E) return id;
-    ++nbad;
-    return -1;
+    if ((unsigned)id < (unsigned)E) atomicAdd(h + id, 1);
+    else ++nbad;
 }
 
 __global__ void __launch_bounds__(kLoadWarps * 32)
@@ -44,8 +35,13 @@ k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
        int32_t *__restrict__ counts, int32_t *__restrict__ bad)
 {
     extern __shared__ __align__(16) int32_t sm_load[];
-    int32_t *hist = sm_load;          // [E]
-    int32_t *sbad = sm_load + E;      // [1]
+    int32_t *hist = sm_load;                     // [kCopies][E] counts
+    int32_t *tot = hist + kCopies * E;           // [E]    CTA counts (read by the cluster)
+    int32_t *sbad = tot + E;                     // [1]
+
+    // The planner (launched with programmatic dependent launch) may start
+    // now; it waits for this grid's completion before reading counts.
+    pdl_trigger();
 
     cg::cluster_group cluster = cg::this_cluster();
     const int C = (int)cluster.num_blocks();
@@ -53,7 +49,7 @@ k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
     const int r = blockIdx.x / C;
     const int lane = lane_id(), warp = threadIdx.x >> 5;
 
-    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+    for (int i = threadIdx.x; i < kCopies * E; i += blockDim.x) hist[i] = 0;
     if (threadIdx.x == 0) *sbad = 0;
     __syncthreads();
 
@@ -65,38 +61,38 @@ k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
     // int4 body [vlo, vhi) on 16-byte boundaries (ids is 16-byte aligned).
     const int64_t vlo = min(hi, (lo + 3) / 4 * 4);
     const int64_t vhi = max(vlo, hi / 4 * 4);
+    int32_t *h = hist + (warp % kCopies) * E;
     int nbad = 0;
 
-    // Ragged head (< 4 ids) and tail (< 4 ids), one warp step.
+    // Ragged head (< 4 ids) and tail (< 4 ids).
     if (warp == 0) {
         int64_t i = -1;
         if (lane < vlo - lo) i = lo + lane;
         else if (lane >= 4 && lane - 4 < hi - vhi) i = vhi + (lane - 4);
-        const int id = i >= 0 ? __ldg(ids + i) : -1;
-        warp_hist_add(hist, valid_key(id, E, i >= 0, nbad));
+        if (i >= 0) count_id(h, __ldg(ids + i), E, nbad);
     }
-
-    // Body: each warp walks int4 vectors; two vectors in flight per lane.
+    // Body: every thread walks int4 vectors, two in flight.
     const int4 *vec = reinterpret_cast<const int4 *>(ids + vlo);
     const int64_t nvec = (vhi - vlo) / 4;
-    constexpr int kStride = kLoadWarps * 32;
-    for (int64_t w0 = (int64_t)warp * 32; w0 < nvec; w0 += 2 * kStride) {
-        const int64_t i0 = w0 + lane, i1 = w0 + kStride + lane;
-        const bool v0 = i0 < nvec, v1 = i1 < nvec;
-        int4 a = v0 ? __ldg(vec + i0) : make_int4(0, 0, 0, 0);
-        int4 b = v1 ? __ldg(vec + i1) : make_int4(0, 0, 0, 0);
-        warp_hist_add(hist, valid_key(a.x, E, v0, nbad));
-        warp_hist_add(hist, valid_key(a.y, E, v0, nbad));
-        warp_hist_add(hist, valid_key(a.z, E, v0, nbad));
-        warp_hist_add(hist, valid_key(a.w, E, v0, nbad));
-        if (w0 + kStride < nvec) {   // warp-uniform
-            warp_hist_add(hist, valid_key(b.x, E, v1, nbad));
-            warp_hist_add(hist, valid_key(b.y, E, v1, nbad));
-            warp_hist_add(hist, valid_key(b.z, E, v1, nbad));
-            warp_hist_add(hist, valid_key(b.w, E, v1, nbad));
-        }
+    const int64_t stride = (int64_t)blockDim.x;
+    int64_t v = threadIdx.x;
+    for (; v + stride < nvec; v += 2 * stride) {
+        const int4 a = __ldg(vec + v), b = __ldg(vec + v + stride);
+        count_id(h, a.x, E, nbad); count_id(h, a.y, E, nbad); count_id(h, a.z, E, nbad); count_id(h, a.w, E, nbad);
+        count_id(h, b.x, E, nbad); count_id(h, b.y, E, nbad); count_id(h, b.z, E, nbad); count_id(h, b.w, E, nbad);
+    }
+    if (v < nvec) {
+        const int4 a = __ldg(vec + v);
+        count_id(h, a.x, E, nbad); count_id(h, a.y, E, nbad); count_id(h, a.z, E, nbad); count_id(h, a.w, E, nbad);
     }
     if (nbad) atomicAdd(sbad, nbad);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int s = 0;
+#pragma unroll
+        for (int w = 0; w < kCopies; ++w) s += hist[w * E + e];
+        tot[e] = s;
+    }
 
     // Cluster reduction over distributed shared memory.
     cluster.sync();
@@ -104,7 +100,7 @@ k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
     const int e0 = c * cols, e1 = min(E, e0 + cols);
     for (int e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
         int s = 0;
-        for (int q = 0; q < C; ++q) s += cluster.map_shared_rank(hist, q)[e];
+        for (int q = 0; q < C; ++q) s += cluster.map_shared_rank(tot, q)[e];
         counts[(int64_t)r * E + e] = s;
     }
     if (bad != nullptr && c == 0 && threadIdx.x == 0) {
@@ -112,29 +108,18 @@ k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
         for (int q = 0; q < C; ++q) s += *cluster.map_shared_rank(sbad, q);
         bad[r] = s;
     }
-    cluster.sync();   // peers may still read this CTA's histogram
+    cluster.sync();   // peers may still read this CTA's totals
 }
 
 }  // namespace
 
-size_t load_smem_bytes(const Shape &sh) { return (size_t)(sh.E + 4) * sizeof(int32_t); }
+size_t load_smem_bytes(const Shape &sh) { return (size_t)((kCopies + 1) * sh.E + 4) * sizeof(int32_t); }
 
 cudaError_t launch_load(const Shape &sh, const Launch &ln, const int32_t *ids, int32_t *counts,
                         int32_t *bad, cudaStream_t st)
 {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(sh.N * ln.cluster));
-    cfg.blockDim = dim3(kLoadWarps * 32);
-    cfg.dynamicSmemBytes = load_smem_bytes(sh);
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)ln.cluster;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_load, ids, sh.per_rank, sh.E, counts, bad);
+    return launch_ex(k_load, (unsigned)(sh.N * ln.cluster), kLoadWarps * 32, load_smem_bytes(sh), st,
+                     (unsigned)ln.cluster, false, ids, sh.per_rank, sh.E, counts, bad);
 }
 
 cudaError_t set_load_attributes(size_t max_smem)

@@ -14,17 +14,27 @@
 //   rep_cum = exclusive prefix of their quotas.
 //
 // Design (sm_100a): one thread-block cluster of up to 8 CTAs x 1024 threads.
-//   Phase A (all CTAs, column blocks of 32 experts): column sums of counts
-//     give load[e]; the exclusive column scan over ranks gives rank_off[r][e]
-//     (what the reroute kernel needs).  CTA 0 then pulls every expert's load
-//     from the owning CTA's shared memory over DSMEM.
-//   Phase B (CTA 0): the home pass in closed form from a block-wide prefix
-//     sum (the home rank's load before e is min(Q, in-rank prefix), so
-//     take = min(Q, prefix + load) - min(Q, prefix)); the overflow order by
-//     a rank-by-counting sort; the greedy in one warp, each rank's spare and
-//     used-slot count held in the registers of lane r % 32, the argmax with
-//     two redux.sync instructions per chunk (max spare, then min rank among
-//     the lanes holding it); then all 1024 threads write the tables.
+//   Peer CTAs (cluster rank >= 1) own 32-expert column groups of counts: they
+//     sum their columns (loads) and arrive on the cluster barrier, then - off
+//     the critical path, while CTA 0 plans - write the exclusive column scan
+//     over ranks, rank_off[r][e], that the reroute kernel needs.
+//   CTA 0 pulls the loads over DSMEM and plans:
+//     * home pass in closed form from a block-wide prefix sum: the home rank's
+//       load before e is min(Q, in-rank prefix), so
+//       take = min(Q, prefix + load) - min(Q, prefix);
+//     * overflow order by a rank-by-counting sort of packed (overflow, id) keys;
+//     * R = 1: a rank can be chosen at most once and its spare never changes
+//       before that, so the greedy visits the eligible ranks in the order of
+//       their initial spare (descending, lowest rank first).  The ranks are
+//       sorted once, their spares prefix-summed, and each overflow expert takes
+//       the next run of ranks whose spares cover it: one warp-wide search per
+//       expert instead of one argmax per chunk;
+//     * R > 1: the chunk-by-chunk greedy in one warp, each rank's spare and
+//       used slots in the registers of lane r % 32, the argmax as two
+//       redux.sync (largest spare, then lowest rank holding it);
+//     * once no rank is eligible none becomes eligible again (spares only
+//       shrink, used slots only grow): the rest of the overflow stays home;
+//     * then all 1024 threads write the tables.
 #include <climits>
 
 #include <cooperative_groups.h>
@@ -39,56 +49,62 @@ namespace {
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanWarps = kPlanThreads / 32;
 
-// Shared-memory layout of the planner CTA (all int32).
+// Shared-memory layout of a planner CTA (all 4-byte words unless noted).
 struct PlanSmem {
-    int32_t *part;      // [32][33] phase-A partial sums
-    int32_t *ws;        // [64] scan / reduction scratch
-    int32_t *misc;      // [8]  n_asg, flags
-    int32_t *sload;     // [E]  loads of this CTA's column groups (CTA 0: all of them)
-    int32_t *pre;       // [E]  exclusive prefix of load over experts
-    int32_t *qh;        // [E]  home quota (plus any residual)
-    int32_t *ovf;       // [E]
-    int32_t *cl;        // [E]  experts with overflow (compacted)
-    int32_t *order;     // [E]  overflow order
-    int32_t *afirst;    // [E]  first assignment of e
-    int32_t *acnt;      // [E]  number of assignments of e
-    int32_t *before;    // [N]
-    int32_t *spare;     // [N]
-    int32_t *extra;     // [N]  residual overflow kept home
-    int32_t *ar;        // [NR] assignment rank
-    int32_t *au;        // [NR] assignment redundant index on that rank
-    int32_t *ac;        // [NR] assignment quota
-    int32_t *ae;        // [NR] assignment expert
-    int32_t *sasg;      // [NR] (rank, redundant index) -> assignment or -1
+    int32_t *part;        // [32][33] column-group partial sums
+    int32_t *ws;          // [96] scan / reduction scratch
+    int32_t *misc;        // [8]  assignments, stop position, remainder at the stop
+    int32_t *sload;       // [E]  loads (peers: of their own column groups)
+    int32_t *pre;         // [E]  exclusive prefix of load over experts
+    int32_t *qh;          // [E]  home quota (plus any residual)
+    int32_t *ovf;         // [E]
+    int32_t *order;       // [E]  overflow order
+    int32_t *afirst;      // [E]  first assignment of e
+    int32_t *acnt;        // [E]  number of assignments of e
+    int32_t *before;      // [N]
+    int32_t *spare;       // [N]
+    int32_t *extra;       // [N]  residual overflow kept home
+    int32_t *rsorted;     // [N]  R = 1: eligible ranks by initial spare
+    int32_t *rsum;        // [N+1] R = 1: exclusive prefix of their spares
+    int32_t *ar;          // [NR] assignment rank
+    int32_t *au;          // [NR] assignment redundant index on that rank
+    int32_t *ac;          // [NR] assignment quota
+    int32_t *ae;          // [NR] assignment expert
+    int32_t *sasg;        // [NR] (rank, redundant index) -> assignment or -1
+    unsigned long long *key;   // [max(E, N)] packed sort keys (8-byte aligned)
 };
 
 __host__ __device__ inline size_t plan_smem_words(int E, int N, int NR)
 {
-    return (size_t)32 * 33 + 64 + 8 + (size_t)8 * E + (size_t)3 * N + (size_t)5 * NR;
+    const int K = E > N ? E : N;
+    return (size_t)32 * 33 + 96 + 8 + (size_t)7 * E + (size_t)5 * N + 1 + (size_t)5 * NR + 2 + (size_t)2 * K;
 }
 
 __device__ __forceinline__ PlanSmem carve(int32_t *p, int E, int N, int NR)
 {
     PlanSmem s;
-    s.part = p;            p += 32 * 33;
-    s.ws = p;              p += 64;
-    s.misc = p;            p += 8;
-    s.sload = p;           p += E;
-    s.pre = p;             p += E;
-    s.qh = p;              p += E;
-    s.ovf = p;             p += E;
-    s.cl = p;              p += E;
-    s.order = p;           p += E;
-    s.afirst = p;          p += E;
-    s.acnt = p;            p += E;
-    s.before = p;          p += N;
-    s.spare = p;           p += N;
-    s.extra = p;           p += N;
-    s.ar = p;              p += NR;
-    s.au = p;              p += NR;
-    s.ac = p;              p += NR;
-    s.ae = p;              p += NR;
-    s.sasg = p;
+    s.part = p;      p += 32 * 33;
+    s.ws = p;        p += 96;
+    s.misc = p;      p += 8;
+    s.sload = p;     p += E;
+    s.pre = p;       p += E;
+    s.qh = p;        p += E;
+    s.ovf = p;       p += E;
+    s.order = p;     p += E;
+    s.afirst = p;    p += E;
+    s.acnt = p;      p += E;
+    s.before = p;    p += N;
+    s.spare = p;     p += N;
+    s.extra = p;     p += N;
+    s.rsorted = p;   p += N;
+    s.rsum = p;      p += N + 1;
+    s.ar = p;        p += NR;
+    s.au = p;        p += NR;
+    s.ac = p;        p += NR;
+    s.ae = p;        p += NR;
+    s.sasg = p;      p += NR;
+    p += (reinterpret_cast<uintptr_t>(p) & 7) ? 1 : 0;
+    s.key = reinterpret_cast<unsigned long long *>(p);
     return s;
 }
 
@@ -120,22 +136,63 @@ __device__ int block_excl_scan(int v, int32_t *ws, int *total)
     return r;
 }
 
-__device__ int block_max(int v, int32_t *ws)
+// Sum of counts[r][g*32 + lane] over this thread's rows [r0, r1).
+__device__ __forceinline__ int column_part(const int32_t *__restrict__ counts, int E, int g, int r0, int r1)
 {
-    const int lane = lane_id(), warp = threadIdx.x >> 5;
-    v = __reduce_max_sync(0xffffffffu, v);
-    if (lane == 0) ws[warp] = v;
-    __syncthreads();
-    int m = ws[0];
-    for (int w = 1; w < kPlanWarps; ++w) m = max(m, ws[w]);
-    __syncthreads();
-    return m;
+    const int e = g * 32 + lane_id();
+    int sum = 0;
+    if (e < E)
+        for (int r = r0; r < r1; ++r) sum += __ldg(counts + (int64_t)r * E + e);
+    return sum;
 }
 
-// The greedy overflow placement, run by warp 0.  Lane l owns ranks l, l+32, ...
-// (NRL per lane), keeping spare capacity and used redundant slots in registers.
+// Column totals of group g from part[row group][column]; writes sload and the plan's load.
+__device__ __forceinline__ void column_totals(int E, int g, const int32_t *part, int32_t *sload, int32_t *load_out)
+{
+    const int tid = threadIdx.x;
+    if (tid < 32) {
+        const int e = g * 32 + tid;
+        int t = 0;
+#pragma unroll 8
+        for (int w = 0; w < 32; ++w) t += part[w * 33 + tid];
+        if (e < E) {
+            sload[e] = t;
+            load_out[e] = t;
+        }
+    }
+}
+
+// Exclusive scan of column group g over the row groups (part[row group][column]),
+// then rank_off[r][e] for this thread's rows [r0, r1).
+__device__ void column_rank_off(const int32_t *__restrict__ counts, int E, int g, int r0, int r1, int32_t *part,
+                                int32_t *rank_off)
+{
+    const int lane = lane_id(), warp = threadIdx.x >> 5;
+    __syncthreads();   // column_totals has read part
+    {   // warp w scans column w of the group over the row groups (lane = row group)
+        const int v = part[lane * 33 + warp];
+        int x = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        part[lane * 33 + warp] = x - v;
+    }
+    __syncthreads();
+    const int e = g * 32 + lane;
+    int run = part[warp * 33 + lane];
+    if (e < E)
+        for (int r = r0; r < r1; ++r) {
+            rank_off[(int64_t)r * E + e] = run;
+            run += __ldg(counts + (int64_t)r * E + e);
+        }
+    __syncthreads();
+}
+
+// R > 1: the chunk-by-chunk greedy, run by warp 0.
 template <int NRL>
-__device__ void greedy(const PlanSmem &s, int N, int R, int H, int M1)
+__device__ void greedy_chunks(const PlanSmem &s, int N, int R, int M1)
 {
     const int lane = lane_id();
     unsigned sp[NRL];
@@ -146,61 +203,66 @@ __device__ void greedy(const PlanSmem &s, int N, int R, int H, int M1)
         sp[i] = r < N ? (unsigned)s.spare[r] : 0u;
         us[i] = 0;
     }
-    unsigned bs = 0;
-    int br = INT_MAX;
+    unsigned bs;
+    int br;
     auto lane_best = [&]() {
         bs = 0;
         br = INT_MAX;
 #pragma unroll
         for (int i = 0; i < NRL; ++i) {
-            const int r = lane + 32 * i;
-            const bool eligible = r < N && us[i] < R && sp[i] > 0u;
-            if (eligible && sp[i] > bs) { bs = sp[i]; br = r; }   // strict: lowest rank on ties
+            const bool better = us[i] < R && sp[i] > bs;    // strict: lowest rank on ties
+            bs = better ? sp[i] : bs;
+            br = better ? lane + 32 * i : br;
         }
     };
     lane_best();
 
-    int na = 0, flags = 0;
-    for (int m = 0; m < M1; ++m) {
-        const int e = s.order[m];
-        int rem = s.ovf[e];
-        const int first = na;
-        while (rem > 0) {
-            const unsigned mx = __reduce_max_sync(0xffffffffu, bs);
-            if (mx == 0u) {                       // slots ran out: remainder stays home
-                if (lane == 0) {
-                    s.qh[e] += rem;
-                    s.extra[e / H] += rem;
-                }
-                flags |= 1;
-                break;
-            }
-            const int rs = __reduce_min_sync(0xffffffffu, bs == mx ? br : INT_MAX);
-            const int c = rem < (int)mx ? rem : (int)mx;
-            if (lane == (rs & 31)) {
-                const int slot_i = rs >> 5;
+    int na = 0, stop_pos = M1, stop_rem = 0;
+    for (int m0 = 0; m0 < M1 && stop_pos == M1; m0 += 32) {
+        const int idx = m0 + lane;
+        const int e_l = idx < M1 ? s.order[idx] : 0;
+        const int o_l = idx < M1 ? s.ovf[e_l] : 0;
+        const int cnt = min(32, M1 - m0);
+        for (int j = 0; j < cnt; ++j) {
+            const int e = __shfl_sync(0xffffffffu, e_l, j);
+            int rem = __shfl_sync(0xffffffffu, o_l, j);
+            const int first = na;
+            while (rem > 0) {
+                const unsigned mx = __reduce_max_sync(0xffffffffu, bs);
+                if (mx == 0u) break;                             // no eligible rank left
+                const int rs = __reduce_min_sync(0xffffffffu, bs == mx ? br : INT_MAX);
+                const int c = rem < (int)mx ? rem : (int)mx;
+                const bool own = lane == (rs & 31);
+                const int si = rs >> 5;
                 int u = 0;
 #pragma unroll
                 for (int i = 0; i < NRL; ++i) {
-                    if (i == slot_i) {
-                        u = us[i];
-                        us[i] += 1;
-                        sp[i] -= (unsigned)c;
-                    }
+                    const bool hit = own && i == si;
+                    u = hit ? us[i] : u;
+                    us[i] += hit ? 1 : 0;
+                    sp[i] -= hit ? (unsigned)c : 0u;
                 }
-                s.ar[na] = rs;
-                s.au[na] = u;
-                s.ac[na] = c;
-                s.ae[na] = e;
-                s.sasg[rs * R + u] = na;
                 lane_best();
+                u = __shfl_sync(0xffffffffu, u, rs & 31);
+                if (lane == 0) {
+                    s.ar[na] = rs;
+                    s.au[na] = u;
+                    s.ac[na] = c;
+                    s.ae[na] = e;
+                    s.sasg[rs * R + u] = na;
+                }
+                rem -= c;
+                ++na;
             }
-            rem -= c;
-            ++na;
-        }
-        if (lane == 0) {
-            s.afirst[e] = first;
-            s.acnt[e] = na - first;
+            if (lane == 0) {
+                s.afirst[e] = first;
+                s.acnt[e] = na - first;
+            }
+            if (rem > 0) {                                       // ran out at this expert
+                stop_pos = m0 + j;
+                stop_rem = rem;
+                break;
+            }
         }
     }
 #pragma unroll
@@ -210,10 +272,63 @@ __device__ void greedy(const PlanSmem &s, int N, int R, int H, int M1)
     }
     if (lane == 0) {
         s.misc[0] = na;
-        s.misc[1] = flags;
+        s.misc[1] = stop_pos;
+        s.misc[2] = stop_rem;
     }
 }
 
+// R = 1: walk the eligible ranks in sorted order (s.rsorted, exclusive prefix
+// s.rsum, K of them); run by warp 0.  Assignment a is sorted position a.
+__device__ void greedy_sorted(const PlanSmem &s, int K, int M1)
+{
+    const int lane = lane_id();
+    int p = 0, stop_pos = M1, stop_rem = 0;
+    for (int m = 0; m < M1; ++m) {
+        const int e = s.order[m];
+        const int rem = s.ovf[e];
+        const long long target = (long long)s.rsum[p] + rem;   // smallest q > p with rsum[q] >= target
+        int q = -1;
+        for (int base = p + 1; base <= K; base += 32) {
+            const int cand = base + lane;
+            const bool hit = cand <= K && (long long)s.rsum[cand] >= target;
+            const unsigned b = __ballot_sync(0xffffffffu, hit);
+            if (b) {
+                q = base + __ffs(b) - 1;
+                break;
+            }
+        }
+        const int end = q < 0 ? K : q;            // ranks [p, end) go to e
+        for (int a = p + lane; a < end; a += 32) {
+            const int r = s.rsorted[a];
+            const int full = s.rsum[a + 1] - s.rsum[a];
+            s.ar[a] = r;
+            s.au[a] = 0;
+            s.ac[a] = (q >= 0 && a == end - 1) ? rem - (s.rsum[a] - s.rsum[p]) : full;
+            s.ae[a] = e;
+            s.sasg[r] = a;
+        }
+        if (lane == 0) {
+            s.afirst[e] = p;
+            s.acnt[e] = end - p;
+        }
+        if (q < 0) {                              // every remaining rank used: the rest stays home
+            stop_pos = m;
+            stop_rem = rem - (s.rsum[K] - s.rsum[p]);
+            p = K;
+            break;
+        }
+        p = q;
+    }
+    __syncwarp();
+    for (int a = lane; a < p; a += 32) s.spare[s.ar[a]] -= s.ac[a];
+    if (lane == 0) {
+        s.misc[0] = p;
+        s.misc[1] = stop_pos;
+        s.misc[2] = stop_rem;
+    }
+}
+
+template <int NRL>
 __global__ void __launch_bounds__(kPlanThreads, 1)
 k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
 {
@@ -224,71 +339,68 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
     cg::cluster_group cluster = cg::this_cluster();
     const int C = (int)cluster.num_blocks();
     const int c = (int)cluster.block_rank();
-    const int tid = threadIdx.x, lane = lane_id(), warp = tid >> 5;
-
-    // ---- phase A: loads and rank offsets, 32-expert column groups ----------
-    const int rpg = (N + 31) / 32;               // ranks per row group
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int groups = (E + 31) / 32;
+    const int rpg = (N + 31) / 32;                 // ranks per row group
     const int r0 = min(N, warp * rpg), r1 = min(N, r0 + rpg);
-    for (int g = c; g * 32 < E; g += C) {
-        const int e = g * 32 + lane;
-        const bool ve = e < E;
-        int sum = 0;
-        if (ve)
-            for (int r = r0; r < r1; ++r) sum += __ldg(counts + (int64_t)r * E + e);
-        s.part[warp * 33 + lane] = sum;
-        __syncthreads();
-        {   // warp w scans column w of the group over the 32 row groups (lane = row group)
-            const int col = warp;
-            const int v = s.part[lane * 33 + col];
-            int x = v;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, x, o);
-                if (lane >= o) x += y;
-            }
-            s.part[lane * 33 + col] = x - v;
-            const int ec = g * 32 + col;
-            if (lane == 31 && ec < E) {
-                plan.load[ec] = x;
-                s.sload[ec] = x;          // pulled by CTA 0 after the cluster barrier
-            }
+
+    // The reroute grid may launch now (its first pass needs only the ids);
+    // the counts of the load grid are read after it completes.
+    pdl_trigger();
+    pdl_wait();
+
+    if (C > 1 && c != 0) {
+        // Peer: loads of the own column groups, then (off the critical path) rank_off.
+        for (int g = c - 1; g < groups; g += C - 1) {
+            s.part[warp * 33 + lane_id()] = column_part(counts, E, g, r0, r1);
+            __syncthreads();
+            column_totals(E, g, s.part, s.sload, plan.load);
+            __syncthreads();
         }
-        __syncthreads();
-        int run = s.part[warp * 33 + lane];
-        if (ve)
-            for (int r = r0; r < r1; ++r) {
-                plan.rank_off[(int64_t)r * E + e] = run;
-                run += __ldg(counts + (int64_t)r * E + e);
-            }
-        __syncthreads();
-    }
-    cluster.sync();
-    if (c != 0) {              // keep this CTA's loads readable until CTA 0 has pulled them
-        cluster_arrive();
+        cluster_arrive();      // #1: loads ready for CTA 0
+        for (int g = c - 1; g < groups; g += C - 1) {
+            s.part[warp * 33 + lane_id()] = column_part(counts, E, g, r0, r1);
+            __syncthreads();
+            column_rank_off(counts, E, g, r0, r1, s.part, plan.rank_off);
+        }
+        cluster_wait();
+        cluster_arrive();      // #2: completes once CTA 0 has pulled the loads
         cluster_wait();
         return;
     }
-
-    // ---- phase B: the plan, CTA 0 ---------------------------------------------
-    const int e = tid;
-    const bool ve = e < E;
-    const int ld = ve ? cluster.map_shared_rank(s.sload, (e >> 5) % C)[e] : 0;
+    if (C == 1) {
+        for (int g = 0; g < groups; ++g) {
+            s.part[warp * 33 + lane_id()] = column_part(counts, E, g, r0, r1);
+            __syncthreads();
+            column_totals(E, g, s.part, s.sload, plan.load);
+            column_rank_off(counts, E, g, r0, r1, s.part, plan.rank_off);
+        }
+    }
     cluster_arrive();
     cluster_wait();
+    const int e = tid;
+    const bool ve = e < E;
+    const int ld = !ve ? 0 : (C == 1 ? s.sload[e] : cluster.map_shared_rank(s.sload, 1 + (e >> 5) % (C - 1))[e]);
+    cluster_arrive();          // #2; the matching wait is at the end of the kernel
+
+    // ---- the plan ---------------------------------------------------------------
     int L;
     const int pre = block_excl_scan(ld, s.ws, &L);
     const int Q = L == 0 ? 0 : (L - 1) / N + 1;
     if (ve) s.pre[e] = pre;
     for (int r = tid; r < N; r += kPlanThreads) s.extra[r] = 0;
+    for (int i = tid; i < NR; i += kPlanThreads) s.sasg[i] = -1;
     __syncthreads();
 
     // Home pass in closed form.
+    int my_ovf = 0;
     if (ve) {
         const int h = e / H;
         const int pin = pre - s.pre[h * H];      // load of earlier experts of the same home rank
         const int take = min(Q, pin + ld) - min(Q, pin);
+        my_ovf = ld - take;
         s.qh[e] = take;
-        s.ovf[e] = ld - take;
+        s.ovf[e] = my_ovf;
         s.acnt[e] = 0;
         s.afirst[e] = 0;
         if (e % H == H - 1) {
@@ -297,42 +409,75 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
             s.spare[h] = Q - min(Q, rank_sum);
         }
     }
-    for (int i = tid; i < NR; i += kPlanThreads) s.sasg[i] = -1;
-
-    // Overflow experts, then their order: overflow descending, lower id first.
-    const int has_ovf = (ve && s.ovf[e] > 0) ? 1 : 0;   // read after the scan's barriers
+    // Overflow experts as packed keys: larger overflow first, then lower id.
     int M1;
-    const int pos = block_excl_scan(has_ovf, s.ws, &M1);
-    if (has_ovf) s.cl[pos] = e;
+    const int pos = block_excl_scan(my_ovf > 0 ? 1 : 0, s.ws, &M1);
+    if (my_ovf > 0) s.key[pos] = ((unsigned long long)(unsigned)my_ovf << 32) | (0xffffffffu - (unsigned)e);
     __syncthreads();
     if (tid < M1) {
-        const int ei = s.cl[tid], oi = s.ovf[ei];
+        const unsigned long long mine = s.key[tid];
         int rank = 0;
-        for (int k = 0; k < M1; ++k) {
-            const int ek = s.cl[k], ok = s.ovf[ek];
-            rank += (ok > oi) || (ok == oi && ek < ei);
+#pragma unroll 8
+        for (int k = 0; k < M1; ++k) rank += s.key[k] > mine ? 1 : 0;
+        s.order[rank] = (int)(0xffffffffu - (unsigned)(mine & 0xffffffffu));
+    }
+    __syncthreads();
+
+    if (R == 1) {
+        // Eligible ranks (spare > 0) sorted by spare descending, lowest rank first.
+        const int sp_r = tid < N ? s.spare[tid] : 0;
+        int K;
+        const int kpos = block_excl_scan(sp_r > 0 ? 1 : 0, s.ws, &K);
+        if (sp_r > 0) s.key[kpos] = ((unsigned long long)(unsigned)sp_r << 32) | (0xffffffffu - (unsigned)tid);
+        __syncthreads();
+        int my_rank = 0, my_sp = 0;
+        if (tid < K) {
+            const unsigned long long mine = s.key[tid];
+            int rank = 0;
+#pragma unroll 8
+            for (int k = 0; k < K; ++k) rank += s.key[k] > mine ? 1 : 0;
+            my_rank = rank;
+            my_sp = (int)(mine >> 32);
+            s.rsorted[rank] = (int)(0xffffffffu - (unsigned)(mine & 0xffffffffu));
         }
-        s.order[rank] = ei;
+        __syncthreads();
+        if (tid < K) s.rsum[my_rank] = my_sp;   // spares in sorted order
+        __syncthreads();
+        const int sp_sorted = tid < K ? s.rsum[tid] : 0;
+        int tot;
+        const int ex = block_excl_scan(sp_sorted, s.ws, &tot);
+        if (tid < K) s.rsum[tid] = ex;
+        if (tid == 0) s.rsum[K] = tot;
+        __syncthreads();
+        if (warp == 0) greedy_sorted(s, K, M1);
+    } else if (warp == 0) {
+        greedy_chunks<NRL>(s, N, R, M1);
+    }
+    __syncthreads();
+    const int n_asg = s.misc[0], stop_pos = s.misc[1], stop_rem = s.misc[2];
+    const int flags = stop_pos < M1 ? 1 : 0;
+    // Slots ran out at overflow position stop_pos: that expert's remainder and
+    // the whole overflow of every later expert stay on their home slots.
+    for (int p = stop_pos + tid; p < M1; p += kPlanThreads) {
+        const int ep = s.order[p];
+        const int res = p == stop_pos ? stop_rem : s.ovf[ep];
+        s.qh[ep] += res;
+        atomicAdd(&s.extra[ep / H], res);
+        if (p != stop_pos) {
+            s.afirst[ep] = 0;
+            s.acnt[ep] = 0;
+        }
     }
     __syncthreads();
 
-    // Greedy placement in warp 0.
-    if (warp == 0) {
-        const int nrl = (N + 31) / 32;
-        if (nrl <= 1) greedy<1>(s, N, R, H, M1);
-        else if (nrl <= 2) greedy<2>(s, N, R, H, M1);
-        else if (nrl <= 4) greedy<4>(s, N, R, H, M1);
-        else if (nrl <= 8) greedy<8>(s, N, R, H, M1);
-        else if (nrl <= 16) greedy<16>(s, N, R, H, M1);
-        else greedy<32>(s, N, R, H, M1);
-    }
-    __syncthreads();
-    const int n_asg = s.misc[0], flags = s.misc[1];
-
-    // Replica lists (CSR): home first, then allocation order.
-    const int nrep = ve ? 1 + s.acnt[e] : 0;
-    int tot_rep;
-    const int off = block_excl_scan(nrep, s.ws, &tot_rep);
+    // Replica lists (CSR) and the replicated-expert list from one packed scan:
+    // the low 16 bits count replica entries, the high bits replicated experts.
+    const int na_e = ve ? s.acnt[e] : 0;
+    const int packed = ve ? (1 + na_e) | ((na_e > 0 ? 1 : 0) << 16) : 0;
+    int tot_packed;
+    const int pk = block_excl_scan(packed, s.ws, &tot_packed);
+    const int off = pk & 0xffff, mpos = pk >> 16;
+    const int tot_rep = tot_packed & 0xffff, M = tot_packed >> 16;
     if (ve) {
         const int h = e / H;
         plan.rep_off[e] = off;
@@ -340,18 +485,20 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
         plan.rep_cum[off] = 0;
         int cum = s.qh[e];
         const int a0 = s.afirst[e];
-        for (int i = 0; i < s.acnt[e]; ++i) {
+        for (int i = 0; i < na_e; ++i) {
             const int a = a0 + i;
             plan.rep_slot[off + 1 + i] = s.ar[a] * HR + H + s.au[a];
             plan.rep_cum[off + 1 + i] = cum;
             cum += s.ac[a];
         }
+        if (na_e > 0) plan.rep_experts[mpos] = e;
     }
     if (tid == 0) plan.rep_off[E] = tot_rep;
     for (int p = tot_rep + tid; p < cap; p += kPlanThreads) {
         plan.rep_slot[p] = -1;
         plan.rep_cum[p] = -1;
     }
+    for (int p = M + tid; p < E; p += kPlanThreads) plan.rep_experts[p] = -1;
 
     // Slot table.
     for (int sl = tid; sl < S; sl += kPlanThreads) {
@@ -369,14 +516,7 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
         plan.slot_quota[sl] = sq;
     }
 
-    // Experts holding redundant replicas, increasing id.
-    const int rep_flag = (ve && s.acnt[e] > 0) ? 1 : 0;
-    int M;
-    const int mpos = block_excl_scan(rep_flag, s.ws, &M);
-    if (rep_flag) plan.rep_experts[mpos] = e;
-    for (int p = M + tid; p < E; p += kPlanThreads) plan.rep_experts[p] = -1;
-
-    // Rank loads before / after.
+    // Rank loads before / after and their maxima.
     int mb = 0, ma = 0;
     for (int r = tid; r < N; r += kPlanThreads) {
         const int after = Q - s.spare[r] + s.extra[r];
@@ -385,9 +525,18 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
         mb = max(mb, s.before[r]);
         ma = max(ma, after);
     }
-    mb = block_max(mb, s.ws);
-    ma = block_max(ma, s.ws);
+    mb = __reduce_max_sync(0xffffffffu, mb);
+    ma = __reduce_max_sync(0xffffffffu, ma);
+    if (lane_id() == 0) {
+        s.ws[warp] = mb;
+        s.ws[32 + warp] = ma;
+    }
+    __syncthreads();
     if (tid == 0) {
+        for (int w = 1; w < kPlanWarps; ++w) {
+            mb = max(mb, s.ws[w]);
+            ma = max(ma, s.ws[32 + w]);
+        }
         plan.info[0] = Q;
         plan.info[1] = L;
         plan.info[2] = flags;
@@ -397,6 +546,7 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
         plan.info[6] = ma;
         plan.info[7] = 0;
     }
+    cluster_wait();
 }
 
 }  // namespace
@@ -406,30 +556,36 @@ size_t plan_smem_bytes(const Shape &sh) { return plan_smem_words(sh.E, sh.N, sh.
 int plan_cluster(const Shape &sh)
 {
     const int groups = (sh.E + 31) / 32;
-    return groups < kMaxCluster ? groups : kMaxCluster;
+    if (groups <= 1) return 1;
+    return groups + 1 < kMaxCluster ? groups + 1 : kMaxCluster;   // CTA 0 plans, peers own column groups
 }
 
-cudaError_t launch_plan(const Shape &sh, const int32_t *counts, const PlanDev &plan, cudaStream_t st)
+cudaError_t launch_plan(const Shape &sh, const int32_t *counts, const PlanDev &plan, cudaStream_t st, bool pdl)
 {
-    const int C = plan_cluster(sh);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)C);
-    cfg.blockDim = dim3(kPlanThreads);
-    cfg.dynamicSmemBytes = plan_smem_bytes(sh);
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_plan, counts, sh.E, sh.N, sh.R, plan);
+    const unsigned C = (unsigned)plan_cluster(sh);
+    const int nrl = (sh.N + 31) / 32;
+    const size_t smem = plan_smem_bytes(sh);
+#define UE_PLAN_LAUNCH(V) launch_ex(k_plan<V>, C, kPlanThreads, smem, st, C, pdl, counts, sh.E, sh.N, sh.R, plan)
+    if (nrl <= 1) return UE_PLAN_LAUNCH(1);
+    if (nrl <= 2) return UE_PLAN_LAUNCH(2);
+    if (nrl <= 4) return UE_PLAN_LAUNCH(4);
+    if (nrl <= 8) return UE_PLAN_LAUNCH(8);
+    if (nrl <= 16) return UE_PLAN_LAUNCH(16);
+    return UE_PLAN_LAUNCH(32);
+#undef UE_PLAN_LAUNCH
 }
 
 cudaError_t set_plan_attributes(size_t max_smem)
 {
-    return cudaFuncSetAttribute(k_plan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)max_smem);
+    const int m = (int)max_smem;
+    const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
+    cudaError_t e = cudaFuncSetAttribute(k_plan<1>, a, m);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_plan<2>, a, m);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_plan<4>, a, m);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_plan<8>, a, m);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_plan<16>, a, m);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_plan<32>, a, m);
+    return e;
 }
 
 }  // namespace ue

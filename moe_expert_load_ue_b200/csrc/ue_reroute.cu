@@ -6,16 +6,21 @@
 // replica i of e whose cumulative-quota range [rep_cum[i], rep_cum[i] + q_i)
 // holds j.
 //
-// Design (sm_100a): the same rank-per-cluster decomposition as the load
-// kernel.  j = (occurrences of e in earlier ranks: plan.rank_off[r][e])
-//           + (occurrences in earlier CTAs of this rank's cluster, read from
-//              the peers' shared-memory histograms over DSMEM)
-//           + (occurrences in earlier warps of this CTA: exclusive scan of
-//              per-warp histograms)
-//           + (running count inside the warp: __match_any_sync groups equal
-//              ids, the rank inside a group is popc(group & lanemask_lt)).
-// The replica tables of the plan sit in shared memory; the lookup scans the
-// (typically 1-3) replicas of e from the last one down.
+// Design (sm_100a): the rank-per-cluster decomposition of the load kernel.
+// Each warp owns a contiguous part of its CTA's ids, and the occurrence index
+// of the warp's first occurrence of e is
+//     rank_off[r][e]                         (earlier ranks, from the plan)
+//   + totals of e in earlier CTAs of the rank's cluster (peers' shared memory, DSMEM)
+//   + counts of e in earlier warps of this CTA (exclusive scan of per-warp histograms).
+// Pass 1 (per-warp histograms) needs only the ids, so it runs before
+// griddepcontrol.wait: launched with programmatic dependent launch, it
+// overlaps the planner.  From the counts and the bases each warp then knows,
+// per expert, whether all its occurrences fall into one replica's quota range
+// ("uniform": every expert with one replica, and almost every (warp, expert)
+// pair of a replicated one).  Pass 2 is then one shared-memory lookup per id;
+// only ids of an expert whose quota boundary falls inside the warp's part are
+// ranked exactly, by ballots over the bits of the expert's compact index in
+// plan.rep_experts.
 #include <cooperative_groups.h>
 
 #include "ue_internal.cuh"
@@ -29,32 +34,51 @@ constexpr int kRerouteWarps = 16;
 constexpr int kUnroll = 4;
 
 struct RerouteSmem {
-    int32_t *hist;   // [W][E]  per-warp counts, then per-warp base occurrence index
-    int32_t *tot;    // [E]     this CTA's counts (read by later CTAs of the cluster)
-    int32_t *roff;   // [E+1]
-    int32_t *rslot;  // [cap]
-    int32_t *rcum;   // [cap]
+    int32_t *hist;   // [W][E] per-warp counts; then ~slot (uniform) or running occurrence index
+    int32_t *tot;    // [E]    this CTA's counts (read by later CTAs of the cluster)
+    int2 *tab;       // [E]    {first replica entry, (compact index << 16) | replica count}
+    int2 *rc;        // [cap]  {cumulative quota, slot} of each replica entry
 };
 
-__device__ __forceinline__ RerouteSmem carve(int32_t *base, int E, int cap)
+__host__ __device__ inline size_t reroute_smem_words(int E, int cap)
+{
+    return (size_t)kRerouteWarps * E + E + 2 * (size_t)E + 2 * (size_t)cap + 4;
+}
+
+__device__ __forceinline__ RerouteSmem carve(int32_t *base, int E)
 {
     RerouteSmem s;
     s.hist = base;
     s.tot = s.hist + kRerouteWarps * E;
-    s.roff = s.tot + E;
-    s.rslot = s.roff + E + 1;
-    s.rcum = s.rslot + cap;
+    int32_t *p = s.tot + E;
+    p += (reinterpret_cast<uintptr_t>(p) & 7) ? 1 : 0;   // 8-byte alignment for int2
+    s.tab = reinterpret_cast<int2 *>(p);
+    s.rc = s.tab + E;
     return s;
+}
+
+// Lanes of the warp holding the same key as this lane (keys in [0, 2^nb), or -1).
+__device__ __forceinline__ unsigned match_key(int key, int nb)
+{
+    const unsigned none = __ballot_sync(0xffffffffu, key < 0);
+    unsigned m = key < 0 ? none : ~none;
+    for (int b = 0; b < nb; ++b) {
+        const bool bit = (key >> b) & 1;
+        const unsigned v = __ballot_sync(0xffffffffu, bit);
+        m &= bit ? v : ~v;
+    }
+    return m;
 }
 
 __global__ void __launch_bounds__(kRerouteWarps * 32)
 k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
           const int32_t *__restrict__ rep_off, const int32_t *__restrict__ rep_slot,
-          const int32_t *__restrict__ rep_cum, const int32_t *__restrict__ rank_off,
+          const int32_t *__restrict__ rep_cum, const int32_t *__restrict__ rep_experts,
+          const int32_t *__restrict__ info, const int32_t *__restrict__ rank_off,
           int32_t *__restrict__ phys)
 {
     extern __shared__ __align__(16) int32_t sm_rr[];
-    const RerouteSmem s = carve(sm_rr, E, cap);
+    const RerouteSmem s = carve(sm_rr, E);
 
     cg::cluster_group cluster = cg::this_cluster();
     const int C = (int)cluster.num_blocks();
@@ -62,12 +86,6 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
     const int r = blockIdx.x / C;
     const int lane = lane_id(), warp = threadIdx.x >> 5;
 
-    // Plan tables -> shared memory (clamped so a malformed plan cannot index out of bounds).
-    for (int i = threadIdx.x; i <= E; i += blockDim.x) s.roff[i] = clampi(__ldg(rep_off + i), 0, cap);
-    for (int i = threadIdx.x; i < cap; i += blockDim.x) {
-        s.rslot[i] = __ldg(rep_slot + i);
-        s.rcum[i] = __ldg(rep_cum + i);
-    }
     for (int i = threadIdx.x; i < kRerouteWarps * E; i += blockDim.x) s.hist[i] = 0;
     __syncthreads();
 
@@ -82,73 +100,95 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
     const int64_t whi = min(hi, wlo + wshare);
     int32_t *h = s.hist + warp * E;
 
-    // Pass 1: per-warp histogram of the warp's part (warp-private: no atomics).
+    // Pass 1: per-warp histogram of the warp's part (ids only; overlaps the planner).
     for (int64_t x0 = wlo; x0 < whi; x0 += 32 * kUnroll) {
-        int key[kUnroll];
+        int id[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             const int64_t i = x0 + u * 32 + lane;
-            const int id = i < whi ? __ldg(ids + i) : -1;
-            key[u] = (unsigned)id < (unsigned)E ? id : -1;
+            id[u] = i < whi ? __ldg(ids + i) : -1;
         }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const unsigned m = __match_any_sync(0xffffffffu, key[u]);
-            if (key[u] >= 0 && (lanemask_lt() & m) == 0) h[key[u]] += __popc(m);
-            __syncwarp();
-        }
+        for (int u = 0; u < kUnroll; ++u)
+            if ((unsigned)id[u] < (unsigned)E) atomicAdd(h + id[u], 1);
     }
     __syncthreads();
-
-    // Exclusive scan over warps per expert; CTA totals for the cluster peers.
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int run = 0;
+        int t = 0;
 #pragma unroll
-        for (int w = 0; w < kRerouteWarps; ++w) {
-            const int t = s.hist[w * E + e];
-            s.hist[w * E + e] = run;
-            run += t;
-        }
-        s.tot[e] = run;
+        for (int w = 0; w < kRerouteWarps; ++w) t += s.hist[w * E + e];
+        s.tot[e] = t;
     }
     cluster.sync();
-    // Base occurrence index of this CTA = earlier ranks + earlier CTAs of this rank.
+
+    // The plan (and rank_off) of the preceding planner grid.
+    pdl_wait();
+    for (int i = threadIdx.x; i < cap; i += blockDim.x) s.rc[i] = make_int2(__ldg(rep_cum + i), __ldg(rep_slot + i));
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int b = __ldg(rank_off + (int64_t)r * E + e);
-        for (int q = 0; q < c; ++q) b += cluster.map_shared_rank(s.tot, q)[e];
-#pragma unroll
-        for (int w = 0; w < kRerouteWarps; ++w) s.hist[w * E + e] += b;
+        const int off = clampi(__ldg(rep_off + e), 0, cap - 1);
+        const int n = clampi(__ldg(rep_off + e + 1) - off, 1, min(cap - off, 0xffff));
+        s.tab[e] = make_int2(off, n);
     }
-    cluster_arrive();          // done reading peers; they may exit once all arrive
+    const int M = clampi(__ldg(info + 3), 0, E);
+    __syncthreads();
+    for (int m = threadIdx.x; m < M; m += blockDim.x) {
+        const int e = clampi(__ldg(rep_experts + m), 0, E - 1);
+        s.tab[e].y |= m << 16;
+    }
+    // Per (warp, expert): ~slot when all the warp's occurrences of e share one
+    // replica, else the warp's first occurrence index of e.
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = __ldg(rank_off + (int64_t)r * E + e);
+        for (int q = 0; q < c; ++q) run += cluster.map_shared_rank(s.tot, q)[e];
+        const int2 t = s.tab[e];
+        const int n = t.y & 0xffff;
+        for (int w = 0; w < kRerouteWarps; ++w) {
+            const int cnt = s.hist[w * E + e];
+            int v = ~s.rc[t.x].y;                       // home slot: the only replica
+            if (n > 1) {
+                int k = n - 1;
+                while (k > 0 && s.rc[t.x + k].x > run) --k;
+                const bool uniform = k == n - 1 || run + cnt <= s.rc[t.x + k + 1].x;
+                v = uniform ? ~s.rc[t.x + k].y : run;
+            }
+            s.hist[w * E + e] = v;
+            run += cnt;
+        }
+    }
+    cluster_arrive();          // done reading peers; they may exit once all have arrived
+    const int nb = M > 1 ? 32 - __clz(M - 1) : 0;   // bits of the compact index
     __syncthreads();
 
-    // Pass 2: stable occurrence index and replica lookup.
+    // Pass 2: replica of every (t, k).
     for (int64_t x0 = wlo; x0 < whi; x0 += 32 * kUnroll) {
-        int key[kUnroll];
+        int id[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             const int64_t i = x0 + u * 32 + lane;
-            const int id = i < whi ? __ldg(ids + i) : -1;
-            key[u] = (unsigned)id < (unsigned)E ? id : -1;
+            id[u] = i < whi ? __ldg(ids + i) : -1;
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             const int64_t i = x0 + u * 32 + lane;
-            const int k = key[u];
-            const unsigned m = __match_any_sync(0xffffffffu, k);
-            const int before = __popc(m & lanemask_lt());
-            int out = -1;
-            int j = 0;
-            if (k >= 0) {
-                j = h[k] + before;
-                const int off = min(s.roff[k], cap - 1);
-                int i_rep = clampi(s.roff[k + 1] - off, 1, cap - off) - 1;
-                while (i_rep > 0 && s.rcum[off + i_rep] > j) --i_rep;
-                out = s.rslot[off + i_rep];
+            const bool valid = (unsigned)id[u] < (unsigned)E;
+            const int v = valid ? h[id[u]] : -1;
+            int out = ~v;                                  // uniform replica (or -1 for a bad id)
+            const bool rank_it = valid && v >= 0;
+            if (__any_sync(0xffffffffu, rank_it)) {
+                const int2 t = rank_it ? s.tab[id[u]] : make_int2(0, 0);
+                const int key = rank_it ? (t.y >> 16) : -1;
+                const unsigned m = match_key(key, nb);
+                const int before = __popc(m & lanemask_lt());
+                if (rank_it) {
+                    const int j = v + before;
+                    int k = (t.y & 0xffff) - 1;
+                    while (k > 0 && s.rc[t.x + k].x > j) --k;
+                    out = s.rc[t.x + k].y;
+                }
+                __syncwarp();
+                if (rank_it && before == 0) h[id[u]] = v + __popc(m);
+                __syncwarp();
             }
-            __syncwarp();
-            if (k >= 0 && before == 0) h[k] += __popc(m);
-            __syncwarp();
             if (i < whi) phys[i] = out;
         }
     }
@@ -157,29 +197,14 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
 
 }  // namespace
 
-size_t reroute_smem_bytes(const Shape &sh)
-{
-    const int cap = sh.E + sh.NR;
-    return (size_t)(kRerouteWarps * sh.E + sh.E + sh.E + 1 + 2 * cap) * sizeof(int32_t);
-}
+size_t reroute_smem_bytes(const Shape &sh) { return reroute_smem_words(sh.E, sh.E + sh.NR) * sizeof(int32_t); }
 
 cudaError_t launch_reroute(const Shape &sh, const Launch &ln, const int32_t *ids, const PlanDev &plan,
-                           int32_t *phys, cudaStream_t st)
+                           int32_t *phys, cudaStream_t st, bool pdl)
 {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(sh.N * ln.cluster));
-    cfg.blockDim = dim3(kRerouteWarps * 32);
-    cfg.dynamicSmemBytes = reroute_smem_bytes(sh);
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)ln.cluster;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_reroute, ids, sh.per_rank, sh.E, sh.E + sh.NR, plan.rep_off,
-                              plan.rep_slot, plan.rep_cum, plan.rank_off, phys);
+    return launch_ex(k_reroute, (unsigned)(sh.N * ln.cluster), kRerouteWarps * 32, reroute_smem_bytes(sh), st,
+                     (unsigned)ln.cluster, pdl, ids, sh.per_rank, sh.E, sh.E + sh.NR, plan.rep_off, plan.rep_slot,
+                     plan.rep_cum, plan.rep_experts, plan.info, plan.rank_off, phys);
 }
 
 cudaError_t set_reroute_attributes(size_t max_smem)
