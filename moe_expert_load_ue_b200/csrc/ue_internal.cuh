@@ -94,6 +94,18 @@ cudaError_t launch_ex(void (*kernel)(KArgs...), unsigned grid, unsigned block, s
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// Opt a kernel into `max_smem` bytes of shared memory per block in total
+// (dynamic plus the kernel's static shared memory).
+template <typename... KArgs>
+cudaError_t allow_smem(void (*kernel)(KArgs...), size_t max_smem)
+{
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+    if (e != cudaSuccess) return e;
+    const size_t dyn = max_smem > fa.sharedSizeBytes ? max_smem - fa.sharedSizeBytes : 0;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+}
+
 // ---- device helpers ---------------------------------------------------------
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }

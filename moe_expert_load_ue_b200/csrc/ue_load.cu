@@ -49,10 +49,6 @@ k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
     const int r = blockIdx.x / C;
     const int lane = lane_id(), warp = threadIdx.x >> 5;
 
-    for (int i = threadIdx.x; i < kCopies * E; i += blockDim.x) hist[i] = 0;
-    if (threadIdx.x == 0) *sbad = 0;
-    __syncthreads();
-
     // This CTA's share [lo, hi) of rank r's flat id range, 32-id aligned shares.
     const int64_t share = ((per_rank + C - 1) / C + 31) / 32 * 32;
     const int64_t base = (int64_t)r * per_rank;
@@ -61,6 +57,20 @@ k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
     // int4 body [vlo, vhi) on 16-byte boundaries (ids is 16-byte aligned).
     const int64_t vlo = min(hi, (lo + 3) / 4 * 4);
     const int64_t vhi = max(vlo, hi / 4 * 4);
+    const int4 *vec = reinterpret_cast<const int4 *>(ids + vlo);
+    const int64_t nvec = (vhi - vlo) / 4;
+    const int64_t stride = (int64_t)blockDim.x;
+    // The first four vectors of every thread are in flight while the
+    // histograms are cleared.
+    int4 q0[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int64_t v = threadIdx.x + k * stride;
+        q0[k] = v < nvec ? __ldg(vec + v) : make_int4(-1, -1, -1, -1);
+    }
+    for (int i = threadIdx.x; i < kCopies * E; i += blockDim.x) hist[i] = 0;
+    if (threadIdx.x == 0) *sbad = 0;
+    __syncthreads();
     int32_t *h = hist + (warp % kCopies) * E;
     int nbad = 0;
 
@@ -71,17 +81,26 @@ k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
         else if (lane >= 4 && lane - 4 < hi - vhi) i = vhi + (lane - 4);
         if (i >= 0) count_id(h, __ldg(ids + i), E, nbad);
     }
-    // Body: every thread walks int4 vectors, two in flight.
-    const int4 *vec = reinterpret_cast<const int4 *>(ids + vlo);
-    const int64_t nvec = (vhi - vlo) / 4;
-    const int64_t stride = (int64_t)blockDim.x;
-    int64_t v = threadIdx.x;
-    for (; v + stride < nvec; v += 2 * stride) {
-        const int4 a = __ldg(vec + v), b = __ldg(vec + v + stride);
-        count_id(h, a.x, E, nbad); count_id(h, a.y, E, nbad); count_id(h, a.z, E, nbad); count_id(h, a.w, E, nbad);
-        count_id(h, b.x, E, nbad); count_id(h, b.y, E, nbad); count_id(h, b.z, E, nbad); count_id(h, b.w, E, nbad);
+    // Body: every thread walks int4 vectors, four in flight.
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        if (threadIdx.x + k * stride < nvec) {
+            count_id(h, q0[k].x, E, nbad); count_id(h, q0[k].y, E, nbad);
+            count_id(h, q0[k].z, E, nbad); count_id(h, q0[k].w, E, nbad);
+        }
     }
-    if (v < nvec) {
+    int64_t v = threadIdx.x + 4 * stride;
+    for (; v + 3 * stride < nvec; v += 4 * stride) {
+        int4 q[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) q[k] = __ldg(vec + v + k * stride);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            count_id(h, q[k].x, E, nbad); count_id(h, q[k].y, E, nbad);
+            count_id(h, q[k].z, E, nbad); count_id(h, q[k].w, E, nbad);
+        }
+    }
+    for (; v < nvec; v += stride) {
         const int4 a = __ldg(vec + v);
         count_id(h, a.x, E, nbad); count_id(h, a.y, E, nbad); count_id(h, a.z, E, nbad); count_id(h, a.w, E, nbad);
     }
@@ -99,8 +118,12 @@ k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
     const int cols = (E + C - 1) / C;
     const int e0 = c * cols, e1 = min(E, e0 + cols);
     for (int e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
+        int part[kMaxCluster];
+#pragma unroll
+        for (int q = 0; q < kMaxCluster; ++q) part[q] = q < C ? cluster.map_shared_rank(tot, q)[e] : 0;
         int s = 0;
-        for (int q = 0; q < C; ++q) s += cluster.map_shared_rank(tot, q)[e];
+#pragma unroll
+        for (int q = 0; q < kMaxCluster; ++q) s += part[q];
         counts[(int64_t)r * E + e] = s;
     }
     if (bad != nullptr && c == 0 && threadIdx.x == 0) {
@@ -124,7 +147,7 @@ cudaError_t launch_load(const Shape &sh, const Launch &ln, const int32_t *ids, i
 
 cudaError_t set_load_attributes(size_t max_smem)
 {
-    return cudaFuncSetAttribute(k_load, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)max_smem);
+    return allow_smem(k_load, max_smem);
 }
 
 }  // namespace ue

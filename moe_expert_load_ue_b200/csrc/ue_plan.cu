@@ -13,12 +13,13 @@
 //   Replica list of e: home slot, then redundant slots in allocation order;
 //   rep_cum = exclusive prefix of their quotas.
 //
-// Design (sm_100a): one thread-block cluster of up to 8 CTAs x 1024 threads.
-//   Peer CTAs (cluster rank >= 1) own 32-expert column groups of counts: they
-//     sum their columns (loads) and arrive on the cluster barrier, then - off
-//     the critical path, while CTA 0 plans - write the exclusive column scan
-//     over ranks, rank_off[r][e], that the reroute kernel needs.
-//   CTA 0 pulls the loads over DSMEM and plans:
+// Design (sm_100a): one thread-block cluster of up to 8 CTAs.  Every CTA sums
+//   a slice of the rank rows of counts into a partial load vector in shared
+//   memory and arrives on the cluster barrier.  CTA 0 adds the partial vectors
+//   over DSMEM (the loads) and plans; meanwhile - off the critical path - the
+//   other CTAs write the exclusive scan over ranks of their row slices,
+//   rank_off[r][e], that the reroute kernel needs (the partial vectors of the
+//   earlier slices give each slice its starting offsets).  CTA 0 plans:
 //     * home pass in closed form from a block-wide prefix sum: the home rank's
 //       load before e is min(Q, in-rank prefix), so
 //       take = min(Q, prefix + load) - min(Q, prefix);
@@ -46,8 +47,7 @@ namespace cg = cooperative_groups;
 namespace ue {
 namespace {
 
-constexpr int kPlanThreads = 1024;
-constexpr int kPlanWarps = kPlanThreads / 32;
+constexpr int kPlanMaxThreads = 1024;
 
 // Shared-memory layout of a planner CTA (all 4-byte words unless noted).
 struct PlanSmem {
@@ -108,10 +108,11 @@ __device__ __forceinline__ PlanSmem carve(int32_t *p, int E, int N, int NR)
     return s;
 }
 
-// Block-wide exclusive prefix sum of one value per thread (all 1024 threads call it).
+// Block-wide exclusive prefix sum of one value per thread (every thread of the
+// block calls it; blockDim.x is a multiple of 32).
 __device__ int block_excl_scan(int v, int32_t *ws, int *total)
 {
-    const int lane = lane_id(), warp = threadIdx.x >> 5;
+    const int lane = lane_id(), warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     int x = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -121,7 +122,7 @@ __device__ int block_excl_scan(int v, int32_t *ws, int *total)
     if (lane == 31) ws[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        int w = ws[lane];
+        int w = lane < nw ? ws[lane] : 0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, w, o);
@@ -131,63 +132,52 @@ __device__ int block_excl_scan(int v, int32_t *ws, int *total)
     }
     __syncthreads();
     const int r = (warp ? ws[32 + warp - 1] : 0) + x - v;
-    *total = ws[32 + kPlanWarps - 1];
+    *total = ws[32 + nw - 1];
     __syncthreads();
     return r;
 }
 
-// Sum of counts[r][g*32 + lane] over this thread's rows [r0, r1).
-__device__ __forceinline__ int column_part(const int32_t *__restrict__ counts, int E, int g, int r0, int r1)
-{
-    const int e = g * 32 + lane_id();
-    int sum = 0;
-    if (e < E)
-        for (int r = r0; r < r1; ++r) sum += __ldg(counts + (int64_t)r * E + e);
-    return sum;
-}
+constexpr int kRowBatch = 8;   // rows of counts loaded per batch (all loads in flight together)
 
-// Column totals of group g from part[row group][column]; writes sload and the plan's load.
-__device__ __forceinline__ void column_totals(int E, int g, const int32_t *part, int32_t *sload, int32_t *load_out)
+// Row slice [r0, r1) of counts summed per expert into part[e].
+__device__ __forceinline__ void slice_sums(const int32_t *__restrict__ counts, int E, int r0, int r1, int32_t *part)
 {
-    const int tid = threadIdx.x;
-    if (tid < 32) {
-        const int e = g * 32 + tid;
-        int t = 0;
-#pragma unroll 8
-        for (int w = 0; w < 32; ++w) t += part[w * 33 + tid];
-        if (e < E) {
-            sload[e] = t;
-            load_out[e] = t;
-        }
-    }
-}
-
-// Exclusive scan of column group g over the row groups (part[row group][column]),
-// then rank_off[r][e] for this thread's rows [r0, r1).
-__device__ void column_rank_off(const int32_t *__restrict__ counts, int E, int g, int r0, int r1, int32_t *part,
-                                int32_t *rank_off)
-{
-    const int lane = lane_id(), warp = threadIdx.x >> 5;
-    __syncthreads();   // column_totals has read part
-    {   // warp w scans column w of the group over the row groups (lane = row group)
-        const int v = part[lane * 33 + warp];
-        int x = v;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int acc = 0;
+        for (int rb = r0; rb < r1; rb += kRowBatch) {
+            int v[kRowBatch];
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
+            for (int k = 0; k < kRowBatch; ++k) v[k] = rb + k < r1 ? __ldg(counts + (int64_t)(rb + k) * E + e) : 0;
+#pragma unroll
+            for (int k = 0; k < kRowBatch; ++k) acc += v[k];
         }
-        part[lane * 33 + warp] = x - v;
+        part[e] = acc;
     }
-    __syncthreads();
-    const int e = g * 32 + lane;
-    int run = part[warp * 33 + lane];
-    if (e < E)
-        for (int r = r0; r < r1; ++r) {
-            rank_off[(int64_t)r * E + e] = run;
-            run += __ldg(counts + (int64_t)r * E + e);
+}
+
+// rank_off[r][e] for the rows [r0, r1), starting from the occurrences in the
+// rows before r0 (the partial vectors of the earlier slices, over DSMEM).
+__device__ void slice_rank_off(cg::cluster_group &cluster, const int32_t *__restrict__ counts, int E, int r0,
+                               int r1, int c, int32_t *part, int32_t *__restrict__ rank_off)
+{
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int prev[kMaxCluster];
+#pragma unroll
+        for (int q = 0; q < kMaxCluster; ++q) prev[q] = q < c ? cluster.map_shared_rank(part, q)[e] : 0;
+        int run = 0;
+#pragma unroll
+        for (int q = 0; q < kMaxCluster; ++q) run += prev[q];
+        for (int rb = r0; rb < r1; rb += kRowBatch) {
+            int v[kRowBatch];
+#pragma unroll
+            for (int k = 0; k < kRowBatch; ++k) v[k] = rb + k < r1 ? __ldg(counts + (int64_t)(rb + k) * E + e) : 0;
+#pragma unroll
+            for (int k = 0; k < kRowBatch; ++k) {
+                if (rb + k < r1) rank_off[(int64_t)(rb + k) * E + e] = run;
+                run += v[k];
+            }
         }
-    __syncthreads();
+    }
 }
 
 // R > 1: the chunk-by-chunk greedy, run by warp 0.
@@ -277,50 +267,55 @@ __device__ void greedy_chunks(const PlanSmem &s, int N, int R, int M1)
     }
 }
 
-// R = 1: walk the eligible ranks in sorted order (s.rsorted, exclusive prefix
-// s.rsum, K of them); run by warp 0.  Assignment a is sorted position a.
+// R = 1: walk the eligible ranks in sorted order (exclusive spare prefix
+// s.rsum over K ranks); run by warp 0.  Expert m of the overflow order takes
+// the sorted positions [cut[m], cut[m+1]) (recorded in s.afirst / s.acnt);
+// assignment a is sorted position a, filled in by the whole block afterwards.
+// The prefix values are held in registers, a window of 32 at a time, so each
+// expert costs one compare, one ballot and one shuffle.
 __device__ void greedy_sorted(const PlanSmem &s, int K, int M1)
 {
     const int lane = lane_id();
     int p = 0, stop_pos = M1, stop_rem = 0;
-    for (int m = 0; m < M1; ++m) {
-        const int e = s.order[m];
-        const int rem = s.ovf[e];
-        const long long target = (long long)s.rsum[p] + rem;   // smallest q > p with rsum[q] >= target
-        int q = -1;
-        for (int base = p + 1; base <= K; base += 32) {
-            const int cand = base + lane;
-            const bool hit = cand <= K && (long long)s.rsum[cand] >= target;
-            const unsigned b = __ballot_sync(0xffffffffu, hit);
-            if (b) {
-                q = base + __ffs(b) - 1;
+    int rsum_p = 0;                                   // s.rsum[p]
+    int wbase = 1;                                    // window: lane holds s.rsum[wbase + lane]
+    int wv = wbase + lane <= K ? s.rsum[wbase + lane] : INT_MAX;
+    for (int m0 = 0; m0 < M1 && stop_pos == M1; m0 += 32) {
+        const int idx = m0 + lane;
+        const int e_l = idx < M1 ? s.order[idx] : 0;
+        const int o_l = idx < M1 ? s.ovf[e_l] : 0;
+        const int cnt = min(32, M1 - m0);
+        for (int j = 0; j < cnt; ++j) {
+            const int e = __shfl_sync(0xffffffffu, e_l, j);
+            const int rem = __shfl_sync(0xffffffffu, o_l, j);
+            const long long target = (long long)rsum_p + rem;   // smallest q > p with rsum[q] >= target
+            int q = -1, rsum_q = 0;
+            while (wbase <= K) {
+                const bool cand = wbase + lane > p && wbase + lane <= K;
+                const unsigned b = __ballot_sync(0xffffffffu, cand && (long long)wv >= target);
+                if (b) {
+                    const int src = __ffs(b) - 1;
+                    q = wbase + src;
+                    rsum_q = __shfl_sync(0xffffffffu, wv, src);
+                    break;
+                }
+                wbase += 32;                          // the whole window is below the target
+                wv = wbase + lane <= K ? s.rsum[wbase + lane] : INT_MAX;
+            }
+            if (lane == 0) {
+                s.afirst[e] = p;
+                s.acnt[e] = (q < 0 ? K : q) - p;
+            }
+            if (q < 0) {                              // every remaining rank used: the rest stays home
+                stop_pos = m0 + j;
+                stop_rem = rem - (s.rsum[K] - rsum_p);
+                p = K;
                 break;
             }
+            p = q;
+            rsum_p = rsum_q;
         }
-        const int end = q < 0 ? K : q;            // ranks [p, end) go to e
-        for (int a = p + lane; a < end; a += 32) {
-            const int r = s.rsorted[a];
-            const int full = s.rsum[a + 1] - s.rsum[a];
-            s.ar[a] = r;
-            s.au[a] = 0;
-            s.ac[a] = (q >= 0 && a == end - 1) ? rem - (s.rsum[a] - s.rsum[p]) : full;
-            s.ae[a] = e;
-            s.sasg[r] = a;
-        }
-        if (lane == 0) {
-            s.afirst[e] = p;
-            s.acnt[e] = end - p;
-        }
-        if (q < 0) {                              // every remaining rank used: the rest stays home
-            stop_pos = m;
-            stop_rem = rem - (s.rsum[K] - s.rsum[p]);
-            p = K;
-            break;
-        }
-        p = q;
     }
-    __syncwarp();
-    for (int a = lane; a < p; a += 32) s.spare[s.ar[a]] -= s.ac[a];
     if (lane == 0) {
         s.misc[0] = p;
         s.misc[1] = stop_pos;
@@ -329,7 +324,7 @@ __device__ void greedy_sorted(const PlanSmem &s, int K, int M1)
 }
 
 template <int NRL>
-__global__ void __launch_bounds__(kPlanThreads, 1)
+__global__ void __launch_bounds__(kPlanMaxThreads, 1)
 k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
 {
     extern __shared__ __align__(16) int32_t sm_plan[];
@@ -339,57 +334,48 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
     cg::cluster_group cluster = cg::this_cluster();
     const int C = (int)cluster.num_blocks();
     const int c = (int)cluster.block_rank();
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int groups = (E + 31) / 32;
-    const int rpg = (N + 31) / 32;                 // ranks per row group
-    const int r0 = min(N, warp * rpg), r1 = min(N, r0 + rpg);
+    const int tid = threadIdx.x, nt = blockDim.x, warp = tid >> 5;
+    // This CTA's slice of the rank rows of counts.
+    const int rows = (N + C - 1) / C;
+    const int r0 = min(N, c * rows), r1 = min(N, r0 + rows);
 
     // The reroute grid may launch now (its first pass needs only the ids);
     // the counts of the load grid are read after it completes.
     pdl_trigger();
     pdl_wait();
 
-    if (C > 1 && c != 0) {
-        // Peer: loads of the own column groups, then (off the critical path) rank_off.
-        for (int g = c - 1; g < groups; g += C - 1) {
-            s.part[warp * 33 + lane_id()] = column_part(counts, E, g, r0, r1);
-            __syncthreads();
-            column_totals(E, g, s.part, s.sload, plan.load);
-            __syncthreads();
-        }
-        cluster_arrive();      // #1: loads ready for CTA 0
-        for (int g = c - 1; g < groups; g += C - 1) {
-            s.part[warp * 33 + lane_id()] = column_part(counts, E, g, r0, r1);
-            __syncthreads();
-            column_rank_off(counts, E, g, r0, r1, s.part, plan.rank_off);
-        }
-        cluster_wait();
-        cluster_arrive();      // #2: completes once CTA 0 has pulled the loads
+    slice_sums(counts, E, r0, r1, s.sload);
+    cluster_arrive();          // #1: this slice's partial loads are ready
+    cluster_wait();
+    if (c != 0) {
+        // Off the critical path: rank_off for this slice, then stay resident
+        // until every CTA has read the partial vectors.
+        slice_rank_off(cluster, counts, E, r0, r1, c, s.sload, plan.rank_off);
+        cluster_arrive();      // #2
         cluster_wait();
         return;
     }
-    if (C == 1) {
-        for (int g = 0; g < groups; ++g) {
-            s.part[warp * 33 + lane_id()] = column_part(counts, E, g, r0, r1);
-            __syncthreads();
-            column_totals(E, g, s.part, s.sload, plan.load);
-            column_rank_off(counts, E, g, r0, r1, s.part, plan.rank_off);
-        }
-    }
-    cluster_arrive();
-    cluster_wait();
     const int e = tid;
     const bool ve = e < E;
-    const int ld = !ve ? 0 : (C == 1 ? s.sload[e] : cluster.map_shared_rank(s.sload, 1 + (e >> 5) % (C - 1))[e]);
-    cluster_arrive();          // #2; the matching wait is at the end of the kernel
+    int ld = 0;
+    if (ve) {
+        int part[kMaxCluster];
+#pragma unroll
+        for (int q = 1; q < kMaxCluster; ++q) part[q] = q < C ? cluster.map_shared_rank(s.sload, q)[e] : 0;
+        ld = s.sload[e];
+#pragma unroll
+        for (int q = 1; q < kMaxCluster; ++q) ld += part[q];
+        plan.load[e] = ld;
+    }
+    cluster_arrive();          // #2: done reading the peers (they still read this CTA's slice)
 
-    // ---- the plan ---------------------------------------------------------------
+    // ---- the plan (CTA 0; blockDim >= max(E, N)) ---------------------------------
     int L;
     const int pre = block_excl_scan(ld, s.ws, &L);
     const int Q = L == 0 ? 0 : (L - 1) / N + 1;
     if (ve) s.pre[e] = pre;
-    for (int r = tid; r < N; r += kPlanThreads) s.extra[r] = 0;
-    for (int i = tid; i < NR; i += kPlanThreads) s.sasg[i] = -1;
+    for (int r = tid; r < N; r += nt) s.extra[r] = 0;
+    for (int i = tid; i < NR; i += nt) s.sasg[i] = -1;
     __syncthreads();
 
     // Home pass in closed form.
@@ -450,6 +436,27 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
         if (tid == 0) s.rsum[K] = tot;
         __syncthreads();
         if (warp == 0) greedy_sorted(s, K, M1);
+        __syncthreads();
+        // Fill the assignments: expert m of the overflow order owns the sorted
+        // positions of its cut; every rank is full except the last rank of an
+        // expert that was placed completely (m before the stop), which takes
+        // what is left of the expert's overflow.
+        if (tid < M1) {
+            const int em = s.order[tid];
+            const int a0 = s.afirst[em], na = s.acnt[em];
+            const bool placed = tid < s.misc[1];
+            for (int a = a0; a < a0 + na; ++a) {
+                const int r = s.rsorted[a];
+                int q = s.rsum[a + 1] - s.rsum[a];
+                if (placed && a == a0 + na - 1) q = s.ovf[em] - (s.rsum[a] - s.rsum[a0]);
+                s.ar[a] = r;
+                s.au[a] = 0;
+                s.ac[a] = q;
+                s.ae[a] = em;
+                s.sasg[r] = a;
+                s.spare[r] -= q;
+            }
+        }
     } else if (warp == 0) {
         greedy_chunks<NRL>(s, N, R, M1);
     }
@@ -458,7 +465,7 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
     const int flags = stop_pos < M1 ? 1 : 0;
     // Slots ran out at overflow position stop_pos: that expert's remainder and
     // the whole overflow of every later expert stay on their home slots.
-    for (int p = stop_pos + tid; p < M1; p += kPlanThreads) {
+    for (int p = stop_pos + tid; p < M1; p += nt) {
         const int ep = s.order[p];
         const int res = p == stop_pos ? stop_rem : s.ovf[ep];
         s.qh[ep] += res;
@@ -494,14 +501,14 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
         if (na_e > 0) plan.rep_experts[mpos] = e;
     }
     if (tid == 0) plan.rep_off[E] = tot_rep;
-    for (int p = tot_rep + tid; p < cap; p += kPlanThreads) {
+    for (int p = tot_rep + tid; p < cap; p += nt) {
         plan.rep_slot[p] = -1;
         plan.rep_cum[p] = -1;
     }
-    for (int p = M + tid; p < E; p += kPlanThreads) plan.rep_experts[p] = -1;
+    for (int p = M + tid; p < E; p += nt) plan.rep_experts[p] = -1;
 
     // Slot table.
-    for (int sl = tid; sl < S; sl += kPlanThreads) {
+    for (int sl = tid; sl < S; sl += nt) {
         const int r = sl / HR, u = sl % HR;
         int se, sq;
         if (u < H) {
@@ -518,7 +525,7 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
 
     // Rank loads before / after and their maxima.
     int mb = 0, ma = 0;
-    for (int r = tid; r < N; r += kPlanThreads) {
+    for (int r = tid; r < N; r += nt) {
         const int after = Q - s.spare[r] + s.extra[r];
         plan.rank_load_before[r] = s.before[r];
         plan.rank_load_after[r] = after;
@@ -532,20 +539,24 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
         s.ws[32 + warp] = ma;
     }
     __syncthreads();
-    if (tid == 0) {
-        for (int w = 1; w < kPlanWarps; ++w) {
-            mb = max(mb, s.ws[w]);
-            ma = max(ma, s.ws[32 + w]);
+    if (warp == 0) {
+        const int nw = nt >> 5;
+        mb = __reduce_max_sync(0xffffffffu, lane_id() < nw ? s.ws[lane_id()] : 0);
+        ma = __reduce_max_sync(0xffffffffu, lane_id() < nw ? s.ws[32 + lane_id()] : 0);
+        if (tid == 0) {
+            plan.info[0] = Q;
+            plan.info[1] = L;
+            plan.info[2] = flags;
+            plan.info[3] = M;
+            plan.info[4] = n_asg;
+            plan.info[5] = mb;
+            plan.info[6] = ma;
+            plan.info[7] = 0;
         }
-        plan.info[0] = Q;
-        plan.info[1] = L;
-        plan.info[2] = flags;
-        plan.info[3] = M;
-        plan.info[4] = n_asg;
-        plan.info[5] = mb;
-        plan.info[6] = ma;
-        plan.info[7] = 0;
     }
+    // rank_off of CTA 0's own slice (it starts at zero); stay resident until
+    // the peers have read this CTA's partial loads.
+    slice_rank_off(cluster, counts, E, r0, r1, 0, s.sload, plan.rank_off);
     cluster_wait();
 }
 
@@ -553,19 +564,34 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
 
 size_t plan_smem_bytes(const Shape &sh) { return plan_smem_words(sh.E, sh.N, sh.NR) * sizeof(int32_t); }
 
+// Threads of a planner CTA: one per expert and one per rank at least; more
+// when counts is large so that each thread sums at most ~8 values per slice.
+int plan_threads(const Shape &sh)
+{
+    int t = sh.E > sh.N ? sh.E : sh.N;
+    t = (t + 31) / 32 * 32;
+    if (t < 64) t = 64;
+    const int64_t cells = (int64_t)sh.N * sh.E;
+    while (t < kPlanMaxThreads && cells > (int64_t)8 * kMaxCluster * t) t *= 2;
+    return t < kPlanMaxThreads ? t : kPlanMaxThreads;
+}
+
+// CTAs of the planner cluster: enough row slices that each thread sums at most ~8 rows.
 int plan_cluster(const Shape &sh)
 {
-    const int groups = (sh.E + 31) / 32;
-    if (groups <= 1) return 1;
-    return groups + 1 < kMaxCluster ? groups + 1 : kMaxCluster;   // CTA 0 plans, peers own column groups
+    const int64_t per_cta = (int64_t)8 * plan_threads(sh);
+    int C = 1;
+    while (C < kMaxCluster && (int64_t)sh.N * sh.E > per_cta * C) C *= 2;
+    return C < sh.N ? C : (sh.N < 1 ? 1 : sh.N);
 }
 
 cudaError_t launch_plan(const Shape &sh, const int32_t *counts, const PlanDev &plan, cudaStream_t st, bool pdl)
 {
     const unsigned C = (unsigned)plan_cluster(sh);
+    const unsigned threads = (unsigned)plan_threads(sh);
     const int nrl = (sh.N + 31) / 32;
     const size_t smem = plan_smem_bytes(sh);
-#define UE_PLAN_LAUNCH(V) launch_ex(k_plan<V>, C, kPlanThreads, smem, st, C, pdl, counts, sh.E, sh.N, sh.R, plan)
+#define UE_PLAN_LAUNCH(V) launch_ex(k_plan<V>, C, threads, smem, st, C, pdl, counts, sh.E, sh.N, sh.R, plan)
     if (nrl <= 1) return UE_PLAN_LAUNCH(1);
     if (nrl <= 2) return UE_PLAN_LAUNCH(2);
     if (nrl <= 4) return UE_PLAN_LAUNCH(4);
@@ -577,14 +603,12 @@ cudaError_t launch_plan(const Shape &sh, const int32_t *counts, const PlanDev &p
 
 cudaError_t set_plan_attributes(size_t max_smem)
 {
-    const int m = (int)max_smem;
-    const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
-    cudaError_t e = cudaFuncSetAttribute(k_plan<1>, a, m);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_plan<2>, a, m);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_plan<4>, a, m);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_plan<8>, a, m);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_plan<16>, a, m);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_plan<32>, a, m);
+    cudaError_t e = allow_smem(k_plan<1>, max_smem);
+    if (e == cudaSuccess) e = allow_smem(k_plan<2>, max_smem);
+    if (e == cudaSuccess) e = allow_smem(k_plan<4>, max_smem);
+    if (e == cudaSuccess) e = allow_smem(k_plan<8>, max_smem);
+    if (e == cudaSuccess) e = allow_smem(k_plan<16>, max_smem);
+    if (e == cudaSuccess) e = allow_smem(k_plan<32>, max_smem);
     return e;
 }
 

@@ -16,11 +16,11 @@
 // griddepcontrol.wait: launched with programmatic dependent launch, it
 // overlaps the planner.  From the counts and the bases each warp then knows,
 // per expert, whether all its occurrences fall into one replica's quota range
-// ("uniform": every expert with one replica, and almost every (warp, expert)
-// pair of a replicated one).  Pass 2 is then one shared-memory lookup per id;
-// only ids of an expert whose quota boundary falls inside the warp's part are
-// ranked exactly, by ballots over the bits of the expert's compact index in
-// plan.rep_experts.
+// ("uniform": almost every (warp, expert) pair of a replicated expert; an
+// expert with one replica always is).  Pass 2 is then one or two shared-memory
+// lookups per id; only ids of an expert whose quota boundary falls inside the
+// warp's part are ranked exactly, by ballots over the bits of the expert's
+// compact index in plan.rep_experts.
 #include <cooperative_groups.h>
 
 #include "ue_internal.cuh"
@@ -34,23 +34,29 @@ constexpr int kRerouteWarps = 16;
 constexpr int kUnroll = 4;
 
 struct RerouteSmem {
-    int32_t *hist;   // [W][E] per-warp counts; then ~slot (uniform) or running occurrence index
+    int32_t *hist;   // [W][E] per-warp counts, then their exclusive scan over the warps
+    int32_t *code;   // [W][M] per warp and replicated expert: ~slot (uniform) or running occurrence index
     int32_t *tot;    // [E]    this CTA's counts (read by later CTAs of the cluster)
-    int2 *tab;       // [E]    {first replica entry, (compact index << 16) | replica count}
+    int32_t *base;   // [E]    occurrences of e before this CTA's ids
+    int32_t *rexp;   // [E]    replicated experts (plan.rep_experts)
+    int2 *tab;       // [E]    {home slot if one replica, else first replica entry; (compact index << 16) | count}
     int2 *rc;        // [cap]  {cumulative quota, slot} of each replica entry
 };
 
 __host__ __device__ inline size_t reroute_smem_words(int E, int cap)
 {
-    return (size_t)kRerouteWarps * E + E + 2 * (size_t)E + 2 * (size_t)cap + 4;
+    return (size_t)2 * kRerouteWarps * E + 3 * (size_t)E + 2 * (size_t)E + 2 * (size_t)cap + 4;
 }
 
 __device__ __forceinline__ RerouteSmem carve(int32_t *base, int E)
 {
     RerouteSmem s;
     s.hist = base;
-    s.tot = s.hist + kRerouteWarps * E;
-    int32_t *p = s.tot + E;
+    s.code = s.hist + kRerouteWarps * E;
+    s.tot = s.code + kRerouteWarps * E;
+    s.base = s.tot + E;
+    s.rexp = s.base + E;
+    int32_t *p = s.rexp + E;
     p += (reinterpret_cast<uintptr_t>(p) & 7) ? 1 : 0;   // 8-byte alignment for int2
     s.tab = reinterpret_cast<int2 *>(p);
     s.rc = s.tab + E;
@@ -113,49 +119,65 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
             if ((unsigned)id[u] < (unsigned)E) atomicAdd(h + id[u], 1);
     }
     __syncthreads();
+    // Exclusive scan over the warps per expert (in place) and CTA totals.
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int t = 0;
+        int run = 0;
 #pragma unroll
-        for (int w = 0; w < kRerouteWarps; ++w) t += s.hist[w * E + e];
-        s.tot[e] = t;
+        for (int w = 0; w < kRerouteWarps; ++w) {
+            const int t = s.hist[w * E + e];
+            s.hist[w * E + e] = run;
+            run += t;
+        }
+        s.tot[e] = run;
     }
     cluster.sync();
 
-    // The plan (and rank_off) of the preceding planner grid.
+    // The plan (and rank_off) of the preceding planner grid: every global load
+    // of the plan is issued in one round.
     pdl_wait();
+    const int M = clampi(__ldg(info + 3), 0, E);
     for (int i = threadIdx.x; i < cap; i += blockDim.x) s.rc[i] = make_int2(__ldg(rep_cum + i), __ldg(rep_slot + i));
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        const int off = clampi(__ldg(rep_off + e), 0, cap - 1);
-        const int n = clampi(__ldg(rep_off + e + 1) - off, 1, min(cap - off, 0xffff));
+        const int o0 = __ldg(rep_off + e), o1 = __ldg(rep_off + e + 1);
+        int b = __ldg(rank_off + (int64_t)r * E + e);
+        int peer[kMaxCluster];
+#pragma unroll
+        for (int q = 0; q < kMaxCluster; ++q) peer[q] = q < c ? cluster.map_shared_rank(s.tot, q)[e] : 0;
+        const int off = clampi(o0, 0, cap - 1);
+        const int n = clampi(o1 - off, 1, min(cap - off, 0xffff));
         s.tab[e] = make_int2(off, n);
+#pragma unroll
+        for (int q = 0; q < kMaxCluster; ++q) b += peer[q];
+        s.base[e] = b;            // occurrences of e before this CTA's ids
     }
-    const int M = clampi(__ldg(info + 3), 0, E);
+    for (int m = threadIdx.x; m < M; m += blockDim.x) s.rexp[m] = clampi(__ldg(rep_experts + m), 0, E - 1);
+    cluster_arrive();          // done reading peers; they may exit once all have arrived
     __syncthreads();
-    for (int m = threadIdx.x; m < M; m += blockDim.x) {
-        const int e = clampi(__ldg(rep_experts + m), 0, E - 1);
-        s.tab[e].y |= m << 16;
-    }
-    // Per (warp, expert): ~slot when all the warp's occurrences of e share one
-    // replica, else the warp's first occurrence index of e.
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int run = __ldg(rank_off + (int64_t)r * E + e);
-        for (int q = 0; q < c; ++q) run += cluster.map_shared_rank(s.tot, q)[e];
+    // Replicated experts get their compact index; every other expert's table
+    // entry becomes its home slot (its only replica).
+    for (int m = threadIdx.x; m < M; m += blockDim.x) s.tab[s.rexp[m]].y |= m << 16;
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        if ((s.tab[e].y & 0xffff) == 1) s.tab[e].x = s.rc[s.tab[e].x].y;
+    __syncthreads();
+    // Per (warp, replicated expert): ~slot when all the warp's occurrences of
+    // the expert share one replica, else the warp's first occurrence index.
+    for (int i = threadIdx.x; i < kRerouteWarps * M; i += blockDim.x) {
+        const int w = i / M, m = i - w * M;
+        const int e = s.rexp[m];
         const int2 t = s.tab[e];
         const int n = t.y & 0xffff;
-        for (int w = 0; w < kRerouteWarps; ++w) {
-            const int cnt = s.hist[w * E + e];
-            int v = ~s.rc[t.x].y;                       // home slot: the only replica
-            if (n > 1) {
-                int k = n - 1;
-                while (k > 0 && s.rc[t.x + k].x > run) --k;
-                const bool uniform = k == n - 1 || run + cnt <= s.rc[t.x + k + 1].x;
-                v = uniform ? ~s.rc[t.x + k].y : run;
-            }
-            s.hist[w * E + e] = v;
-            run += cnt;
+        const int excl = s.hist[w * E + e];
+        const int cnt = (w + 1 < kRerouteWarps ? s.hist[(w + 1) * E + e] : s.tot[e]) - excl;
+        const int j0 = s.base[e] + excl;
+        int lo = 0, hi = n - 1;                         // largest k with cum[k] <= j0
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s.rc[t.x + mid].x <= j0) lo = mid;
+            else hi = mid - 1;
         }
+        const bool uniform = lo == n - 1 || j0 + cnt <= s.rc[t.x + lo + 1].x;
+        s.code[w * M + m] = uniform ? ~s.rc[t.x + lo].y : j0;
     }
-    cluster_arrive();          // done reading peers; they may exit once all have arrived
     const int nb = M > 1 ? 32 - __clz(M - 1) : 0;   // bits of the compact index
     __syncthreads();
 
@@ -171,22 +193,26 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
         for (int u = 0; u < kUnroll; ++u) {
             const int64_t i = x0 + u * 32 + lane;
             const bool valid = (unsigned)id[u] < (unsigned)E;
-            const int v = valid ? h[id[u]] : -1;
-            int out = ~v;                                  // uniform replica (or -1 for a bad id)
-            const bool rank_it = valid && v >= 0;
+            const int2 t = valid ? s.tab[id[u]] : make_int2(-1, 1);
+            const int n = t.y & 0xffff, cm = t.y >> 16;
+            int out = t.x;                                 // the home slot (a single replica); -1 for a bad id
+            int v = 0;
+            if (n > 1) {
+                v = s.code[warp * M + cm];
+                out = ~v;                                  // the warp's uniform replica, if v < 0
+            }
+            const bool rank_it = n > 1 && v >= 0;
             if (__any_sync(0xffffffffu, rank_it)) {
-                const int2 t = rank_it ? s.tab[id[u]] : make_int2(0, 0);
-                const int key = rank_it ? (t.y >> 16) : -1;
-                const unsigned m = match_key(key, nb);
+                const unsigned m = match_key(rank_it ? cm : -1, nb);
                 const int before = __popc(m & lanemask_lt());
                 if (rank_it) {
                     const int j = v + before;
-                    int k = (t.y & 0xffff) - 1;
+                    int k = n - 1;
                     while (k > 0 && s.rc[t.x + k].x > j) --k;
                     out = s.rc[t.x + k].y;
                 }
                 __syncwarp();
-                if (rank_it && before == 0) h[id[u]] = v + __popc(m);
+                if (rank_it && before == 0) s.code[warp * M + cm] = v + __popc(m);
                 __syncwarp();
             }
             if (i < whi) phys[i] = out;
@@ -209,7 +235,11 @@ cudaError_t launch_reroute(const Shape &sh, const Launch &ln, const int32_t *ids
 
 cudaError_t set_reroute_attributes(size_t max_smem)
 {
-    return cudaFuncSetAttribute(k_reroute, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)max_smem);
+    cudaError_t e = allow_smem(k_reroute, max_smem);
+    // Enough shared memory for three CTAs per SM, so that the grid runs in one
+    // wave beside the planner (the default split may leave room for one).
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_reroute, cudaFuncAttributePreferredSharedMemoryCarveout, 60);
+    return e;
 }
 
 }  // namespace ue

@@ -189,7 +189,7 @@ cudaError_t launch_sync(const Shape &sh, const Launch &ln, uint8_t *weights, int
 
 cudaError_t set_sync_attributes(size_t max_smem)
 {
-    return cudaFuncSetAttribute(k_sync, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)max_smem);
+    return allow_smem(k_sync, max_smem);
 }
 
 }  // namespace ue
