@@ -37,10 +37,37 @@ from moe_expert_load_ue_b200 import inputs  # noqa: E402
 METRIC = "rebalance µs/layer-microbatch (load+plan+reroute); sync & grad-reduce HBM GB/s"
 UNIT = "µs"
 FALLBACK_HBM_GBS = 6650.0
-# DRAM bytes per launch of the dominant kernel from the committed ncu capture
-# (profiles/), scaled to this workload; None until a capture of the current
-# kernel exists.
-TRAFFIC_BYTES = {}
+# DRAM bytes of one launch from an ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum) next to that launch's algorithmic bytes, per kernel
+# and full-size workload; summarised in profiles/.  The JSON's roofline.traffic
+# scales the measured ratio to the mean launch of the run, and is null when the
+# kernel's source no longer matches the one that was captured.
+TRAFFIC = {
+    ("grad_reduce", "671B-class"): {
+        "source": "moe_expert_load_ue_b200/csrc/ue_grad_reduce.cu",
+        "sha256": "3503a95d76ce7d9ac8808ca3d9a351d3e71755bfeb60fc4a02b0e73bc6855973",
+        "dram_bytes": 7905447680, "algorithmic_bytes": 7927234560,
+        "profile": "profiles/grad_reduce_and_sync_dram_671B-class.md"},
+    ("sync", "671B-class"): {
+        "source": "moe_expert_load_ue_b200/csrc/ue_sync.cu",
+        "sha256": "91512a937a653f349c4cd0560db05baf8b6173feef146d5e1abb6919fb878111",
+        "dram_bytes": 4962545920, "algorithmic_bytes": 5020581888,
+        "profile": "profiles/grad_reduce_and_sync_dram_671B-class.md"},
+}
+
+
+def traffic_per_launch(kernel: str, workload: str, full_size: bool, mean_alg: float):
+    t = TRAFFIC.get((kernel, workload))
+    if t is None or not full_size:
+        return None
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, t["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != t["sha256"]:
+                return None
+    except OSError:
+        return None
+    return round(t["dram_bytes"] / t["algorithmic_bytes"] * mean_alg)
 
 
 def parse_args(argv=None):
@@ -349,7 +376,8 @@ def run_ours(args, dist: Dist):
     roofline = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(ach / peak, 4), "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6650 GB/s",
-                "traffic": TRAFFIC_BYTES.get((dom, args.workload)),
+                "traffic": traffic_per_launch(dom, w.name, not args.expert_shape, per_launch),
+                "traffic_source": (TRAFFIC.get((dom, w.name)) or {}).get("profile"),
                 "algorithmic_bytes_per_launch": per_launch}
 
     cpu = None
