@@ -80,37 +80,41 @@ __host__ __device__ inline size_t plan_smem_words(int E, int N, int NR)
     return (size_t)32 * 33 + 96 + 8 + (size_t)7 * E + (size_t)5 * N + 1 + (size_t)5 * NR + 2 + (size_t)2 * K;
 }
 
+// Word offsets are computed as integers from the (16-byte aligned) base of the
+// dynamic shared memory, so every pointer stays visibly derived from it and
+// compiles to shared-memory instructions.
 __device__ __forceinline__ PlanSmem carve(int32_t *p, int E, int N, int NR)
 {
     PlanSmem s;
-    s.part = p;      p += 32 * 33;
-    s.ws = p;        p += 96;
-    s.misc = p;      p += 8;
-    s.sload = p;     p += E;
-    s.pre = p;       p += E;
-    s.qh = p;        p += E;
-    s.ovf = p;       p += E;
-    s.order = p;     p += E;
-    s.afirst = p;    p += E;
-    s.acnt = p;      p += E;
-    s.before = p;    p += N;
-    s.spare = p;     p += N;
-    s.extra = p;     p += N;
-    s.rsorted = p;   p += N;
-    s.rsum = p;      p += N + 1;
-    s.ar = p;        p += NR;
-    s.au = p;        p += NR;
-    s.ac = p;        p += NR;
-    s.ae = p;        p += NR;
-    s.sasg = p;      p += NR;
-    p += (reinterpret_cast<uintptr_t>(p) & 7) ? 1 : 0;
-    s.key = reinterpret_cast<unsigned long long *>(p);
+    int o = 0;
+    s.part = p + o;      o += 32 * 33;
+    s.ws = p + o;        o += 96;
+    s.misc = p + o;      o += 8;
+    s.sload = p + o;     o += E;
+    s.pre = p + o;       o += E;
+    s.qh = p + o;        o += E;
+    s.ovf = p + o;       o += E;
+    s.order = p + o;     o += E;
+    s.afirst = p + o;    o += E;
+    s.acnt = p + o;      o += E;
+    s.before = p + o;    o += N;
+    s.spare = p + o;     o += N;
+    s.extra = p + o;     o += N;
+    s.rsorted = p + o;   o += N;
+    s.rsum = p + o;      o += N + 1;
+    s.ar = p + o;        o += NR;
+    s.au = p + o;        o += NR;
+    s.ac = p + o;        o += NR;
+    s.ae = p + o;        o += NR;
+    s.sasg = p + o;      o += NR;
+    o = (o + 1) & ~1;                       // 8-byte alignment for the keys
+    s.key = reinterpret_cast<unsigned long long *>(p + o);
     return s;
 }
 
 // Block-wide exclusive prefix sum of one value per thread (every thread of the
 // block calls it; blockDim.x is a multiple of 32).
-__device__ int block_excl_scan(int v, int32_t *ws, int *total)
+__device__ __forceinline__ int block_excl_scan(int v, int32_t *ws, int *total)
 {
     const int lane = lane_id(), warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     int x = v;
@@ -157,7 +161,7 @@ __device__ __forceinline__ void slice_sums(const int32_t *__restrict__ counts, i
 
 // rank_off[r][e] for the rows [r0, r1), starting from the occurrences in the
 // rows before r0 (the partial vectors of the earlier slices, over DSMEM).
-__device__ void slice_rank_off(cg::cluster_group &cluster, const int32_t *__restrict__ counts, int E, int r0,
+__device__ __forceinline__ void slice_rank_off(cg::cluster_group &cluster, const int32_t *__restrict__ counts, int E, int r0,
                                int r1, int c, int32_t *part, int32_t *__restrict__ rank_off)
 {
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -182,7 +186,7 @@ __device__ void slice_rank_off(cg::cluster_group &cluster, const int32_t *__rest
 
 // R > 1: the chunk-by-chunk greedy, run by warp 0.
 template <int NRL>
-__device__ void greedy_chunks(const PlanSmem &s, int N, int R, int M1)
+__device__ __forceinline__ void greedy_chunks(const PlanSmem &s, int N, int R, int M1)
 {
     const int lane = lane_id();
     unsigned sp[NRL];
@@ -273,7 +277,7 @@ __device__ void greedy_chunks(const PlanSmem &s, int N, int R, int M1)
 // assignment a is sorted position a, filled in by the whole block afterwards.
 // The prefix values are held in registers, a window of 32 at a time, so each
 // expert costs one compare, one ballot and one shuffle.
-__device__ void greedy_sorted(const PlanSmem &s, int K, int M1)
+__device__ __forceinline__ void greedy_sorted(const PlanSmem &s, int K, int M1)
 {
     const int lane = lane_id();
     int p = 0, stop_pos = M1, stop_rem = 0;

@@ -48,17 +48,20 @@ __host__ __device__ inline size_t reroute_smem_words(int E, int cap)
     return (size_t)2 * kRerouteWarps * E + 3 * (size_t)E + 2 * (size_t)E + 2 * (size_t)cap + 4;
 }
 
+// Word offsets are computed as integers from the (16-byte aligned) base of the
+// dynamic shared memory, so every pointer stays visibly derived from it and
+// compiles to shared-memory instructions.
 __device__ __forceinline__ RerouteSmem carve(int32_t *base, int E)
 {
     RerouteSmem s;
-    s.hist = base;
-    s.code = s.hist + kRerouteWarps * E;
-    s.tot = s.code + kRerouteWarps * E;
-    s.base = s.tot + E;
-    s.rexp = s.base + E;
-    int32_t *p = s.rexp + E;
-    p += (reinterpret_cast<uintptr_t>(p) & 7) ? 1 : 0;   // 8-byte alignment for int2
-    s.tab = reinterpret_cast<int2 *>(p);
+    int o = 0;
+    s.hist = base + o;   o += kRerouteWarps * E;
+    s.code = base + o;   o += kRerouteWarps * E;
+    s.tot = base + o;    o += E;
+    s.base = base + o;   o += E;
+    s.rexp = base + o;   o += E;
+    o = (o + 1) & ~1;                       // 8-byte alignment for the int2 tables
+    s.tab = reinterpret_cast<int2 *>(base + o);
     s.rc = s.tab + E;
     return s;
 }
