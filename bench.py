@@ -81,6 +81,9 @@ def parse_args(argv=None):
                     help="distinct resident microbatches cycled by the steps (default: the workload's)")
     ap.add_argument("--expert-shape", default=None,
                     help="override the expert matrices' rows x cols (e.g. 1024x512) for small profiling cases")
+    ap.add_argument("--sweep", action="store_true",
+                    help="rebalance latency and imbalance over the sweep grid (one JSON line per point)")
+    ap.add_argument("--sweep-seeds", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args(argv)
@@ -505,9 +508,53 @@ def run_reference(args, dist: Dist):
     }
 
 
+def run_sweep(args, dist: Dist):
+    """Rebalance over the sweep grid: E=256, top-8, R=1 (E + N slots), tokens per
+    rank x N x Zipf s; inputs drawn on the device.  One JSON line per point."""
+    import torch
+
+    from moe_expert_load_ue_b200 import ue
+    torch.cuda.set_device(dist.local_rank)
+    dev = torch.device("cuda", dist.local_rank)
+    ctx = ue.Context(dist.local_rank)
+    stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for w in inputs.sweep(seeds=args.sweep_seeds):
+        cfg = ue.Config(E=w.E, N=w.N, R=w.R, K=w.K, T=w.T)
+        ids = inputs.topk_ids_device(w, 0, dev)
+        counts = torch.empty((w.N, w.E), dtype=torch.int32, device=dev)
+        bad = torch.empty(w.N, dtype=torch.int32, device=dev)
+        plan = ue.Plan(cfg, device=dev)
+        phys = torch.empty_like(ids)
+        times = []
+        with torch.cuda.stream(stream):
+            for k in range(args.warmup + 10):
+                flush.zero_()                       # ids leave L2 between repetitions
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                ue.ue_rebalance(ctx, cfg, ids, counts, bad, plan, phys, stream=stream)
+                b.record(stream)
+                if k >= args.warmup:
+                    times.append((a, b))
+        stream.synchronize()
+        info = plan["info"].cpu().tolist()
+        us = [a.elapsed_time(b) * 1e3 for a, b in times]
+        mean = w.L / w.N
+        print(json.dumps({"sweep_point": w.name, "tokens_per_rank": w.tokens_per_rank, "N": w.N, "zipf_s": w.s,
+                          "seed": w.base_seed, "T": w.T, "rebalance_us_median": round(statistics.median(us), 2),
+                          "imbalance_before": round(info[5] / mean, 4), "imbalance_after": round(info[6] / mean, 4),
+                          "slots_ran_out": bool(info[2] & 1), "replicated_experts": info[3],
+                          "filled_redundant_slots": info[4]}), flush=True)
+        del ids, phys, plan
+    ctx.close()
+
+
 def main(argv=None):
     args = parse_args(argv)
     dist = Dist()
+    if args.sweep:
+        run_sweep(args, dist)
+        return
     if args.impl == "reference":
         res = run_reference(args, dist)
     else:

@@ -178,6 +178,23 @@ def topk_ids(w: Workload, microbatch: int = 0) -> np.ndarray:
     return ids
 
 
+def topk_ids_device(w: Workload, microbatch: int = 0, device="cuda"):
+    """Same routing model drawn with torch on `device` (for large sweeps; a
+    different random stream from topk_ids).  Returns int32 [T, K] on device."""
+    import torch
+    p = torch.as_tensor(popularity(w, microbatch), dtype=torch.float32, device=device)
+    g = torch.Generator(device=device).manual_seed(w.seed(microbatch) * 7919 + 17)
+    out = torch.empty((w.T, w.K), dtype=torch.int32, device=device)
+    inv = 1.0 / p
+    chunk = 1 << 16
+    for a in range(0, w.T, chunk):
+        b = min(w.T, a + chunk)
+        x = torch.empty((b - a, w.E), dtype=torch.float32, device=device).exponential_(generator=g)
+        x *= inv                       # exponential race: the K smallest X / p are the Gumbel-top-k
+        out[a:b] = torch.topk(x, w.K, dim=1, largest=False, sorted=True).indices.to(torch.int32)
+    return out
+
+
 def hot_expert(w: Workload, microbatch: int = 0) -> int:
     """The forced hot expert of an extreme-skew microbatch (same draw as topk_ids)."""
     ss_hot = np.random.SeedSequence(w.seed(microbatch)).spawn(3)[1]

@@ -61,3 +61,13 @@ def test_bf16_bits_round_to_nearest():
     x = inputs.random_bf16_bits((1000,), 0.02, 3)
     f = (x.astype(np.uint32) << 16).view(np.float32)
     assert abs(float(f.std()) - 0.02) < 0.003
+
+
+def test_device_generator_shapes_and_distinct():
+    w = inputs.CLASS_671B.with_(tokens_per_rank=64)
+    a = inputs.topk_ids_device(w, 1, "cpu").numpy()
+    assert a.shape == (w.T, w.K) and a.dtype == np.int32
+    assert (np.diff(np.sort(a, axis=1), axis=1) > 0).all()
+    assert a.min() >= 0 and a.max() < w.E
+    b = inputs.topk_ids_device(w, 1, "cpu").numpy()
+    assert np.array_equal(a, b)
