@@ -521,11 +521,15 @@ def run_sweep(args, dist: Dist):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     for w in inputs.sweep(seeds=args.sweep_seeds):
         cfg = ue.Config(E=w.E, N=w.N, R=w.R, K=w.K, T=w.T)
-        ids = inputs.topk_ids_device(w, 0, dev)
-        counts = torch.empty((w.N, w.E), dtype=torch.int32, device=dev)
-        bad = torch.empty(w.N, dtype=torch.int32, device=dev)
-        plan = ue.Plan(cfg, device=dev)
-        phys = torch.empty_like(ids)
+        # Inputs drawn and buffers allocated on the stream the kernels run on,
+        # and the device drained before timing: no cross-stream reuse of memory.
+        with torch.cuda.stream(stream):
+            ids = inputs.topk_ids_device(w, 0, dev)
+            counts = torch.empty((w.N, w.E), dtype=torch.int32, device=dev)
+            bad = torch.empty(w.N, dtype=torch.int32, device=dev)
+            plan = ue.Plan(cfg, device=dev)
+            phys = torch.empty_like(ids)
+        torch.cuda.synchronize(dev)
         times = []
         with torch.cuda.stream(stream):
             for k in range(args.warmup + 10):
@@ -545,7 +549,8 @@ def run_sweep(args, dist: Dist):
                           "imbalance_before": round(info[5] / mean, 4), "imbalance_after": round(info[6] / mean, 4),
                           "slots_ran_out": bool(info[2] & 1), "replicated_experts": info[3],
                           "filled_redundant_slots": info[4]}), flush=True)
-        del ids, phys, plan
+        del ids, phys, plan, counts, bad
+        torch.cuda.synchronize(dev)
     ctx.close()
 
 

@@ -119,6 +119,13 @@ __device__ __forceinline__ unsigned lanemask_lt()
 
 __device__ __forceinline__ int clampi(int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi : v); }
 
+// Shared-memory increment as one native reduction (red.shared.add), so that
+// the compiler does not rewrite it into a per-address warp aggregation loop.
+__device__ __forceinline__ void smem_add(int32_t *p, int v)
+{
+    asm volatile("red.shared.add.u32 [%0], %1;" ::"r"((uint32_t)__cvta_generic_to_shared(p)), "r"(v) : "memory");
+}
+
 // Programmatic dependent launch: wait for the previous grid on the stream to
 // complete (and its writes to be visible); allow the next grid to launch.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -127,5 +134,11 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
 // Split cluster barrier (release on arrive, acquire on wait).
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+// Arrive without release semantics: only says "this CTA is done reading its
+// peers' shared memory", so it does not wait for the CTA's own global stores.
+__device__ __forceinline__ void cluster_arrive_relaxed()
+{
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
 
 }  // namespace ue

@@ -6,8 +6,8 @@
 //
 // Design (sm_100a): one thread-block cluster per simulated rank.  Each CTA of
 // the cluster histograms a contiguous share of the rank's ids with 16-byte
-// (int4) loads into shared-memory histograms (8 copies, one per pair of
-// warps, so that shared atomics on a popular expert collide rarely), sums the
+// (int4) loads into shared-memory histograms (one copy per warp, so that
+// shared atomics on a popular expert collide only inside a warp), sums the
 // copies, and the cluster then reduces its CTA histograms over distributed
 // shared memory, each CTA summing a slice of the E columns.  The rank's row
 // of counts is written with plain stores: no global atomics, no pre-zeroing,
@@ -22,11 +22,11 @@ namespace ue {
 namespace {
 
 constexpr int kLoadWarps = 16;
-constexpr int kCopies = 8;       // shared-memory histogram copies per CTA
+constexpr int kCopies = 16;      // shared-memory histogram copies per CTA (one per warp)
 
 __device__ __forceinline__ void count_id(int32_t *h, int id, int E, int &nbad)
 {
-    if ((unsigned)id < (unsigned)E) atomicAdd(h + id, 1);
+    if ((unsigned)id < (unsigned)E) smem_add(h + id, 1);
     else ++nbad;
 }
 
@@ -131,7 +131,8 @@ k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
         for (int q = 0; q < C; ++q) s += *cluster.map_shared_rank(sbad, q);
         bad[r] = s;
     }
-    cluster.sync();   // peers may still read this CTA's totals
+    cluster_arrive_relaxed();   // done reading the peers; they may still read this CTA's totals
+    cluster_wait();
 }
 
 }  // namespace

@@ -13,13 +13,14 @@
 //   Replica list of e: home slot, then redundant slots in allocation order;
 //   rep_cum = exclusive prefix of their quotas.
 //
-// Design (sm_100a): one thread-block cluster of up to 8 CTAs.  Every CTA sums
-//   a slice of the rank rows of counts into a partial load vector in shared
-//   memory and arrives on the cluster barrier.  CTA 0 adds the partial vectors
-//   over DSMEM (the loads) and plans; meanwhile - off the critical path - the
-//   other CTAs write the exclusive scan over ranks of their row slices,
-//   rank_off[r][e], that the reroute kernel needs (the partial vectors of the
-//   earlier slices give each slice its starting offsets).  CTA 0 plans:
+// Design (sm_100a): one thread-block cluster of up to 8 CTAs.  Every
+//   CTA other than CTA 0 sums a slice of the rank rows of counts into a partial
+//   load vector in shared memory and arrives on the cluster barrier.  CTA 0
+//   adds the partial vectors over DSMEM (the loads) and plans; meanwhile - off
+//   the critical path - the other CTAs write the exclusive scan over ranks of
+//   their row slices, rank_off[r][e], that the reroute kernel needs (the
+//   partial vectors of the earlier slices give each slice its starting
+//   offsets).  CTA 0 plans:
 //     * home pass in closed form from a block-wide prefix sum: the home rank's
 //       load before e is min(Q, in-rank prefix), so
 //       take = min(Q, prefix + load) - min(Q, prefix);
@@ -160,14 +161,15 @@ __device__ __forceinline__ void slice_sums(const int32_t *__restrict__ counts, i
 }
 
 // rank_off[r][e] for the rows [r0, r1), starting from the occurrences in the
-// rows before r0 (the partial vectors of the earlier slices, over DSMEM).
-__device__ __forceinline__ void slice_rank_off(cg::cluster_group &cluster, const int32_t *__restrict__ counts, int E, int r0,
-                               int r1, int c, int32_t *part, int32_t *__restrict__ rank_off)
+// rows before r0: the partial vectors of the CTAs q0 <= q < c (over DSMEM).
+__device__ __forceinline__ void slice_rank_off(cg::cluster_group &cluster, const int32_t *__restrict__ counts, int E,
+                                               int r0, int r1, int c, int q0, int32_t *part,
+                                               int32_t *__restrict__ rank_off)
 {
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int prev[kMaxCluster];
 #pragma unroll
-        for (int q = 0; q < kMaxCluster; ++q) prev[q] = q < c ? cluster.map_shared_rank(part, q)[e] : 0;
+        for (int q = 0; q < kMaxCluster; ++q) prev[q] = (q >= q0 && q < c) ? cluster.map_shared_rank(part, q)[e] : 0;
         int run = 0;
 #pragma unroll
         for (int q = 0; q < kMaxCluster; ++q) run += prev[q];
@@ -275,8 +277,9 @@ __device__ __forceinline__ void greedy_chunks(const PlanSmem &s, int N, int R, i
 // s.rsum over K ranks); run by warp 0.  Expert m of the overflow order takes
 // the sorted positions [cut[m], cut[m+1]) (recorded in s.afirst / s.acnt);
 // assignment a is sorted position a, filled in by the whole block afterwards.
-// The prefix values are held in registers, a window of 32 at a time, so each
-// expert costs one compare, one ballot and one shuffle.
+// The prefix values are held in registers, a window of 32 at a time, and the
+// cuts of a batch of 32 experts are kept by their lanes and stored together,
+// so each expert costs a compare, a ballot and two shuffles.
 __device__ __forceinline__ void greedy_sorted(const PlanSmem &s, int K, int M1)
 {
     const int lane = lane_id();
@@ -289,8 +292,9 @@ __device__ __forceinline__ void greedy_sorted(const PlanSmem &s, int K, int M1)
         const int e_l = idx < M1 ? s.order[idx] : 0;
         const int o_l = idx < M1 ? s.ovf[e_l] : 0;
         const int cnt = min(32, M1 - m0);
-        for (int j = 0; j < cnt; ++j) {
-            const int e = __shfl_sync(0xffffffffu, e_l, j);
+        int my_first = 0, my_end = 0;                 // the cut of expert m0 + lane
+        int j = 0;
+        for (; j < cnt; ++j) {
             const int rem = __shfl_sync(0xffffffffu, o_l, j);
             const long long target = (long long)rsum_p + rem;   // smallest q > p with rsum[q] >= target
             int q = -1, rsum_q = 0;
@@ -306,18 +310,22 @@ __device__ __forceinline__ void greedy_sorted(const PlanSmem &s, int K, int M1)
                 wbase += 32;                          // the whole window is below the target
                 wv = wbase + lane <= K ? s.rsum[wbase + lane] : INT_MAX;
             }
-            if (lane == 0) {
-                s.afirst[e] = p;
-                s.acnt[e] = (q < 0 ? K : q) - p;
-            }
+            const int end = q < 0 ? K : q;
+            my_first = lane == j ? p : my_first;
+            my_end = lane == j ? end : my_end;
             if (q < 0) {                              // every remaining rank used: the rest stays home
                 stop_pos = m0 + j;
                 stop_rem = rem - (s.rsum[K] - rsum_p);
                 p = K;
+                ++j;
                 break;
             }
             p = q;
             rsum_p = rsum_q;
+        }
+        if (lane < j) {
+            s.afirst[e_l] = my_first;
+            s.acnt[e_l] = my_end - my_first;
         }
     }
     if (lane == 0) {
@@ -339,23 +347,27 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
     const int C = (int)cluster.num_blocks();
     const int c = (int)cluster.block_rank();
     const int tid = threadIdx.x, nt = blockDim.x, warp = tid >> 5;
-    // This CTA's slice of the rank rows of counts.
-    const int rows = (N + C - 1) / C;
-    const int r0 = min(N, c * rows), r1 = min(N, r0 + rows);
+    // This CTA's slice of the rank rows of counts.  With a cluster, CTA 0 holds
+    // no rows (it only plans) and the other CTAs split them.
+    const int slices = C > 1 ? C - 1 : 1, sl_id = C > 1 ? c - 1 : 0;
+    const int rows = (N + slices - 1) / slices;
+    const int r0 = (C > 1 && c == 0) ? N : min(N, sl_id * rows);
+    const int r1 = (C > 1 && c == 0) ? N : min(N, r0 + rows);
 
     // The reroute grid may launch now (its first pass needs only the ids);
     // the counts of the load grid are read after it completes.
     pdl_trigger();
     pdl_wait();
 
-    slice_sums(counts, E, r0, r1, s.sload);
+    if (C == 1 || c != 0) slice_sums(counts, E, r0, r1, s.sload);
     cluster_arrive();          // #1: this slice's partial loads are ready
     cluster_wait();
     if (c != 0) {
-        // Off the critical path: rank_off for this slice, then stay resident
-        // until every CTA has read the partial vectors.
-        slice_rank_off(cluster, counts, E, r0, r1, c, s.sload, plan.rank_off);
-        cluster_arrive();      // #2
+        // Off the critical path: rank_off for this slice (the slices of the
+        // lower peers give its start), then stay resident until every CTA has
+        // read this CTA's partial vector.
+        slice_rank_off(cluster, counts, E, r0, r1, c, 1, s.sload, plan.rank_off);
+        cluster_arrive_relaxed();   // #2: done reading the lower peers
         cluster_wait();
         return;
     }
@@ -363,15 +375,18 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
     const bool ve = e < E;
     int ld = 0;
     if (ve) {
-        int part[kMaxCluster];
+        if (C == 1) {
+            ld = s.sload[e];
+        } else {
+            int part[kMaxCluster];
 #pragma unroll
-        for (int q = 1; q < kMaxCluster; ++q) part[q] = q < C ? cluster.map_shared_rank(s.sload, q)[e] : 0;
-        ld = s.sload[e];
+            for (int q = 1; q < kMaxCluster; ++q) part[q] = q < C ? cluster.map_shared_rank(s.sload, q)[e] : 0;
 #pragma unroll
-        for (int q = 1; q < kMaxCluster; ++q) ld += part[q];
+            for (int q = 1; q < kMaxCluster; ++q) ld += part[q];
+        }
         plan.load[e] = ld;
     }
-    cluster_arrive();          // #2: done reading the peers (they still read this CTA's slice)
+    cluster_arrive_relaxed();  // #2: done reading the peers; CTA 0 holds nothing they read
 
     // ---- the plan (CTA 0; blockDim >= max(E, N)) ---------------------------------
     int L;
@@ -558,9 +573,7 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
             plan.info[7] = 0;
         }
     }
-    // rank_off of CTA 0's own slice (it starts at zero); stay resident until
-    // the peers have read this CTA's partial loads.
-    slice_rank_off(cluster, counts, E, r0, r1, 0, s.sload, plan.rank_off);
+    if (C == 1) slice_rank_off(cluster, counts, E, r0, r1, 0, 0, s.sload, plan.rank_off);
     cluster_wait();
 }
 
