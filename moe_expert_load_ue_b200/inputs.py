@@ -202,7 +202,7 @@ def hot_expert(w: Workload, microbatch: int = 0) -> int:
 
 
 def gates(ids: np.ndarray, w: Workload, microbatch: int = 0) -> np.ndarray:
-    """fp32 softmax gates over each token's K chosen experts (unused by the path)."""
+    """fp32 softmax gates over each token's K chosen experts (carried along by the dispatch layout)."""
     rng = np.random.default_rng(w.seed(microbatch) + 7_000_000)
     logits = rng.standard_normal(ids.shape).astype(np.float32)
     logits = -np.sort(-logits, axis=1)

@@ -19,6 +19,10 @@ Pinning status (what fixes each function other than itself; the tests under
                 integer max-flow on tiny inputs.
   reroute       numpy stable argsort + searchsorted; per-slot counts equal
                 quotas; every phys slot holds the token's expert.
+  dispatch      hand-worked layouts (tests/golden/dispatch_cases.json); numpy
+                stable argsort of the slots; segment lengths equal the plan's
+                slot quotas; every segment holds only its slot, in increasing
+                flat index; gates carried bit for bit.
   sync          byte-map conservation: every byte of every filled redundant
                 slot comes from the right home byte exactly once, other slots
                 untouched.
@@ -27,8 +31,8 @@ Pinning status (what fixes each function other than itself; the tests under
 
 None of these pins comes from the UltraEP pages themselves, which print no
 worked example, table or value for any step: parity against the pages is
-"unpinned by the pages" for all five steps; the pins above are the
-mathematics and hand-worked cases of the stated rule.
+"unpinned by the pages" for all five steps and the dispatch layout; the pins
+above are the mathematics and hand-worked cases of the stated rule.
 """
 from __future__ import annotations
 
@@ -68,10 +72,11 @@ def _get():
             lib.ue_oracle_expert_load.argtypes = [vp, ci, ci, vp, vp]
             lib.ue_oracle_plan.argtypes = [ci, ci, ci, vp] + [vp] * 9
             lib.ue_oracle_reroute.argtypes = [vp, i64, ci, ci, vp, vp, vp, vp, vp]
+            lib.ue_oracle_dispatch.argtypes = [vp, i64, ci, vp, vp, vp, vp]
             lib.ue_oracle_sync.argtypes = [vp, i64, i64, ci, ci, ci, vp]
             lib.ue_oracle_grad_reduce.argtypes = [vp, i64, vp, ci, i64, i64, ci, ci, ci, vp, vp]
             for f in ("ue_oracle_load", "ue_oracle_expert_load", "ue_oracle_plan",
-                      "ue_oracle_reroute", "ue_oracle_sync", "ue_oracle_grad_reduce"):
+                      "ue_oracle_reroute", "ue_oracle_dispatch", "ue_oracle_sync", "ue_oracle_grad_reduce"):
                 getattr(lib, f).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -148,6 +153,24 @@ def reroute(ids: np.ndarray, E: int, pl: dict) -> np.ndarray:
                                   _p(_c(pl["slot_quota"], np.int32)), _p(phys))
     _check(rc, "reroute")
     return phys
+
+
+def dispatch(phys: np.ndarray, S: int, gates: np.ndarray | None = None):
+    """Dispatch layout of the physical routing: (slot_off [S+1], src_index, gates_out).
+
+    src_index (and gates_out, None without gates) hold the slot_off[S] valid
+    assignments grouped by slot, in increasing flat index within a slot."""
+    phys = _c(phys, np.int32).ravel()
+    L = phys.shape[0]
+    slot_off = np.empty(S + 1, np.int32)
+    src = np.empty(L, np.int32)
+    g = None if gates is None else _c(gates, np.float32).ravel()
+    if g is not None and g.shape[0] != L:
+        raise OracleError("gates must have one value per assignment")
+    gout = None if g is None else np.empty(L, np.float32)
+    _check(_get().ue_oracle_dispatch(_p(phys), L, S, _p(g), _p(slot_off), _p(src), _p(gout)), "dispatch")
+    n = int(slot_off[S])
+    return slot_off, src[:n], (None if gout is None else gout[:n])
 
 
 def sync(W: np.ndarray, nbytes: int, E: int, N: int, R: int, slot_expert: np.ndarray) -> None:

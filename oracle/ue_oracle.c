@@ -282,6 +282,49 @@ int ue_oracle_reroute(const int32_t *ids, int64_t T, int K, int E,
     return rc;
 }
 
+/* ---- after step 3: dispatch layout -----------------------------------------
+ * Routing expansion hands its physical routing to token dispatch, which groups
+ * the assignments by physical slot before expert compute.  The layout:
+ *   slot_off[s]  = number of valid assignments routed to slots below s
+ *                  (slot_off[S] = every valid assignment);
+ *   src_index    = for s = 0, 1, ..., S-1 in turn, the flat indices x = t*K + k
+ *                  with phys[x] = s, in increasing x (a stable counting sort of
+ *                  the assignments by slot);
+ *   gates_out[p] = gates[src_index[p]] when gates is given.
+ * Assignments with phys[x] = -1 (invalid ids) are not dispatched; the entries
+ * of src_index / gates_out past slot_off[S] are left untouched.
+ */
+int ue_oracle_dispatch(const int32_t *phys, int64_t L, int S, const float *gates,
+                       int32_t *slot_off, int32_t *src_index, float *gates_out)
+{
+    if (L < 0 || S < 1) return ORC_BAD_ARG;
+    int64_t *cnt = calloc((size_t)S, sizeof(int64_t));
+    if (!cnt) return ORC_BAD_ARG;
+    for (int64_t x = 0; x < L; ++x) {
+        int32_t s = phys[x];
+        if (s == -1) continue;
+        if (s < 0 || s >= S) { free(cnt); return ORC_BAD_ARG; }
+        cnt[s]++;
+    }
+    int64_t run = 0;
+    for (int s = 0; s < S; ++s) {
+        slot_off[s] = (int32_t)run;
+        int64_t c = cnt[s];
+        cnt[s] = run;                    /* from here on: next free position of slot s */
+        run += c;
+    }
+    slot_off[S] = (int32_t)run;
+    for (int64_t x = 0; x < L; ++x) {
+        int32_t s = phys[x];
+        if (s == -1) continue;
+        int64_t p = cnt[s]++;
+        src_index[p] = (int32_t)x;
+        if (gates) gates_out[p] = gates[x];
+    }
+    free(cnt);
+    return ORC_OK;
+}
+
 /* ---- step 4: replica weight sync ------------------------------------------
  * Every filled redundant slot s (slot_expert[s] = e >= 0, s % (H+R) >= H)
  * receives a copy of e's home slot.  Slot s starts at byte s * slot_stride of
