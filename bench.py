@@ -304,6 +304,37 @@ def run_ours(args, dist: Dist):
     stream.synchronize()
     bd = np.array([[evb[k][i].elapsed_time(evb[k][i + 1]) for i in range(3)] for k in range(n_bd)]) * 1e3
 
+    # The rebalance with the dispatch layout (slot offsets, per-slot source
+    # indices and gates carried along), and the dispatch call alone after a
+    # plan; events around each call, a weight sync between reps as in the step.
+    gates_dev = torch.empty((n_mb, w.T, w.K), dtype=torch.float32, device=dev)
+    for mb in range(n_mb):
+        gates_dev[mb].copy_(torch.from_numpy(inputs.gates(ids_host[mb], w, mb)))
+    disp = ue.Dispatch(cfg, with_gates=True, device=dev)
+    n_dp = max(8, min(args.steps, 64))
+    evd = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_dp)]
+    with torch.cuda.stream(stream):
+        for k in range(args.warmup + n_dp):
+            mb = k % n_mb
+            e = evd[k - args.warmup] if k >= args.warmup else None
+            if e:
+                e[0].record(stream)
+            ue.ue_rebalance_dispatch(ctx, cfg, ids_dev[mb], counts, bad, plan, phys, disp, gates_dev[mb],
+                                     stream=stream)
+            if e:
+                e[1].record(stream)
+            ue.ue_sync(ctx, cfg, weights, slot_bytes, plan, stream=stream)
+            if e:
+                e[2].record(stream)
+            ue.ue_dispatch(ctx, cfg, ids_dev[mb], plan, phys, disp, gates_dev[mb], stream=stream)
+            if e:
+                e[3].record(stream)
+            ue.ue_sync(ctx, cfg, weights, slot_bytes, plan, stream=stream)
+    stream.synchronize()
+    reb_disp_us = float(np.mean([e[0].elapsed_time(e[1]) for e in evd])) * 1e3
+    disp_call_us = float(np.mean([e[2].elapsed_time(e[3]) for e in evd])) * 1e3
+    del gates_dev
+
     # The rebalance of every microbatch captured once into a CUDA graph (the
     # programmatic launch edges are kept) and replayed back to back: launch
     # overhead is amortised; the ids of all microbatches together exceed L2.
@@ -431,6 +462,13 @@ def run_ours(args, dist: Dist):
             "sync": round(sync_us_max, 1), "grad_reduce": round(grad_us_max, 1),
             "launch_floor": round(launch_floor_us, 2),
             "rebalance_graph": None if graph_us is None else round(graph_us, 2),
+            "rebalance_dispatch": round(reb_disp_us, 2),
+            "dispatch_call": round(disp_call_us, 2),
+        },
+        "dispatch_layout": {
+            "note": "ue_rebalance_dispatch: load + plan + reroute with the per-slot grouping of (t, k) and gates",
+            "algorithmic_bytes": 20 * w.L,
+            "hbm_floor_us": round(20 * w.L / (peak * 1e9) * 1e6, 2),
         },
         "rebalance_hbm_floor_us": round(rebalance_alg_bytes / (peak * 1e9) * 1e6, 2),
         "sync_gbs": round(sync_gbs, 1), "sync_frac": round(sync_gbs / peak, 4),

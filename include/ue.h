@@ -88,7 +88,8 @@ ue_status ue_ctx_create(int device, ue_ctx **out);
 ue_status ue_ctx_destroy(ue_ctx *ctx);
 
 /* Copy the context's device status word to *host_word (synchronizes
- * `stream`) and clear it.  Nonzero means a kernel gave up a bounded wait. */
+ * `stream`) and clear it.  Bit 0: a kernel gave up a bounded wait; bit 1:
+ * ue_dispatch met ids that do not match the plan. */
 ue_status ue_ctx_device_error(ue_ctx *ctx, int32_t *host_word, void *stream);
 
 /* ---- step 1: load computation ----------------------------------------------
@@ -130,6 +131,39 @@ ue_status ue_reroute(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids,
 ue_status ue_rebalance(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids,
                        int32_t *counts, int32_t *bad, const ue_plan_buffers *plan,
                        int32_t *phys, void *stream);
+
+/* ---- dispatch layout (after step 3) ------------------------------------------
+ * Routing expansion hands the physical routing to token dispatch, which groups
+ * the assignments by physical slot for expert compute ("Routing expansion ->
+ * Token dispatch: physical routing", "Token dispatch -> Expert compute:
+ * dispatches tokens" in "How dots-infra/ultraep works").  Layout:
+ *   slot_off[s]  = assignments routed to slots below s (exclusive prefix of
+ *                  plan.slot_quota; slot_off[S] = all valid assignments);
+ *   src_index[p] for p in [slot_off[s], slot_off[s+1]): the flat indices
+ *                  x = t*K + k with phys[x] = s, increasing (stable grouping);
+ *   gates_out[p] = gates[src_index[p]] (bit copy) when gates is given.
+ * Ids outside [0, E) are not dispatched; entries past slot_off[S] are left
+ * untouched. */
+typedef struct {
+    const float *gates;   /* [T*K] fp32 gate of each (t, k), or NULL                    */
+    int32_t *slot_off;    /* [S+1] out                                                  */
+    int32_t *src_index;   /* [T*K] out                                                  */
+    float *gates_out;     /* [T*K] out; required when gates is given, else ignored      */
+} ue_dispatch_buffers;
+
+/* Routing expansion with the dispatch layout: writes phys exactly as
+ * ue_reroute does, plus *disp.  ids must be the ids the plan was computed
+ * from: an assignment that falls outside its slot's segment (a plan from other
+ * ids) is not written and sets bit 1 (value 2) of the context's device status
+ * word (ue_ctx_device_error). */
+ue_status ue_dispatch(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids,
+                      const ue_plan_buffers *plan, int32_t *phys,
+                      const ue_dispatch_buffers *disp, void *stream);
+
+/* Steps 1-3 with the dispatch layout, back to back on one stream (three launches). */
+ue_status ue_rebalance_dispatch(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids,
+                                int32_t *counts, int32_t *bad, const ue_plan_buffers *plan,
+                                int32_t *phys, const ue_dispatch_buffers *disp, void *stream);
 
 /* ---- step 4: replica weight sync ---------------------------------------------
  * "Replica weight sync" (csrc/kernels/weight_sync.cu; "persistent tile

@@ -105,6 +105,7 @@ ue::Launch launch_of(const ue_ctx *ctx, const ue::Shape &sh)
 {
     ue::Launch ln;
     ln.sms = ctx->sms;
+    ln.max_smem = (size_t)ctx->max_smem;
     ln.cluster = choose_cluster(sh, ctx->sms);
     return ln;
 }
@@ -265,9 +266,9 @@ ue_status ue_reroute(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids, cons
     if (sh.T > 0 && (!ids || !aligned16(ids))) return fail(UE_ERR_INVALID_ARG, "ids must be non-NULL and 16-byte aligned");
     if (sh.T > 0 && !phys) return fail(UE_ERR_INVALID_ARG, "phys is NULL");
     if ((s = check_ctx(ctx)) != UE_OK) return s;
-    if (ue::reroute_smem_bytes(sh) > (size_t)ctx->max_smem)
-        return fail(UE_ERR_INVALID_ARG, "reroute needs %zu bytes of shared memory (> %d)", ue::reroute_smem_bytes(sh),
-                    ctx->max_smem);
+    if (ue::reroute_smem_bytes(sh, false, 0, false) > (size_t)ctx->max_smem)
+        return fail(UE_ERR_INVALID_ARG, "reroute needs %zu bytes of shared memory (> %d)",
+                    ue::reroute_smem_bytes(sh, false, 0, false), ctx->max_smem);
     return on_device(ctx, [&]() -> ue_status {
         cudaError_t e = ue::launch_reroute(sh, launch_of(ctx, sh), ids, ue::to_dev(*plan), phys,
                                            static_cast<cudaStream_t>(stream), false);
@@ -287,7 +288,7 @@ ue_status ue_rebalance(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids, in
     if (sh.T > 0 && (!ids || !aligned16(ids))) return fail(UE_ERR_INVALID_ARG, "ids must be non-NULL and 16-byte aligned");
     if (sh.T > 0 && !phys) return fail(UE_ERR_INVALID_ARG, "phys is NULL");
     if ((s = check_ctx(ctx)) != UE_OK) return s;
-    if (ue::plan_smem_bytes(sh) > (size_t)ctx->max_smem || ue::reroute_smem_bytes(sh) > (size_t)ctx->max_smem)
+    if (ue::plan_smem_bytes(sh) > (size_t)ctx->max_smem || ue::reroute_smem_bytes(sh, false, 0, false) > (size_t)ctx->max_smem)
         return fail(UE_ERR_INVALID_ARG, "shape needs more shared memory than the device offers");
     return on_device(ctx, [&]() -> ue_status {
         const cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -301,6 +302,72 @@ ue_status ue_rebalance(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids, in
         if ((e = ue::launch_plan(sh, counts, pd, st, true)) != cudaSuccess) return cuda_fail(e, "plan launch");
         if ((e = ue::launch_reroute(sh, ln, ids, pd, phys, st, true)) != cudaSuccess)
             return cuda_fail(e, "reroute launch");
+        return UE_OK;
+    });
+}
+
+namespace {
+ue_status check_dispatch(const ue::Shape &sh, const ue_dispatch_buffers *d, ue::DispatchOut *out)
+{
+    if (!d) return fail(UE_ERR_INVALID_ARG, "dispatch buffers are NULL");
+    if (!d->slot_off) return fail(UE_ERR_INVALID_ARG, "slot_off is NULL");
+    if (sh.T > 0 && !d->src_index) return fail(UE_ERR_INVALID_ARG, "src_index is NULL");
+    if (sh.T > 0 && d->gates && !d->gates_out) return fail(UE_ERR_INVALID_ARG, "gates given but gates_out is NULL");
+    out->gates = sh.T > 0 ? d->gates : nullptr;
+    out->slot_off = d->slot_off;
+    out->src_index = d->src_index;
+    out->gates_out = d->gates_out;
+    return UE_OK;
+}
+}  // namespace
+
+ue_status ue_dispatch(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids, const ue_plan_buffers *plan,
+                      int32_t *phys, const ue_dispatch_buffers *disp, void *stream)
+{
+    ue::Shape sh{};
+    ue::DispatchOut out{};
+    ue_status s = make_shape(cfg, true, &sh);
+    if (s == UE_OK) s = check_plan(plan);
+    if (s == UE_OK) s = check_dispatch(sh, disp, &out);
+    if (s != UE_OK) return s;
+    if (sh.T > 0 && (!ids || !aligned16(ids))) return fail(UE_ERR_INVALID_ARG, "ids must be non-NULL and 16-byte aligned");
+    if (sh.T > 0 && !phys) return fail(UE_ERR_INVALID_ARG, "phys is NULL");
+    if ((s = check_ctx(ctx)) != UE_OK) return s;
+    if (ue::reroute_smem_bytes(sh, true, 0, false) > (size_t)ctx->max_smem)
+        return fail(UE_ERR_INVALID_ARG, "dispatch needs %zu bytes of shared memory (> %d)",
+                    ue::reroute_smem_bytes(sh, true, 0, false), ctx->max_smem);
+    return on_device(ctx, [&]() -> ue_status {
+        cudaError_t e = ue::launch_dispatch(sh, launch_of(ctx, sh), ids, ue::to_dev(*plan), phys, out, ctx->dev_err,
+                                            static_cast<cudaStream_t>(stream), false);
+        return e == cudaSuccess ? UE_OK : cuda_fail(e, "dispatch launch");
+    });
+}
+
+ue_status ue_rebalance_dispatch(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids, int32_t *counts,
+                                int32_t *bad, const ue_plan_buffers *plan, int32_t *phys,
+                                const ue_dispatch_buffers *disp, void *stream)
+{
+    ue::Shape sh{};
+    ue::DispatchOut out{};
+    ue_status s = make_shape(cfg, true, &sh);
+    if (s == UE_OK) s = check_plan(plan);
+    if (s == UE_OK) s = check_dispatch(sh, disp, &out);
+    if (s != UE_OK) return s;
+    if (!counts) return fail(UE_ERR_INVALID_ARG, "counts is NULL");
+    if (sh.T > 0 && (!ids || !aligned16(ids))) return fail(UE_ERR_INVALID_ARG, "ids must be non-NULL and 16-byte aligned");
+    if (sh.T > 0 && !phys) return fail(UE_ERR_INVALID_ARG, "phys is NULL");
+    if ((s = check_ctx(ctx)) != UE_OK) return s;
+    if (ue::plan_smem_bytes(sh) > (size_t)ctx->max_smem || ue::reroute_smem_bytes(sh, true, 0, false) > (size_t)ctx->max_smem)
+        return fail(UE_ERR_INVALID_ARG, "shape needs more shared memory than the device offers");
+    return on_device(ctx, [&]() -> ue_status {
+        const cudaStream_t st = static_cast<cudaStream_t>(stream);
+        const ue::Launch ln = launch_of(ctx, sh);
+        const ue::PlanDev pd = ue::to_dev(*plan);
+        cudaError_t e = ue::launch_load(sh, ln, ids, counts, bad, st);
+        if (e != cudaSuccess) return cuda_fail(e, "load launch");
+        if ((e = ue::launch_plan(sh, counts, pd, st, true)) != cudaSuccess) return cuda_fail(e, "plan launch");
+        if ((e = ue::launch_dispatch(sh, ln, ids, pd, phys, out, ctx->dev_err, st, true)) != cudaSuccess)
+            return cuda_fail(e, "dispatch launch");
         return UE_OK;
     });
 }

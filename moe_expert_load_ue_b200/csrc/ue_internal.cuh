@@ -38,6 +38,14 @@ struct Shape {
 struct Launch {
     int sms;               // SM count of the device
     int cluster;           // CTAs per simulated rank for load / reroute
+    size_t max_smem;       // opt-in shared memory per block
+};
+
+// Outputs of the dispatch layout (ue_dispatch_buffers without the caller's struct).
+struct DispatchOut {
+    const float *gates;
+    int32_t *slot_off, *src_index;
+    float *gates_out;
 };
 
 // Host launchers (one per kernel file).  Each returns cudaGetLastError().
@@ -52,7 +60,12 @@ int plan_cluster(const Shape &sh);
 
 cudaError_t launch_reroute(const Shape &sh, const Launch &ln, const int32_t *ids, const PlanDev &plan,
                            int32_t *phys, cudaStream_t st, bool pdl);
-size_t reroute_smem_bytes(const Shape &sh);
+cudaError_t launch_dispatch(const Shape &sh, const Launch &ln, const int32_t *ids, const PlanDev &plan,
+                            int32_t *phys, const DispatchOut &out, int32_t *dev_err, cudaStream_t st, bool pdl);
+// Shared memory of the reroute kernel (dispatch variant or not) with a
+// staging buffer of stage_cap ids (0: ids are read twice from memory), and as
+// many gates when the dispatch variant carries them.
+size_t reroute_smem_bytes(const Shape &sh, bool dispatch, int stage_cap, bool gates);
 
 cudaError_t launch_sync(const Shape &sh, const Launch &ln, uint8_t *weights, int64_t slot_bytes,
                         const PlanDev &plan, int32_t *dev_err, cudaStream_t st);

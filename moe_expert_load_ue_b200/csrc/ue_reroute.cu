@@ -23,6 +23,18 @@
 // lookups per id; only ids of an expert whose quota boundary falls inside the
 // warp's part are ranked exactly, by ballots over the bits of the expert's
 // compact index in plan.rep_experts.
+//
+// Dispatch layout (token dispatch consumes the physical routing: "Routing
+// expansion -> Token dispatch: physical routing", "Token dispatch -> Expert
+// compute: dispatches tokens").  The dispatch variant of the kernel also groups
+// the assignments by slot: with slot_off the exclusive prefix of the plan's
+// slot quotas, the assignment with occurrence index j that replica entry p
+// (slot rep_slot[p], cumulative quota rep_cum[p]) serves lands at position
+//     slot_off[rep_slot[p]] + j - rep_cum[p]
+// of src_index (its flat index t*K + k) and gates_out (its gate), i.e. a
+// stable grouping by slot computed in the same pass.  Every valid id then
+// needs its occurrence index, so this variant ranks every id of a warp step
+// by ballots over the bits of the expert id.
 #include <cooperative_groups.h>
 
 #include "ue_internal.cuh"
@@ -36,41 +48,75 @@ constexpr int kRerouteWarps = 16;
 constexpr int kUnroll = 4;
 constexpr int kStageIds = 8192;   // ids of a CTA share kept in shared memory between the passes
 
+// Kernel-side view of the dispatch outputs (unused by the plain variant).
+struct DispatchArgs {
+    const float *gates;            // [T*K] or nullptr
+    const int32_t *slot_quota;     // [S] the plan's slot quotas
+    int32_t *slot_off;             // [S+1] out (written by CTA 0)
+    int32_t *src_index;            // [T*K] out
+    float *gates_out;              // [T*K] out when gates != nullptr
+    int32_t *err;                  // device status word: bit 1 = ids do not match the plan's quotas
+    int64_t L;                     // T*K: capacity of src_index / gates_out
+    int S;
+};
+
 struct RerouteSmem {
     int32_t *hist;   // [W][E] per-warp counts, then their exclusive scan over the warps
     int32_t *code;   // [W][M] per warp and replicated expert: ~slot (uniform) or running occurrence index
+                     //        (dispatch variant: [32] partial sums of the slot-offset scan)
     int32_t *tot;    // [E]    this CTA's counts (read by later CTAs of the cluster)
     int32_t *base;   // [E]    occurrences of e before this CTA's ids
-    int32_t *rexp;   // [E]    replicated experts (plan.rep_experts)
+    int32_t *rexp;   // [E+1]  replicated experts (plan.rep_experts); dispatch variant:
+                     //        exclusive prefix of this CTA's per-expert counts
     int2 *tab;       // [E]    {home slot if one replica, else first replica entry; (compact index << 16) | count}
     int2 *rc;        // [cap]  {cumulative quota, slot} of each replica entry
-    int32_t *stage;  // [kStageIds] the CTA's ids, read once from HBM in pass 1 (when they fit)
+    int32_t *soff;   // [S+1]  dispatch only: exclusive prefix of the slot quotas
+    uint8_t *tag;    // [W][E] dispatch only: per warp and expert, a lane of the current step holding it
+    int32_t *stage;  // [stage_cap] the CTA's ids, read once from HBM in pass 1 (when they fit)
+    float *gstage;   // [stage_cap] dispatch with gates: the CTA's gates, read in pass 1 likewise
+    uint16_t *oli;   // [stage_cap] dispatch: local indices of the CTA's assignments in (expert, j) order
 };
 
-__host__ __device__ inline size_t reroute_smem_words(int E, int cap)
+// Words of code[]: per (warp, replicated expert) for the plain variant; the
+// dispatch variant keeps only the warps' partial sums there.
+__host__ __device__ inline int code_words(int E, int S_disp) { return S_disp > 0 ? 32 : kRerouteWarps * E; }
+
+// Shared-memory words; S_disp = S for the dispatch variant, else 0; the
+// gates are staged beside the ids (gstage_cap = stage_cap) when carried.
+__host__ __device__ inline size_t reroute_smem_words(int E, int cap, int S_disp, int stage_cap, int gstage_cap)
 {
-    return (size_t)2 * kRerouteWarps * E + 3 * (size_t)E + 2 * (size_t)E + 2 * (size_t)cap + 8 + kStageIds;
+    const size_t dwords = S_disp > 0 ? (size_t)S_disp + 1 + ((size_t)kRerouteWarps * E + 3) / 4 : 0;
+    const size_t oli_words = S_disp > 0 ? ((size_t)stage_cap + 1) / 2 : 0;
+    return (size_t)kRerouteWarps * E + code_words(E, S_disp) + 3 * (size_t)E + 1 + 2 * (size_t)E + 2 * (size_t)cap +
+           dwords + 8 + (size_t)stage_cap + (size_t)gstage_cap + oli_words;
 }
 
 // Word offsets are computed as integers from the (16-byte aligned) base of the
 // dynamic shared memory, so every pointer stays visibly derived from it and
 // compiles to shared-memory instructions.
-__device__ __forceinline__ RerouteSmem carve(int32_t *base, int E, int cap)
+__device__ __forceinline__ RerouteSmem carve(int32_t *base, int E, int cap, int S_disp, int stage_cap,
+                                             int gstage_cap)
 {
     RerouteSmem s;
     int o = 0;
     s.hist = base + o;   o += kRerouteWarps * E;
-    s.code = base + o;   o += kRerouteWarps * E;
+    s.code = base + o;   o += code_words(E, S_disp);
     s.tot = base + o;    o += E;
     s.base = base + o;   o += E;
-    s.rexp = base + o;   o += E;
+    s.rexp = base + o;   o += E + 1;
     o = (o + 1) & ~1;                       // 8-byte alignment for the int2 tables
     s.tab = reinterpret_cast<int2 *>(base + o);
     o += 2 * E;
     s.rc = reinterpret_cast<int2 *>(base + o);
     o += 2 * cap;
-    o = (o + 3) & ~3;                       // 16-byte alignment for the staged ids
-    s.stage = base + o;
+    s.soff = base + o;   o += S_disp > 0 ? S_disp + 1 : 0;
+    s.tag = reinterpret_cast<uint8_t *>(base + o);
+    o += S_disp > 0 ? (kRerouteWarps * E + 3) / 4 : 0;
+    o = (o + 3) & ~3;                       // 16-byte alignment for the staged ids and gates
+    s.stage = base + o;  o += (stage_cap + 3) & ~3;
+    s.gstage = reinterpret_cast<float *>(base + o);
+    o += (gstage_cap + 3) & ~3;
+    s.oli = reinterpret_cast<uint16_t *>(base + o);
     return s;
 }
 
@@ -87,15 +133,67 @@ __device__ __forceinline__ unsigned match_key(int key, int nb)
     return m;
 }
 
+// Largest k in [0, n) with rc[k].x <= j (rc[0].x = 0 <= j): the replica entry
+// whose cumulative-quota range holds occurrence j.  A replica with quota 0 has
+// an empty range and is skipped, since the next entry has the same cum.
+__device__ __forceinline__ int covering_entry(const int2 *rc, int n, int j)
+{
+    int lo = 0, hi = n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (rc[mid].x <= j) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Exclusive prefix of get(0..n-1) into out[0..n] (out[n] = the total), each
+// thread a contiguous run; tmp holds 32 words.  Every thread of the block
+// calls it; out may be written while get reads other memory.
+template <class Get>
+__device__ __forceinline__ void runs_excl_scan(Get get, int n, int32_t *out, int32_t *tmp)
+{
+    const int lane = lane_id(), warp = threadIdx.x >> 5;
+    const int per = (n + (int)blockDim.x - 1) / (int)blockDim.x;
+    const int a0 = min(n, (int)threadIdx.x * per), a1 = min(n, a0 + per);
+    int sum = 0;
+    for (int a = a0; a < a1; ++a) {
+        const int q = get(a);
+        out[a] = q;
+        sum += q;
+    }
+    int x = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    __syncthreads();                       // tmp may still be read by a previous call
+    if (lane == 31) tmp[warp] = x;
+    __syncthreads();
+    int run = x - sum;
+    for (int w = 0; w < warp; ++w) run += tmp[w];
+    for (int a = a0; a < a1; ++a) {
+        const int q = out[a];
+        out[a] = run;
+        run += q;
+    }
+    if (a0 < n && a1 == n) out[n] = run;   // the thread owning the last entry
+    if (n == 0 && threadIdx.x == 0) out[0] = 0;
+    __syncthreads();
+}
+
+template <bool kDispatch>
 __global__ void __launch_bounds__(kRerouteWarps * 32)
 k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
           const int32_t *__restrict__ rep_off, const int32_t *__restrict__ rep_slot,
           const int32_t *__restrict__ rep_cum, const int32_t *__restrict__ rep_experts,
           const int32_t *__restrict__ info, const int32_t *__restrict__ rank_off,
-          int32_t *__restrict__ phys)
+          int32_t *__restrict__ phys, int stage_cap, DispatchArgs da)
 {
     extern __shared__ __align__(16) int32_t sm_rr[];
-    const RerouteSmem s = carve(sm_rr, E, cap);
+    const RerouteSmem s = carve(sm_rr, E, cap, kDispatch ? da.S : 0, stage_cap,
+                                (kDispatch && da.gates != nullptr) ? stage_cap : 0);
 
     cg::cluster_group cluster = cg::this_cluster();
     const int C = (int)cluster.num_blocks();
@@ -116,7 +214,7 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
     const int64_t wlo = min(hi, lo + warp * wshare);
     const int64_t whi = min(hi, wlo + wshare);
     int32_t *h = s.hist + warp * E;
-    const bool staged = hi - lo <= kStageIds;     // then pass 2 reads the ids from shared memory
+    const bool staged = hi - lo <= stage_cap;     // then pass 2 reads the ids from shared memory
     // Vector mode: 16-byte loads and stores, four ids per lane, when the CTA's
     // share and phys are 16-byte aligned and the share fits in shared memory.
     const bool vec = staged && (lo % 4) == 0 && ((hi - lo) % 4) == 0 &&
@@ -156,6 +254,39 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
             if ((unsigned)id[u] < (unsigned)E) smem_add(h + id[u], 1);
         }
     }
+    // Dispatch with gates: the warp's gates are staged beside its ids.
+    const bool gstaged = kDispatch && da.gates != nullptr && staged;
+    if (gstaged) {
+        if ((lo % 4) == 0 && ((hi - lo) % 4) == 0 && (reinterpret_cast<uintptr_t>(da.gates) & 15) == 0) {
+            for (int64_t v0 = wlo; v0 < whi; v0 += 128 * kUnroll) {
+                float4 g[kUnroll];
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) {
+                    const int64_t i = v0 + 128 * u + 4 * lane;
+                    if (i < whi) g[u] = __ldg(reinterpret_cast<const float4 *>(da.gates + i));
+                }
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) {
+                    const int64_t i = v0 + 128 * u + 4 * lane;
+                    if (i < whi) *reinterpret_cast<float4 *>(s.gstage + (i - lo)) = g[u];
+                }
+            }
+        } else {
+            for (int64_t x0 = wlo; x0 < whi; x0 += 32 * kUnroll) {
+                float g[kUnroll];
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) {
+                    const int64_t i = x0 + u * 32 + lane;
+                    g[u] = i < whi ? __ldg(da.gates + i) : 0.0f;
+                }
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) {
+                    const int64_t i = x0 + u * 32 + lane;
+                    if (i < whi) s.gstage[i - lo] = g[u];
+                }
+            }
+        }
+    }
     __syncthreads();
     // Exclusive scan over the warps per expert (in place) and CTA totals.
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -188,108 +319,197 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
         for (int q = 0; q < kMaxCluster; ++q) b += peer[q];
         s.base[e] = b;            // occurrences of e before this CTA's ids
     }
-    for (int m = threadIdx.x; m < M; m += blockDim.x) s.rexp[m] = clampi(__ldg(rep_experts + m), 0, E - 1);
+    if (!kDispatch)
+        for (int m = threadIdx.x; m < M; m += blockDim.x) s.rexp[m] = clampi(__ldg(rep_experts + m), 0, E - 1);
     cluster_arrive_relaxed();  // done reading peers; they may exit once all have arrived
-    __syncthreads();
-    // Replicated experts get their compact index; every other expert's table
-    // entry becomes its home slot (its only replica).
-    for (int m = threadIdx.x; m < M; m += blockDim.x) s.tab[s.rexp[m]].y |= m << 16;
-    for (int e = threadIdx.x; e < E; e += blockDim.x)
-        if ((s.tab[e].y & 0xffff) == 1) s.tab[e].x = s.rc[s.tab[e].x].y;
-    __syncthreads();
-    // Per (warp, replicated expert): ~slot when all the warp's occurrences of
-    // the expert share one replica, else the warp's first occurrence index.
-    for (int i = threadIdx.x; i < kRerouteWarps * M; i += blockDim.x) {
-        const int w = i / M, m = i - w * M;
-        const int e = s.rexp[m];
-        const int2 t = s.tab[e];
-        const int n = t.y & 0xffff;
-        const int excl = s.hist[w * E + e];
-        const int cnt = (w + 1 < kRerouteWarps ? s.hist[(w + 1) * E + e] : s.tot[e]) - excl;
-        const int j0 = s.base[e] + excl;
-        int lo = 0, hi = n - 1;                         // largest k with cum[k] <= j0
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (s.rc[t.x + mid].x <= j0) lo = mid;
-            else hi = mid - 1;
-        }
-        const bool uniform = lo == n - 1 || j0 + cnt <= s.rc[t.x + lo + 1].x;
-        s.code[w * M + m] = uniform ? ~s.rc[t.x + lo].y : j0;
-    }
-    const int nb = M > 1 ? 32 - __clz(M - 1) : 0;   // bits of the compact index
-    __syncthreads();
+    if constexpr (kDispatch) {
+        // Slot offsets (exclusive prefix of the slot quotas; CTA 0 writes
+        // them out) and, for the local grouping below, the exclusive prefix
+        // of this CTA's per-expert counts (in rexp[], unused by this variant).
+        runs_excl_scan([&](int a) { return __ldg(da.slot_quota + a); }, da.S, s.soff, s.code);
+        runs_excl_scan([&](int e) { return s.tot[e]; }, E, s.rexp, s.code);
+        const int S = da.S;
+        if (blockIdx.x == 0)
+            for (int a = threadIdx.x; a <= S; a += blockDim.x) da.slot_off[a] = s.soff[a];
+        // Running occurrence index of each (warp, expert): base + earlier warps.
+        for (int w = 0; w < kRerouteWarps; ++w)
+            for (int e = threadIdx.x; e < E; e += blockDim.x) s.hist[w * E + e] += s.base[e];
+        __syncthreads();
 
-    // Replica of one id; rank_it when its expert's quota boundary falls inside
-    // this warp's part (the occurrence index j is then needed).
-    auto lookup = [&](int id, int &out, int &v, int2 &t, bool &rank_it) {
-        const bool valid = (unsigned)id < (unsigned)E;
-        t = valid ? s.tab[id] : make_int2(-1, 1);
-        out = t.x;                                     // the home slot (a single replica); -1 for a bad id
-        v = 0;
-        if ((t.y & 0xffff) > 1) {
-            v = s.code[warp * M + (t.y >> 16)];
-            out = ~v;                                  // the warp's uniform replica, if v < 0
-        }
-        rank_it = (t.y & 0xffff) > 1 && v >= 0;
-    };
-    // One scalar step of 32 consecutive ids (lane order = token-major order).
-    auto step = [&](int id, int64_t i) {
-        int out, v;
-        int2 t;
-        bool rank_it;
-        lookup(id, out, v, t, rank_it);
-        if (__any_sync(0xffffffffu, rank_it)) {
-            const int cm = t.y >> 16;
-            const unsigned m = match_key(rank_it ? cm : -1, nb);
-            const int before = __popc(m & lanemask_lt());
-            if (rank_it) {
-                const int j = v + before;
-                int k = (t.y & 0xffff) - 1;
-                while (k > 0 && s.rc[t.x + k].x > j) --k;
-                out = s.rc[t.x + k].y;
+        // Pass 2: every valid id is ranked among the warp's equal ids (lane
+        // order = token-major order) to get its occurrence index j; the
+        // replica entry p covering j is the slot, and the assignment lands at
+        // soff[slot] + j - rep_cum[p].  Equal ids of a step are found by a
+        // per-warp tag table: each lane writes its lane number at its expert,
+        // one lane per expert wins, and the winning lane number is a 5-bit key
+        // that is equal exactly for equal ids.  With the ids staged, the
+        // position replaces the id in stage[] and the CTA orders its
+        // assignments by (expert, j) in oli[] (local indices), so that each
+        // slot's run of this CTA is written out contiguously below; otherwise
+        // every assignment is stored where it lands.
+        uint8_t *tag = s.tag + warp * E;
+        int32_t *wh = s.hist + warp * E;
+        const unsigned lt = lanemask_lt();
+        const int nloc = (int)(whi - wlo);       // this warp's ids, local index lbase + k
+        const int lbase = (int)(wlo - lo);
+        for (int k0 = 0; k0 < nloc; k0 += 32) {
+            const int k = k0 + lane;
+            const int li = lbase + k;
+            const int id = k < nloc ? (staged ? s.stage[li] : __ldg(ids + lo + li)) : -1;
+            const bool valid = (unsigned)id < (unsigned)E;
+            if (valid) tag[id] = (uint8_t)lane;
+            __syncwarp();
+            const int key = valid ? tag[id] : 0;
+            unsigned m = __ballot_sync(0xffffffffu, valid);
+#pragma unroll
+            for (int b = 0; b < 5; ++b) {
+                const unsigned v = __ballot_sync(0xffffffffu, (key >> b) & 1);
+                m &= ((key >> b) & 1) ? v : ~v;
+            }
+            const int before = __popc(m & lt);
+            int out = -1;
+            if (valid) {
+                const int j = wh[id] + before;
+                const int2 t = s.tab[id];
+                const int2 q = s.rc[t.x + covering_entry(s.rc + t.x, t.y & 0xffff, j)];
+                out = q.y;
+                int pos = -1;
+                // Inside the slot's segment whenever the ids are the ones the
+                // plan was computed from; anything else is reported, not written.
+                if (out >= 0 && out < S) {
+                    pos = s.soff[out] + (j - q.x);
+                    if (pos < s.soff[out] || pos >= s.soff[out + 1] || (int64_t)pos >= da.L) pos = -1;
+                }
+                if (pos < 0) atomicOr(da.err, 2);
+                if (staged) {
+                    s.stage[li] = pos;
+                    s.oli[s.rexp[id] + (j - s.base[id])] = (uint16_t)li;
+                } else if (pos >= 0) {
+                    da.src_index[pos] = (int32_t)(lo + li);
+                    if (da.gates != nullptr) da.gates_out[pos] = __ldg(da.gates + lo + li);
+                }
             }
             __syncwarp();
-            if (rank_it && before == 0) s.code[warp * M + cm] = v + __popc(m);
+            if (valid && before == 0) wh[id] += __popc(m);
             __syncwarp();
+            if (k < nloc) phys[lo + li] = out;
         }
-        if (i < whi) phys[i] = out;
-    };
-
-    // Pass 2: replica of every (t, k).
-    if (vec) {
-        // Blocks of 128 ids, four per lane: when no id of the block needs its
-        // occurrence index, one 16-byte store per lane; otherwise the block is
-        // replayed as four ordered scalar steps.
-        for (int64_t v0 = wlo; v0 < whi; v0 += 128) {
-            const int64_t i = v0 + 4 * lane;
-            const int4 q = i < whi ? *reinterpret_cast<const int4 *>(s.stage + (i - lo)) : make_int4(-1, -1, -1, -1);
-            int o0, o1, o2, o3, v;
-            int2 t;
-            bool r0, r1, r2, r3;
-            lookup(q.x, o0, v, t, r0);
-            lookup(q.y, o1, v, t, r1);
-            lookup(q.z, o2, v, t, r2);
-            lookup(q.w, o3, v, t, r3);
-            if (!__any_sync(0xffffffffu, r0 || r1 || r2 || r3)) {
-                if (i < whi) *reinterpret_cast<int4 *>(phys + i) = make_int4(o0, o1, o2, o3);
-            } else {
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int64_t iu = v0 + 32 * u + lane;
-                    step(iu < whi ? s.stage[iu - lo] : -1, iu);
-                }
+        if (staged) {
+            // Write-out in (expert, j) order: consecutive threads take
+            // consecutive positions of one slot's run.
+            __syncthreads();
+            const int nvalid = s.rexp[E];
+            for (int lp = threadIdx.x; lp < nvalid; lp += blockDim.x) {
+                const int li = s.oli[lp];
+                const int pos = s.stage[li];
+                if (pos < 0) continue;
+                da.src_index[pos] = (int32_t)(lo + li);
+                if (gstaged) da.gates_out[pos] = s.gstage[li];
+                else if (da.gates != nullptr) da.gates_out[pos] = __ldg(da.gates + lo + li);
             }
         }
     } else {
-        for (int64_t x0 = wlo; x0 < whi; x0 += 32 * kUnroll) {
-            int id[kUnroll];
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const int64_t i = x0 + u * 32 + lane;
-                id[u] = i >= whi ? -1 : (staged ? s.stage[i - lo] : __ldg(ids + i));
+        __syncthreads();
+        // Replicated experts get their compact index; every other expert's table
+        // entry becomes its home slot (its only replica).
+        for (int m = threadIdx.x; m < M; m += blockDim.x) s.tab[s.rexp[m]].y |= m << 16;
+        for (int e = threadIdx.x; e < E; e += blockDim.x)
+            if ((s.tab[e].y & 0xffff) == 1) s.tab[e].x = s.rc[s.tab[e].x].y;
+        __syncthreads();
+        // Per (warp, replicated expert): ~slot when all the warp's occurrences of
+        // the expert share one replica, else the warp's first occurrence index.
+        for (int i = threadIdx.x; i < kRerouteWarps * M; i += blockDim.x) {
+            const int w = i / M, m = i - w * M;
+            const int e = s.rexp[m];
+            const int2 t = s.tab[e];
+            const int n = t.y & 0xffff;
+            const int excl = s.hist[w * E + e];
+            const int cnt = (w + 1 < kRerouteWarps ? s.hist[(w + 1) * E + e] : s.tot[e]) - excl;
+            const int j0 = s.base[e] + excl;
+            int lo = 0, hi = n - 1;                         // largest k with cum[k] <= j0
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (s.rc[t.x + mid].x <= j0) lo = mid;
+                else hi = mid - 1;
             }
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) step(id[u], x0 + u * 32 + lane);
+            const bool uniform = lo == n - 1 || j0 + cnt <= s.rc[t.x + lo + 1].x;
+            s.code[w * M + m] = uniform ? ~s.rc[t.x + lo].y : j0;
+        }
+        const int nb = M > 1 ? 32 - __clz(M - 1) : 0;   // bits of the compact index
+        __syncthreads();
+
+        // Replica of one id; rank_it when its expert's quota boundary falls inside
+        // this warp's part (the occurrence index j is then needed).
+        auto lookup = [&](int id, int &out, int &v, int2 &t, bool &rank_it) {
+            const bool valid = (unsigned)id < (unsigned)E;
+            t = valid ? s.tab[id] : make_int2(-1, 1);
+            out = t.x;                                     // the home slot (a single replica); -1 for a bad id
+            v = 0;
+            if ((t.y & 0xffff) > 1) {
+                v = s.code[warp * M + (t.y >> 16)];
+                out = ~v;                                  // the warp's uniform replica, if v < 0
+            }
+            rank_it = (t.y & 0xffff) > 1 && v >= 0;
+        };
+        // One scalar step of 32 consecutive ids (lane order = token-major order).
+        auto step = [&](int id, int64_t i) {
+            int out, v;
+            int2 t;
+            bool rank_it;
+            lookup(id, out, v, t, rank_it);
+            if (__any_sync(0xffffffffu, rank_it)) {
+                const int cm = t.y >> 16;
+                const unsigned m = match_key(rank_it ? cm : -1, nb);
+                const int before = __popc(m & lanemask_lt());
+                if (rank_it) {
+                    const int j = v + before;
+                    int k = (t.y & 0xffff) - 1;
+                    while (k > 0 && s.rc[t.x + k].x > j) --k;
+                    out = s.rc[t.x + k].y;
+                }
+                __syncwarp();
+                if (rank_it && before == 0) s.code[warp * M + cm] = v + __popc(m);
+                __syncwarp();
+            }
+            if (i < whi) phys[i] = out;
+        };
+
+        // Pass 2: replica of every (t, k).
+        if (vec) {
+            // Blocks of 128 ids, four per lane: when no id of the block needs its
+            // occurrence index, one 16-byte store per lane; otherwise the block is
+            // replayed as four ordered scalar steps.
+            for (int64_t v0 = wlo; v0 < whi; v0 += 128) {
+                const int64_t i = v0 + 4 * lane;
+                const int4 q = i < whi ? *reinterpret_cast<const int4 *>(s.stage + (i - lo)) : make_int4(-1, -1, -1, -1);
+                int o0, o1, o2, o3, v;
+                int2 t;
+                bool r0, r1, r2, r3;
+                lookup(q.x, o0, v, t, r0);
+                lookup(q.y, o1, v, t, r1);
+                lookup(q.z, o2, v, t, r2);
+                lookup(q.w, o3, v, t, r3);
+                if (!__any_sync(0xffffffffu, r0 || r1 || r2 || r3)) {
+                    if (i < whi) *reinterpret_cast<int4 *>(phys + i) = make_int4(o0, o1, o2, o3);
+                } else {
+    #pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int64_t iu = v0 + 32 * u + lane;
+                        step(iu < whi ? s.stage[iu - lo] : -1, iu);
+                    }
+                }
+            }
+        } else {
+            for (int64_t x0 = wlo; x0 < whi; x0 += 32 * kUnroll) {
+                int id[kUnroll];
+    #pragma unroll
+                for (int u = 0; u < kUnroll; ++u) {
+                    const int64_t i = x0 + u * 32 + lane;
+                    id[u] = i >= whi ? -1 : (staged ? s.stage[i - lo] : __ldg(ids + i));
+                }
+    #pragma unroll
+                for (int u = 0; u < kUnroll; ++u) step(id[u], x0 + u * 32 + lane);
+            }
         }
     }
     cluster_wait();            // keep this CTA's shared memory alive for its peers
@@ -297,23 +517,55 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
 
 }  // namespace
 
-size_t reroute_smem_bytes(const Shape &sh) { return reroute_smem_words(sh.E, sh.E + sh.NR) * sizeof(int32_t); }
+size_t reroute_smem_bytes(const Shape &sh, bool dispatch, int stage_cap, bool gates)
+{
+    const int cap = sh.E + sh.NR;
+    return reroute_smem_words(sh.E, cap, dispatch ? sh.S : 0, stage_cap, dispatch && gates ? stage_cap : 0) *
+           sizeof(int32_t);
+}
+
+namespace {
+// The ids of a CTA are kept in shared memory between the passes when the
+// staging buffer fits beside the tables.
+int stage_cap_for(const Shape &sh, const Launch &ln, bool dispatch, bool gates)
+{
+    return reroute_smem_bytes(sh, dispatch, kStageIds, gates) <= ln.max_smem ? kStageIds : 0;
+}
+}  // namespace
 
 cudaError_t launch_reroute(const Shape &sh, const Launch &ln, const int32_t *ids, const PlanDev &plan,
                            int32_t *phys, cudaStream_t st, bool pdl)
 {
-    return launch_ex(k_reroute, (unsigned)(sh.N * ln.cluster), kRerouteWarps * 32, reroute_smem_bytes(sh), st,
-                     (unsigned)ln.cluster, pdl, ids, sh.per_rank, sh.E, sh.E + sh.NR, plan.rep_off, plan.rep_slot,
-                     plan.rep_cum, plan.rep_experts, plan.info, plan.rank_off, phys);
+    const int stage = stage_cap_for(sh, ln, false, false);
+    return launch_ex(k_reroute<false>, (unsigned)(sh.N * ln.cluster), kRerouteWarps * 32,
+                     reroute_smem_bytes(sh, false, stage, false), st, (unsigned)ln.cluster, pdl, ids, sh.per_rank, sh.E,
+                     sh.E + sh.NR, plan.rep_off, plan.rep_slot, plan.rep_cum, plan.rep_experts, plan.info,
+                     plan.rank_off, phys, stage, DispatchArgs{});
+}
+
+cudaError_t launch_dispatch(const Shape &sh, const Launch &ln, const int32_t *ids, const PlanDev &plan,
+                            int32_t *phys, const DispatchOut &out, int32_t *dev_err, cudaStream_t st, bool pdl)
+{
+    const bool gates = out.gates != nullptr;
+    const int stage = stage_cap_for(sh, ln, true, gates);
+    const DispatchArgs da{out.gates, plan.slot_quota, out.slot_off, out.src_index, out.gates_out, dev_err,
+                          sh.N * sh.per_rank, sh.S};
+    return launch_ex(k_reroute<true>, (unsigned)(sh.N * ln.cluster), kRerouteWarps * 32,
+                     reroute_smem_bytes(sh, true, stage, gates), st, (unsigned)ln.cluster, pdl, ids, sh.per_rank, sh.E,
+                     sh.E + sh.NR, plan.rep_off, plan.rep_slot, plan.rep_cum, plan.rep_experts, plan.info,
+                     plan.rank_off, phys, stage, da);
 }
 
 cudaError_t set_reroute_attributes(size_t max_smem)
 {
-    cudaError_t e = allow_smem(k_reroute, max_smem);
     // The largest shared-memory split, so that two CTAs per SM fit and the grid
     // runs in one wave beside the planner (the default split may leave room for one).
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_reroute, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    return e;
+    for (auto k : {k_reroute<false>, k_reroute<true>}) {
+        cudaError_t e = allow_smem(k, max_smem);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace ue

@@ -24,8 +24,8 @@ PLAN_FIELDS = ("slot_expert", "slot_quota", "rep_off", "rep_slot", "rep_cum", "r
 
 # Entry points declared in include/ue.h (checked against the header by the tests).
 EXPORTS = ("ue_plan_sizes", "ue_ctx_create", "ue_ctx_destroy", "ue_ctx_device_error", "ue_load",
-           "ue_plan", "ue_reroute", "ue_rebalance", "ue_sync", "ue_grad_reduce",
-           "ue_status_string", "ue_last_error")
+           "ue_plan", "ue_reroute", "ue_rebalance", "ue_dispatch", "ue_rebalance_dispatch", "ue_sync",
+           "ue_grad_reduce", "ue_status_string", "ue_last_error")
 
 
 class UeConfig(ctypes.Structure):
@@ -35,6 +35,11 @@ class UeConfig(ctypes.Structure):
 
 class UePlanBuffers(ctypes.Structure):
     _fields_ = [(f, ctypes.c_void_p) for f in PLAN_FIELDS]
+
+
+class UeDispatchBuffers(ctypes.Structure):
+    _fields_ = [("gates", ctypes.c_void_p), ("slot_off", ctypes.c_void_p), ("src_index", ctypes.c_void_p),
+                ("gates_out", ctypes.c_void_p)]
 
 
 class UeError(RuntimeError):
@@ -58,6 +63,7 @@ def lib() -> ctypes.CDLL:
             L = ctypes.CDLL(LIB_PATH)
             vp, i64, ci = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
             cfgp, planp = ctypes.POINTER(UeConfig), ctypes.POINTER(UePlanBuffers)
+            dispp = ctypes.POINTER(UeDispatchBuffers)
             sig = {
                 "ue_plan_sizes": [cfgp, ctypes.POINTER(ctypes.c_int64)],
                 "ue_ctx_create": [ci, ctypes.POINTER(vp)],
@@ -67,6 +73,8 @@ def lib() -> ctypes.CDLL:
                 "ue_plan": [vp, cfgp, vp, planp, vp],
                 "ue_reroute": [vp, cfgp, vp, planp, vp, vp],
                 "ue_rebalance": [vp, cfgp, vp, vp, vp, planp, vp, vp],
+                "ue_dispatch": [vp, cfgp, vp, planp, vp, dispp, vp],
+                "ue_rebalance_dispatch": [vp, cfgp, vp, vp, vp, planp, vp, dispp, vp],
                 "ue_sync": [vp, cfgp, vp, i64, planp, vp],
                 "ue_grad_reduce": [vp, cfgp, vp, vp, ci, i64, planp, vp],
             }
@@ -207,6 +215,43 @@ def ue_rebalance(ctx: Context, cfg: Config, ids: torch.Tensor, counts: torch.Ten
                  bad: torch.Tensor | None, plan: Plan, phys: torch.Tensor, stream=None) -> None:
     _check(lib().ue_rebalance(ctx.handle, ctypes.byref(cfg.c()), _ptr(ids), _ptr(counts), _ptr(bad),
                               plan.ref(), _ptr(phys), _stream(stream)), "ue_rebalance")
+
+
+class Dispatch:
+    """Device buffers of one dispatch layout: slot_off [S+1], src_index [T*K]
+    and, when gates are carried, gates_out [T*K] (torch tensors)."""
+
+    def __init__(self, cfg: Config, with_gates: bool = True, device="cuda"):
+        L = cfg.T * cfg.K
+        self.slot_off = torch.empty(cfg.S + 1, dtype=torch.int32, device=device)
+        self.src_index = torch.empty(L, dtype=torch.int32, device=device)
+        self.gates_out = torch.empty(L, dtype=torch.float32, device=device) if with_gates else None
+
+    def buffers(self, gates: torch.Tensor | None) -> UeDispatchBuffers:
+        if gates is not None and self.gates_out is None:
+            raise ValueError("this Dispatch was made without a gates_out buffer")
+        return UeDispatchBuffers(_ptr(gates), _ptr(self.slot_off), _ptr(self.src_index),
+                                 _ptr(self.gates_out) if gates is not None else None)
+
+    def nbytes(self, with_gates: bool = True) -> int:
+        n = (self.slot_off.numel() + self.src_index.numel()) * 4
+        return n + (self.gates_out.numel() * 4 if with_gates and self.gates_out is not None else 0)
+
+
+def ue_dispatch(ctx: Context, cfg: Config, ids: torch.Tensor, plan: Plan, phys: torch.Tensor,
+                disp: Dispatch, gates: torch.Tensor | None = None, stream=None) -> None:
+    b = disp.buffers(gates)
+    _check(lib().ue_dispatch(ctx.handle, ctypes.byref(cfg.c()), _ptr(ids), plan.ref(), _ptr(phys),
+                             ctypes.byref(b), _stream(stream)), "ue_dispatch")
+
+
+def ue_rebalance_dispatch(ctx: Context, cfg: Config, ids: torch.Tensor, counts: torch.Tensor,
+                          bad: torch.Tensor | None, plan: Plan, phys: torch.Tensor, disp: Dispatch,
+                          gates: torch.Tensor | None = None, stream=None) -> None:
+    b = disp.buffers(gates)
+    _check(lib().ue_rebalance_dispatch(ctx.handle, ctypes.byref(cfg.c()), _ptr(ids), _ptr(counts), _ptr(bad),
+                                       plan.ref(), _ptr(phys), ctypes.byref(b), _stream(stream)),
+           "ue_rebalance_dispatch")
 
 
 def ue_sync(ctx: Context, cfg: Config, weights: torch.Tensor, slot_bytes: int, plan: Plan,

@@ -150,3 +150,32 @@ def test_null_context_refused(L):
     assert L.ue_load(None, ctypes.byref(c), ids.ctypes.data, counts.ctypes.data, None, None) == 1
     assert "context" in L.ue_last_error().decode()
     assert (counts == 7).all()
+
+
+def test_dispatch_refusals(L):
+    hp = _HostPlan()
+    c = ue.UeConfig(16, 4, 1, 8, 64)
+    ids = np.zeros(64 * 8 + 4, np.int32)
+    ids_p = ids.ctypes.data + (-ids.ctypes.data % 16)
+    phys = np.full(512, 7, np.int32)
+    slot_off = np.full(21, 7, np.int32)
+    src = np.full(512, 7, np.int32)
+    gates = np.zeros(512, np.float32)
+    counts = np.zeros(64, np.int32)
+
+    def call(d, ids_ptr=ids_p, rebalance=False):
+        if rebalance:
+            return L.ue_rebalance_dispatch(FAKE_CTX, ctypes.byref(c), ids_ptr, counts.ctypes.data, None,
+                                           ctypes.byref(hp.c), phys.ctypes.data, d, None)
+        return L.ue_dispatch(FAKE_CTX, ctypes.byref(c), ids_ptr, ctypes.byref(hp.c), phys.ctypes.data, d, None)
+
+    assert call(None) == 1 and "dispatch buffers" in L.ue_last_error().decode()
+    d = ue.UeDispatchBuffers(None, None, src.ctypes.data, None)
+    assert call(ctypes.byref(d)) == 1 and "slot_off" in L.ue_last_error().decode()
+    d = ue.UeDispatchBuffers(gates.ctypes.data, slot_off.ctypes.data, src.ctypes.data, None)
+    assert call(ctypes.byref(d)) == 1 and "gates_out" in L.ue_last_error().decode()
+    d = ue.UeDispatchBuffers(None, slot_off.ctypes.data, None, None)
+    assert call(ctypes.byref(d), rebalance=True) == 1 and "src_index" in L.ue_last_error().decode()
+    d = ue.UeDispatchBuffers(None, slot_off.ctypes.data, src.ctypes.data, None)
+    assert call(ctypes.byref(d), ids_ptr=ids_p + 4) == 1 and "aligned" in L.ue_last_error().decode()
+    assert hp.untouched() and (phys == 7).all() and (slot_off == 7).all() and (src == 7).all()
