@@ -26,6 +26,10 @@ Pinning status (what fixes each function other than itself; the tests under
   sync          byte-map conservation: every byte of every filled redundant
                 slot comes from the right home byte exactly once, other slots
                 untouched.
+  sync_delta    byte map over a microbatch sequence: after a sync under the
+                previous plan, the incremental sync leaves exactly the state a
+                full sync gives; slots whose expert is unchanged are untouched;
+                the copied-slot count equals a numpy count.
   grad_reduce   exact closed-form sums on dyadic values; zero gradients
                 leave the master unchanged; numpy float32 reference order.
 
@@ -74,9 +78,11 @@ def _get():
             lib.ue_oracle_reroute.argtypes = [vp, i64, ci, ci, vp, vp, vp, vp, vp]
             lib.ue_oracle_dispatch.argtypes = [vp, i64, ci, vp, vp, vp, vp]
             lib.ue_oracle_sync.argtypes = [vp, i64, i64, ci, ci, ci, vp]
+            lib.ue_oracle_sync_delta.argtypes = [vp, i64, i64, ci, ci, ci, vp, vp, vp]
             lib.ue_oracle_grad_reduce.argtypes = [vp, i64, vp, ci, i64, i64, ci, ci, ci, vp, vp]
             for f in ("ue_oracle_load", "ue_oracle_expert_load", "ue_oracle_plan",
-                      "ue_oracle_reroute", "ue_oracle_dispatch", "ue_oracle_sync", "ue_oracle_grad_reduce"):
+                      "ue_oracle_reroute", "ue_oracle_dispatch", "ue_oracle_sync",
+                      "ue_oracle_sync_delta", "ue_oracle_grad_reduce"):
                 getattr(lib, f).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -180,6 +186,22 @@ def sync(W: np.ndarray, nbytes: int, E: int, N: int, R: int, slot_expert: np.nda
     stride = W.shape[1] * W.itemsize
     rc = _get().ue_oracle_sync(_p(W), stride, nbytes, E, N, R, _p(_c(slot_expert, np.int32)))
     _check(rc, "sync")
+
+
+def sync_delta(W: np.ndarray, nbytes: int, E: int, N: int, R: int, slot_expert: np.ndarray,
+               prev_slot_expert: np.ndarray | None) -> int:
+    """Step 4, incremental: copies only filled redundant slots whose expert
+    differs from the previous plan's (all of them when prev is None); returns
+    the number of slots copied."""
+    if not (W.flags.c_contiguous and W.ndim == 2):
+        raise OracleError("W must be a C-contiguous [S][stride] array")
+    stride = W.shape[1] * W.itemsize
+    n = ctypes.c_int64(0)
+    prev = None if prev_slot_expert is None else _c(prev_slot_expert, np.int32)
+    rc = _get().ue_oracle_sync_delta(_p(W), stride, nbytes, E, N, R, _p(_c(slot_expert, np.int32)), _p(prev),
+                                     ctypes.byref(n))
+    _check(rc, "sync_delta")
+    return int(n.value)
 
 
 def grad_reduce(master: np.ndarray, grads: np.ndarray, n: int, E: int, N: int, R: int,

@@ -346,6 +346,34 @@ int ue_oracle_sync(uint8_t *W, int64_t slot_stride, int64_t nbytes,
     return ORC_OK;
 }
 
+/* ---- step 4, incremental form ---------------------------------------------
+ * Within one training step the expert weights do not change between
+ * microbatches, so a redundant slot that held expert e under the previous
+ * microbatch's plan (prev_slot_expert[s] = e) already holds e's home weights:
+ * only filled redundant slots whose expert differs from prev are copied.  With
+ * prev_slot_expert NULL every filled redundant slot is copied (a full sync,
+ * as after the optimizer step).  *copied = number of slots copied.
+ */
+int ue_oracle_sync_delta(uint8_t *W, int64_t slot_stride, int64_t nbytes,
+                         int E, int N, int R, const int32_t *slot_expert,
+                         const int32_t *prev_slot_expert, int64_t *copied)
+{
+    if (E < 1 || N < 1 || R < 0 || E % N != 0 || nbytes > slot_stride || nbytes < 0) return ORC_BAD_ARG;
+    const int H = E / N, HR = H + R, S = N * HR;
+    int64_t n = 0;
+    for (int s = 0; s < S; ++s) {
+        int e = slot_expert[s];
+        if (s % HR < H || e < 0) continue;
+        if (e >= E) return ORC_BAD_ARG;
+        if (prev_slot_expert && prev_slot_expert[s] == e) continue;
+        int64_t home = (int64_t)(e / H) * HR + (e % H);
+        memcpy(W + (int64_t)s * slot_stride, W + home * slot_stride, (size_t)nbytes);
+        ++n;
+    }
+    if (copied) *copied = n;
+    return ORC_OK;
+}
+
 /* ---- step 5: replica gradient reduction -----------------------------------
  * For each expert e with redundant replicas, in replica order i = 1, 2, ...:
  *     master[e][x] = master[e][x] + float(grad[g(i)][x])

@@ -279,3 +279,51 @@ def test_grad_reduce_zero_grads_identity_and_order():
             s = pl["rep_slot"][i]
             ref[e] = np.add(ref[e], g[(s // HR) * R + (s % HR - H)], dtype=np.float32)
     assert np.array_equal(out, ref)
+
+
+# ---- weight sync, incremental form -----------------------------------------------
+
+def _plans_sequence(E, N, R, n, seed):
+    rng = np.random.default_rng(seed)
+    out = []
+    for _ in range(n):
+        p = rng.permutation(E) + 1.0
+        ld = rng.multinomial(4000, (p ** -1.5) / (p ** -1.5).sum()).astype(np.int32)
+        out.append(oracle.plan(ld, N, R))
+    return out
+
+
+@pytest.mark.parametrize("R", [1, 2])
+def test_sync_delta_equals_full_sync_state(R):
+    """After a sync under plan A, the incremental sync under plan B (prev = A)
+    must leave the bytes a full sync under B leaves; slots whose expert did not
+    change are not written; the copy count is the numpy count of changed slots."""
+    E, N = 16, 4
+    H, HR = E // N, E // N + R
+    S, B = N * HR, 512
+    plans = _plans_sequence(E, N, R, 6, seed=R)
+    W = _tagged_slots(S, B)
+    assert oracle.sync_delta(W, B, E, N, R, plans[0]["slot_expert"], None) == plans[0]["info"][4]
+    for a, b in zip(plans, plans[1:]):
+        full = W.copy()
+        oracle.sync(full, B, E, N, R, b["slot_expert"])
+        before = W.copy()
+        n = oracle.sync_delta(W, B, E, N, R, b["slot_expert"], a["slot_expert"])
+        assert np.array_equal(W, full)
+        red = (np.arange(S) % HR) >= H
+        changed = red & (b["slot_expert"] >= 0) & (b["slot_expert"] != a["slot_expert"])
+        assert n == int(changed.sum())
+        assert np.array_equal(W[~changed], before[~changed])      # unchanged slots untouched
+
+
+def test_sync_delta_same_plan_copies_nothing_and_none_is_full():
+    E, N, R = 8, 4, 1
+    pl = oracle.plan(np.array([40, 1, 1, 1, 1, 1, 1, 9], np.int32), N, R)
+    S, B = N * (E // N + R), 256
+    W = _tagged_slots(S, B)
+    before = W.copy()
+    assert oracle.sync_delta(W, B, E, N, R, pl["slot_expert"], pl["slot_expert"]) == 0
+    assert np.array_equal(W, before)
+    n = oracle.sync_delta(W, B, E, N, R, pl["slot_expert"], None)
+    assert n == pl["info"][4] > 0
+    assert _byte_map_check(before, W, E, N, R, pl["slot_expert"])
