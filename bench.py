@@ -84,6 +84,8 @@ def parse_args(argv=None):
     ap.add_argument("--sweep", action="store_true",
                     help="rebalance latency and imbalance over the sweep grid (one JSON line per point)")
     ap.add_argument("--sweep-seeds", type=int, default=1)
+    ap.add_argument("--stationary", action="store_true",
+                    help="keep the expert popularity fixed across microbatches (no re-permutation)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args(argv)
@@ -213,6 +215,8 @@ def run_ours(args, dist: Dist):
     dev = torch.device("cuda", dist.local_rank)
     dist.init("nccl")
     w = inputs.WORKLOADS[args.workload].with_(base_seed=dist.rank)
+    if args.stationary:
+        w = w.with_(repermute=False)
     if args.expert_shape:
         rows, cols = (int(x) for x in args.expert_shape.lower().split("x"))
         w = w.with_(rows=rows, cols=cols)
@@ -367,7 +371,8 @@ def run_ours(args, dist: Dist):
             stream.synchronize()
             info = plan["info"].cpu().numpy()
             per_mb.append({"Q": int(info[0]), "L": int(info[1]), "ran_out": int(info[2] & 1), "M": int(info[3]),
-                           "filled": int(info[4]), "max_before": int(info[5]), "max_after": int(info[6])})
+                           "filled": int(info[4]), "max_before": int(info[5]), "max_after": int(info[6]),
+                           "slot_expert": plan["slot_expert"].cpu().numpy()})
     gsize = 2 if w.grad_dtype == "bf16" else 4
     sync_bytes = np.array([(p["M"] + p["filled"]) * slot_bytes for p in per_mb], dtype=np.float64)
     grad_bytes = np.array([p["M"] * P * 8 + p["filled"] * P * gsize for p in per_mb], dtype=np.float64)
@@ -375,6 +380,36 @@ def run_ours(args, dist: Dist):
     sync_gbs = sync_bytes[step_mb].sum() / (seg[:, 1].sum() * 1e-6) / 1e9
     grad_gbs = grad_bytes[step_mb].sum() / (seg[:, 2].sum() * 1e-6) / 1e9
     rebalance_alg_bytes = 3.0 * w.L * 4
+
+    # Incremental weight sync over the microbatch sequence of one training
+    # step: the first microbatch syncs in full, each later one copies only the
+    # redundant slots whose expert changed; two plan buffers alternate.
+    plans2 = [plan, ue.Plan(cfg, device=dev)]
+    evs_d = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_mb)]
+    with torch.cuda.stream(stream):
+        for mb in range(n_mb):
+            cur, prv = plans2[mb % 2], plans2[(mb + 1) % 2]
+            ue.ue_rebalance(ctx, cfg, ids_dev[mb], counts, bad, cur, phys, stream=stream)
+            evs_d[mb][0].record(stream)
+            ue.ue_sync_delta(ctx, cfg, weights, slot_bytes, cur, None if mb == 0 else prv["slot_expert"],
+                             stream=stream)
+            evs_d[mb][1].record(stream)
+    stream.synchronize()
+    red = (np.arange(w.S) % (w.H + w.R)) >= w.H
+    delta_bytes = 0
+    for mb in range(n_mb):
+        se = per_mb[mb]["slot_expert"]
+        ch = red & (se >= 0)
+        if mb:
+            ch &= se != per_mb[mb - 1]["slot_expert"]
+        delta_bytes += (len(np.unique(se[ch])) + int(ch.sum())) * slot_bytes
+    delta_full = float(sync_bytes.sum())
+    delta_us = float(sum(a.elapsed_time(b) for a, b in evs_d)) * 1e3
+    sync_delta = {"microbatches": n_mb, "bytes_full": int(delta_full), "bytes_delta": int(delta_bytes),
+                  "saved_frac": round(1.0 - delta_bytes / delta_full, 4) if delta_full else None,
+                  "us_total": round(delta_us, 1),
+                  "gbs": round(delta_bytes / (delta_us * 1e-6) / 1e9, 1) if delta_us > 0 else None}
+    del plans2
 
     # Launch floor: one tiny kernel bracketed by events on the same stream.
     tiny = torch.zeros(1, device=dev)
@@ -450,6 +485,7 @@ def run_ours(args, dist: Dist):
         "config": {"workload": w.name, "E": w.E, "N": w.N, "H": w.H, "R": w.R, "K": w.K, "T": w.T,
                    "P": P, "slot_bytes": slot_bytes, "grad_dtype": w.grad_dtype, "zipf_s": w.s,
                    "microbatches_cycled": n_mb, "parallelism": f"replicas x{dist.world}",
+                   "popularity": "re-drawn every microbatch" if w.repermute else "stationary",
                    "l2": "inputs larger than L2: every step streams > 1 GB (sync + grad reduce), "
                          "so each rebalance reads its ids from HBM"},
         "breakdown_us": {
@@ -474,6 +510,7 @@ def run_ours(args, dist: Dist):
         "sync_gbs": round(sync_gbs, 1), "sync_frac": round(sync_gbs / peak, 4),
         "grad_reduce_gbs": round(grad_gbs, 1), "grad_reduce_frac": round(grad_gbs / peak, 4),
         "frac_of_8000_gbs": {"sync": round(sync_gbs / 8000, 4), "grad_reduce": round(grad_gbs / 8000, 4)},
+        "sync_delta": sync_delta,
         "imbalance": {
             "before": round(float(np.mean([p["max_before"] / (p["L"] / w.N) for p in per_mb])), 4),
             "after": round(float(np.mean([p["max_after"] / (p["L"] / w.N) for p in per_mb])), 4),

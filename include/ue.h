@@ -178,6 +178,16 @@ ue_status ue_rebalance_dispatch(ue_ctx *ctx, const ue_config *cfg, const int32_t
 ue_status ue_sync(ue_ctx *ctx, const ue_config *cfg, void *weights, int64_t slot_bytes,
                   const ue_plan_buffers *plan, void *stream);
 
+/* Incremental weight sync for the microbatches of one training step, whose
+ * expert weights do not change between microbatches: a filled redundant slot
+ * whose expert equals prev_slot_expert[s] (the previous microbatch's
+ * plan.slot_expert, [S] device memory, read only) already holds that expert's
+ * weights and is not written; every other filled redundant slot is copied as
+ * in ue_sync.  prev_slot_expert = NULL gives the full sync (the first
+ * microbatch after an optimizer step). */
+ue_status ue_sync_delta(ue_ctx *ctx, const ue_config *cfg, void *weights, int64_t slot_bytes,
+                        const ue_plan_buffers *plan, const int32_t *prev_slot_expert, void *stream);
+
 /* ---- step 5: replica gradient reduction ------------------------------------
  * "Replica gradient reduction" (csrc/kernels/grad_reduce.cu; "Expert compute
  * -> Replica gradient reduction: replica gradients", "-> MoE framework:

@@ -372,8 +372,9 @@ ue_status ue_rebalance_dispatch(ue_ctx *ctx, const ue_config *cfg, const int32_t
     });
 }
 
-ue_status ue_sync(ue_ctx *ctx, const ue_config *cfg, void *weights, int64_t slot_bytes, const ue_plan_buffers *plan,
-                  void *stream)
+namespace {
+ue_status sync_common(ue_ctx *ctx, const ue_config *cfg, void *weights, int64_t slot_bytes,
+                      const ue_plan_buffers *plan, const int32_t *prev, void *stream)
 {
     ue::Shape sh{};
     ue_status s = make_shape(cfg, false, &sh);
@@ -388,9 +389,22 @@ ue_status ue_sync(ue_ctx *ctx, const ue_config *cfg, void *weights, int64_t slot
                     ctx->max_smem);
     return on_device(ctx, [&]() -> ue_status {
         cudaError_t e = ue::launch_sync(sh, launch_of(ctx, sh), static_cast<uint8_t *>(weights), slot_bytes,
-                                        ue::to_dev(*plan), ctx->dev_err, static_cast<cudaStream_t>(stream));
+                                        ue::to_dev(*plan), prev, ctx->dev_err, static_cast<cudaStream_t>(stream));
         return e == cudaSuccess ? UE_OK : cuda_fail(e, "sync launch");
     });
+}
+}  // namespace
+
+ue_status ue_sync(ue_ctx *ctx, const ue_config *cfg, void *weights, int64_t slot_bytes, const ue_plan_buffers *plan,
+                  void *stream)
+{
+    return sync_common(ctx, cfg, weights, slot_bytes, plan, nullptr, stream);
+}
+
+ue_status ue_sync_delta(ue_ctx *ctx, const ue_config *cfg, void *weights, int64_t slot_bytes,
+                        const ue_plan_buffers *plan, const int32_t *prev_slot_expert, void *stream)
+{
+    return sync_common(ctx, cfg, weights, slot_bytes, plan, prev_slot_expert, stream);
 }
 
 ue_status ue_grad_reduce(ue_ctx *ctx, const ue_config *cfg, float *master, const void *grads, int grad_dtype,

@@ -67,8 +67,9 @@ cudaError_t launch_dispatch(const Shape &sh, const Launch &ln, const int32_t *id
 // many gates when the dispatch variant carries them.
 size_t reroute_smem_bytes(const Shape &sh, bool dispatch, int stage_cap, bool gates);
 
+// prev_slot_expert: the previous plan's slot_expert for the incremental form, or nullptr.
 cudaError_t launch_sync(const Shape &sh, const Launch &ln, uint8_t *weights, int64_t slot_bytes,
-                        const PlanDev &plan, int32_t *dev_err, cudaStream_t st);
+                        const PlanDev &plan, const int32_t *prev_slot_expert, int32_t *dev_err, cudaStream_t st);
 size_t sync_smem_bytes(const Shape &sh);
 
 cudaError_t launch_grad_reduce(const Shape &sh, const Launch &ln, float *master, const void *grads,

@@ -15,6 +15,11 @@
 // Stage reuse waits on cp.async.bulk.wait_group.read.  No multicast anywhere.
 // Every mbarrier wait is bounded by the global timer; on timeout the kernel
 // records an error in the context's status word, drains its stores and exits.
+//
+// Incremental form: given the previous microbatch's slot_expert, a redundant
+// slot that already held its expert is not copied (the expert weights do not
+// change between the microbatches of one training step), and experts left
+// with nothing to copy produce no work items.
 #include "ue_internal.cuh"
 
 namespace ue {
@@ -92,7 +97,7 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
 k_sync(uint8_t *__restrict__ W, int64_t slot_bytes, int E, int S, int cap,
        const int32_t *__restrict__ rep_off, const int32_t *__restrict__ rep_slot,
        const int32_t *__restrict__ rep_experts, const int32_t *__restrict__ info,
-       int32_t *__restrict__ dev_err)
+       const int32_t *__restrict__ prev, int32_t *__restrict__ dev_err)
 {
     extern __shared__ __align__(128) uint8_t sm_sync[];
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm_sync);                 // [stages]
@@ -100,8 +105,11 @@ k_sync(uint8_t *__restrict__ W, int64_t slot_bytes, int E, int S, int cap,
     int32_t *x_home = reinterpret_cast<int32_t *>(stage + (size_t)kSyncStages * kSyncTile);  // [E]
     int32_t *x_first = x_home + E;                                         // [E] first redundant entry
     int32_t *x_cnt = x_first + E;                                          // [E] redundant replicas
-    int32_t *x_slot = x_cnt + E;                                           // [cap]
+    int32_t *x_slot = x_cnt + E;                                           // [cap] slots to write
+    int32_t *x_act = x_slot + cap;                                         // [E+1] experts with work; count
 
+    // Per replicated expert: its home slot and the redundant slots to write
+    // (all of them, or those whose expert changed since the previous plan).
     const int M = clampi(__ldg(info + 3), 0, E);
     for (int m = threadIdx.x; m < M; m += blockDim.x) {
         const int e = clampi(__ldg(rep_experts + m), 0, E - 1);
@@ -109,26 +117,44 @@ k_sync(uint8_t *__restrict__ W, int64_t slot_bytes, int E, int S, int cap,
         const int end = clampi(__ldg(rep_off + e + 1), off + 1, cap);
         x_home[m] = clampi(__ldg(rep_slot + off), 0, S - 1);
         x_first[m] = off + 1;
-        x_cnt[m] = end - off - 1;
+        int c = 0;
+        for (int p = off + 1; p < end; ++p) {
+            const int slot = clampi(__ldg(rep_slot + p), 0, S - 1);
+            if (prev == nullptr || __ldg(prev + slot) != e) x_slot[off + 1 + c++] = slot;
+        }
+        x_cnt[m] = c;
     }
-    for (int p = threadIdx.x; p < cap; p += blockDim.x) x_slot[p] = clampi(__ldg(rep_slot + p), 0, S - 1);
     if (threadIdx.x == 0) {
         for (int i = 0; i < kSyncStages; ++i) mbar_init(&bar[i], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
-    if (threadIdx.x != 0 || M == 0) return;
+    if (threadIdx.x < 32) {                  // compact the experts that have slots to write
+        const int lane = threadIdx.x;
+        int n = 0;
+        for (int m0 = 0; m0 < M; m0 += 32) {
+            const int m = m0 + lane;
+            const bool a = m < M && x_cnt[m] > 0;
+            const unsigned b = __ballot_sync(0xffffffffu, a);
+            if (a) x_act[n + __popc(b & lanemask_lt())] = m;
+            n += __popc(b);
+        }
+        if (lane == 0) x_act[E] = n;
+    }
+    __syncthreads();
+    const int MA = x_act[E];
+    if (threadIdx.x != 0 || MA == 0) return;
 
     const int64_t ntiles = (slot_bytes + kSyncTile - 1) / kSyncTile;
-    const int64_t total = (int64_t)M * ntiles;
+    const int64_t total = (int64_t)MA * ntiles;
     if ((int64_t)blockIdx.x >= total) return;
     const int64_t nmy = (total - 1 - blockIdx.x) / gridDim.x + 1;
 
     auto item = [&](int64_t k) {
         const int64_t i = (int64_t)blockIdx.x + k * gridDim.x;
         SyncItem it;
-        it.m = (int)(i % M);
-        const int64_t t = i / M;
+        it.m = x_act[(int)(i % MA)];
+        const int64_t t = i / MA;
         it.offset = t * kSyncTile;
         const int64_t left = slot_bytes - it.offset;
         it.bytes = (unsigned)(left < kSyncTile ? left : kSyncTile);
@@ -175,15 +201,15 @@ k_sync(uint8_t *__restrict__ W, int64_t slot_bytes, int E, int S, int cap,
 
 size_t sync_smem_bytes(const Shape &sh)
 {
-    return 128 + (size_t)kSyncStages * kSyncTile + (size_t)(3 * sh.E + sh.E + sh.NR) * sizeof(int32_t);
+    return 128 + (size_t)kSyncStages * kSyncTile + (size_t)(3 * sh.E + sh.E + sh.NR + sh.E + 1) * sizeof(int32_t);
 }
 
 cudaError_t launch_sync(const Shape &sh, const Launch &ln, uint8_t *weights, int64_t slot_bytes,
-                        const PlanDev &plan, int32_t *dev_err, cudaStream_t st)
+                        const PlanDev &plan, const int32_t *prev_slot_expert, int32_t *dev_err, cudaStream_t st)
 {
     k_sync<<<ln.sms, kSyncThreads, sync_smem_bytes(sh), st>>>(weights, slot_bytes, sh.E, sh.S, sh.E + sh.NR,
                                                                plan.rep_off, plan.rep_slot, plan.rep_experts,
-                                                               plan.info, dev_err);
+                                                               plan.info, prev_slot_expert, dev_err);
     return cudaGetLastError();
 }
 

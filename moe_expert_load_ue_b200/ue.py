@@ -24,7 +24,7 @@ PLAN_FIELDS = ("slot_expert", "slot_quota", "rep_off", "rep_slot", "rep_cum", "r
 
 # Entry points declared in include/ue.h (checked against the header by the tests).
 EXPORTS = ("ue_plan_sizes", "ue_ctx_create", "ue_ctx_destroy", "ue_ctx_device_error", "ue_load",
-           "ue_plan", "ue_reroute", "ue_rebalance", "ue_dispatch", "ue_rebalance_dispatch", "ue_sync",
+           "ue_plan", "ue_reroute", "ue_rebalance", "ue_dispatch", "ue_rebalance_dispatch", "ue_sync", "ue_sync_delta",
            "ue_grad_reduce", "ue_status_string", "ue_last_error")
 
 
@@ -76,6 +76,7 @@ def lib() -> ctypes.CDLL:
                 "ue_dispatch": [vp, cfgp, vp, planp, vp, dispp, vp],
                 "ue_rebalance_dispatch": [vp, cfgp, vp, vp, vp, planp, vp, dispp, vp],
                 "ue_sync": [vp, cfgp, vp, i64, planp, vp],
+                "ue_sync_delta": [vp, cfgp, vp, i64, planp, vp, vp],
                 "ue_grad_reduce": [vp, cfgp, vp, vp, ci, i64, planp, vp],
             }
             for name, args in sig.items():
@@ -258,6 +259,12 @@ def ue_sync(ctx: Context, cfg: Config, weights: torch.Tensor, slot_bytes: int, p
             stream=None) -> None:
     _check(lib().ue_sync(ctx.handle, ctypes.byref(cfg.c()), _ptr(weights), int(slot_bytes), plan.ref(),
                          _stream(stream)), "ue_sync")
+
+
+def ue_sync_delta(ctx: Context, cfg: Config, weights: torch.Tensor, slot_bytes: int, plan: Plan,
+                  prev_slot_expert: torch.Tensor | None, stream=None) -> None:
+    _check(lib().ue_sync_delta(ctx.handle, ctypes.byref(cfg.c()), _ptr(weights), int(slot_bytes), plan.ref(),
+                               _ptr(prev_slot_expert), _stream(stream)), "ue_sync_delta")
 
 
 def ue_grad_reduce(ctx: Context, cfg: Config, master: torch.Tensor, grads: torch.Tensor, P: int,

@@ -179,3 +179,14 @@ def test_dispatch_refusals(L):
     d = ue.UeDispatchBuffers(None, slot_off.ctypes.data, src.ctypes.data, None)
     assert call(ctypes.byref(d), ids_ptr=ids_p + 4) == 1 and "aligned" in L.ue_last_error().decode()
     assert hp.untouched() and (phys == 7).all() and (slot_off == 7).all() and (src == 7).all()
+
+
+def test_sync_delta_refusals(L):
+    hp = _HostPlan()
+    c = ue.UeConfig(16, 4, 1, 8, 64)
+    w = np.zeros(1024, np.uint8)
+    prev = np.zeros(20, np.int32)
+    assert L.ue_sync_delta(FAKE_CTX, ctypes.byref(c), w.ctypes.data, 24, ctypes.byref(hp.c),
+                           prev.ctypes.data, None) == 1
+    assert L.ue_sync_delta(FAKE_CTX, ctypes.byref(c), None, 32, ctypes.byref(hp.c), None, None) == 1
+    assert hp.untouched() and (w == 0).all()
