@@ -75,12 +75,13 @@ def _get():
             lib.ue_oracle_load.argtypes = [vp, i64, ci, ci, ci, vp, vp]
             lib.ue_oracle_expert_load.argtypes = [vp, ci, ci, vp, vp]
             lib.ue_oracle_plan.argtypes = [ci, ci, ci, vp] + [vp] * 9
+            lib.ue_oracle_plan_ex.argtypes = [ci, ci, ci, vp, ci] + [vp] * 9
             lib.ue_oracle_reroute.argtypes = [vp, i64, ci, ci, vp, vp, vp, vp, vp]
             lib.ue_oracle_dispatch.argtypes = [vp, i64, ci, vp, vp, vp, vp]
             lib.ue_oracle_sync.argtypes = [vp, i64, i64, ci, ci, ci, vp]
             lib.ue_oracle_sync_delta.argtypes = [vp, i64, i64, ci, ci, ci, vp, vp, vp]
             lib.ue_oracle_grad_reduce.argtypes = [vp, i64, vp, ci, i64, i64, ci, ci, ci, vp, vp]
-            for f in ("ue_oracle_load", "ue_oracle_expert_load", "ue_oracle_plan",
+            for f in ("ue_oracle_load", "ue_oracle_expert_load", "ue_oracle_plan", "ue_oracle_plan_ex",
                       "ue_oracle_reroute", "ue_oracle_dispatch", "ue_oracle_sync",
                       "ue_oracle_sync_delta", "ue_oracle_grad_reduce"):
                 getattr(lib, f).restype = ctypes.c_int
@@ -129,8 +130,13 @@ PLAN_FIELDS = ("slot_expert", "slot_quota", "rep_off", "rep_slot", "rep_cum", "r
                "rank_load_before", "rank_load_after", "info")
 
 
-def plan(load_e: np.ndarray, N: int, R: int) -> dict:
-    """Step 2: the quota-driven plan (see ue_oracle.c for the exact rule)."""
+REQUEUE, SPREAD = 1, 2     # plan variants (bit flags), see ue_oracle.c
+
+
+def plan(load_e: np.ndarray, N: int, R: int, variant: int = 0) -> dict:
+    """Step 2: the quota-driven plan (see ue_oracle.c for the exact rule and
+    the variants: REQUEUE re-queues partly placed experts, SPREAD spreads the
+    remainder of stuck experts over their replicas)."""
     load_e = _c(load_e, np.int32)
     E = load_e.shape[0]
     if E % N:
@@ -144,7 +150,7 @@ def plan(load_e: np.ndarray, N: int, R: int) -> dict:
         "rank_load_before": np.empty(N, np.int32), "rank_load_after": np.empty(N, np.int32),
         "info": np.empty(8, np.int32),
     }
-    rc = _get().ue_oracle_plan(E, N, R, _p(load_e), *[_p(out[f]) for f in PLAN_FIELDS])
+    rc = _get().ue_oracle_plan_ex(E, N, R, _p(load_e), int(variant), *[_p(out[f]) for f in PLAN_FIELDS])
     _check(rc, "plan")
     return out
 
@@ -220,10 +226,10 @@ def grad_reduce(master: np.ndarray, grads: np.ndarray, n: int, E: int, N: int, R
     _check(rc, "grad_reduce")
 
 
-def rebalance(ids: np.ndarray, E: int, N: int, R: int):
+def rebalance(ids: np.ndarray, E: int, N: int, R: int, variant: int = 0):
     """Steps 1-3 chained: counts, expert loads, rank offsets, plan, phys."""
     counts, bad = load(ids, E, N)
     ld, off = expert_load(counts)
-    pl = plan(ld, N, R)
+    pl = plan(ld, N, R, variant)
     phys = reroute(ids, E, pl)
     return {"counts": counts, "bad": bad, "load": ld, "rank_off": off, "plan": pl, "phys": phys}

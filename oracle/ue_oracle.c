@@ -110,14 +110,28 @@ static int orc_ovf_cmp(const void *a, const void *b)
     return x->e < y->e ? -1 : (x->e > y->e ? 1 : 0);         /* tie: lower expert id */
 }
 
-int ue_oracle_plan(int E, int N, int R, const int32_t *load,
-                   int32_t *slot_expert, int32_t *slot_quota,
-                   int32_t *rep_off, int32_t *rep_slot, int32_t *rep_cum,
-                   int32_t *rep_experts,
-                   int32_t *rank_load_before, int32_t *rank_load_after,
-                   int32_t *info)
+/* Plan variants (bit flags; 0 = the stated rule):
+ *   ORC_REQUEUE  the overflow is a priority queue: after every chunk the expert
+ *                with the largest remaining overflow (ties: lower id) is placed
+ *                next, instead of placing each expert fully in the order fixed
+ *                after the home pass;
+ *   ORC_SPREAD   when slots run out, each stuck expert's remainder (in the
+ *                order the experts are visited) is spread over its replicas one
+ *                token at a time, each token to the replica whose rank has the
+ *                lowest load (ties: the earlier replica, home first), instead of
+ *                staying on the home slot.
+ */
+#define ORC_REQUEUE 1
+#define ORC_SPREAD 2
+
+int ue_oracle_plan_ex(int E, int N, int R, const int32_t *load, int variant,
+                      int32_t *slot_expert, int32_t *slot_quota,
+                      int32_t *rep_off, int32_t *rep_slot, int32_t *rep_cum,
+                      int32_t *rep_experts,
+                      int32_t *rank_load_before, int32_t *rank_load_after,
+                      int32_t *info)
 {
-    if (E < 1 || N < 1 || R < 0 || E % N != 0) return ORC_BAD_ARG;
+    if (E < 1 || N < 1 || R < 0 || E % N != 0 || variant < 0 || variant > 3) return ORC_BAD_ARG;
     const int H = E / N, HR = H + R, S = N * HR, NR = N * R;
     int64_t L = 0;
     for (int e = 0; e < E; ++e) {
@@ -135,8 +149,10 @@ int ue_oracle_plan(int E, int N, int R, const int32_t *load,
     int32_t *asg_e = calloc((size_t)NR + 1, sizeof(int32_t)); /* assignments, allocation order */
     int32_t *asg_s = calloc((size_t)NR + 1, sizeof(int32_t));
     int64_t *asg_c = calloc((size_t)NR + 1, sizeof(int64_t));
+    int64_t *rem_e = calloc((size_t)E, sizeof(int64_t));      /* remaining overflow (variants) */
+    int32_t *stuck = calloc((size_t)E, sizeof(int32_t));      /* experts left with a remainder, in visit order */
     int rc = ORC_OK;
-    if (!cur || !used || !home_quota || !ovf || !order || !asg_e || !asg_s || !asg_c) {
+    if (!cur || !used || !home_quota || !ovf || !order || !asg_e || !asg_s || !asg_c || !rem_e || !stuck) {
         rc = ORC_BAD_ARG;
         goto done;
     }
@@ -157,35 +173,86 @@ int ue_oracle_plan(int E, int N, int R, const int32_t *load,
         if (ovf[e] > 0) { order[n_ovf].ovf = (int32_t)ovf[e]; order[n_ovf].e = e; ++n_ovf; }
     qsort(order, (size_t)n_ovf, sizeof(orc_ovf), orc_ovf_cmp);
 
-    /* Greedy: each chunk goes to the eligible rank with most spare capacity. */
-    for (int m = 0; m < n_ovf; ++m) {
-        int e = order[m].e, h = e / H;
-        int64_t rem = ovf[e];
-        while (rem > 0) {
-            int best = -1;
-            for (int r = 0; r < N; ++r) {
-                if (used[r] >= R || Q - cur[r] <= 0) continue;   /* not eligible */
-                if (best < 0 || Q - cur[r] > Q - cur[best]) best = r;   /* ties keep lowest r */
+    /* Greedy: each chunk goes to the eligible rank with most spare capacity,
+     * min(remaining, spare) tokens.  The stated rule places the experts one
+     * after the other in the fixed order; with ORC_REQUEUE the next chunk is
+     * always for the expert with the largest remaining overflow.  Experts
+     * still holding overflow when no rank is eligible are "stuck". */
+    int n_stuck = 0;
+    for (int e = 0; e < E; ++e) rem_e[e] = ovf[e];
+    int m_next = 0;                       /* fixed order: next expert to place */
+    for (;;) {
+        int e = -1;
+        if (variant & ORC_REQUEUE) {
+            for (int x = 0; x < E; ++x)   /* largest remaining overflow, ties to lower id */
+                if (rem_e[x] > 0 && (e < 0 || rem_e[x] > rem_e[e])) e = x;
+        } else {
+            while (m_next < n_ovf && rem_e[order[m_next].e] == 0) ++m_next;
+            if (m_next < n_ovf) e = order[m_next].e;
+        }
+        if (e < 0) break;                 /* every overflow placed */
+        int h = e / H;
+        int best = -1;
+        for (int r = 0; r < N; ++r) {
+            if (used[r] >= R || Q - cur[r] <= 0) continue;   /* not eligible */
+            if (best < 0 || Q - cur[r] > Q - cur[best]) best = r;   /* ties keep lowest r */
+        }
+        if (best < 0) {                   /* slots ran out; none becomes eligible again */
+            flags |= 1;
+            break;
+        }
+        if (best == h) { rc = ORC_INVARIANT; goto done; }  /* home is full whenever ovf > 0 */
+        for (int a = 0; a < n_asg; ++a)                      /* one replica of e per rank */
+            if (asg_e[a] == e && asg_s[a] / HR == best) { rc = ORC_INVARIANT; goto done; }
+        int64_t spare = Q - cur[best];
+        int64_t c = rem_e[e] < spare ? rem_e[e] : spare;
+        asg_e[n_asg] = e;
+        asg_s[n_asg] = best * HR + H + used[best];
+        asg_c[n_asg] = c;
+        ++n_asg;
+        used[best] += 1;
+        cur[best] += c;
+        rem_e[e] -= c;
+    }
+    /* The stuck experts, in the order the greedy would have visited them:
+     * the fixed order, or (requeue) largest remaining first, ties lower id. */
+    if (variant & ORC_REQUEUE) {
+        for (;;) {
+            int e = -1;
+            for (int x = 0; x < E; ++x) {
+                int taken = 0;
+                for (int k = 0; k < n_stuck; ++k) taken |= stuck[k] == x;
+                if (!taken && rem_e[x] > 0 && (e < 0 || rem_e[x] > rem_e[e])) e = x;
             }
-            if (best < 0) {               /* slots ran out: the rest stays home */
-                home_quota[e] += rem;
-                cur[h] += rem;
-                rem = 0;
-                flags |= 1;
-                break;
+            if (e < 0) break;
+            stuck[n_stuck++] = e;
+        }
+    } else {
+        for (int m = 0; m < n_ovf; ++m)
+            if (rem_e[order[m].e] > 0) stuck[n_stuck++] = order[m].e;
+    }
+    /* Their remainders: on the home slot (the stated rule), or spread token by
+     * token over the expert's replicas (home first, then allocation order),
+     * each token to the replica whose rank has the lowest load. */
+    for (int k = 0; k < n_stuck; ++k) {
+        int e = stuck[k], h = e / H;
+        if (!(variant & ORC_SPREAD)) {
+            home_quota[e] += rem_e[e];
+            cur[h] += rem_e[e];
+            rem_e[e] = 0;
+            continue;
+        }
+        while (rem_e[e] > 0) {
+            int best_a = -1;              /* -1: the home replica */
+            int64_t best_load = cur[h];
+            for (int a = 0; a < n_asg; ++a) {
+                if (asg_e[a] != e) continue;
+                int r = asg_s[a] / HR;
+                if (cur[r] < best_load) { best_load = cur[r]; best_a = a; }
             }
-            if (best == h) { rc = ORC_INVARIANT; goto done; }  /* home is full whenever ovf > 0 */
-            for (int a = 0; a < n_asg; ++a)                      /* one replica of e per rank */
-                if (asg_e[a] == e && asg_s[a] / HR == best) { rc = ORC_INVARIANT; goto done; }
-            int64_t spare = Q - cur[best];
-            int64_t c = rem < spare ? rem : spare;
-            asg_e[n_asg] = e;
-            asg_s[n_asg] = best * HR + H + used[best];
-            asg_c[n_asg] = c;
-            ++n_asg;
-            used[best] += 1;
-            cur[best] += c;
-            rem -= c;
+            if (best_a < 0) { home_quota[e] += 1; cur[h] += 1; }
+            else { asg_c[best_a] += 1; cur[asg_s[best_a] / HR] += 1; }
+            rem_e[e] -= 1;
         }
     }
 
@@ -246,8 +313,19 @@ int ue_oracle_plan(int E, int N, int R, const int32_t *load,
 
 done:
     free(cur); free(used); free(home_quota); free(ovf); free(order);
-    free(asg_e); free(asg_s); free(asg_c);
+    free(asg_e); free(asg_s); free(asg_c); free(rem_e); free(stuck);
     return rc;
+}
+
+int ue_oracle_plan(int E, int N, int R, const int32_t *load,
+                   int32_t *slot_expert, int32_t *slot_quota,
+                   int32_t *rep_off, int32_t *rep_slot, int32_t *rep_cum,
+                   int32_t *rep_experts,
+                   int32_t *rank_load_before, int32_t *rank_load_after,
+                   int32_t *info)
+{
+    return ue_oracle_plan_ex(E, N, R, load, 0, slot_expert, slot_quota, rep_off, rep_slot, rep_cum,
+                             rep_experts, rank_load_before, rank_load_after, info);
 }
 
 /* ---- step 3: routing expansion -------------------------------------------
