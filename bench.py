@@ -37,6 +37,7 @@ from moe_expert_load_ue_b200 import inputs  # noqa: E402
 METRIC = "rebalance µs/layer-microbatch (load+plan+reroute); sync & grad-reduce HBM GB/s"
 UNIT = "µs"
 FALLBACK_HBM_GBS = 6650.0
+VARIANTS = {"requeue": 1, "spread": 2, "requeue+spread": 3}     # plan variant bits (UE_PLAN_*)
 # DRAM bytes of one launch from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum) next to that launch's algorithmic bytes, per kernel
 # and full-size workload; summarised in profiles/.  The JSON's roofline.traffic
@@ -381,6 +382,26 @@ def run_ours(args, dist: Dist):
     grad_gbs = grad_bytes[step_mb].sum() / (seg[:, 2].sum() * 1e-6) / 1e9
     rebalance_alg_bytes = 3.0 * w.L * 4
 
+    # Plan variants on the same microbatches: rebalance latency (events around
+    # each ue_rebalance_ex) and the imbalance after the plan.
+    plan_variants = {}
+    for name, v in VARIANTS.items():
+        evv = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_mb)]
+        after = []
+        with torch.cuda.stream(stream):
+            for k in range(args.warmup):        # first launches of the variant's kernels
+                ue.ue_rebalance_ex(ctx, cfg, ids_dev[k % n_mb], counts, bad, plan, phys, v, stream=stream)
+            for mb in range(n_mb):
+                ue.ue_sync(ctx, cfg, weights, slot_bytes, plan, stream=stream)     # keeps L2 cold as in the step
+                evv[mb][0].record(stream)
+                ue.ue_rebalance_ex(ctx, cfg, ids_dev[mb], counts, bad, plan, phys, v, stream=stream)
+                evv[mb][1].record(stream)
+                stream.synchronize()
+                vi = plan["info"].cpu().numpy()
+                after.append(vi[6] / (vi[1] / w.N))
+        plan_variants[name] = {"rebalance_us": round(float(np.mean([a.elapsed_time(b) for a, b in evv])) * 1e3, 2),
+                               "imbalance_after": round(float(np.mean(after)), 4)}
+
     # Incremental weight sync over the microbatch sequence of one training
     # step: the first microbatch syncs in full, each later one copies only the
     # redundant slots whose expert changed; two plan buffers alternate.
@@ -511,6 +532,7 @@ def run_ours(args, dist: Dist):
         "grad_reduce_gbs": round(grad_gbs, 1), "grad_reduce_frac": round(grad_gbs / peak, 4),
         "frac_of_8000_gbs": {"sync": round(sync_gbs / 8000, 4), "grad_reduce": round(grad_gbs / 8000, 4)},
         "sync_delta": sync_delta,
+        "plan_variants": plan_variants,
         "imbalance": {
             "before": round(float(np.mean([p["max_before"] / (p["L"] / w.N) for p in per_mb])), 4),
             "after": round(float(np.mean([p["max_after"] / (p["L"] / w.N) for p in per_mb])), 4),
@@ -644,11 +666,29 @@ def run_sweep(args, dist: Dist):
         info = plan["info"].cpu().tolist()
         us = [a.elapsed_time(b) * 1e3 for a, b in times]
         mean = w.L / w.N
+        # The plan variants on the same ids: imbalance after and latency.
+        variants = {}
+        for name, v in VARIANTS.items():
+            vt = []
+            with torch.cuda.stream(stream):
+                for k in range(args.warmup + 5):
+                    flush.zero_()
+                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                    ue.ue_rebalance_ex(ctx, cfg, ids, counts, bad, plan, phys, v, stream=stream)
+                    b.record(stream)
+                    if k >= args.warmup:
+                        vt.append((a, b))
+            stream.synchronize()
+            vi = plan["info"].cpu().tolist()
+            variants[name] = {"imbalance_after": round(vi[6] / mean, 4),
+                              "rebalance_us_median": round(statistics.median(a.elapsed_time(b) * 1e3 for a, b in vt),
+                                                           2)}
         print(json.dumps({"sweep_point": w.name, "tokens_per_rank": w.tokens_per_rank, "N": w.N, "zipf_s": w.s,
                           "seed": w.base_seed, "T": w.T, "rebalance_us_median": round(statistics.median(us), 2),
                           "imbalance_before": round(info[5] / mean, 4), "imbalance_after": round(info[6] / mean, 4),
                           "slots_ran_out": bool(info[2] & 1), "replicated_experts": info[3],
-                          "filled_redundant_slots": info[4]}), flush=True)
+                          "filled_redundant_slots": info[4], "plan_variants": variants}), flush=True)
         del ids, phys, plan, counts, bad
         torch.cuda.synchronize(dev)
     ctx.close()

@@ -117,6 +117,23 @@ ue_status ue_load(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids,
 ue_status ue_plan(ue_ctx *ctx, const ue_config *cfg, const int32_t *counts,
                   const ue_plan_buffers *plan, void *stream);
 
+/* Plan variants for the two points the rule leaves open (bit flags for
+ * ue_plan_ex / ue_rebalance_ex; 0 = ue_plan):
+ *   UE_PLAN_REQUEUE  the overflow is a priority queue: after every chunk the
+ *                    expert with the largest remaining overflow (ties: lower
+ *                    id) is placed next, instead of each expert being placed
+ *                    fully in the order fixed after the home pass;
+ *   UE_PLAN_SPREAD   when slots run out, each stuck expert's remainder (in
+ *                    visit order) goes token by token to the replica whose rank
+ *                    has the lowest load (ties: earlier replica, home first)
+ *                    instead of staying on the home slot.
+ * Everything else (quota, home pass, eligibility, chunk size, replica order,
+ * cumulative quotas, outputs) is as in ue_plan. */
+#define UE_PLAN_REQUEUE 1
+#define UE_PLAN_SPREAD 2
+ue_status ue_plan_ex(ue_ctx *ctx, const ue_config *cfg, const int32_t *counts,
+                     const ue_plan_buffers *plan, int variant, void *stream);
+
 /* ---- step 3: routing expansion ---------------------------------------------
  * "Routing expansion" (csrc/kernels/reroute.cu; "Routing expansion -> Token
  * dispatch: physical routing").  The j-th occurrence (0-based, token-major
@@ -131,6 +148,11 @@ ue_status ue_reroute(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids,
 ue_status ue_rebalance(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids,
                        int32_t *counts, int32_t *bad, const ue_plan_buffers *plan,
                        int32_t *phys, void *stream);
+
+/* ue_rebalance with a plan variant (UE_PLAN_REQUEUE | UE_PLAN_SPREAD bits). */
+ue_status ue_rebalance_ex(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids,
+                          int32_t *counts, int32_t *bad, const ue_plan_buffers *plan,
+                          int32_t *phys, int variant, void *stream);
 
 /* ---- dispatch layout (after step 3) ------------------------------------------
  * Routing expansion hands the physical routing to token dispatch, which groups

@@ -238,22 +238,31 @@ ue_status ue_load(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids, int32_t
     });
 }
 
-ue_status ue_plan(ue_ctx *ctx, const ue_config *cfg, const int32_t *counts, const ue_plan_buffers *plan,
-                  void *stream)
+ue_status ue_plan_ex(ue_ctx *ctx, const ue_config *cfg, const int32_t *counts, const ue_plan_buffers *plan,
+                     int variant, void *stream)
 {
     ue::Shape sh{};
     ue_status s = make_shape(cfg, false, &sh);
     if (s == UE_OK) s = check_plan(plan);
     if (s != UE_OK) return s;
+    if (variant < 0 || variant > (UE_PLAN_REQUEUE | UE_PLAN_SPREAD))
+        return fail(UE_ERR_INVALID_ARG, "variant=%d (bits: 1 requeue, 2 spread)", variant);
     if (!counts) return fail(UE_ERR_INVALID_ARG, "counts is NULL");
     if ((s = check_ctx(ctx)) != UE_OK) return s;
     if (ue::plan_smem_bytes(sh) > (size_t)ctx->max_smem)
         return fail(UE_ERR_INVALID_ARG, "plan needs %zu bytes of shared memory (> %d)", ue::plan_smem_bytes(sh),
                     ctx->max_smem);
     return on_device(ctx, [&]() -> ue_status {
-        cudaError_t e = ue::launch_plan(sh, counts, ue::to_dev(*plan), static_cast<cudaStream_t>(stream), false);
+        cudaError_t e = ue::launch_plan(sh, counts, ue::to_dev(*plan), static_cast<cudaStream_t>(stream), false,
+                                        variant);
         return e == cudaSuccess ? UE_OK : cuda_fail(e, "plan launch");
     });
+}
+
+ue_status ue_plan(ue_ctx *ctx, const ue_config *cfg, const int32_t *counts, const ue_plan_buffers *plan,
+                  void *stream)
+{
+    return ue_plan_ex(ctx, cfg, counts, plan, 0, stream);
 }
 
 ue_status ue_reroute(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids, const ue_plan_buffers *plan,
@@ -276,14 +285,16 @@ ue_status ue_reroute(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids, cons
     });
 }
 
-ue_status ue_rebalance(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids, int32_t *counts, int32_t *bad,
-                       const ue_plan_buffers *plan, int32_t *phys, void *stream)
+ue_status ue_rebalance_ex(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids, int32_t *counts, int32_t *bad,
+                          const ue_plan_buffers *plan, int32_t *phys, int variant, void *stream)
 {
     // Validate everything before the first launch so a refusal leaves all outputs untouched.
     ue::Shape sh{};
     ue_status s = make_shape(cfg, true, &sh);
     if (s == UE_OK) s = check_plan(plan);
     if (s != UE_OK) return s;
+    if (variant < 0 || variant > (UE_PLAN_REQUEUE | UE_PLAN_SPREAD))
+        return fail(UE_ERR_INVALID_ARG, "variant=%d (bits: 1 requeue, 2 spread)", variant);
     if (!counts) return fail(UE_ERR_INVALID_ARG, "counts is NULL");
     if (sh.T > 0 && (!ids || !aligned16(ids))) return fail(UE_ERR_INVALID_ARG, "ids must be non-NULL and 16-byte aligned");
     if (sh.T > 0 && !phys) return fail(UE_ERR_INVALID_ARG, "phys is NULL");
@@ -299,11 +310,18 @@ ue_status ue_rebalance(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids, in
         // The planner and the reroute kernel use programmatic dependent launch:
         // each may start while its predecessor drains, and waits for it
         // (griddepcontrol.wait) before reading what it wrote.
-        if ((e = ue::launch_plan(sh, counts, pd, st, true)) != cudaSuccess) return cuda_fail(e, "plan launch");
+        if ((e = ue::launch_plan(sh, counts, pd, st, true, variant)) != cudaSuccess)
+            return cuda_fail(e, "plan launch");
         if ((e = ue::launch_reroute(sh, ln, ids, pd, phys, st, true)) != cudaSuccess)
             return cuda_fail(e, "reroute launch");
         return UE_OK;
     });
+}
+
+ue_status ue_rebalance(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids, int32_t *counts, int32_t *bad,
+                       const ue_plan_buffers *plan, int32_t *phys, void *stream)
+{
+    return ue_rebalance_ex(ctx, cfg, ids, counts, bad, plan, phys, 0, stream);
 }
 
 namespace {
@@ -365,7 +383,7 @@ ue_status ue_rebalance_dispatch(ue_ctx *ctx, const ue_config *cfg, const int32_t
         const ue::PlanDev pd = ue::to_dev(*plan);
         cudaError_t e = ue::launch_load(sh, ln, ids, counts, bad, st);
         if (e != cudaSuccess) return cuda_fail(e, "load launch");
-        if ((e = ue::launch_plan(sh, counts, pd, st, true)) != cudaSuccess) return cuda_fail(e, "plan launch");
+        if ((e = ue::launch_plan(sh, counts, pd, st, true, 0)) != cudaSuccess) return cuda_fail(e, "plan launch");
         if ((e = ue::launch_dispatch(sh, ln, ids, pd, phys, out, ctx->dev_err, st, true)) != cudaSuccess)
             return cuda_fail(e, "dispatch launch");
         return UE_OK;

@@ -53,8 +53,10 @@ cudaError_t launch_load(const Shape &sh, const Launch &ln, const int32_t *ids, i
                         int32_t *bad, cudaStream_t st);
 size_t load_smem_bytes(const Shape &sh);
 
+// variant: bit 0 re-queues partly placed overflow, bit 1 spreads stuck
+// remainders over the expert's replicas (0 = the stated rule).
 cudaError_t launch_plan(const Shape &sh, const int32_t *counts, const PlanDev &plan, cudaStream_t st,
-                        bool pdl);
+                        bool pdl, int variant);
 size_t plan_smem_bytes(const Shape &sh);
 int plan_cluster(const Shape &sh);
 

@@ -52,7 +52,6 @@ constexpr int kPlanMaxThreads = 1024;
 
 // Shared-memory layout of a planner CTA (all 4-byte words unless noted).
 struct PlanSmem {
-    int32_t *part;        // [32][33] column-group partial sums
     int32_t *ws;          // [96] scan / reduction scratch
     int32_t *misc;        // [8]  assignments, stop position, remainder at the stop
     int32_t *sload;       // [E]  loads (peers: of their own column groups)
@@ -72,13 +71,19 @@ struct PlanSmem {
     int32_t *ac;          // [NR] assignment quota
     int32_t *ae;          // [NR] assignment expert
     int32_t *sasg;        // [NR] (rank, redundant index) -> assignment or -1
+    int32_t *rem;         // [E]  variants: remaining overflow of order[p]
+    int32_t *alast;       // [E]  requeue: last assignment of e
+    int32_t *anext;       // [NR] requeue: next assignment of the same expert, -1 at the end
+    int32_t *stuck;       // [E]  experts left with overflow when slots ran out, in visit order
+    int32_t *srem;        // [E]  their remainders
+    int32_t *tmp;         // [NR+1] spread: the assignments of the expert being spread
     unsigned long long *key;   // [max(E, N)] packed sort keys (8-byte aligned)
 };
 
 __host__ __device__ inline size_t plan_smem_words(int E, int N, int NR)
 {
     const int K = E > N ? E : N;
-    return (size_t)32 * 33 + 96 + 8 + (size_t)7 * E + (size_t)5 * N + 1 + (size_t)5 * NR + 2 + (size_t)2 * K;
+    return (size_t)96 + 8 + (size_t)11 * E + (size_t)5 * N + 1 + (size_t)7 * NR + 1 + 2 + (size_t)2 * K;
 }
 
 // Word offsets are computed as integers from the (16-byte aligned) base of the
@@ -88,7 +93,6 @@ __device__ __forceinline__ PlanSmem carve(int32_t *p, int E, int N, int NR)
 {
     PlanSmem s;
     int o = 0;
-    s.part = p + o;      o += 32 * 33;
     s.ws = p + o;        o += 96;
     s.misc = p + o;      o += 8;
     s.sload = p + o;     o += E;
@@ -108,6 +112,12 @@ __device__ __forceinline__ PlanSmem carve(int32_t *p, int E, int N, int NR)
     s.ac = p + o;        o += NR;
     s.ae = p + o;        o += NR;
     s.sasg = p + o;      o += NR;
+    s.rem = p + o;       o += E;
+    s.alast = p + o;     o += E;
+    s.anext = p + o;     o += NR;
+    s.stuck = p + o;     o += E;
+    s.srem = p + o;      o += E;
+    s.tmp = p + o;       o += NR + 1;
     o = (o + 1) & ~1;                       // 8-byte alignment for the keys
     s.key = reinterpret_cast<unsigned long long *>(p + o);
     return s;
@@ -335,9 +345,248 @@ __device__ __forceinline__ void greedy_sorted(const PlanSmem &s, int K, int M1)
     }
 }
 
+// Variant REQUEUE: after every chunk the expert with the largest remaining
+// overflow (ties: lower id) is placed next; run by warp 0.  Lane l owns the
+// overflow-order positions l, l + 32, ... (rem[p] = what order[p] still has to
+// place) and keeps the best of them as one 32-bit key (remaining << 10 |
+// 1023 - id, so that one redux.sync max picks the expert, ties to the lower id)
+// while every overflow is below 2^22; otherwise the pick takes two redux.sync.
+// Only the owner of the expert just served rescans its positions.  Ranks: with
+// R = 1 a rank is chosen at most once and its spare does not change before, so
+// the k-th chunk goes to the k-th rank of the ranks sorted by initial spare
+// (rsorted, K of them); with R > 1 the argmax of greedy_chunks.  An expert's
+// assignments are chained in allocation order through afirst / anext.
 template <int NRL>
+__device__ __forceinline__ void greedy_requeue(const PlanSmem &s, int N, int R, int M1, int K)
+{
+    const int lane = lane_id();
+    unsigned sp[NRL];
+    int us[NRL];
+    unsigned bs = 0;
+    int br = INT_MAX;
+    auto lane_best = [&]() {
+        bs = 0;
+        br = INT_MAX;
+#pragma unroll
+        for (int i = 0; i < NRL; ++i) {
+            const bool better = us[i] < R && sp[i] > bs;    // strict: lowest rank on ties
+            bs = better ? sp[i] : bs;
+            br = better ? lane + 32 * i : br;
+        }
+    };
+    if (R > 1) {
+#pragma unroll
+        for (int i = 0; i < NRL; ++i) {
+            const int r = lane + 32 * i;
+            sp[i] = r < N ? (unsigned)s.spare[r] : 0u;
+            us[i] = 0;
+        }
+        lane_best();
+    }
+    int omax = 0;
+    for (int p = lane; p < M1; p += 32) {
+        const int o = s.ovf[s.order[p]];
+        s.rem[p] = o;
+        omax = max(omax, o);
+    }
+    const bool packed = __reduce_max_sync(0xffffffffu, omax) < (1 << 22);
+    __syncwarp();
+    unsigned bkey;                 // packed: the lane's best key
+    int brem, bid, bpos;
+    auto expert_best = [&]() {
+        brem = 0;
+        bid = INT_MAX;
+        bpos = 0;
+        for (int p = lane; p < M1; p += 32) {
+            const int r = s.rem[p], e = s.order[p];
+            if (r > brem || (r == brem && r > 0 && e < bid)) {
+                brem = r;
+                bid = e;
+                bpos = p;
+            }
+        }
+        bkey = brem > 0 ? ((unsigned)brem << 10) | (1023u - (unsigned)bid) : 0u;
+    };
+    expert_best();
+    int na = 0;
+    bool ran_out = false;
+    for (;;) {
+        int mx, e, el;
+        if (packed) {
+            const unsigned k = __reduce_max_sync(0xffffffffu, bkey);
+            if (k == 0u) break;                                  // every overflow placed
+            mx = (int)(k >> 10);
+            e = 1023 - (int)(k & 1023u);
+            el = __ffs(__ballot_sync(0xffffffffu, bkey == k)) - 1;
+        } else {
+            mx = __reduce_max_sync(0xffffffffu, brem);
+            if (mx == 0) break;
+            e = __reduce_min_sync(0xffffffffu, brem == mx ? bid : INT_MAX);
+            el = __ffs(__ballot_sync(0xffffffffu, brem == mx && bid == e)) - 1;
+        }
+        int rs, spare_rs, u = 0;
+        if (R == 1) {
+            if (na >= K) {                                       // every eligible rank used
+                ran_out = true;
+                break;
+            }
+            rs = s.rsorted[na];
+            spare_rs = s.rsum[na + 1] - s.rsum[na];
+        } else {
+            const unsigned ms = __reduce_max_sync(0xffffffffu, bs);
+            if (ms == 0u) {                                      // no eligible rank left
+                ran_out = true;
+                break;
+            }
+            rs = __reduce_min_sync(0xffffffffu, bs == ms ? br : INT_MAX);
+            spare_rs = (int)ms;
+        }
+        const int c = mx < spare_rs ? mx : spare_rs;
+        if (R > 1) {
+            const bool own = lane == (rs & 31);
+            const int si = rs >> 5;
+#pragma unroll
+            for (int i = 0; i < NRL; ++i) {
+                const bool hit = own && i == si;
+                u = hit ? us[i] : u;
+                us[i] += hit ? 1 : 0;
+                sp[i] -= hit ? (unsigned)c : 0u;
+            }
+            lane_best();
+            u = __shfl_sync(0xffffffffu, u, rs & 31);
+        }
+        if (lane == el) {                                        // the owner of e records the chunk
+            s.ar[na] = rs;
+            s.au[na] = u;
+            s.ac[na] = c;
+            s.ae[na] = e;
+            s.sasg[rs * R + u] = na;
+            s.anext[na] = -1;
+            const int last = s.alast[e];
+            if (last >= 0) s.anext[last] = na;
+            else s.afirst[e] = na;
+            s.alast[e] = na;
+            s.acnt[e] += 1;
+            s.rem[bpos] = mx - c;
+            if (R == 1) s.spare[rs] -= c;
+            expert_best();
+        }
+        ++na;
+    }
+    if (R > 1) {
+#pragma unroll
+        for (int i = 0; i < NRL; ++i) {
+            const int r = lane + 32 * i;
+            if (r < N) s.spare[r] = (int)sp[i];
+        }
+    }
+    if (lane == 0) {
+        s.misc[0] = na;
+        s.misc[1] = ran_out ? 0 : M1;
+        s.misc[2] = 0;
+    }
+}
+
+// Variant SPREAD, run by warp 0 over the ns stuck experts in visit order:
+// each remainder goes token by token to the replica whose rank has the lowest
+// load (ties: the earlier replica, home first).  In closed form: the replicas
+// are filled up to the level lam with f(lam) = sum_i max(0, lam - l_i) <= res
+// < f(lam + 1), and the t = res - f(lam) tokens left go one each to the first
+// t replicas (in replica order) whose load is then lam.  Rank load =
+// Q - spare + extra.  chained: assignments linked through anext (REQUEUE),
+// else contiguous from afirst.  With at most 32 replicas and res < 2^26 the
+// loads stay in registers and f is one redux.sync add of terms clamped to
+// res + 1 (the sum then fits 32 bits); otherwise a 64-bit shuffle sum.
+__device__ __forceinline__ void spread_stuck(const PlanSmem &s, int ns, int Q, int H, bool chained)
+{
+    const int lane = lane_id();
+    for (int k = 0; k < ns; ++k) {
+        const int e = s.stuck[k], h = e / H, res = s.srem[k];
+        const int nred = s.acnt[e];
+        if (nred == 0 || res == 0) {
+            if (lane == 0) {
+                s.qh[e] += res;
+                s.extra[h] += res;
+            }
+            __syncwarp();
+            continue;
+        }
+        if (lane == 0) {
+            int a = s.afirst[e];
+            for (int i = 0; i < nred; ++i) {
+                s.tmp[i] = a;
+                a = chained ? s.anext[a] : a + 1;
+            }
+        }
+        __syncwarp();
+        const int n = 1 + nred;
+        auto rank_of = [&](int i) { return i == 0 ? h : s.ar[s.tmp[i - 1]]; };
+        auto load_of = [&](int i) {
+            const int r = rank_of(i);
+            return Q - s.spare[r] + s.extra[r];
+        };
+        int lam;
+        if (n <= 32 && res < (1 << 26)) {
+            const int my = lane < n ? load_of(lane) : INT_MAX;
+            const int minl = __reduce_min_sync(0xffffffffu, my);
+            int lo = minl, hi = minl + res;
+            while (lo < hi) {
+                const int mid = lo + (hi - lo + 1) / 2;
+                const unsigned term = lane < n && mid > my ? (unsigned)min(mid - my, res + 1) : 0u;
+                if (__reduce_add_sync(0xffffffffu, term) <= (unsigned)res) lo = mid;
+                else hi = mid - 1;
+            }
+            lam = lo;
+        } else {
+            int minl = INT_MAX;
+            for (int i = lane; i < n; i += 32) minl = min(minl, load_of(i));
+            minl = __reduce_min_sync(0xffffffffu, minl);
+            auto fill = [&](int x) {
+                long long f = 0;
+                for (int i = lane; i < n; i += 32) f += max(0, x - load_of(i));
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) f += __shfl_xor_sync(0xffffffffu, f, o);
+                return f;
+            };
+            int lo = minl, hi = minl + res;
+            while (lo < hi) {
+                const int mid = lo + (hi - lo + 1) / 2;
+                if (fill(mid) <= res) lo = mid;
+                else hi = mid - 1;
+            }
+            lam = lo;
+        }
+        // f(lam) and the replicas at or below lam, in replica order.
+        long long f = 0;
+        for (int i = lane; i < n; i += 32) f += max(0, lam - load_of(i));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) f += __shfl_xor_sync(0xffffffffu, f, o);
+        const int t = res - (int)f;           // < number of replicas at or below lam
+        int seen = 0;
+        for (int i0 = 0; i0 < n; i0 += 32) {
+            const int i = i0 + lane;
+            const int l = i < n ? load_of(i) : INT_MAX;
+            const bool at = i < n && l <= lam;
+            const unsigned b = __ballot_sync(0xffffffffu, at);
+            const int add = at ? (lam - l) + ((seen + __popc(b & lanemask_lt())) < t ? 1 : 0) : 0;
+            __syncwarp();                     // every load of the batch read before any update
+            if (add > 0) {
+                const int r = rank_of(i);
+                if (i == 0) s.qh[e] += add;
+                else s.ac[s.tmp[i - 1]] += add;
+                s.extra[r] += add;            // replicas of one expert sit on distinct ranks
+            }
+            seen += __popc(b);
+            __syncwarp();
+        }
+    }
+}
+
+// kVariants = false compiles the stated rule alone (variant is ignored), so
+// the default planner carries none of the variants' code.
+template <int NRL, bool kVariants>
 __global__ void __launch_bounds__(kPlanMaxThreads, 1)
-k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
+k_plan(const int32_t *__restrict__ counts, int E, int N, int R, int variant, PlanDev plan)
 {
     extern __shared__ __align__(16) int32_t sm_plan[];
     const int H = E / N, HR = H + R, S = N * HR, NR = N * R, cap = E + NR;
@@ -408,6 +657,7 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
         s.ovf[e] = my_ovf;
         s.acnt[e] = 0;
         s.afirst[e] = 0;
+        s.alast[e] = -1;
         if (e % H == H - 1) {
             const int rank_sum = pin + ld;
             s.before[h] = rank_sum;
@@ -428,6 +678,7 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
     }
     __syncthreads();
 
+    const bool requeue = kVariants && (variant & 1) != 0, spread = kVariants && (variant & 2) != 0;
     if (R == 1) {
         // Eligible ranks (spare > 0) sorted by spare descending, lowest rank first.
         const int sp_r = tid < N ? s.spare[tid] : 0;
@@ -454,44 +705,87 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
         if (tid < K) s.rsum[tid] = ex;
         if (tid == 0) s.rsum[K] = tot;
         __syncthreads();
-        if (warp == 0) greedy_sorted(s, K, M1);
-        __syncthreads();
-        // Fill the assignments: expert m of the overflow order owns the sorted
-        // positions of its cut; every rank is full except the last rank of an
-        // expert that was placed completely (m before the stop), which takes
-        // what is left of the expert's overflow.
-        if (tid < M1) {
-            const int em = s.order[tid];
-            const int a0 = s.afirst[em], na = s.acnt[em];
-            const bool placed = tid < s.misc[1];
-            for (int a = a0; a < a0 + na; ++a) {
-                const int r = s.rsorted[a];
-                int q = s.rsum[a + 1] - s.rsum[a];
-                if (placed && a == a0 + na - 1) q = s.ovf[em] - (s.rsum[a] - s.rsum[a0]);
-                s.ar[a] = r;
-                s.au[a] = 0;
-                s.ac[a] = q;
-                s.ae[a] = em;
-                s.sasg[r] = a;
-                s.spare[r] -= q;
+        if (requeue) {
+            if (warp == 0) greedy_requeue<NRL>(s, N, R, M1, K);
+        } else {
+            if (warp == 0) greedy_sorted(s, K, M1);
+            __syncthreads();
+            // Fill the assignments: expert m of the overflow order owns the sorted
+            // positions of its cut; every rank is full except the last rank of an
+            // expert that was placed completely (m before the stop), which takes
+            // what is left of the expert's overflow.
+            if (tid < M1) {
+                const int em = s.order[tid];
+                const int a0 = s.afirst[em], na = s.acnt[em];
+                const bool placed = tid < s.misc[1];
+                for (int a = a0; a < a0 + na; ++a) {
+                    const int r = s.rsorted[a];
+                    int q = s.rsum[a + 1] - s.rsum[a];
+                    if (placed && a == a0 + na - 1) q = s.ovf[em] - (s.rsum[a] - s.rsum[a0]);
+                    s.ar[a] = r;
+                    s.au[a] = 0;
+                    s.ac[a] = q;
+                    s.ae[a] = em;
+                    s.sasg[r] = a;
+                    s.spare[r] -= q;
+                }
             }
         }
+    } else if (requeue) {
+        if (warp == 0) greedy_requeue<NRL>(s, N, R, M1, 0);
     } else if (warp == 0) {
         greedy_chunks<NRL>(s, N, R, M1);
     }
     __syncthreads();
     const int n_asg = s.misc[0], stop_pos = s.misc[1], stop_rem = s.misc[2];
     const int flags = stop_pos < M1 ? 1 : 0;
-    // Slots ran out at overflow position stop_pos: that expert's remainder and
-    // the whole overflow of every later expert stay on their home slots.
-    for (int p = stop_pos + tid; p < M1; p += nt) {
-        const int ep = s.order[p];
-        const int res = p == stop_pos ? stop_rem : s.ovf[ep];
-        s.qh[ep] += res;
-        atomicAdd(&s.extra[ep / H], res);
-        if (p != stop_pos) {
-            s.afirst[ep] = 0;
-            s.acnt[ep] = 0;
+    if (!requeue) {
+        // Slots ran out at overflow position stop_pos: that expert's remainder
+        // and the whole overflow of every later expert are stuck, in this order.
+        for (int p = stop_pos + tid; p < M1; p += nt) {
+            const int ep = s.order[p];
+            const int res = p == stop_pos ? stop_rem : s.ovf[ep];
+            if (p != stop_pos) {
+                s.afirst[ep] = 0;
+                s.acnt[ep] = 0;
+            }
+            if (spread) {
+                s.stuck[p - stop_pos] = ep;
+                s.srem[p - stop_pos] = res;
+            } else {                      // the stated rule: the remainder stays home
+                s.qh[ep] += res;
+                atomicAdd(&s.extra[ep / H], res);
+            }
+        }
+        if (spread) {
+            __syncthreads();
+            if (warp == 0) spread_stuck(s, M1 - stop_pos, Q, H, false);
+        }
+    } else if (flags) {
+        // Re-queued overflow: the stuck experts are those with overflow left,
+        // visited largest remainder first (ties: lower id).
+        const int rp = tid < M1 ? s.rem[tid] : 0;
+        const int ep = tid < M1 ? s.order[tid] : 0;
+        int ns;
+        const int kp = block_excl_scan(rp > 0 ? 1 : 0, s.ws, &ns);
+        if (rp > 0) s.key[kp] = ((unsigned long long)(unsigned)rp << 32) | (0xffffffffu - (unsigned)ep);
+        __syncthreads();
+        if (tid < ns) {
+            const unsigned long long mine = s.key[tid];
+            int rank = 0;
+            for (int k = 0; k < ns; ++k) rank += s.key[k] > mine ? 1 : 0;
+            const int ek = (int)(0xffffffffu - (unsigned)(mine & 0xffffffffu));
+            const int rk = (int)(mine >> 32);
+            s.stuck[rank] = ek;
+            s.srem[rank] = rk;
+            if (!spread) {
+                s.qh[ek] += rk;
+                atomicAdd(&s.extra[ek / H], rk);
+            }
+        }
+        if (spread) {
+            __syncthreads();
+            if (warp == 0) spread_stuck(s, ns, Q, H, true);
         }
     }
     __syncthreads();
@@ -510,12 +804,12 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, PlanDev plan)
         plan.rep_slot[off] = h * HR + e % H;
         plan.rep_cum[off] = 0;
         int cum = s.qh[e];
-        const int a0 = s.afirst[e];
+        int a = s.afirst[e];
         for (int i = 0; i < na_e; ++i) {
-            const int a = a0 + i;
             plan.rep_slot[off + 1 + i] = s.ar[a] * HR + H + s.au[a];
             plan.rep_cum[off + 1 + i] = cum;
             cum += s.ac[a];
+            a = requeue ? s.anext[a] : a + 1;
         }
         if (na_e > 0) plan.rep_experts[mpos] = e;
     }
@@ -602,13 +896,16 @@ int plan_cluster(const Shape &sh)
     return C < sh.N ? C : (sh.N < 1 ? 1 : sh.N);
 }
 
-cudaError_t launch_plan(const Shape &sh, const int32_t *counts, const PlanDev &plan, cudaStream_t st, bool pdl)
+cudaError_t launch_plan(const Shape &sh, const int32_t *counts, const PlanDev &plan, cudaStream_t st, bool pdl,
+                        int variant)
 {
     const unsigned C = (unsigned)plan_cluster(sh);
     const unsigned threads = (unsigned)plan_threads(sh);
     const int nrl = (sh.N + 31) / 32;
     const size_t smem = plan_smem_bytes(sh);
-#define UE_PLAN_LAUNCH(V) launch_ex(k_plan<V>, C, threads, smem, st, C, pdl, counts, sh.E, sh.N, sh.R, plan)
+#define UE_PLAN_LAUNCH(V)                                                                                       \
+    (variant ? launch_ex(k_plan<V, true>, C, threads, smem, st, C, pdl, counts, sh.E, sh.N, sh.R, variant, plan)  \
+             : launch_ex(k_plan<V, false>, C, threads, smem, st, C, pdl, counts, sh.E, sh.N, sh.R, 0, plan))
     if (nrl <= 1) return UE_PLAN_LAUNCH(1);
     if (nrl <= 2) return UE_PLAN_LAUNCH(2);
     if (nrl <= 4) return UE_PLAN_LAUNCH(4);
@@ -620,13 +917,13 @@ cudaError_t launch_plan(const Shape &sh, const int32_t *counts, const PlanDev &p
 
 cudaError_t set_plan_attributes(size_t max_smem)
 {
-    cudaError_t e = allow_smem(k_plan<1>, max_smem);
-    if (e == cudaSuccess) e = allow_smem(k_plan<2>, max_smem);
-    if (e == cudaSuccess) e = allow_smem(k_plan<4>, max_smem);
-    if (e == cudaSuccess) e = allow_smem(k_plan<8>, max_smem);
-    if (e == cudaSuccess) e = allow_smem(k_plan<16>, max_smem);
-    if (e == cudaSuccess) e = allow_smem(k_plan<32>, max_smem);
-    return e;
+    for (auto k : {k_plan<1, false>, k_plan<2, false>, k_plan<4, false>, k_plan<8, false>, k_plan<16, false>,
+                   k_plan<32, false>, k_plan<1, true>, k_plan<2, true>, k_plan<4, true>, k_plan<8, true>,
+                   k_plan<16, true>, k_plan<32, true>}) {
+        const cudaError_t e = allow_smem(k, max_smem);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace ue

@@ -18,13 +18,14 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libue.so")
 
 UE_OK, UE_ERR_INVALID_ARG, UE_ERR_CUDA, UE_ERR_UNSUPPORTED, UE_ERR_DEVICE = range(5)
+UE_PLAN_REQUEUE, UE_PLAN_SPREAD = 1, 2      # plan variant bits (include/ue.h)
 
 PLAN_FIELDS = ("slot_expert", "slot_quota", "rep_off", "rep_slot", "rep_cum", "rep_experts",
                "load", "rank_off", "rank_load_before", "rank_load_after", "info")
 
 # Entry points declared in include/ue.h (checked against the header by the tests).
 EXPORTS = ("ue_plan_sizes", "ue_ctx_create", "ue_ctx_destroy", "ue_ctx_device_error", "ue_load",
-           "ue_plan", "ue_reroute", "ue_rebalance", "ue_dispatch", "ue_rebalance_dispatch", "ue_sync", "ue_sync_delta",
+           "ue_plan", "ue_plan_ex", "ue_reroute", "ue_rebalance", "ue_rebalance_ex", "ue_dispatch", "ue_rebalance_dispatch", "ue_sync", "ue_sync_delta",
            "ue_grad_reduce", "ue_status_string", "ue_last_error")
 
 
@@ -71,8 +72,10 @@ def lib() -> ctypes.CDLL:
                 "ue_ctx_device_error": [vp, ctypes.POINTER(ctypes.c_int32), vp],
                 "ue_load": [vp, cfgp, vp, vp, vp, vp],
                 "ue_plan": [vp, cfgp, vp, planp, vp],
+                "ue_plan_ex": [vp, cfgp, vp, planp, ci, vp],
                 "ue_reroute": [vp, cfgp, vp, planp, vp, vp],
                 "ue_rebalance": [vp, cfgp, vp, vp, vp, planp, vp, vp],
+                "ue_rebalance_ex": [vp, cfgp, vp, vp, vp, planp, vp, ci, vp],
                 "ue_dispatch": [vp, cfgp, vp, planp, vp, dispp, vp],
                 "ue_rebalance_dispatch": [vp, cfgp, vp, vp, vp, planp, vp, dispp, vp],
                 "ue_sync": [vp, cfgp, vp, i64, planp, vp],
@@ -206,6 +209,11 @@ def ue_plan(ctx: Context, cfg: Config, counts: torch.Tensor, plan: Plan, stream=
            "ue_plan")
 
 
+def ue_plan_ex(ctx: Context, cfg: Config, counts: torch.Tensor, plan: Plan, variant: int, stream=None) -> None:
+    _check(lib().ue_plan_ex(ctx.handle, ctypes.byref(cfg.c()), _ptr(counts), plan.ref(), int(variant),
+                            _stream(stream)), "ue_plan_ex")
+
+
 def ue_reroute(ctx: Context, cfg: Config, ids: torch.Tensor, plan: Plan, phys: torch.Tensor,
                stream=None) -> None:
     _check(lib().ue_reroute(ctx.handle, ctypes.byref(cfg.c()), _ptr(ids), plan.ref(), _ptr(phys),
@@ -253,6 +261,12 @@ def ue_rebalance_dispatch(ctx: Context, cfg: Config, ids: torch.Tensor, counts: 
     _check(lib().ue_rebalance_dispatch(ctx.handle, ctypes.byref(cfg.c()), _ptr(ids), _ptr(counts), _ptr(bad),
                                        plan.ref(), _ptr(phys), ctypes.byref(b), _stream(stream)),
            "ue_rebalance_dispatch")
+
+
+def ue_rebalance_ex(ctx: Context, cfg: Config, ids: torch.Tensor, counts: torch.Tensor,
+                    bad: torch.Tensor | None, plan: Plan, phys: torch.Tensor, variant: int, stream=None) -> None:
+    _check(lib().ue_rebalance_ex(ctx.handle, ctypes.byref(cfg.c()), _ptr(ids), _ptr(counts), _ptr(bad),
+                                 plan.ref(), _ptr(phys), int(variant), _stream(stream)), "ue_rebalance_ex")
 
 
 def ue_sync(ctx: Context, cfg: Config, weights: torch.Tensor, slot_bytes: int, plan: Plan,

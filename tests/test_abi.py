@@ -190,3 +190,17 @@ def test_sync_delta_refusals(L):
                            prev.ctypes.data, None) == 1
     assert L.ue_sync_delta(FAKE_CTX, ctypes.byref(c), None, 32, ctypes.byref(hp.c), None, None) == 1
     assert hp.untouched() and (w == 0).all()
+
+
+def test_plan_variant_refused(L):
+    hp = _HostPlan()
+    counts = np.zeros(64, np.int32)
+    c = ue.UeConfig(16, 4, 1, 8, 64)
+    assert L.ue_plan_ex(FAKE_CTX, ctypes.byref(c), counts.ctypes.data, ctypes.byref(hp.c), 4, None) == 1
+    assert "variant" in L.ue_last_error().decode()
+    phys = np.full(512, 7, np.int32)
+    ids = np.zeros(64 * 8 + 4, np.int32)
+    ids_p = ids.ctypes.data + (-ids.ctypes.data % 16)
+    assert L.ue_rebalance_ex(FAKE_CTX, ctypes.byref(c), ids_p, counts.ctypes.data, None, ctypes.byref(hp.c),
+                             phys.ctypes.data, -1, None) == 1
+    assert hp.untouched() and (phys == 7).all()
