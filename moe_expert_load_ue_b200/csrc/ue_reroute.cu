@@ -16,13 +16,16 @@
 // griddepcontrol.wait: launched with programmatic dependent launch, it
 // overlaps the planner.  Pass 1 also keeps the CTA's ids in shared memory
 // (when they fit), so pass 2 does not read them from memory again; both passes
-// move four ids per lane with 16-byte accesses when the share is aligned.  From the counts and the bases each warp then knows,
-// per expert, whether all its occurrences fall into one replica's quota range
-// ("uniform": almost every (warp, expert) pair of a replicated expert; an
-// expert with one replica always is).  Pass 2 is then one or two shared-memory
-// lookups per id; only ids of an expert whose quota boundary falls inside the
-// warp's part are ranked exactly, by ballots over the bits of the expert's
-// compact index in plan.rep_experts.
+// move four ids per lane with 16-byte accesses when the share is aligned.
+// From the counts and the bases each warp then knows, per expert, whether all
+// of its occurrences fall into one replica's quota range (an expert with one
+// replica always does; so does almost every (warp, expert) pair of a
+// replicated one), and a per-warp table maps every expert to that slot, or
+// marks it with the warp's running occurrence index.  Pass 2 is one shared
+// load per id; a block of 128 ids whose marked ids all belong to one expert
+// and stay inside one replica range advances the running index by their
+// count; only a block that straddles a quota boundary ranks its ids exactly,
+// by ballots over the bits of the expert id.
 //
 // Dispatch layout (token dispatch consumes the physical routing: "Routing
 // expansion -> Token dispatch: physical routing", "Token dispatch -> Expert
@@ -35,6 +38,8 @@
 // stable grouping by slot computed in the same pass.  Every valid id then
 // needs its occurrence index, so this variant ranks every id of a warp step
 // by ballots over the bits of the expert id.
+#include <climits>
+
 #include <cooperative_groups.h>
 
 #include "ue_internal.cuh"
@@ -62,12 +67,11 @@ struct DispatchArgs {
 
 struct RerouteSmem {
     int32_t *hist;   // [W][E] per-warp counts, then their exclusive scan over the warps
-    int32_t *code;   // [W][M] per warp and replicated expert: ~slot (uniform) or running occurrence index
+    int32_t *code;   // [W][E] per warp and expert: its slot, or -2 - the warp's next occurrence index
                      //        (dispatch variant: [32] partial sums of the slot-offset scan)
     int32_t *tot;    // [E]    this CTA's counts (read by later CTAs of the cluster)
     int32_t *base;   // [E]    occurrences of e before this CTA's ids
-    int32_t *rexp;   // [E+1]  replicated experts (plan.rep_experts); dispatch variant:
-                     //        exclusive prefix of this CTA's per-expert counts
+    int32_t *rexp;   // [E+1]  dispatch variant: exclusive prefix of this CTA's per-expert counts
     int2 *tab;       // [E]    {home slot if one replica, else first replica entry; (compact index << 16) | count}
     int2 *rc;        // [cap]  {cumulative quota, slot} of each replica entry
     int32_t *soff;   // [S+1]  dispatch only: exclusive prefix of the slot quotas
@@ -187,8 +191,7 @@ template <bool kDispatch>
 __global__ void __launch_bounds__(kRerouteWarps * 32)
 k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
           const int32_t *__restrict__ rep_off, const int32_t *__restrict__ rep_slot,
-          const int32_t *__restrict__ rep_cum, const int32_t *__restrict__ rep_experts,
-          const int32_t *__restrict__ info, const int32_t *__restrict__ rank_off,
+          const int32_t *__restrict__ rep_cum, const int32_t *__restrict__ rank_off,
           int32_t *__restrict__ phys, int stage_cap, DispatchArgs da)
 {
     extern __shared__ __align__(16) int32_t sm_rr[];
@@ -216,9 +219,9 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
     int32_t *h = s.hist + warp * E;
     const bool staged = hi - lo <= stage_cap;     // then pass 2 reads the ids from shared memory
     // Vector mode: 16-byte loads and stores, four ids per lane, when the CTA's
-    // share and phys are 16-byte aligned and the share fits in shared memory.
-    const bool vec = staged && (lo % 4) == 0 && ((hi - lo) % 4) == 0 &&
-                     (reinterpret_cast<uintptr_t>(phys) & 15) == 0;
+    // share and phys are 16-byte aligned (ids is); the ids come from shared
+    // memory in pass 2 when the share was staged, else from memory again.
+    const bool vec = (lo % 4) == 0 && ((hi - lo) % 4) == 0 && (reinterpret_cast<uintptr_t>(phys) & 15) == 0;
 
     // Pass 1: per-warp histogram of the warp's part (ids only; overlaps the planner).
     if (vec) {
@@ -232,7 +235,7 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u) {
                 const int64_t i = v0 + 128 * u + 4 * lane;
-                if (i < whi) *reinterpret_cast<int4 *>(s.stage + (i - lo)) = q[u];
+                if (staged && i < whi) *reinterpret_cast<int4 *>(s.stage + (i - lo)) = q[u];
                 if ((unsigned)q[u].x < (unsigned)E) smem_add(h + q[u].x, 1);
                 if ((unsigned)q[u].y < (unsigned)E) smem_add(h + q[u].y, 1);
                 if ((unsigned)q[u].z < (unsigned)E) smem_add(h + q[u].z, 1);
@@ -304,7 +307,6 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
     // The plan (and rank_off) of the preceding planner grid: every global load
     // of the plan is issued in one round.
     pdl_wait();
-    const int M = clampi(__ldg(info + 3), 0, E);
     for (int i = threadIdx.x; i < cap; i += blockDim.x) s.rc[i] = make_int2(__ldg(rep_cum + i), __ldg(rep_slot + i));
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         const int o0 = __ldg(rep_off + e), o1 = __ldg(rep_off + e + 1);
@@ -319,8 +321,6 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
         for (int q = 0; q < kMaxCluster; ++q) b += peer[q];
         s.base[e] = b;            // occurrences of e before this CTA's ids
     }
-    if (!kDispatch)
-        for (int m = threadIdx.x; m < M; m += blockDim.x) s.rexp[m] = clampi(__ldg(rep_experts + m), 0, E - 1);
     cluster_arrive_relaxed();  // done reading peers; they may exit once all have arrived
     if constexpr (kDispatch) {
         // Slot offsets (exclusive prefix of the slot quotas; CTA 0 writes
@@ -352,47 +352,58 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
         const unsigned lt = lanemask_lt();
         const int nloc = (int)(whi - wlo);       // this warp's ids, local index lbase + k
         const int lbase = (int)(wlo - lo);
-        for (int k0 = 0; k0 < nloc; k0 += 32) {
-            const int k = k0 + lane;
-            const int li = lbase + k;
-            const int id = k < nloc ? (staged ? s.stage[li] : __ldg(ids + lo + li)) : -1;
-            const bool valid = (unsigned)id < (unsigned)E;
-            if (valid) tag[id] = (uint8_t)lane;
-            __syncwarp();
-            const int key = valid ? tag[id] : 0;
-            unsigned m = __ballot_sync(0xffffffffu, valid);
+        for (int k00 = 0; k00 < nloc; k00 += 32 * kUnroll) {
+            int idv[kUnroll];                // the ids of four steps in flight together
 #pragma unroll
-            for (int b = 0; b < 5; ++b) {
-                const unsigned v = __ballot_sync(0xffffffffu, (key >> b) & 1);
-                m &= ((key >> b) & 1) ? v : ~v;
+            for (int u = 0; u < kUnroll; ++u) {
+                const int k = k00 + 32 * u + lane;
+                idv[u] = k < nloc ? (staged ? s.stage[lbase + k] : __ldg(ids + lo + lbase + k)) : -1;
             }
-            const int before = __popc(m & lt);
-            int out = -1;
-            if (valid) {
-                const int j = wh[id] + before;
-                const int2 t = s.tab[id];
-                const int2 q = s.rc[t.x + covering_entry(s.rc + t.x, t.y & 0xffff, j)];
-                out = q.y;
-                int pos = -1;
-                // Inside the slot's segment whenever the ids are the ones the
-                // plan was computed from; anything else is reported, not written.
-                if (out >= 0 && out < S) {
-                    pos = s.soff[out] + (j - q.x);
-                    if (pos < s.soff[out] || pos >= s.soff[out + 1] || (int64_t)pos >= da.L) pos = -1;
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int k0 = k00 + 32 * u;
+                if (k0 >= nloc) break;
+                const int k = k0 + lane;
+                const int li = lbase + k;
+                const int id = idv[u];
+                const bool valid = (unsigned)id < (unsigned)E;
+                if (valid) tag[id] = (uint8_t)lane;
+                __syncwarp();
+                const int key = valid ? tag[id] : 0;
+                unsigned m = __ballot_sync(0xffffffffu, valid);
+#pragma unroll
+                for (int b = 0; b < 5; ++b) {
+                    const unsigned v = __ballot_sync(0xffffffffu, (key >> b) & 1);
+                    m &= ((key >> b) & 1) ? v : ~v;
                 }
-                if (pos < 0) atomicOr(da.err, 2);
-                if (staged) {
-                    s.stage[li] = pos;
-                    s.oli[s.rexp[id] + (j - s.base[id])] = (uint16_t)li;
-                } else if (pos >= 0) {
-                    da.src_index[pos] = (int32_t)(lo + li);
-                    if (da.gates != nullptr) da.gates_out[pos] = __ldg(da.gates + lo + li);
+                const int before = __popc(m & lt);
+                int out = -1;
+                if (valid) {
+                    const int j = wh[id] + before;
+                    const int2 t = s.tab[id];
+                    const int2 q = s.rc[t.x + covering_entry(s.rc + t.x, t.y & 0xffff, j)];
+                    out = q.y;
+                    int pos = -1;
+                    // Inside the slot's segment whenever the ids are the ones the
+                    // plan was computed from; anything else is reported, not written.
+                    if (out >= 0 && out < S) {
+                        pos = s.soff[out] + (j - q.x);
+                        if (pos < s.soff[out] || pos >= s.soff[out + 1] || (int64_t)pos >= da.L) pos = -1;
+                    }
+                    if (pos < 0) atomicOr(da.err, 2);
+                    if (staged) {
+                        s.stage[li] = pos;
+                        s.oli[s.rexp[id] + (j - s.base[id])] = (uint16_t)li;
+                    } else if (pos >= 0) {
+                        da.src_index[pos] = (int32_t)(lo + li);
+                        if (da.gates != nullptr) da.gates_out[pos] = __ldg(da.gates + lo + li);
+                    }
                 }
+                __syncwarp();
+                if (valid && before == 0) wh[id] += __popc(m);
+                __syncwarp();
+                if (k < nloc) phys[lo + li] = out;
             }
-            __syncwarp();
-            if (valid && before == 0) wh[id] += __popc(m);
-            __syncwarp();
-            if (k < nloc) phys[lo + li] = out;
         }
         if (staged) {
             // Write-out in (expert, j) order: consecutive threads take
@@ -410,65 +421,50 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
         }
     } else {
         __syncthreads();
-        // Replicated experts get their compact index; every other expert's table
-        // entry becomes its home slot (its only replica).
-        for (int m = threadIdx.x; m < M; m += blockDim.x) s.tab[s.rexp[m]].y |= m << 16;
+        // Every expert with one replica: its table entry becomes its home slot.
         for (int e = threadIdx.x; e < E; e += blockDim.x)
             if ((s.tab[e].y & 0xffff) == 1) s.tab[e].x = s.rc[s.tab[e].x].y;
         __syncthreads();
-        // Per (warp, replicated expert): ~slot when all the warp's occurrences of
-        // the expert share one replica, else the warp's first occurrence index.
-        for (int i = threadIdx.x; i < kRerouteWarps * M; i += blockDim.x) {
-            const int w = i / M, m = i - w * M;
-            const int e = s.rexp[m];
+        // Per-warp direct table code[w][e], each warp filling its own row: the
+        // slot of every id of e in warp w's part when they all fall into one
+        // replica (an expert with one replica always does), else -2 - j with j
+        // the occurrence index of the warp's next occurrence of e (updated as
+        // the warp goes).
+        int32_t *tb = s.code + warp * E;
+        for (int e = lane; e < E; e += 32) {
             const int2 t = s.tab[e];
             const int n = t.y & 0xffff;
-            const int excl = s.hist[w * E + e];
-            const int cnt = (w + 1 < kRerouteWarps ? s.hist[(w + 1) * E + e] : s.tot[e]) - excl;
-            const int j0 = s.base[e] + excl;
-            int lo = 0, hi = n - 1;                         // largest k with cum[k] <= j0
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (s.rc[t.x + mid].x <= j0) lo = mid;
-                else hi = mid - 1;
+            int c = t.x;
+            if (n > 1) {
+                const int excl = s.hist[warp * E + e];
+                const int cnt = (warp + 1 < kRerouteWarps ? s.hist[(warp + 1) * E + e] : s.tot[e]) - excl;
+                const int j0 = s.base[e] + excl;
+                const int k = covering_entry(s.rc + t.x, n, j0);
+                const bool uniform = k == n - 1 || j0 + cnt <= s.rc[t.x + k + 1].x;
+                c = uniform ? s.rc[t.x + k].y : -2 - j0;
             }
-            const bool uniform = lo == n - 1 || j0 + cnt <= s.rc[t.x + lo + 1].x;
-            s.code[w * M + m] = uniform ? ~s.rc[t.x + lo].y : j0;
+            tb[e] = c;
         }
-        const int nb = M > 1 ? 32 - __clz(M - 1) : 0;   // bits of the compact index
-        __syncthreads();
+        const int nbe = E > 1 ? 32 - __clz(E - 1) : 0;   // bits of an expert id
+        __syncwarp();
 
-        // Replica of one id; rank_it when its expert's quota boundary falls inside
-        // this warp's part (the occurrence index j is then needed).
-        auto lookup = [&](int id, int &out, int &v, int2 &t, bool &rank_it) {
-            const bool valid = (unsigned)id < (unsigned)E;
-            t = valid ? s.tab[id] : make_int2(-1, 1);
-            out = t.x;                                     // the home slot (a single replica); -1 for a bad id
-            v = 0;
-            if ((t.y & 0xffff) > 1) {
-                v = s.code[warp * M + (t.y >> 16)];
-                out = ~v;                                  // the warp's uniform replica, if v < 0
-            }
-            rank_it = (t.y & 0xffff) > 1 && v >= 0;
-        };
+        // Table entry of one id: its slot (>= 0), -1 for a bad id, or -2 - j
+        // (<= -2) when the id must be ranked to find its replica.
+        auto lookup = [&](int id) { return (unsigned)id < (unsigned)E ? tb[id] : -1; };
         // One scalar step of 32 consecutive ids (lane order = token-major order).
         auto step = [&](int id, int64_t i) {
-            int out, v;
-            int2 t;
-            bool rank_it;
-            lookup(id, out, v, t, rank_it);
-            if (__any_sync(0xffffffffu, rank_it)) {
-                const int cm = t.y >> 16;
-                const unsigned m = match_key(rank_it ? cm : -1, nb);
+            const int c = lookup(id);
+            int out = c;
+            if (__any_sync(0xffffffffu, c <= -2)) {
+                const unsigned m = match_key(c <= -2 ? id : -1, nbe);
                 const int before = __popc(m & lanemask_lt());
-                if (rank_it) {
-                    const int j = v + before;
-                    int k = (t.y & 0xffff) - 1;
-                    while (k > 0 && s.rc[t.x + k].x > j) --k;
-                    out = s.rc[t.x + k].y;
+                if (c <= -2) {
+                    const int j = -2 - c + before;
+                    const int2 t = s.tab[id];
+                    out = s.rc[t.x + covering_entry(s.rc + t.x, t.y & 0xffff, j)].y;
                 }
                 __syncwarp();
-                if (rank_it && before == 0) s.code[warp * M + cm] = v + __popc(m);
+                if (c <= -2 && before == 0) tb[id] = c - __popc(m);
                 __syncwarp();
             }
             if (i < whi) phys[i] = out;
@@ -476,38 +472,72 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
 
         // Pass 2: replica of every (t, k).
         if (vec) {
-            // Blocks of 128 ids, four per lane: when no id of the block needs its
-            // occurrence index, one 16-byte store per lane; otherwise the block is
-            // replayed as four ordered scalar steps.
-            for (int64_t v0 = wlo; v0 < whi; v0 += 128) {
-                const int64_t i = v0 + 4 * lane;
-                const int4 q = i < whi ? *reinterpret_cast<const int4 *>(s.stage + (i - lo)) : make_int4(-1, -1, -1, -1);
-                int o0, o1, o2, o3, v;
-                int2 t;
-                bool r0, r1, r2, r3;
-                lookup(q.x, o0, v, t, r0);
-                lookup(q.y, o1, v, t, r1);
-                lookup(q.z, o2, v, t, r2);
-                lookup(q.w, o3, v, t, r3);
-                if (!__any_sync(0xffffffffu, r0 || r1 || r2 || r3)) {
-                    if (i < whi) *reinterpret_cast<int4 *>(phys + i) = make_int4(o0, o1, o2, o3);
-                } else {
-    #pragma unroll
+            // Blocks of 128 ids, four per lane: when no id of the block needs
+            // ranking, one 16-byte store per lane; when the ids to rank all
+            // belong to one expert and the block's occurrences of it fall into
+            // one replica, likewise (the warp's running index just advances);
+            // otherwise the block is replayed as four ordered scalar steps.
+            for (int64_t v00 = wlo; v00 < whi; v00 += 128 * kUnroll) {
+                int4 qs[kUnroll];            // every block's ids in flight together
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) {
+                    const int64_t i = v00 + 128 * u + 4 * lane;
+                    qs[u] = i >= whi ? make_int4(-1, -1, -1, -1)
+                            : staged ? *reinterpret_cast<const int4 *>(s.stage + (i - lo))
+                                     : __ldg(reinterpret_cast<const int4 *>(ids + i));
+                }
+#pragma unroll
+                for (int ub = 0; ub < kUnroll; ++ub) {
+                    const int64_t v0 = v00 + 128 * ub;
+                    if (v0 >= whi) break;
+                    const int64_t i = v0 + 4 * lane;
+                    const int4 q = qs[ub];
+                    const int o0 = lookup(q.x), o1 = lookup(q.y), o2 = lookup(q.z), o3 = lookup(q.w);
+                    const bool r0 = o0 <= -2, r1 = o1 <= -2, r2 = o2 <= -2, r3 = o3 <= -2;
+                    if (!__any_sync(0xffffffffu, r0 || r1 || r2 || r3)) {
+                        if (i < whi) *reinterpret_cast<int4 *>(phys + i) = make_int4(o0, o1, o2, o3);
+                        continue;
+                    }
+                    int emn = INT_MAX, emx = -1;   // experts of this lane's ids to rank
+                    if (r0) emn = min(emn, q.x), emx = max(emx, q.x);
+                    if (r1) emn = min(emn, q.y), emx = max(emx, q.y);
+                    if (r2) emn = min(emn, q.z), emx = max(emx, q.z);
+                    if (r3) emn = min(emn, q.w), emx = max(emx, q.w);
+                    const int gmin = __reduce_min_sync(0xffffffffu, emn);
+                    const int gmax = __reduce_max_sync(0xffffffffu, emx);
+                    if (gmin == gmax) {
+                        const int cnt = (int)__reduce_add_sync(0xffffffffu, (unsigned)(r0 + r1 + r2 + r3));
+                        const int2 te = s.tab[gmin];
+                        const int vv = -2 - tb[gmin];     // the warp's next occurrence index of gmin
+                        const int k1 = covering_entry(s.rc + te.x, te.y & 0xffff, vv);
+                        const int k2 = covering_entry(s.rc + te.x, te.y & 0xffff, vv + cnt - 1);
+                        if (k1 == k2) {
+                            const int sl = s.rc[te.x + k1].y;
+                            if (i < whi)
+                                *reinterpret_cast<int4 *>(phys + i) =
+                                    make_int4(r0 ? sl : o0, r1 ? sl : o1, r2 ? sl : o2, r3 ? sl : o3);
+                            __syncwarp();
+                            if (lane == 0) tb[gmin] = -2 - (vv + cnt);
+                            __syncwarp();
+                            continue;
+                        }
+                    }
+#pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const int64_t iu = v0 + 32 * u + lane;
-                        step(iu < whi ? s.stage[iu - lo] : -1, iu);
+                        step(iu >= whi ? -1 : staged ? s.stage[iu - lo] : __ldg(ids + iu), iu);
                     }
                 }
             }
         } else {
             for (int64_t x0 = wlo; x0 < whi; x0 += 32 * kUnroll) {
                 int id[kUnroll];
-    #pragma unroll
+#pragma unroll
                 for (int u = 0; u < kUnroll; ++u) {
                     const int64_t i = x0 + u * 32 + lane;
                     id[u] = i >= whi ? -1 : (staged ? s.stage[i - lo] : __ldg(ids + i));
                 }
-    #pragma unroll
+#pragma unroll
                 for (int u = 0; u < kUnroll; ++u) step(id[u], x0 + u * 32 + lane);
             }
         }
@@ -539,8 +569,7 @@ cudaError_t launch_reroute(const Shape &sh, const Launch &ln, const int32_t *ids
     const int stage = stage_cap_for(sh, ln, false, false);
     return launch_ex(k_reroute<false>, (unsigned)(sh.N * ln.cluster), kRerouteWarps * 32,
                      reroute_smem_bytes(sh, false, stage, false), st, (unsigned)ln.cluster, pdl, ids, sh.per_rank, sh.E,
-                     sh.E + sh.NR, plan.rep_off, plan.rep_slot, plan.rep_cum, plan.rep_experts, plan.info,
-                     plan.rank_off, phys, stage, DispatchArgs{});
+                     sh.E + sh.NR, plan.rep_off, plan.rep_slot, plan.rep_cum, plan.rank_off, phys, stage, DispatchArgs{});
 }
 
 cudaError_t launch_dispatch(const Shape &sh, const Launch &ln, const int32_t *ids, const PlanDev &plan,
@@ -552,8 +581,7 @@ cudaError_t launch_dispatch(const Shape &sh, const Launch &ln, const int32_t *id
                           sh.N * sh.per_rank, sh.S};
     return launch_ex(k_reroute<true>, (unsigned)(sh.N * ln.cluster), kRerouteWarps * 32,
                      reroute_smem_bytes(sh, true, stage, gates), st, (unsigned)ln.cluster, pdl, ids, sh.per_rank, sh.E,
-                     sh.E + sh.NR, plan.rep_off, plan.rep_slot, plan.rep_cum, plan.rep_experts, plan.info,
-                     plan.rank_off, phys, stage, da);
+                     sh.E + sh.NR, plan.rep_off, plan.rep_slot, plan.rep_cum, plan.rank_off, phys, stage, da);
 }
 
 cudaError_t set_reroute_attributes(size_t max_smem)
