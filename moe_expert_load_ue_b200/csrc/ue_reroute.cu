@@ -291,14 +291,17 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
         }
     }
     __syncthreads();
-    // Exclusive scan over the warps per expert (in place) and CTA totals.
+    // Exclusive scan over the warps per expert (in place) and CTA totals; the
+    // 16 counts of an expert are loaded together before any is overwritten.
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int c[kRerouteWarps];
+#pragma unroll
+        for (int w = 0; w < kRerouteWarps; ++w) c[w] = s.hist[w * E + e];
         int run = 0;
 #pragma unroll
         for (int w = 0; w < kRerouteWarps; ++w) {
-            const int t = s.hist[w * E + e];
             s.hist[w * E + e] = run;
-            run += t;
+            run += c[w];
         }
         s.tot[e] = run;
     }
@@ -474,9 +477,10 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
         if (vec) {
             // Blocks of 128 ids, four per lane: when no id of the block needs
             // ranking, one 16-byte store per lane; when the ids to rank all
-            // belong to one expert and the block's occurrences of it fall into
-            // one replica, likewise (the warp's running index just advances);
-            // otherwise the block is replayed as four ordered scalar steps.
+            // belong to one expert, a scan of the lanes' counts ranks them (and
+            // when they fall into one replica, no search is needed); only a
+            // block with ids of two or more experts to rank is replayed as four
+            // ordered scalar steps.
             for (int64_t v00 = wlo; v00 < whi; v00 += 128 * kUnroll) {
                 int4 qs[kUnroll];            // every block's ids in flight together
 #pragma unroll
@@ -506,21 +510,42 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
                     const int gmin = __reduce_min_sync(0xffffffffu, emn);
                     const int gmax = __reduce_max_sync(0xffffffffu, emx);
                     if (gmin == gmax) {
-                        const int cnt = (int)__reduce_add_sync(0xffffffffu, (unsigned)(r0 + r1 + r2 + r3));
-                        const int2 te = s.tab[gmin];
-                        const int vv = -2 - tb[gmin];     // the warp's next occurrence index of gmin
-                        const int k1 = covering_entry(s.rc + te.x, te.y & 0xffff, vv);
-                        const int k2 = covering_entry(s.rc + te.x, te.y & 0xffff, vv + cnt - 1);
-                        if (k1 == k2) {
-                            const int sl = s.rc[te.x + k1].y;
-                            if (i < whi)
-                                *reinterpret_cast<int4 *>(phys + i) =
-                                    make_int4(r0 ? sl : o0, r1 ? sl : o1, r2 ? sl : o2, r3 ? sl : o3);
-                            __syncwarp();
-                            if (lane == 0) tb[gmin] = -2 - (vv + cnt);
-                            __syncwarp();
-                            continue;
+                        // One expert to rank: its occurrences in the block, in
+                        // token-major order, are lane by lane and x, y, z, w
+                        // within a lane, so an exclusive scan of the lanes'
+                        // counts gives each its occurrence index.
+                        const int mine = r0 + r1 + r2 + r3;
+                        int incl = mine;
+#pragma unroll
+                        for (int o = 1; o < 32; o <<= 1) {
+                            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                            if (lane >= o) incl += y;
                         }
+                        const int cnt = __shfl_sync(0xffffffffu, incl, 31);
+                        const int2 te = s.tab[gmin];
+                        const int n = te.y & 0xffff;
+                        const int vv = -2 - tb[gmin];     // the warp's next occurrence index of gmin
+                        const int k1 = covering_entry(s.rc + te.x, n, vv);
+                        const int k2 = covering_entry(s.rc + te.x, n, vv + cnt - 1);
+                        int j = vv + incl - mine;
+                        int p0 = o0, p1 = o1, p2 = o2, p3 = o3;
+                        if (k1 == k2) {                   // one replica for all of them
+                            const int sl = s.rc[te.x + k1].y;
+                            p0 = r0 ? sl : o0;
+                            p1 = r1 ? sl : o1;
+                            p2 = r2 ? sl : o2;
+                            p3 = r3 ? sl : o3;
+                        } else {
+                            if (r0) p0 = s.rc[te.x + covering_entry(s.rc + te.x, n, j++)].y;
+                            if (r1) p1 = s.rc[te.x + covering_entry(s.rc + te.x, n, j++)].y;
+                            if (r2) p2 = s.rc[te.x + covering_entry(s.rc + te.x, n, j++)].y;
+                            if (r3) p3 = s.rc[te.x + covering_entry(s.rc + te.x, n, j++)].y;
+                        }
+                        if (i < whi) *reinterpret_cast<int4 *>(phys + i) = make_int4(p0, p1, p2, p3);
+                        __syncwarp();
+                        if (lane == 0) tb[gmin] = -2 - (vv + cnt);
+                        __syncwarp();
+                        continue;
                     }
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
