@@ -47,12 +47,12 @@ TRAFFIC = {
     ("grad_reduce", "671B-class"): {
         "source": "moe_expert_load_ue_b200/csrc/ue_grad_reduce.cu",
         "sha256": "3503a95d76ce7d9ac8808ca3d9a351d3e71755bfeb60fc4a02b0e73bc6855973",
-        "dram_bytes": 7905447680, "algorithmic_bytes": 7927234560,
+        "dram_bytes": 7905546496, "algorithmic_bytes": 7927234560,
         "profile": "profiles/grad_reduce_and_sync_dram_671B-class.md"},
     ("sync", "671B-class"): {
         "source": "moe_expert_load_ue_b200/csrc/ue_sync.cu",
-        "sha256": "91512a937a653f349c4cd0560db05baf8b6173feef146d5e1abb6919fb878111",
-        "dram_bytes": 4962545920, "algorithmic_bytes": 5020581888,
+        "sha256": "b665e6bdb8798ed602856a77a966653df27c20822157ce0b62ea2de003b35571",
+        "dram_bytes": 4962380288, "algorithmic_bytes": 5020581888,
         "profile": "profiles/grad_reduce_and_sync_dram_671B-class.md"},
 }
 
