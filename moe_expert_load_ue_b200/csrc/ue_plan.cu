@@ -78,12 +78,14 @@ struct PlanSmem {
     int32_t *srem;        // [E]  their remainders
     int32_t *tmp;         // [NR+1] spread: the assignments of the expert being spread
     unsigned long long *key;   // [max(E, N)] packed sort keys (8-byte aligned)
+    unsigned long long *key2;  // [N] R = 1: packed keys of the eligible ranks
 };
 
 __host__ __device__ inline size_t plan_smem_words(int E, int N, int NR)
 {
     const int K = E > N ? E : N;
-    return (size_t)96 + 8 + (size_t)11 * E + (size_t)5 * N + 1 + (size_t)7 * NR + 1 + 2 + (size_t)2 * K;
+    return (size_t)96 + 8 + (size_t)11 * E + (size_t)5 * N + 1 + (size_t)7 * NR + 1 + 2 + (size_t)2 * K +
+           (size_t)2 * N;
 }
 
 // Word offsets are computed as integers from the (16-byte aligned) base of the
@@ -120,6 +122,7 @@ __device__ __forceinline__ PlanSmem carve(int32_t *p, int E, int N, int NR)
     s.tmp = p + o;       o += NR + 1;
     o = (o + 1) & ~1;                       // 8-byte alignment for the keys
     s.key = reinterpret_cast<unsigned long long *>(p + o);
+    s.key2 = s.key + (E > N ? E : N);
     return s;
 }
 
@@ -336,6 +339,7 @@ __device__ __forceinline__ void greedy_sorted(const PlanSmem &s, int K, int M1)
         if (lane < j) {
             s.afirst[e_l] = my_first;
             s.acnt[e_l] = my_end - my_first;
+            s.rem[m0 + lane] = my_first;          // cut start by overflow position
         }
     }
     if (lane == 0) {
@@ -658,16 +662,25 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, int variant, Pla
         s.acnt[e] = 0;
         s.afirst[e] = 0;
         s.alast[e] = -1;
-        if (e % H == H - 1) {
-            const int rank_sum = pin + ld;
-            s.before[h] = rank_sum;
-            s.spare[h] = Q - min(Q, rank_sum);
-        }
     }
-    // Overflow experts as packed keys: larger overflow first, then lower id.
-    int M1;
-    const int pos = block_excl_scan(my_ovf > 0 ? 1 : 0, s.ws, &M1);
-    if (my_ovf > 0) s.key[pos] = ((unsigned long long)(unsigned)my_ovf << 32) | (0xffffffffu - (unsigned)e);
+    // Rank tid's home load and spare, from the prefix of the loads.
+    int my_spare = 0;
+    if (tid < N) {
+        const int rank_sum = (tid + 1 < N ? s.pre[(tid + 1) * H] : L) - s.pre[tid * H];
+        my_spare = Q - min(Q, rank_sum);
+        s.before[tid] = rank_sum;
+        s.spare[tid] = my_spare;
+    }
+    // Overflow experts (larger overflow first, then lower id) and, for R = 1,
+    // the eligible ranks (spare > 0; larger spare first, then lower rank) as
+    // packed keys, both compacted by one scan (experts in the low 16 bits).
+    const bool eligible = R == 1 && my_spare > 0;
+    int packed_tot;
+    const int pk0 = block_excl_scan((my_ovf > 0 ? 1 : 0) | (eligible ? 1 << 16 : 0), s.ws, &packed_tot);
+    const int M1 = packed_tot & 0xffff, K = packed_tot >> 16;
+    if (my_ovf > 0) s.key[pk0 & 0xffff] = ((unsigned long long)(unsigned)my_ovf << 32) | (0xffffffffu - (unsigned)e);
+    if (eligible) s.key2[pk0 >> 16] = ((unsigned long long)(unsigned)my_spare << 32) | (0xffffffffu - (unsigned)tid);
+    if (tid == 0 && K == 0) s.rsum[0] = 0;        // no eligible rank: an empty prefix
     __syncthreads();
     if (tid < M1) {
         const unsigned long long mine = s.key[tid];
@@ -676,35 +689,25 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, int variant, Pla
         for (int k = 0; k < M1; ++k) rank += s.key[k] > mine ? 1 : 0;
         s.order[rank] = (int)(0xffffffffu - (unsigned)(mine & 0xffffffffu));
     }
+    if (tid < K) {
+        // Sorted position of this rank and the spares of the ranks before it.
+        const unsigned long long mine = s.key2[tid];
+        int rank = 0, before_sp = 0;
+#pragma unroll 8
+        for (int k = 0; k < K; ++k) {
+            const unsigned long long o = s.key2[k];
+            const bool gt = o > mine;
+            rank += gt ? 1 : 0;
+            before_sp += gt ? (int)(o >> 32) : 0;
+        }
+        s.rsorted[rank] = (int)(0xffffffffu - (unsigned)(mine & 0xffffffffu));
+        s.rsum[rank] = before_sp;
+        if (rank == K - 1) s.rsum[K] = before_sp + (int)(mine >> 32);
+    }
     __syncthreads();
 
     const bool requeue = kVariants && (variant & 1) != 0, spread = kVariants && (variant & 2) != 0;
     if (R == 1) {
-        // Eligible ranks (spare > 0) sorted by spare descending, lowest rank first.
-        const int sp_r = tid < N ? s.spare[tid] : 0;
-        int K;
-        const int kpos = block_excl_scan(sp_r > 0 ? 1 : 0, s.ws, &K);
-        if (sp_r > 0) s.key[kpos] = ((unsigned long long)(unsigned)sp_r << 32) | (0xffffffffu - (unsigned)tid);
-        __syncthreads();
-        int my_rank = 0, my_sp = 0;
-        if (tid < K) {
-            const unsigned long long mine = s.key[tid];
-            int rank = 0;
-#pragma unroll 8
-            for (int k = 0; k < K; ++k) rank += s.key[k] > mine ? 1 : 0;
-            my_rank = rank;
-            my_sp = (int)(mine >> 32);
-            s.rsorted[rank] = (int)(0xffffffffu - (unsigned)(mine & 0xffffffffu));
-        }
-        __syncthreads();
-        if (tid < K) s.rsum[my_rank] = my_sp;   // spares in sorted order
-        __syncthreads();
-        const int sp_sorted = tid < K ? s.rsum[tid] : 0;
-        int tot;
-        const int ex = block_excl_scan(sp_sorted, s.ws, &tot);
-        if (tid < K) s.rsum[tid] = ex;
-        if (tid == 0) s.rsum[K] = tot;
-        __syncthreads();
         if (requeue) {
             if (warp == 0) greedy_requeue<NRL>(s, N, R, M1, K);
         } else {
@@ -714,21 +717,29 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, int variant, Pla
             // positions of its cut; every rank is full except the last rank of an
             // expert that was placed completely (m before the stop), which takes
             // what is left of the expert's overflow.
-            if (tid < M1) {
-                const int em = s.order[tid];
-                const int a0 = s.afirst[em], na = s.acnt[em];
-                const bool placed = tid < s.misc[1];
-                for (int a = a0; a < a0 + na; ++a) {
-                    const int r = s.rsorted[a];
-                    int q = s.rsum[a + 1] - s.rsum[a];
-                    if (placed && a == a0 + na - 1) q = s.ovf[em] - (s.rsum[a] - s.rsum[a0]);
-                    s.ar[a] = r;
-                    s.au[a] = 0;
-                    s.ac[a] = q;
-                    s.ae[a] = em;
-                    s.sasg[r] = a;
-                    s.spare[r] -= q;
+            // One thread per assignment: its expert is the last overflow
+            // position (among those the walk reached) whose cut starts at or
+            // before it (s.rem holds the cut starts by position).
+            const int n_a = s.misc[0], stop = s.misc[1];
+            const int nproc = stop < M1 ? stop + 1 : M1;
+            for (int a = tid; a < n_a; a += nt) {
+                int lo = 0, hi = nproc - 1;
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (s.rem[mid] <= a) lo = mid;
+                    else hi = mid - 1;
                 }
+                const int em = s.order[lo];
+                const int a0 = s.rem[lo], na = s.acnt[em];
+                const int r = s.rsorted[a];
+                int q = s.rsum[a + 1] - s.rsum[a];
+                if (lo < stop && a == a0 + na - 1) q = s.ovf[em] - (s.rsum[a] - s.rsum[a0]);
+                s.ar[a] = r;
+                s.au[a] = 0;
+                s.ac[a] = q;
+                s.ae[a] = em;
+                s.sasg[r] = a;
+                s.spare[r] -= q;
             }
         }
     } else if (requeue) {
@@ -798,20 +809,38 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, int variant, Pla
     const int pk = block_excl_scan(packed, s.ws, &tot_packed);
     const int off = pk & 0xffff, mpos = pk >> 16;
     const int tot_rep = tot_packed & 0xffff, M = tot_packed >> 16;
+    // R = 1 under the stated rule: an expert's assignments are consecutive
+    // sorted positions and all but its last are full ranks, so the cumulative
+    // quota before assignment a is qh + rsum[a] - rsum[first]: one thread per
+    // assignment writes its entry.
+    const bool sorted_csr = R == 1 && !requeue && !spread;
     if (ve) {
         const int h = e / H;
         plan.rep_off[e] = off;
         plan.rep_slot[off] = h * HR + e % H;
         plan.rep_cum[off] = 0;
-        int cum = s.qh[e];
-        int a = s.afirst[e];
-        for (int i = 0; i < na_e; ++i) {
-            plan.rep_slot[off + 1 + i] = s.ar[a] * HR + H + s.au[a];
-            plan.rep_cum[off + 1 + i] = cum;
-            cum += s.ac[a];
-            a = requeue ? s.anext[a] : a + 1;
+        if (sorted_csr) {
+            s.pre[e] = off;                       // (reused) replica-list offset of e
+        } else {
+            int cum = s.qh[e];
+            int a = s.afirst[e];
+            for (int i = 0; i < na_e; ++i) {
+                plan.rep_slot[off + 1 + i] = s.ar[a] * HR + H + s.au[a];
+                plan.rep_cum[off + 1 + i] = cum;
+                cum += s.ac[a];
+                a = requeue ? s.anext[a] : a + 1;
+            }
         }
         if (na_e > 0) plan.rep_experts[mpos] = e;
+    }
+    if (sorted_csr) {
+        __syncthreads();
+        for (int a = tid; a < n_asg; a += nt) {
+            const int ea = s.ae[a], a0 = s.afirst[ea];
+            const int entry = s.pre[ea] + 1 + (a - a0);
+            plan.rep_slot[entry] = s.ar[a] * HR + H;
+            plan.rep_cum[entry] = s.qh[ea] + s.rsum[a] - s.rsum[a0];
+        }
     }
     if (tid == 0) plan.rep_off[E] = tot_rep;
     for (int p = tot_rep + tid; p < cap; p += nt) {
