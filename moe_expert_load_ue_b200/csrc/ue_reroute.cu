@@ -71,7 +71,8 @@ struct RerouteSmem {
                      //        (dispatch variant: [32] partial sums of the slot-offset scan)
     int32_t *tot;    // [E]    this CTA's counts (read by later CTAs of the cluster)
     int32_t *base;   // [E]    occurrences of e before this CTA's ids
-    int32_t *rexp;   // [E+1]  dispatch variant: exclusive prefix of this CTA's per-expert counts
+    int32_t *rexp;   // [E+1]  plain: the replicated experts and their count; dispatch variant:
+                     //        exclusive prefix of this CTA's per-expert counts
     int2 *tab;       // [E]    {home slot if one replica, else first replica entry; (compact index << 16) | count}
     int2 *rc;        // [cap]  {cumulative quota, slot} of each replica entry
     int32_t *soff;   // [S+1]  dispatch only: exclusive prefix of the slot quotas
@@ -324,6 +325,7 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
         for (int q = 0; q < kMaxCluster; ++q) b += peer[q];
         s.base[e] = b;            // occurrences of e before this CTA's ids
     }
+    if (!kDispatch && threadIdx.x == 0) s.rexp[E] = 0;   // count of the replicated-expert list
     cluster_arrive_relaxed();  // done reading peers; they may exit once all have arrived
     if constexpr (kDispatch) {
         // Slot offsets (exclusive prefix of the slot quotas; CTA 0 writes
@@ -424,29 +426,35 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
         }
     } else {
         __syncthreads();
-        // Every expert with one replica: its table entry becomes its home slot.
-        for (int e = threadIdx.x; e < E; e += blockDim.x)
-            if ((s.tab[e].y & 0xffff) == 1) s.tab[e].x = s.rc[s.tab[e].x].y;
+        // Every expert with one replica: its table entry becomes its home
+        // slot; the replicated experts are listed in rexp (any order).
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            const int2 t = s.tab[e];
+            if ((t.y & 0xffff) == 1) s.tab[e].x = s.rc[t.x].y;
+            else s.rexp[atomicAdd(&s.rexp[E], 1)] = e;
+        }
         __syncthreads();
         // Per-warp direct table code[w][e], each warp filling its own row: the
         // slot of every id of e in warp w's part when they all fall into one
         // replica (an expert with one replica always does), else -2 - j with j
         // the occurrence index of the warp's next occurrence of e (updated as
-        // the warp goes).
+        // the warp goes).  The row is the home slots copied, then the
+        // replicated experts' entries.
         int32_t *tb = s.code + warp * E;
-        for (int e = lane; e < E; e += 32) {
+#pragma unroll 4
+        for (int e = lane; e < E; e += 32) tb[e] = s.tab[e].x;
+        __syncwarp();
+        const int nrep = s.rexp[E];
+        for (int i = lane; i < nrep; i += 32) {
+            const int e = s.rexp[i];
             const int2 t = s.tab[e];
             const int n = t.y & 0xffff;
-            int c = t.x;
-            if (n > 1) {
-                const int excl = s.hist[warp * E + e];
-                const int cnt = (warp + 1 < kRerouteWarps ? s.hist[(warp + 1) * E + e] : s.tot[e]) - excl;
-                const int j0 = s.base[e] + excl;
-                const int k = covering_entry(s.rc + t.x, n, j0);
-                const bool uniform = k == n - 1 || j0 + cnt <= s.rc[t.x + k + 1].x;
-                c = uniform ? s.rc[t.x + k].y : -2 - j0;
-            }
-            tb[e] = c;
+            const int excl = s.hist[warp * E + e];
+            const int cnt = (warp + 1 < kRerouteWarps ? s.hist[(warp + 1) * E + e] : s.tot[e]) - excl;
+            const int j0 = s.base[e] + excl;
+            const int k = covering_entry(s.rc + t.x, n, j0);
+            const bool uniform = k == n - 1 || j0 + cnt <= s.rc[t.x + k + 1].x;
+            tb[e] = uniform ? s.rc[t.x + k].y : -2 - j0;
         }
         const int nbe = E > 1 ? 32 - __clz(E - 1) : 0;   // bits of an expert id
         __syncwarp();
@@ -476,11 +484,10 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
         // Pass 2: replica of every (t, k).
         if (vec) {
             // Blocks of 128 ids, four per lane: when no id of the block needs
-            // ranking, one 16-byte store per lane; when the ids to rank all
-            // belong to one expert, a scan of the lanes' counts ranks them (and
-            // when they fall into one replica, no search is needed); only a
-            // block with ids of two or more experts to rank is replayed as four
-            // ordered scalar steps.
+            // ranking, one 16-byte store per lane; otherwise the marked ids are
+            // ranked expert by expert with a warp scan of the lanes' counts
+            // (no search when an expert's occurrences here stay in one
+            // replica), then stored the same way.
             for (int64_t v00 = wlo; v00 < whi; v00 += 128 * kUnroll) {
                 int4 qs[kUnroll];            // every block's ids in flight together
 #pragma unroll
@@ -502,19 +509,23 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
                         if (i < whi) *reinterpret_cast<int4 *>(phys + i) = make_int4(o0, o1, o2, o3);
                         continue;
                     }
-                    int emn = INT_MAX, emx = -1;   // experts of this lane's ids to rank
-                    if (r0) emn = min(emn, q.x), emx = max(emx, q.x);
-                    if (r1) emn = min(emn, q.y), emx = max(emx, q.y);
-                    if (r2) emn = min(emn, q.z), emx = max(emx, q.z);
-                    if (r3) emn = min(emn, q.w), emx = max(emx, q.w);
-                    const int gmin = __reduce_min_sync(0xffffffffu, emn);
-                    const int gmax = __reduce_max_sync(0xffffffffu, emx);
-                    if (gmin == gmax) {
-                        // One expert to rank: its occurrences in the block, in
-                        // token-major order, are lane by lane and x, y, z, w
-                        // within a lane, so an exclusive scan of the lanes'
-                        // counts gives each its occurrence index.
-                        const int mine = r0 + r1 + r2 + r3;
+                    // Rank the marked ids expert by expert (the smallest expert
+                    // id first): an expert's occurrences in the block, in
+                    // token-major order, are lane by lane and x, y, z, w within
+                    // a lane, so an exclusive scan of the lanes' counts gives
+                    // each its occurrence index.
+                    int p0 = o0, p1 = o1, p2 = o2, p3 = o3;
+                    bool m0 = r0, m1 = r1, m2 = r2, m3 = r3;   // still to rank
+                    while (__any_sync(0xffffffffu, m0 || m1 || m2 || m3)) {
+                        int emn = INT_MAX;
+                        if (m0) emn = min(emn, q.x);
+                        if (m1) emn = min(emn, q.y);
+                        if (m2) emn = min(emn, q.z);
+                        if (m3) emn = min(emn, q.w);
+                        const int ex = __reduce_min_sync(0xffffffffu, emn);
+                        const bool h0 = m0 && q.x == ex, h1 = m1 && q.y == ex;
+                        const bool h2 = m2 && q.z == ex, h3 = m3 && q.w == ex;
+                        const int mine = h0 + h1 + h2 + h3;
                         int incl = mine;
 #pragma unroll
                         for (int o = 1; o < 32; o <<= 1) {
@@ -522,36 +533,33 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
                             if (lane >= o) incl += y;
                         }
                         const int cnt = __shfl_sync(0xffffffffu, incl, 31);
-                        const int2 te = s.tab[gmin];
+                        const int2 te = s.tab[ex];
                         const int n = te.y & 0xffff;
-                        const int vv = -2 - tb[gmin];     // the warp's next occurrence index of gmin
+                        const int vv = -2 - tb[ex];          // the warp's next occurrence index of ex
                         const int k1 = covering_entry(s.rc + te.x, n, vv);
                         const int k2 = covering_entry(s.rc + te.x, n, vv + cnt - 1);
-                        int j = vv + incl - mine;
-                        int p0 = o0, p1 = o1, p2 = o2, p3 = o3;
-                        if (k1 == k2) {                   // one replica for all of them
+                        if (k1 == k2) {                      // one replica for all of them
                             const int sl = s.rc[te.x + k1].y;
-                            p0 = r0 ? sl : o0;
-                            p1 = r1 ? sl : o1;
-                            p2 = r2 ? sl : o2;
-                            p3 = r3 ? sl : o3;
+                            p0 = h0 ? sl : p0;
+                            p1 = h1 ? sl : p1;
+                            p2 = h2 ? sl : p2;
+                            p3 = h3 ? sl : p3;
                         } else {
-                            if (r0) p0 = s.rc[te.x + covering_entry(s.rc + te.x, n, j++)].y;
-                            if (r1) p1 = s.rc[te.x + covering_entry(s.rc + te.x, n, j++)].y;
-                            if (r2) p2 = s.rc[te.x + covering_entry(s.rc + te.x, n, j++)].y;
-                            if (r3) p3 = s.rc[te.x + covering_entry(s.rc + te.x, n, j++)].y;
+                            int j = vv + incl - mine;
+                            if (h0) p0 = s.rc[te.x + covering_entry(s.rc + te.x, n, j++)].y;
+                            if (h1) p1 = s.rc[te.x + covering_entry(s.rc + te.x, n, j++)].y;
+                            if (h2) p2 = s.rc[te.x + covering_entry(s.rc + te.x, n, j++)].y;
+                            if (h3) p3 = s.rc[te.x + covering_entry(s.rc + te.x, n, j++)].y;
                         }
-                        if (i < whi) *reinterpret_cast<int4 *>(phys + i) = make_int4(p0, p1, p2, p3);
                         __syncwarp();
-                        if (lane == 0) tb[gmin] = -2 - (vv + cnt);
+                        if (lane == 0) tb[ex] = -2 - (vv + cnt);
                         __syncwarp();
-                        continue;
+                        m0 = m0 && !h0;
+                        m1 = m1 && !h1;
+                        m2 = m2 && !h2;
+                        m3 = m3 && !h3;
                     }
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int64_t iu = v0 + 32 * u + lane;
-                        step(iu >= whi ? -1 : staged ? s.stage[iu - lo] : __ldg(ids + iu), iu);
-                    }
+                    if (i < whi) *reinterpret_cast<int4 *>(phys + i) = make_int4(p0, p1, p2, p3);
                 }
             }
         } else {
