@@ -155,7 +155,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int32_t *ws, int *total)
     return r;
 }
 
-constexpr int kRowBatch = 8;   // rows of counts loaded per batch (all loads in flight together)
+constexpr int kRowBatch = 16;  // rows of counts loaded per batch (all loads in flight together)
 
 // Row slice [r0, r1) of counts summed per expert into part[e].
 __device__ __forceinline__ void slice_sums(const int32_t *__restrict__ counts, int E, int r0, int r1, int32_t *part)
