@@ -52,6 +52,7 @@ namespace {
 constexpr int kRerouteWarps = 16;
 constexpr int kUnroll = 4;
 constexpr int kStageIds = 8192;   // ids of a CTA share kept in shared memory between the passes
+constexpr int kRepCache = 64;     // replicated experts whose current replica each warp caches
 
 // Kernel-side view of the dispatch outputs (unused by the plain variant).
 struct DispatchArgs {
@@ -69,6 +70,8 @@ struct RerouteSmem {
     int32_t *hist;   // [W][E] per-warp counts, then their exclusive scan over the warps
     int32_t *code;   // [W][E] per warp and expert: its slot, or -2 - the warp's next occurrence index
                      //        (dispatch variant: [32] partial sums of the slot-offset scan)
+    int2 *cc;        // [W][kRepCache] plain: per warp and replicated expert (list position), the slot of
+                     //        the replica holding the warp's next occurrence and where that replica ends
     int32_t *tot;    // [E]    this CTA's counts (read by later CTAs of the cluster)
     int32_t *base;   // [E]    occurrences of e before this CTA's ids
     int32_t *rexp;   // [E+1]  plain: the replicated experts and their count; dispatch variant:
@@ -84,7 +87,10 @@ struct RerouteSmem {
 
 // Words of code[]: per (warp, replicated expert) for the plain variant; the
 // dispatch variant keeps only the warps' partial sums there.
-__host__ __device__ inline int code_words(int E, int S_disp) { return S_disp > 0 ? 32 : kRerouteWarps * E; }
+__host__ __device__ inline int code_words(int E, int S_disp)
+{
+    return S_disp > 0 ? 32 : kRerouteWarps * E + 2 * kRerouteWarps * kRepCache;
+}
 
 // Shared-memory words; S_disp = S for the dispatch variant, else 0; the
 // gates are staged beside the ids (gstage_cap = stage_cap) when carried.
@@ -106,6 +112,7 @@ __device__ __forceinline__ RerouteSmem carve(int32_t *base, int E, int cap, int 
     int o = 0;
     s.hist = base + o;   o += kRerouteWarps * E;
     s.code = base + o;   o += code_words(E, S_disp);
+    s.cc = reinterpret_cast<int2 *>(s.code + kRerouteWarps * E);   // plain variant (8-byte aligned)
     s.tot = base + o;    o += E;
     s.base = base + o;   o += E;
     s.rexp = base + o;   o += E + 1;
@@ -430,8 +437,13 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
         // slot; the replicated experts are listed in rexp (any order).
         for (int e = threadIdx.x; e < E; e += blockDim.x) {
             const int2 t = s.tab[e];
-            if ((t.y & 0xffff) == 1) s.tab[e].x = s.rc[t.x].y;
-            else s.rexp[atomicAdd(&s.rexp[E], 1)] = e;
+            if ((t.y & 0xffff) == 1) {
+                s.tab[e].x = s.rc[t.x].y;
+            } else {
+                const int pos = atomicAdd(&s.rexp[E], 1);
+                s.rexp[pos] = e;
+                s.tab[e].y = t.y | (pos << 16);   // the expert's position in the list
+            }
         }
         __syncthreads();
         // Per-warp direct table code[w][e], each warp filling its own row: the
@@ -455,6 +467,8 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
             const int k = covering_entry(s.rc + t.x, n, j0);
             const bool uniform = k == n - 1 || j0 + cnt <= s.rc[t.x + k + 1].x;
             tb[e] = uniform ? s.rc[t.x + k].y : -2 - j0;
+            if (!uniform && i < kRepCache)
+                s.cc[warp * kRepCache + i] = make_int2(s.rc[t.x + k].y, s.rc[t.x + k + 1].x);
         }
         const int nbe = E > 1 ? 32 - __clz(E - 1) : 0;   // bits of an expert id
         __syncwarp();
@@ -525,31 +539,46 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
                         const int ex = __reduce_min_sync(0xffffffffu, emn);
                         const bool h0 = m0 && q.x == ex, h1 = m1 && q.y == ex;
                         const bool h2 = m2 && q.z == ex, h3 = m3 && q.w == ex;
-                        const int mine = h0 + h1 + h2 + h3;
-                        int incl = mine;
-#pragma unroll
-                        for (int o = 1; o < 32; o <<= 1) {
-                            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                            if (lane >= o) incl += y;
-                        }
-                        const int cnt = __shfl_sync(0xffffffffu, incl, 31);
+                        const int cnt = __popc(__ballot_sync(0xffffffffu, h0)) + __popc(__ballot_sync(0xffffffffu, h1)) +
+                                        __popc(__ballot_sync(0xffffffffu, h2)) + __popc(__ballot_sync(0xffffffffu, h3));
                         const int2 te = s.tab[ex];
-                        const int n = te.y & 0xffff;
+                        const int n = te.y & 0xffff, ci = te.y >> 16;
                         const int vv = -2 - tb[ex];          // the warp's next occurrence index of ex
-                        const int k1 = covering_entry(s.rc + te.x, n, vv);
-                        const int k2 = covering_entry(s.rc + te.x, n, vv + cnt - 1);
-                        if (k1 == k2) {                      // one replica for all of them
-                            const int sl = s.rc[te.x + k1].y;
-                            p0 = h0 ? sl : p0;
-                            p1 = h1 ? sl : p1;
-                            p2 = h2 ? sl : p2;
-                            p3 = h3 ? sl : p3;
+                        const int2 cur = ci < kRepCache ? s.cc[warp * kRepCache + ci] : make_int2(-1, 0);
+                        if (cur.x >= 0 && vv + cnt < cur.y) {
+                            // All of them, and the next occurrence, in the cached replica.
+                            p0 = h0 ? cur.x : p0;
+                            p1 = h1 ? cur.x : p1;
+                            p2 = h2 ? cur.x : p2;
+                            p3 = h3 ? cur.x : p3;
                         } else {
-                            int j = vv + incl - mine;
-                            if (h0) p0 = s.rc[te.x + covering_entry(s.rc + te.x, n, j++)].y;
-                            if (h1) p1 = s.rc[te.x + covering_entry(s.rc + te.x, n, j++)].y;
-                            if (h2) p2 = s.rc[te.x + covering_entry(s.rc + te.x, n, j++)].y;
-                            if (h3) p3 = s.rc[te.x + covering_entry(s.rc + te.x, n, j++)].y;
+                            const int mine = h0 + h1 + h2 + h3;
+                            int incl = mine;
+#pragma unroll
+                            for (int o = 1; o < 32; o <<= 1) {
+                                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                                if (lane >= o) incl += y;
+                            }
+                            const int k1 = covering_entry(s.rc + te.x, n, vv);
+                            const int k2 = covering_entry(s.rc + te.x, n, vv + cnt - 1);
+                            if (k1 == k2) {                  // one replica for all of them
+                                const int sl = s.rc[te.x + k1].y;
+                                p0 = h0 ? sl : p0;
+                                p1 = h1 ? sl : p1;
+                                p2 = h2 ? sl : p2;
+                                p3 = h3 ? sl : p3;
+                            } else {
+                                int j = vv + incl - mine;
+                                if (h0) p0 = s.rc[te.x + covering_entry(s.rc + te.x, n, j++)].y;
+                                if (h1) p1 = s.rc[te.x + covering_entry(s.rc + te.x, n, j++)].y;
+                                if (h2) p2 = s.rc[te.x + covering_entry(s.rc + te.x, n, j++)].y;
+                                if (h3) p3 = s.rc[te.x + covering_entry(s.rc + te.x, n, j++)].y;
+                            }
+                            if (lane == 0 && ci < kRepCache) {   // the replica of the next occurrence
+                                const int k3 = covering_entry(s.rc + te.x, n, vv + cnt);
+                                s.cc[warp * kRepCache + ci] =
+                                    make_int2(s.rc[te.x + k3].y, k3 + 1 < n ? s.rc[te.x + k3 + 1].x : INT_MAX);
+                            }
                         }
                         __syncwarp();
                         if (lane == 0) tb[ex] = -2 - (vv + cnt);
