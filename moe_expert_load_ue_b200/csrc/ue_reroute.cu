@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(kRerouteWarps * 32)
 k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
           const int32_t *__restrict__ rep_off, const int32_t *__restrict__ rep_slot,
           const int32_t *__restrict__ rep_cum, const int32_t *__restrict__ rank_off,
-          int32_t *__restrict__ phys, int stage_cap, DispatchArgs da)
+          int32_t *__restrict__ phys, int H, int HR, int stage_cap, DispatchArgs da)
 {
     extern __shared__ __align__(16) int32_t sm_rr[];
     const RerouteSmem s = carve(sm_rr, E, cap, kDispatch ? da.S : 0, stage_cap,
@@ -213,6 +213,7 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
     const int lane = lane_id(), warp = threadIdx.x >> 5;
 
     for (int i = threadIdx.x; i < kRerouteWarps * E; i += blockDim.x) s.hist[i] = 0;
+    if (!kDispatch && threadIdx.x == 0) s.rexp[E] = 0;   // count of the replicated-expert list
     __syncthreads();
 
     // CTA share [lo, hi) of rank r's ids, and this warp's part [wlo, whi).
@@ -315,25 +316,45 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
     }
     cluster.sync();
 
+    // Still before the plan: the occurrences of e in the earlier CTAs of the
+    // cluster (peers' totals over DSMEM) and, for the plain variant, each
+    // warp's table row filled with the home slots (the plan never moves them).
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int peer[kMaxCluster];
+#pragma unroll
+        for (int q = 0; q < kMaxCluster; ++q) peer[q] = q < c ? cluster.map_shared_rank(s.tot, q)[e] : 0;
+        int b = 0;
+#pragma unroll
+        for (int q = 0; q < kMaxCluster; ++q) b += peer[q];
+        s.base[e] = b;
+    }
+    if (!kDispatch) {
+        int32_t *row = s.code + warp * E;
+        for (int e = lane; e < E; e += 32) {
+            const int hr = e / H;
+            row[e] = hr * HR + (e - hr * H);
+        }
+    }
+    cluster_arrive_relaxed();  // done reading peers; they may exit once all have arrived
+
     // The plan (and rank_off) of the preceding planner grid: every global load
     // of the plan is issued in one round.
     pdl_wait();
     for (int i = threadIdx.x; i < cap; i += blockDim.x) s.rc[i] = make_int2(__ldg(rep_cum + i), __ldg(rep_slot + i));
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         const int o0 = __ldg(rep_off + e), o1 = __ldg(rep_off + e + 1);
-        int b = __ldg(rank_off + (int64_t)r * E + e);
-        int peer[kMaxCluster];
-#pragma unroll
-        for (int q = 0; q < kMaxCluster; ++q) peer[q] = q < c ? cluster.map_shared_rank(s.tot, q)[e] : 0;
+        const int b = __ldg(rank_off + (int64_t)r * E + e);
         const int off = clampi(o0, 0, cap - 1);
         const int n = clampi(o1 - off, 1, min(cap - off, 0xffff));
-        s.tab[e] = make_int2(off, n);
-#pragma unroll
-        for (int q = 0; q < kMaxCluster; ++q) b += peer[q];
-        s.base[e] = b;            // occurrences of e before this CTA's ids
+        int packed = n;
+        if (!kDispatch && n > 1) {               // plain: list the replicated experts (any order)
+            const int pos = atomicAdd(&s.rexp[E], 1);
+            s.rexp[pos] = e;
+            packed |= pos << 16;                  // the expert's position in the list
+        }
+        s.tab[e] = make_int2(off, packed);
+        s.base[e] += b;           // occurrences of e before this CTA's ids
     }
-    if (!kDispatch && threadIdx.x == 0) s.rexp[E] = 0;   // count of the replicated-expert list
-    cluster_arrive_relaxed();  // done reading peers; they may exit once all have arrived
     if constexpr (kDispatch) {
         // Slot offsets (exclusive prefix of the slot quotas; CTA 0 writes
         // them out) and, for the local grouping below, the exclusive prefix
@@ -433,29 +454,13 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
         }
     } else {
         __syncthreads();
-        // Every expert with one replica: its table entry becomes its home
-        // slot; the replicated experts are listed in rexp (any order).
-        for (int e = threadIdx.x; e < E; e += blockDim.x) {
-            const int2 t = s.tab[e];
-            if ((t.y & 0xffff) == 1) {
-                s.tab[e].x = s.rc[t.x].y;
-            } else {
-                const int pos = atomicAdd(&s.rexp[E], 1);
-                s.rexp[pos] = e;
-                s.tab[e].y = t.y | (pos << 16);   // the expert's position in the list
-            }
-        }
-        __syncthreads();
-        // Per-warp direct table code[w][e], each warp filling its own row: the
-        // slot of every id of e in warp w's part when they all fall into one
-        // replica (an expert with one replica always does), else -2 - j with j
-        // the occurrence index of the warp's next occurrence of e (updated as
-        // the warp goes).  The row is the home slots copied, then the
-        // replicated experts' entries.
+        // Per-warp direct table code[w][e] (each warp its own row): the slot of
+        // every id of e in warp w's part when they all fall into one replica
+        // (an expert with one replica always does: its home slot, filled in
+        // before the plan), else -2 - j with j the occurrence index of the
+        // warp's next occurrence of e (updated as the warp goes).  Only the
+        // replicated experts' entries are computed here.
         int32_t *tb = s.code + warp * E;
-#pragma unroll 4
-        for (int e = lane; e < E; e += 32) tb[e] = s.tab[e].x;
-        __syncwarp();
         const int nrep = s.rexp[E];
         for (int i = lane; i < nrep; i += 32) {
             const int e = s.rexp[i];
@@ -631,7 +636,8 @@ cudaError_t launch_reroute(const Shape &sh, const Launch &ln, const int32_t *ids
     const int stage = stage_cap_for(sh, ln, false, false);
     return launch_ex(k_reroute<false>, (unsigned)(sh.N * ln.cluster), kRerouteWarps * 32,
                      reroute_smem_bytes(sh, false, stage, false), st, (unsigned)ln.cluster, pdl, ids, sh.per_rank, sh.E,
-                     sh.E + sh.NR, plan.rep_off, plan.rep_slot, plan.rep_cum, plan.rank_off, phys, stage, DispatchArgs{});
+                     sh.E + sh.NR, plan.rep_off, plan.rep_slot, plan.rep_cum, plan.rank_off, phys, sh.H, sh.HR, stage,
+                     DispatchArgs{});
 }
 
 cudaError_t launch_dispatch(const Shape &sh, const Launch &ln, const int32_t *ids, const PlanDev &plan,
@@ -643,7 +649,7 @@ cudaError_t launch_dispatch(const Shape &sh, const Launch &ln, const int32_t *id
                           sh.N * sh.per_rank, sh.S};
     return launch_ex(k_reroute<true>, (unsigned)(sh.N * ln.cluster), kRerouteWarps * 32,
                      reroute_smem_bytes(sh, true, stage, gates), st, (unsigned)ln.cluster, pdl, ids, sh.per_rank, sh.E,
-                     sh.E + sh.NR, plan.rep_off, plan.rep_slot, plan.rep_cum, plan.rank_off, phys, stage, da);
+                     sh.E + sh.NR, plan.rep_off, plan.rep_slot, plan.rep_cum, plan.rank_off, phys, sh.H, sh.HR, stage, da);
 }
 
 cudaError_t set_reroute_attributes(size_t max_smem)
