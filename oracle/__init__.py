@@ -30,6 +30,12 @@ Pinning status (what fixes each function other than itself; the tests under
                 previous plan, the incremental sync leaves exactly the state a
                 full sync gives; slots whose expert is unchanged are untouched;
                 the copied-slot count equals a numpy count.
+  sync_relay    after max(1, ceil(log2 G)) relay rounds (or the one direct round) the
+                state equals the single-GPU sync on tagged bytes, so a pull
+                from a GPU that had not yet received its copy shows; holders
+                per round double; every GPU sends at most one copy of an
+                expert per round; hand-worked schedules
+                (tests/golden/relay_cases.json).
   grad_reduce   exact closed-form sums on dyadic values; zero gradients
                 leave the master unchanged; numpy float32 reference order.
 
@@ -81,9 +87,12 @@ def _get():
             lib.ue_oracle_sync.argtypes = [vp, i64, i64, ci, ci, ci, vp]
             lib.ue_oracle_sync_delta.argtypes = [vp, i64, i64, ci, ci, ci, vp, vp, vp]
             lib.ue_oracle_grad_reduce.argtypes = [vp, i64, vp, ci, i64, i64, ci, ci, ci, vp, vp]
+            lib.ue_oracle_relay_rounds.argtypes = [ci]
+            lib.ue_oracle_sync_relay.argtypes = [vp, i64, i64, ci, ci, ci, vp, ci, ci, ci, vp]
             for f in ("ue_oracle_load", "ue_oracle_expert_load", "ue_oracle_plan", "ue_oracle_plan_ex",
                       "ue_oracle_reroute", "ue_oracle_dispatch", "ue_oracle_sync",
-                      "ue_oracle_sync_delta", "ue_oracle_grad_reduce"):
+                      "ue_oracle_sync_delta", "ue_oracle_grad_reduce", "ue_oracle_relay_rounds",
+                      "ue_oracle_sync_relay"):
                 getattr(lib, f).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -208,6 +217,27 @@ def sync_delta(W: np.ndarray, nbytes: int, E: int, N: int, R: int, slot_expert: 
                                      ctypes.byref(n))
     _check(rc, "sync_delta")
     return int(n.value)
+
+
+def relay_rounds(G: int) -> int:
+    """Relay rounds after which every holder of an expert has it: max(1, ceil(log2 G))."""
+    return int(_get().ue_oracle_relay_rounds(G))
+
+
+def sync_relay(W: np.ndarray, nbytes: int, E: int, N: int, R: int, slot_expert: np.ndarray,
+               G: int, round: int, dst_gpu: int = -1) -> np.ndarray:
+    """Step 4 over G GPUs: one relay round (round >= 0) or the direct form
+    (round = -1), in place on W viewed as bytes [S][slot_stride], writing only
+    destinations on GPU dst_gpu (all when -1).  Returns the expert copies each
+    GPU sent to other GPUs in this round."""
+    if not (W.flags.c_contiguous and W.ndim == 2):
+        raise OracleError("W must be a C-contiguous [S][stride] array")
+    stride = W.shape[1] * W.itemsize
+    egress = np.zeros(max(G, 1), np.int64)
+    rc = _get().ue_oracle_sync_relay(_p(W), stride, nbytes, E, N, R, _p(_c(slot_expert, np.int32)), G, round,
+                                     dst_gpu, _p(egress))
+    _check(rc, "sync_relay")
+    return egress
 
 
 def grad_reduce(master: np.ndarray, grads: np.ndarray, n: int, E: int, N: int, R: int,

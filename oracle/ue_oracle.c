@@ -452,6 +452,93 @@ int ue_oracle_sync_delta(uint8_t *W, int64_t slot_stride, int64_t nbytes,
     return ORC_OK;
 }
 
+/* ---- step 4 across GPUs: relay tree against fan-out overload --------------
+ * The news summary ("Comment fonctionne l'équilibrage en 300 microsecondes")
+ * streams expert states between GPUs with a relay mechanism against fan-out
+ * overload.  Reading taken here: the N ranks are spread over G GPUs, GPU g
+ * holding ranks [g*N/G, (g+1)*N/G) and so slots [g*SG, (g+1)*SG), SG = S/G.
+ * For an expert e with filled redundant slots, its holder list is
+ *     [home GPU of e, then every other GPU holding a filled redundant slot of
+ *      e, in increasing GPU id].
+ * Relay round k (k = 0, 1, ...): the holder at list position i, 2^k <= i <
+ * 2^(k+1), receives e from the holder at position i - 2^k (the home slot on
+ * the home GPU, else that GPU's lowest slot holding e, filled in an earlier
+ * round), and the received copy fills every redundant slot of e on that GPU.
+ * In round 0 the home GPU also fills its own redundant slots of e from the
+ * home slot.  After max(1, ceil(log2 G)) rounds every holder has e, and each
+ * GPU sends at most one copy of each expert per round.  round = -1 is the direct form:
+ * every redundant slot of e is filled from the home slot (the single-GPU sync),
+ * so the home GPU sends one copy to every other holder.
+ * Only destinations on GPU dst_gpu are written (every GPU when dst_gpu = -1).
+ * egress[G] (optional) receives, per GPU, the expert copies it sent to other
+ * GPUs in this round (for the destinations written).
+ */
+int ue_oracle_relay_rounds(int G)
+{
+    int k = 1;
+    while ((1 << k) < G) ++k;
+    return k;
+}
+
+int ue_oracle_sync_relay(uint8_t *W, int64_t slot_stride, int64_t nbytes,
+                         int E, int N, int R, const int32_t *slot_expert,
+                         int G, int round, int dst_gpu, int64_t *egress)
+{
+    if (E < 1 || N < 1 || R < 0 || E % N != 0 || nbytes > slot_stride || nbytes < 0) return ORC_BAD_ARG;
+    if (G < 1 || N % G != 0 || round < -1 || round >= 31 || dst_gpu < -1 || dst_gpu >= G) return ORC_BAD_ARG;
+    const int H = E / N, HR = H + R, S = N * HR, SG = S / G;
+    int *holder = (int *)malloc(sizeof(int) * (size_t)(G + 1));
+    if (!holder) return ORC_BAD_ARG;
+    if (egress) memset(egress, 0, sizeof(int64_t) * (size_t)G);
+    for (int s = 0; s < S; ++s)
+        if (slot_expert[s] >= E) { free(holder); return ORC_BAD_ARG; }
+    for (int e = 0; e < E; ++e) {
+        const int home = (e / H) * HR + (e % H);
+        const int hg = home / SG;
+        /* holder list: home GPU, then the other GPUs with a redundant slot of e */
+        int n = 0;
+        holder[n++] = hg;
+        for (int g = 0; g < G; ++g) {
+            if (g == hg) continue;
+            int has = 0;
+            for (int s = g * SG; s < (g + 1) * SG; ++s)
+                if (s % HR >= H && slot_expert[s] == e) has = 1;
+            if (has) holder[n++] = g;
+        }
+        for (int i = 0; i < n; ++i) {
+            const int dst = holder[i];
+            int src_pos;
+            if (round < 0) {
+                src_pos = 0;
+            } else if (i == 0) {
+                if (round != 0) continue;                  /* home's own replicas: round 0 */
+                src_pos = 0;
+            } else {
+                if (i < (1 << round) || i >= (2 << round)) continue;
+                src_pos = i - (1 << round);
+            }
+            if (dst_gpu >= 0 && dst != dst_gpu) continue;
+            const int src_gpu = holder[src_pos];
+            int src = home;
+            if (src_pos > 0) {
+                src = -1;
+                for (int s = src_gpu * SG; s < (src_gpu + 1) * SG && src < 0; ++s)
+                    if (s % HR >= H && slot_expert[s] == e) src = s;
+                if (src < 0) { free(holder); return ORC_INVARIANT; }
+            }
+            int wrote = 0;
+            for (int s = dst * SG; s < (dst + 1) * SG; ++s) {
+                if (s % HR < H || slot_expert[s] != e) continue;
+                memcpy(W + (int64_t)s * slot_stride, W + (int64_t)src * slot_stride, (size_t)nbytes);
+                wrote = 1;
+            }
+            if (wrote && src_gpu != dst && egress) egress[src_gpu] += 1;
+        }
+    }
+    free(holder);
+    return ORC_OK;
+}
+
 /* ---- step 5: replica gradient reduction -----------------------------------
  * For each expert e with redundant replicas, in replica order i = 1, 2, ...:
  *     master[e][x] = master[e][x] + float(grad[g(i)][x])
