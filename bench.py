@@ -432,6 +432,68 @@ def run_ours(args, dist: Dist):
                   "gbs": round(delta_bytes / (delta_us * 1e-6) / 1e9, 1) if delta_us > 0 else None}
     del plans2
 
+    # The calls across GPUs with G GPUs emulated as parts of this GPU's memory
+    # (each GPU's slots, home-expert master rows and replica-gradient rows):
+    # the relay rounds and the direct form of the weight sync, and the
+    # gradient reduction on the home GPUs, events around all launches of one
+    # microbatch.  Bytes that would cross NVLink are HBM traffic here.
+    G = 8 if w.N % 8 == 0 else 1
+    SG, EG, RG = w.S // G, w.E // G, (w.N // G) * w.R
+    slot_tabs = [weights[h * SG] for h in range(G)]
+    grad_tabs = [grads[h * RG] for h in range(G)] if w.R > 0 else None
+    rounds = ue.ue_relay_rounds(G)
+    n_sh = min(n_mb, 4)
+    evs_s = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_sh)]
+    with torch.cuda.stream(stream):
+        for k in range(-1, n_sh):                # one untimed pass first
+            mb = max(k, 0)
+            ue.ue_rebalance(ctx, cfg, ids_dev[mb], counts, bad, plan, phys, stream=stream)
+            e = evs_s[k] if k >= 0 else None
+            if e:
+                e[0].record(stream)
+            for r in range(rounds):
+                for h in range(G):
+                    ue.ue_sync_shard(ctx, cfg, G, h, slot_tabs, slot_bytes, plan, r, stream=stream)
+            if e:
+                e[1].record(stream)
+            for h in range(G):
+                ue.ue_sync_shard(ctx, cfg, G, h, slot_tabs, slot_bytes, plan, -1, stream=stream)
+            if e:
+                e[2].record(stream)
+            for h in range(G):
+                ue.ue_grad_reduce_shard(ctx, cfg, G, h, master[h * EG:(h + 1) * EG], grad_tabs, gdt, P, plan,
+                                        stream=stream)
+            if e:
+                e[3].record(stream)
+    stream.synchronize()
+    sh_pairs, sh_cross = [], []
+    for mb in range(n_sh):
+        se = per_mb[mb]["slot_expert"]
+        pairs = cross = 0
+        for e_ in np.unique(se[red & (se >= 0)]):
+            gpus = set((np.nonzero(red & (se == e_))[0] // SG).tolist())
+            hg = ((e_ // w.H) * (w.H + w.R)) // SG
+            pairs += len(gpus)
+            cross += len(gpus - {hg})
+        sh_pairs.append((pairs + int((red & (se >= 0)).sum())) * slot_bytes)
+        sh_cross.append(cross * slot_bytes)
+    t_relay = np.array([e[0].elapsed_time(e[1]) for e in evs_s]) * 1e3
+    t_direct = np.array([e[1].elapsed_time(e[2]) for e in evs_s]) * 1e3
+    t_grad = np.array([e[2].elapsed_time(e[3]) for e in evs_s]) * 1e3
+    sh_bytes = float(np.sum(sh_pairs))
+    across_gpus = {
+        "G": G, "ranks_per_gpu": w.N // G, "relay_rounds": rounds, "microbatches": n_sh,
+        "note": "G GPUs emulated as parts of one GPU's memory; the bytes that would cross NVLink are HBM traffic here",
+        "sync_alg_bytes_mean": int(sh_bytes / n_sh), "sync_nvlink_bytes_mean": int(np.mean(sh_cross)),
+        "sync_relay_us": round(float(t_relay.mean()), 1),
+        "sync_relay_gbs": round(sh_bytes / (t_relay.sum() * 1e-6) / 1e9, 1),
+        "sync_direct_us": round(float(t_direct.mean()), 1),
+        "sync_direct_gbs": round(sh_bytes / (t_direct.sum() * 1e-6) / 1e9, 1),
+        "grad_reduce_us": round(float(t_grad.mean()), 1),
+        "grad_reduce_gbs": round(float(grad_bytes[:n_sh].sum()) / (t_grad.sum() * 1e-6) / 1e9, 1),
+        "launches_per_microbatch": rounds * G + G + G,
+    }
+
     # Launch floor: one tiny kernel bracketed by events on the same stream.
     tiny = torch.zeros(1, device=dev)
     floor = []
@@ -532,6 +594,7 @@ def run_ours(args, dist: Dist):
         "grad_reduce_gbs": round(grad_gbs, 1), "grad_reduce_frac": round(grad_gbs / peak, 4),
         "frac_of_8000_gbs": {"sync": round(sync_gbs / 8000, 4), "grad_reduce": round(grad_gbs / 8000, 4)},
         "sync_delta": sync_delta,
+        "across_gpus_emulated": across_gpus,
         "plan_variants": plan_variants,
         "imbalance": {
             "before": round(float(np.mean([p["max_before"] / (p["L"] / w.N) for p in per_mb])), 4),

@@ -224,6 +224,72 @@ ue_status ue_grad_reduce(ue_ctx *ctx, const ue_config *cfg, float *master,
                          const void *grads, int grad_dtype, int64_t P,
                          const ue_plan_buffers *plan, void *stream);
 
+/* ---- across the GPUs of one NVLink domain ----------------------------------
+ * The N ranks spread over G GPUs: GPU g holds ranks [g*N/G, (g+1)*N/G), their
+ * tokens [g*T/G, (g+1)*T/G) (ids_local [T/G][K]), slots [g*SG, (g+1)*SG) with
+ * SG = S / G, the experts [g*E/G, (g+1)*E/G) homed on them (master_local
+ * [E/G][P]) and the replica-gradient rows [g*(N/G)*R, (g+1)*(N/G)*R)
+ * (N/G*R rows of P elements).  Per microbatch, on every GPU:
+ *   ue_load_shard -> all-gather of the counts rows (the caller's collective,
+ *   e.g. NCCL) -> ue_plan on the full counts (every GPU computes the same
+ *   plan) -> ue_reroute_shard -> ue_sync_shard for each relay round, with a
+ *   barrier across GPUs before each round after the first and after the last.
+ * In backward, after a barrier (every replica gradient written):
+ *   ue_grad_reduce_shard, then a barrier before replica gradients are reused.
+ * Peer tables are host arrays of G device pointers, entry h = GPU h's buffer
+ * as mapped on the calling GPU (peer access, CUDA IPC or symmetric memory),
+ * entry g = the calling GPU's own; each 16-byte aligned.  No kernel waits on
+ * another GPU; a copy never uses cluster multicast.  Limits: 1 <= G <= 128,
+ * N % G == 0, plus the limits above. */
+typedef struct {
+    int32_t G;   /* GPUs */
+    int32_t g;   /* the calling GPU, 0 <= g < G */
+} ue_shard;
+
+/* Step 1 for GPU g's ranks: writes rows [g*N/G, (g+1)*N/G) of counts [N][E]
+ * and the same entries of bad [N] (may be NULL); other rows are untouched. */
+ue_status ue_load_shard(ue_ctx *ctx, const ue_config *cfg, const ue_shard *shard,
+                        const int32_t *ids_local, int32_t *counts, int32_t *bad, void *stream);
+
+/* Step 3 for GPU g's tokens with the plan of the full counts (its rank_off
+ * rows for GPU g's ranks are read): phys_local [T/G][K] as ue_reroute's rows
+ * [g*T/G, (g+1)*T/G). */
+ue_status ue_reroute_shard(ue_ctx *ctx, const ue_config *cfg, const ue_shard *shard,
+                           const int32_t *ids_local, const ue_plan_buffers *plan,
+                           int32_t *phys_local, void *stream);
+
+/* Relay rounds needed for G GPUs: max(1, ceil(log2 G)); -1 if G is out of range. */
+int32_t ue_relay_rounds(int32_t G);
+
+/* Step 4 across GPUs with the relay against fan-out overload (news summary,
+ * "Comment fonctionne l'équilibrage en 300 microsecondes").  Holders of expert
+ * e = [its home GPU, then every other GPU with a filled redundant slot of e,
+ * in increasing GPU id].  Relay round k (0 <= k < ue_relay_rounds(G)): the
+ * holder at position i, 2^k <= i < 2^(k+1), copies e from the holder at
+ * position i - 2^k (the home slot, else that GPU's lowest slot holding e) into
+ * every one of its redundant slots of e; round 0 also fills the home GPU's own
+ * redundant slots.  round = -1: the direct form, every GPU copies from the home
+ * slot (one call instead of the rounds).  This call writes only GPU g's slots
+ * (slot_bases[g]) and reads home slots and, from round 1, slots other GPUs
+ * filled in earlier rounds.  After all rounds every GPU's slots hold what
+ * ue_sync gives.
+ *   slot_bases  [G] host array of device pointers, each GPU's SG slots of
+ *               slot_bytes bytes (multiple of 16). */
+ue_status ue_sync_shard(ue_ctx *ctx, const ue_config *cfg, const ue_shard *shard,
+                        void *const *slot_bases, int64_t slot_bytes,
+                        const ue_plan_buffers *plan, int32_t round, void *stream);
+
+/* Step 5 across GPUs: for every expert e homed on GPU g with redundant
+ * replicas, in replica order, master_local[e - g*E/G][x] += float(gradient of
+ * the replica), the replica's row read from the GPU holding its slot: row
+ * r*R + u of redundant slot r*(H+R) + H + u lives on GPU h = r / (N/G) at local
+ * row (r - h*N/G)*R + u of grad_bases[h].  The same adds in the same order as
+ * ue_grad_reduce, so the result is bit-identical.
+ *   grad_bases  [G] host array of device pointers (may be NULL when R = 0). */
+ue_status ue_grad_reduce_shard(ue_ctx *ctx, const ue_config *cfg, const ue_shard *shard,
+                               float *master_local, const void *const *grad_bases, int grad_dtype,
+                               int64_t P, const ue_plan_buffers *plan, void *stream);
+
 /* Status name, and the reason for the last non-OK status on this thread. */
 const char *ue_status_string(ue_status s);
 const char *ue_last_error(void);

@@ -12,7 +12,9 @@ cudaError_t set_load_attributes(size_t max_smem);
 cudaError_t set_reroute_attributes(size_t max_smem);
 cudaError_t set_plan_attributes(size_t max_smem);
 cudaError_t set_sync_attributes(size_t max_smem);
+cudaError_t set_shard_attributes(size_t max_smem);
 int grad_blocks_per_sm(int grad_dtype);
+int grad_shard_blocks_per_sm(int grad_dtype);
 }  // namespace ue
 
 struct ue_ctx {
@@ -20,6 +22,7 @@ struct ue_ctx {
     int sms;
     int max_smem;          // opt-in dynamic shared memory per block
     int grad_blocks[2];    // resident grad-reduce CTAs per SM (fp32, bf16)
+    int grad_shard_blocks[2];  // the same for the gradient reduction across GPUs
     int32_t *dev_err;      // device status word for bounded waits
 };
 
@@ -180,6 +183,9 @@ ue_status ue_ctx_create(int device, ue_ctx **out)
         if ((err = ue::set_sync_attributes(m)) != cudaSuccess) return cuda_fail(err, "sync attributes");
         tmp.grad_blocks[0] = ue::grad_blocks_per_sm(0);
         tmp.grad_blocks[1] = ue::grad_blocks_per_sm(1);
+        if ((err = ue::set_shard_attributes(m)) != cudaSuccess) return cuda_fail(err, "shard attributes");
+        tmp.grad_shard_blocks[0] = ue::grad_shard_blocks_per_sm(0);
+        tmp.grad_shard_blocks[1] = ue::grad_shard_blocks_per_sm(1);
         if ((err = cudaMalloc(&tmp.dev_err, sizeof(int32_t))) != cudaSuccess) return cuda_fail(err, "cudaMalloc");
         if ((err = cudaMemset(tmp.dev_err, 0, sizeof(int32_t))) != cudaSuccess) {
             cudaFree(tmp.dev_err);
@@ -443,6 +449,144 @@ ue_status ue_grad_reduce(ue_ctx *ctx, const ue_config *cfg, float *master, const
         ln.sms = ctx->sms * ctx->grad_blocks[grad_dtype];
         cudaError_t e = ue::launch_grad_reduce(sh, ln, master, grads, grad_dtype, P, ue::to_dev(*plan),
                                                static_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? UE_OK : cuda_fail(e, "grad-reduce launch");
+    });
+}
+
+// ---- calls across GPUs ---------------------------------------------------------
+
+namespace {
+ue_status check_shard(const ue::Shape &sh, const ue_shard *shard)
+{
+    if (!shard) return fail(UE_ERR_INVALID_ARG, "shard is NULL");
+    if (shard->G < 1 || shard->G > ue::kMaxGpus)
+        return fail(UE_ERR_INVALID_ARG, "G=%d outside [1, %d]", shard->G, ue::kMaxGpus);
+    if (sh.N % shard->G != 0) return fail(UE_ERR_INVALID_ARG, "N=%d is not a multiple of G=%d", sh.N, shard->G);
+    if (shard->g < 0 || shard->g >= shard->G) return fail(UE_ERR_INVALID_ARG, "g=%d not in [0, %d)", shard->g, shard->G);
+    return UE_OK;
+}
+
+// The shape of this GPU's ranks for the rank-per-cluster kernels: N / G ranks
+// and their tokens; everything that indexes slots or experts stays global.
+ue::Shape local_shape(const ue::Shape &sh, const ue_shard *shard)
+{
+    ue::Shape l = sh;
+    l.N = sh.N / shard->G;
+    l.T = sh.T / shard->G;
+    return l;
+}
+
+ue_status peer_table(const void *const *bases, int G, ue::PeerTable *t, const char *what)
+{
+    if (!bases) return fail(UE_ERR_INVALID_ARG, "%s is NULL", what);
+    for (int h = 0; h < ue::kMaxGpus; ++h) t->p[h] = nullptr;
+    for (int h = 0; h < G; ++h) {
+        if (!bases[h] || !aligned16(bases[h]))
+            return fail(UE_ERR_INVALID_ARG, "%s[%d] must be non-NULL and 16-byte aligned", what, h);
+        t->p[h] = bases[h];
+    }
+    return UE_OK;
+}
+}  // namespace
+
+int32_t ue_relay_rounds(int32_t G) { return G < 1 || G > ue::kMaxGpus ? -1 : ue::relay_rounds(G); }
+
+ue_status ue_load_shard(ue_ctx *ctx, const ue_config *cfg, const ue_shard *shard, const int32_t *ids_local,
+                        int32_t *counts, int32_t *bad, void *stream)
+{
+    ue::Shape sh{};
+    ue_status s = make_shape(cfg, true, &sh);
+    if (s == UE_OK) s = check_shard(sh, shard);
+    if (s != UE_OK) return s;
+    if (!counts) return fail(UE_ERR_INVALID_ARG, "counts is NULL");
+    const ue::Shape l = local_shape(sh, shard);
+    if (l.T > 0 && (!ids_local || !aligned16(ids_local)))
+        return fail(UE_ERR_INVALID_ARG, "ids_local must be non-NULL and 16-byte aligned");
+    if ((s = check_ctx(ctx)) != UE_OK) return s;
+    const int64_t r0 = (int64_t)shard->g * l.N;
+    return on_device(ctx, [&]() -> ue_status {
+        cudaError_t e = ue::launch_load(l, launch_of(ctx, l), ids_local, counts + r0 * sh.E, bad ? bad + r0 : nullptr,
+                                        static_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? UE_OK : cuda_fail(e, "load launch");
+    });
+}
+
+ue_status ue_reroute_shard(ue_ctx *ctx, const ue_config *cfg, const ue_shard *shard, const int32_t *ids_local,
+                           const ue_plan_buffers *plan, int32_t *phys_local, void *stream)
+{
+    ue::Shape sh{};
+    ue_status s = make_shape(cfg, true, &sh);
+    if (s == UE_OK) s = check_shard(sh, shard);
+    if (s == UE_OK) s = check_plan(plan);
+    if (s != UE_OK) return s;
+    const ue::Shape l = local_shape(sh, shard);
+    if (l.T > 0 && (!ids_local || !aligned16(ids_local)))
+        return fail(UE_ERR_INVALID_ARG, "ids_local must be non-NULL and 16-byte aligned");
+    if (l.T > 0 && !phys_local) return fail(UE_ERR_INVALID_ARG, "phys_local is NULL");
+    if ((s = check_ctx(ctx)) != UE_OK) return s;
+    if (ue::reroute_smem_bytes(l, false, 0, false) > (size_t)ctx->max_smem)
+        return fail(UE_ERR_INVALID_ARG, "reroute needs %zu bytes of shared memory (> %d)",
+                    ue::reroute_smem_bytes(l, false, 0, false), ctx->max_smem);
+    ue::PlanDev pd = ue::to_dev(*plan);
+    pd.rank_off += (int64_t)shard->g * l.N * sh.E;     // this GPU's rows of rank_off
+    return on_device(ctx, [&]() -> ue_status {
+        cudaError_t e = ue::launch_reroute(l, launch_of(ctx, l), ids_local, pd, phys_local,
+                                           static_cast<cudaStream_t>(stream), false);
+        return e == cudaSuccess ? UE_OK : cuda_fail(e, "reroute launch");
+    });
+}
+
+ue_status ue_sync_shard(ue_ctx *ctx, const ue_config *cfg, const ue_shard *shard, void *const *slot_bases,
+                        int64_t slot_bytes, const ue_plan_buffers *plan, int32_t round, void *stream)
+{
+    ue::Shape sh{};
+    ue_status s = make_shape(cfg, false, &sh);
+    if (s == UE_OK) s = check_shard(sh, shard);
+    if (s == UE_OK) s = check_plan(plan);
+    if (s != UE_OK) return s;
+    ue::PeerTable t;
+    if ((s = peer_table(const_cast<const void *const *>(slot_bases), shard->G, &t, "slot_bases")) != UE_OK) return s;
+    if (slot_bytes <= 0 || slot_bytes % 16 != 0)
+        return fail(UE_ERR_INVALID_ARG, "slot_bytes=%lld must be a positive multiple of 16", (long long)slot_bytes);
+    if (round < -1 || round >= ue::relay_rounds(shard->G))
+        return fail(UE_ERR_INVALID_ARG, "round=%d not in [-1, %d)", round, ue::relay_rounds(shard->G));
+    if ((s = check_ctx(ctx)) != UE_OK) return s;
+    if (ue::sync_shard_smem_bytes(sh) > (size_t)ctx->max_smem)
+        return fail(UE_ERR_INVALID_ARG, "sync needs %zu bytes of shared memory (> %d)", ue::sync_shard_smem_bytes(sh),
+                    ctx->max_smem);
+    return on_device(ctx, [&]() -> ue_status {
+        cudaError_t e = ue::launch_sync_shard(sh, launch_of(ctx, sh), t, static_cast<uint8_t *>(slot_bases[shard->g]),
+                                              shard->G, shard->g, round, slot_bytes, ue::to_dev(*plan), ctx->dev_err,
+                                              static_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? UE_OK : cuda_fail(e, "sync launch");
+    });
+}
+
+ue_status ue_grad_reduce_shard(ue_ctx *ctx, const ue_config *cfg, const ue_shard *shard, float *master_local,
+                               const void *const *grad_bases, int grad_dtype, int64_t P,
+                               const ue_plan_buffers *plan, void *stream)
+{
+    ue::Shape sh{};
+    ue_status s = make_shape(cfg, false, &sh);
+    if (s == UE_OK) s = check_shard(sh, shard);
+    if (s == UE_OK) s = check_plan(plan);
+    if (s != UE_OK) return s;
+    if (grad_dtype != 0 && grad_dtype != 1) return fail(UE_ERR_INVALID_ARG, "grad_dtype=%d (0 = fp32, 1 = bf16)", grad_dtype);
+    if (P <= 0 || P % 8 != 0) return fail(UE_ERR_INVALID_ARG, "P=%lld must be a positive multiple of 8", (long long)P);
+    if (!master_local || !aligned16(master_local))
+        return fail(UE_ERR_INVALID_ARG, "master_local must be non-NULL and 16-byte aligned");
+    ue::PeerTable t;
+    if (sh.NR > 0) {
+        if ((s = peer_table(grad_bases, shard->G, &t, "grad_bases")) != UE_OK) return s;
+    } else {
+        for (int h = 0; h < ue::kMaxGpus; ++h) t.p[h] = nullptr;
+    }
+    if ((s = check_ctx(ctx)) != UE_OK) return s;
+    return on_device(ctx, [&]() -> ue_status {
+        ue::Launch ln = launch_of(ctx, sh);
+        ln.sms = ctx->sms * ctx->grad_shard_blocks[grad_dtype];
+        cudaError_t e = ue::launch_grad_reduce_shard(sh, ln, master_local, t, shard->G, shard->g, grad_dtype, P,
+                                                     ue::to_dev(*plan), static_cast<cudaStream_t>(stream));
         return e == cudaSuccess ? UE_OK : cuda_fail(e, "grad-reduce launch");
     });
 }

@@ -15,6 +15,7 @@ constexpr int kMaxE = 1024;
 constexpr int kMaxN = 1024;
 constexpr int kMaxNR = 4096;
 constexpr int kMaxCluster = 8;        // portable cluster size
+constexpr int kMaxGpus = 128;         // GPUs of one NVLink domain for the calls across GPUs
 
 // Device-side view of the plan (same arrays as ue_plan_buffers).
 struct PlanDev {
@@ -27,6 +28,11 @@ inline PlanDev to_dev(const ue_plan_buffers &p)
     return PlanDev{p.slot_expert, p.slot_quota, p.rep_off, p.rep_slot, p.rep_cum, p.rep_experts,
                    p.load, p.rank_off, p.rank_load_before, p.rank_load_after, p.info};
 }
+
+// Per-GPU base pointers as mapped on the calling GPU (passed by value).
+struct PeerTable {
+    const void *p[kMaxGpus];
+};
 
 // Shape derived from ue_config.
 struct Shape {
@@ -77,6 +83,17 @@ size_t sync_smem_bytes(const Shape &sh);
 cudaError_t launch_grad_reduce(const Shape &sh, const Launch &ln, float *master, const void *grads,
                                int grad_dtype, int64_t P, const PlanDev &plan, cudaStream_t st);
 size_t grad_smem_bytes(const Shape &sh);
+
+// Calls across G GPUs (GPU g holds ranks [g*N/G, (g+1)*N/G)).  round >= 0 is
+// a relay round, -1 the direct form; relay_rounds(G) = max(1, ceil(log2 G)).
+int relay_rounds(int G);
+cudaError_t launch_sync_shard(const Shape &sh, const Launch &ln, const PeerTable &base, uint8_t *local, int G,
+                              int g, int round, int64_t slot_bytes, const PlanDev &plan, int32_t *dev_err,
+                              cudaStream_t st);
+size_t sync_shard_smem_bytes(const Shape &sh);
+cudaError_t launch_grad_reduce_shard(const Shape &sh, const Launch &ln, float *master, const PeerTable &grads,
+                                     int G, int g, int grad_dtype, int64_t P, const PlanDev &plan, cudaStream_t st);
+size_t grad_shard_smem_bytes(const Shape &sh);
 
 // Launch with an optional thread-block cluster (cluster > 1) and optional
 // programmatic dependent launch (pdl: the kernel may start while the previous

@@ -1,0 +1,363 @@
+// Steps 4 and 5 across the GPUs of one NVLink domain.
+//
+// Replica weight sync and replica gradient reduction when the N ranks are
+// spread over G GPUs: GPU g holds ranks [g*N/G, (g+1)*N/G), hence slots
+// [g*SG, (g+1)*SG) (SG = S / G), the experts homed on those ranks and the
+// replica-gradient rows of their redundant slots.  Transfers between GPUs use
+// the relay mechanism against fan-out overload (UltraEP news summary,
+// "Comment fonctionne l'équilibrage en 300 microsecondes"), read as a
+// doubling tree over each expert's holder GPUs:
+//     holders of e = [home GPU of e, then every other GPU with a filled
+//                     redundant slot of e, in increasing GPU id];
+// in relay round k the holder at position i, 2^k <= i < 2^(k+1), pulls e from
+// the holder at position i - 2^k (the home slot on the home GPU, else that
+// GPU's lowest slot holding e, filled in an earlier round); round 0 also fills
+// the home GPU's own redundant slots of e.  Round -1 is the direct form: every
+// GPU pulls from the home slot.  So a hot expert's home sends one copy per
+// round instead of one per receiving GPU.
+//
+// Design (sm_100a).  Sync: the single-GPU sync kernel's persistent ring of
+// TMA bulk copies, run on each GPU over the experts it receives in the round.
+// The global->shared bulk load reads the source GPU's slot through the
+// caller's peer mapping (no tensor map, no multicast); the shared->global bulk
+// stores write every local slot of the expert, so a tile crosses NVLink once
+// per receiving GPU however many of its ranks hold the expert.
+// Gradient reduction: the home GPU of each replicated expert pulls every
+// replica's gradient row from the GPU holding it, in replica order, with the
+// single-GPU kernel's fp32 adds, so its result is bit-identical to it.
+// Peer pointers are plain arguments; on one GPU the G "GPUs" may be parts of
+// one allocation.  No kernel here waits on another GPU: the caller orders the
+// rounds (a barrier across GPUs between them).
+#include <climits>
+
+#include "ue_internal.cuh"
+#include "ue_bulk.cuh"
+#include "ue_grad.cuh"
+
+namespace ue {
+namespace {
+
+// A set of GPU ids < kMaxGpus kept in registers (every index is unrolled).
+struct GpuSet {
+    uint32_t w[kMaxGpus / 32];
+
+    __device__ __forceinline__ void clear()
+    {
+#pragma unroll
+        for (int i = 0; i < kMaxGpus / 32; ++i) w[i] = 0;
+    }
+    __device__ __forceinline__ void add(int x)
+    {
+#pragma unroll
+        for (int i = 0; i < kMaxGpus / 32; ++i)
+            if ((x >> 5) == i) w[i] |= 1u << (x & 31);
+    }
+    // Members below x.
+    __device__ __forceinline__ int count_below(int x) const
+    {
+        int n = 0;
+#pragma unroll
+        for (int i = 0; i < kMaxGpus / 32; ++i) {
+            const int lo = i * 32;
+            if (x >= lo + 32) n += __popc(w[i]);
+            else if (x > lo) n += __popc(w[i] & ((1u << (x - lo)) - 1u));
+        }
+        return n;
+    }
+    // The q-th member (q >= 1) in increasing order; -1 if there are fewer.
+    __device__ __forceinline__ int select(int q) const
+    {
+#pragma unroll
+        for (int i = 0; i < kMaxGpus / 32; ++i) {
+            const int n = __popc(w[i]);
+            if (q <= n) {
+                uint32_t v = w[i];
+                for (int k = 1; k < q; ++k) v &= v - 1u;
+                return i * 32 + __ffs(v) - 1;
+            }
+            q -= n;
+        }
+        return -1;
+    }
+};
+
+__global__ void __launch_bounds__(kSyncThreads, 1)
+k_sync_shard(PeerTable base, uint8_t *__restrict__ local, int64_t slot_bytes, int E, int S, int SG, int G, int g,
+             int round, int cap, const int32_t *__restrict__ rep_off, const int32_t *__restrict__ rep_slot,
+             const int32_t *__restrict__ rep_experts, const int32_t *__restrict__ info,
+             int32_t *__restrict__ dev_err)
+{
+    extern __shared__ __align__(128) uint8_t sm_sync[];
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm_sync);                 // [stages]
+    uint8_t *stage = sm_sync + 128;                                        // [stages][tile]
+    const uint8_t **x_base = reinterpret_cast<const uint8_t **>(stage + (size_t)kSyncStages * kSyncTile);  // [G]
+    int32_t *x_src = reinterpret_cast<int32_t *>(x_base + kMaxGpus);      // [E] source slot (global id)
+    int32_t *x_first = x_src + E;                                          // [E] first destination entry
+    int32_t *x_cnt = x_first + E;                                          // [E] destinations on this GPU
+    int32_t *x_slot = x_cnt + E;                                           // [cap] local destination slots
+    int32_t *x_act = x_slot + cap;                                         // [E+1] experts with work; count
+
+    for (int i = threadIdx.x; i < G; i += blockDim.x) x_base[i] = static_cast<const uint8_t *>(base.p[i]);
+    // Per replicated expert: this GPU's slots of it, and where this round's copy comes from.
+    const int M = clampi(__ldg(info + 3), 0, E);
+    for (int m = threadIdx.x; m < M; m += blockDim.x) {
+        const int e = clampi(__ldg(rep_experts + m), 0, E - 1);
+        const int off = clampi(__ldg(rep_off + e), 0, cap - 1);
+        const int end = clampi(__ldg(rep_off + e + 1), off + 1, cap);
+        const int home = clampi(__ldg(rep_slot + off), 0, S - 1);
+        const int hg = home / SG;
+        GpuSet others;                       // holders other than the home GPU
+        others.clear();
+        int c = 0;
+        for (int p = off + 1; p < end; ++p) {
+            const int s = clampi(__ldg(rep_slot + p), 0, S - 1);
+            const int gp = s / SG;
+            if (gp != hg) others.add(gp);
+            if (gp == g) x_slot[off + 1 + c++] = s - g * SG;
+        }
+        int src = -1;
+        if (c > 0) {
+            if (g == hg) {
+                if (round <= 0) src = home;  // the home GPU's own replicas: round 0
+            } else {
+                const int i = 1 + others.count_below(g);   // this GPU's holder position
+                int q = -1;
+                if (round < 0) q = 0;
+                else if (i >= (1 << round) && i < (2 << round)) q = i - (1 << round);
+                if (q == 0) {
+                    src = home;
+                } else if (q > 0) {
+                    const int sg = others.select(q);
+                    int lo = INT_MAX;
+                    for (int p = off + 1; p < end; ++p) {
+                        const int s = clampi(__ldg(rep_slot + p), 0, S - 1);
+                        if (s / SG == sg && s < lo) lo = s;
+                    }
+                    src = lo == INT_MAX ? -1 : lo;
+                }
+            }
+        }
+        x_src[m] = src;
+        x_first[m] = off + 1;
+        x_cnt[m] = src >= 0 ? c : 0;
+    }
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kSyncStages; ++i) mbar_init(&bar[i], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {                  // compact the experts this GPU receives in this round
+        const int lane = threadIdx.x;
+        int n = 0;
+        for (int m0 = 0; m0 < M; m0 += 32) {
+            const int m = m0 + lane;
+            const bool a = m < M && x_cnt[m] > 0;
+            const unsigned b = __ballot_sync(0xffffffffu, a);
+            if (a) x_act[n + __popc(b & lanemask_lt())] = m;
+            n += __popc(b);
+        }
+        if (lane == 0) x_act[E] = n;
+    }
+    __syncthreads();
+    const int MA = x_act[E];
+    if (threadIdx.x != 0 || MA == 0) return;
+
+    const int64_t ntiles = (slot_bytes + kSyncTile - 1) / kSyncTile;
+    const int64_t total = (int64_t)MA * ntiles;
+    if ((int64_t)blockIdx.x >= total) return;
+    const int64_t nmy = (total - 1 - blockIdx.x) / gridDim.x + 1;
+
+    struct Item {
+        int m;
+        unsigned bytes;
+        int64_t offset;
+    };
+    auto item = [&](int64_t k) {
+        const int64_t i = (int64_t)blockIdx.x + k * gridDim.x;
+        Item it;
+        it.m = x_act[(int)(i % MA)];
+        it.offset = (i / MA) * kSyncTile;
+        const int64_t left = slot_bytes - it.offset;
+        it.bytes = (unsigned)(left < kSyncTile ? left : kSyncTile);
+        return it;
+    };
+    auto issue_load = [&](int64_t k) {
+        const Item it = item(k);
+        const int src = x_src[it.m];
+        const int sg = src / SG;
+        const uint8_t *p = x_base[sg] + (int64_t)(src - sg * SG) * slot_bytes + it.offset;
+        const int b = (int)(k % kSyncStages);
+        mbar_expect_tx(&bar[b], it.bytes);
+        bulk_load(stage + (size_t)b * kSyncTile, p, it.bytes, &bar[b]);
+    };
+
+    for (int64_t k = 0; k < nmy && k < kSyncStages; ++k) issue_load(k);
+    for (int64_t k = 0; k < nmy; ++k) {
+        const int b = (int)(k % kSyncStages);
+        const unsigned parity = (unsigned)((k / kSyncStages) & 1);
+        if (!mbar_try_wait(&bar[b], parity)) {
+            const unsigned long long t0 = global_ns();
+            while (!mbar_try_wait(&bar[b], parity)) {
+                if (global_ns() - t0 > kWaitLimitNs) {
+                    atomicOr(dev_err, 1);
+                    bulk_wait_all();
+                    return;
+                }
+            }
+        }
+        const Item it = item(k);
+        const uint8_t *src = stage + (size_t)b * kSyncTile;
+        const int first = x_first[it.m], cnt = x_cnt[it.m];
+        for (int j = 0; j < cnt; ++j)
+            bulk_store(local + (int64_t)x_slot[first + j] * slot_bytes + it.offset, src, it.bytes);
+        bulk_commit();
+        if (k >= 1 && k - 1 + kSyncStages < nmy) {
+            bulk_wait_read_1();
+            issue_load(k - 1 + kSyncStages);
+        }
+    }
+    bulk_wait_all();
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kGradThreads)
+k_grad_reduce_shard(float *__restrict__ master, PeerTable grads, int64_t P, int E, int S, int H, int HR, int R,
+                    int NG, int G, int g, int cap, const int32_t *__restrict__ rep_off,
+                    const int32_t *__restrict__ rep_slot, const int32_t *__restrict__ rep_experts,
+                    const int32_t *__restrict__ info)
+{
+    extern __shared__ __align__(16) uint8_t sm_grs[];
+    const void **x_base = reinterpret_cast<const void **>(sm_grs);            // [G]
+    int32_t *x_e = reinterpret_cast<int32_t *>(x_base + kMaxGpus);            // [E] local master row of m
+    int32_t *x_first = x_e + E;                                               // [E]
+    int32_t *x_cnt = x_first + E;                                             // [E]
+    int32_t *x_act = x_cnt + E;                                               // [E+1]
+    int32_t *x_loc = x_act + E + 1;                                           // [cap] gpu << 16 | local row
+
+    for (int i = threadIdx.x; i < G; i += blockDim.x) x_base[i] = grads.p[i];
+    const int EG = E / G;
+    const int M = R > 0 ? clampi(__ldg(info + 3), 0, E) : 0;
+    for (int m = threadIdx.x; m < M; m += blockDim.x) {
+        const int e = clampi(__ldg(rep_experts + m), 0, E - 1);
+        const int off = clampi(__ldg(rep_off + e), 0, cap - 1);
+        const int end = clampi(__ldg(rep_off + e + 1), off + 1, cap);
+        x_e[m] = e - g * EG;
+        x_first[m] = off + 1;
+        x_cnt[m] = e / EG == g ? end - off - 1 : 0;   // reduced on its home GPU only
+    }
+    for (int p = threadIdx.x; p < cap; p += blockDim.x) {
+        const int s = clampi(__ldg(rep_slot + p), 0, S - 1);
+        const int r = s / HR, u = s % HR - H;          // u < 0 for home slots
+        const int h = r / NG;
+        x_loc[p] = u >= 0 ? (h << 16) | ((r - h * NG) * R + u) : 0;
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        int n = 0;
+        for (int m0 = 0; m0 < M; m0 += 32) {
+            const int m = m0 + lane;
+            const bool a = m < M && x_cnt[m] > 0;
+            const unsigned b = __ballot_sync(0xffffffffu, a);
+            if (a) x_act[n + __popc(b & lanemask_lt())] = m;
+            n += __popc(b);
+        }
+        if (lane == 0) x_act[E] = n;
+    }
+    __syncthreads();
+    const int MA = x_act[E];
+
+    const int64_t nchunks = (P + kChunk - 1) / kChunk;
+    const int64_t total = (int64_t)MA * nchunks;
+    for (int64_t it = blockIdx.x; it < total; it += gridDim.x) {
+        const int m = x_act[(int)(it / nchunks)];
+        const int64_t x = (it % nchunks) * kChunk + (int64_t)threadIdx.x * kElemsPerThread;
+        if (x >= P) continue;
+        float4 *mp = reinterpret_cast<float4 *>(master + (int64_t)x_e[m] * P + x);
+        const float4 a = __ldcs(mp), b = __ldcs(mp + 1);
+        F8 acc;
+        acc.v[0] = a.x; acc.v[1] = a.y; acc.v[2] = a.z; acc.v[3] = a.w;
+        acc.v[4] = b.x; acc.v[5] = b.y; acc.v[6] = b.z; acc.v[7] = b.w;
+        const int first = x_first[m], cnt = x_cnt[m];
+        for (int j0 = 0; j0 < cnt; j0 += kBatch) {
+            F8 gv[kBatch];
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j)
+                if (j0 + j < cnt) {
+                    const int loc = x_loc[first + j0 + j];
+                    gv[j] = load8<BF16>(x_base[loc >> 16], (int64_t)(loc & 0xffff) * P + x);
+                }
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j)
+                if (j0 + j < cnt) add8(acc, gv[j]);
+        }
+        __stcs(mp, make_float4(acc.v[0], acc.v[1], acc.v[2], acc.v[3]));
+        __stcs(mp + 1, make_float4(acc.v[4], acc.v[5], acc.v[6], acc.v[7]));
+    }
+}
+
+}  // namespace
+
+int relay_rounds(int G)
+{
+    int k = 1;
+    while ((1 << k) < G) ++k;
+    return k;
+}
+
+size_t sync_shard_smem_bytes(const Shape &sh)
+{
+    return 128 + (size_t)kSyncStages * kSyncTile + kMaxGpus * sizeof(void *) +
+           (size_t)(3 * sh.E + sh.E + sh.NR + sh.E + 1) * sizeof(int32_t);
+}
+
+size_t grad_shard_smem_bytes(const Shape &sh)
+{
+    return kMaxGpus * sizeof(void *) + (size_t)(4 * sh.E + 1 + sh.E + sh.NR) * sizeof(int32_t);
+}
+
+cudaError_t launch_sync_shard(const Shape &sh, const Launch &ln, const PeerTable &base, uint8_t *local, int G,
+                              int g, int round, int64_t slot_bytes, const PlanDev &plan, int32_t *dev_err,
+                              cudaStream_t st)
+{
+    k_sync_shard<<<ln.sms, kSyncThreads, sync_shard_smem_bytes(sh), st>>>(
+        base, local, slot_bytes, sh.E, sh.S, sh.S / G, G, g, round, sh.E + sh.NR, plan.rep_off, plan.rep_slot,
+        plan.rep_experts, plan.info, dev_err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_grad_reduce_shard(const Shape &sh, const Launch &ln, float *master, const PeerTable &grads,
+                                     int G, int g, int grad_dtype, int64_t P, const PlanDev &plan, cudaStream_t st)
+{
+    const size_t smem = grad_shard_smem_bytes(sh);
+    const int cap = sh.E + sh.NR, NG = sh.N / G;
+    if (grad_dtype == 1)
+        k_grad_reduce_shard<true><<<ln.sms, kGradThreads, smem, st>>>(master, grads, P, sh.E, sh.S, sh.H, sh.HR,
+                                                                      sh.R, NG, G, g, cap, plan.rep_off,
+                                                                      plan.rep_slot, plan.rep_experts, plan.info);
+    else
+        k_grad_reduce_shard<false><<<ln.sms, kGradThreads, smem, st>>>(master, grads, P, sh.E, sh.S, sh.H, sh.HR,
+                                                                       sh.R, NG, G, g, cap, plan.rep_off,
+                                                                       plan.rep_slot, plan.rep_experts, plan.info);
+    return cudaGetLastError();
+}
+
+int grad_shard_blocks_per_sm(int grad_dtype)
+{
+    int n = 0;
+    const cudaError_t e =
+        grad_dtype == 1
+            ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_grad_reduce_shard<true>, kGradThreads, 32 * 1024)
+            : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_grad_reduce_shard<false>, kGradThreads, 32 * 1024);
+    return (e == cudaSuccess && n > 0) ? n : 1;
+}
+
+cudaError_t set_shard_attributes(size_t max_smem)
+{
+    cudaError_t e = allow_smem(k_sync_shard, max_smem);
+    if (e == cudaSuccess) e = allow_smem(k_grad_reduce_shard<true>, max_smem);
+    if (e == cudaSuccess) e = allow_smem(k_grad_reduce_shard<false>, max_smem);
+    return e;
+}
+
+}  // namespace ue

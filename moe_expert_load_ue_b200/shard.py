@@ -1,0 +1,102 @@
+"""The balancer across the GPUs of one NVLink domain: the order of the calls.
+
+The N expert-parallel ranks are spread over G GPUs, one process per GPU
+(torch.distributed); GPU g holds ranks [g*N/G, (g+1)*N/G) with their tokens,
+slots, home experts and replica-gradient rows (include/ue.h, "across the GPUs
+of one NVLink domain").  The path has two kinds of exchange between GPUs, and
+this module issues them in order around the library's sharded calls:
+
+- after the per-rank histograms (load computation), an all-gather of the
+  counts rows, so that every GPU plans from the same [N][E] counts and
+  computes the same plan (placement planning is deterministic) with its
+  per-rank offsets for routing expansion;
+- barriers across GPUs that order the relay rounds of the replica weight sync
+  (a GPU pulls in round k only from holders filled before it) and fence the
+  replica gradient reduction (every replica gradient written before the home
+  GPUs read them; all reads done before the buffers are reused).
+
+The device steps go through `ops` (`DeviceOps`: the C ABI on this GPU); the
+exchanges through the process group.  With the NCCL backend a barrier is an
+all-reduce of one element on the current stream, so the kernels after it on
+that stream start only once every GPU has reached it.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+from . import ue
+
+
+class DeviceOps:
+    """The sharded C-ABI calls for GPU g of G."""
+
+    def __init__(self, ctx: ue.Context, cfg: ue.Config, G: int, g: int, variant: int = 0):
+        self.ctx, self.cfg, self.G, self.g, self.variant = ctx, cfg, G, g, variant
+
+    def load(self, ids_local, counts, bad):
+        ue.ue_load_shard(self.ctx, self.cfg, self.G, self.g, ids_local, counts, bad)
+
+    def plan(self, counts, plan):
+        ue.ue_plan_ex(self.ctx, self.cfg, counts, plan, self.variant)
+
+    def reroute(self, ids_local, plan, phys_local):
+        ue.ue_reroute_shard(self.ctx, self.cfg, self.G, self.g, ids_local, plan, phys_local)
+
+    def sync(self, slot_bases, slot_bytes, plan, round):
+        ue.ue_sync_shard(self.ctx, self.cfg, self.G, self.g, slot_bases, slot_bytes, plan, round)
+
+    def grad_reduce(self, master_local, grad_bases, grads_dtype, P, plan):
+        ue.ue_grad_reduce_shard(self.ctx, self.cfg, self.G, self.g, master_local, grad_bases, grads_dtype, P, plan)
+
+
+class ShardedBalancer:
+    """Per-microbatch sequence of one GPU (g of G = the process group's size
+    and rank unless given)."""
+
+    def __init__(self, cfg: ue.Config, ops, G: int | None = None, g: int | None = None, group=None,
+                 device: str | torch.device = "cuda"):
+        self.cfg, self.ops, self.group = cfg, ops, group
+        self.G = G if G is not None else (dist.get_world_size(group) if dist.is_initialized() else 1)
+        self.g = g if g is not None else (dist.get_rank(group) if dist.is_initialized() else 0)
+        if cfg.N % self.G != 0:
+            raise ValueError(f"N={cfg.N} is not a multiple of G={self.G}")
+        self.NG = cfg.N // self.G
+        self._token = torch.zeros(1, dtype=torch.int32, device=device)
+
+    @property
+    def relay_rounds(self) -> int:
+        return ue.ue_relay_rounds(self.G)
+
+    def barrier(self) -> None:
+        if self.G > 1:
+            dist.all_reduce(self._token, group=self.group)
+
+    def rebalance(self, ids_local, counts, bad, plan, phys_local) -> None:
+        """Load computation for this GPU's ranks, all-gather of the counts
+        rows (and bad-id rows), placement planning on the full counts, routing
+        expansion of this GPU's tokens."""
+        self.ops.load(ids_local, counts, bad)
+        if self.G > 1:
+            lo, hi = self.g * self.NG, (self.g + 1) * self.NG
+            dist.all_gather_into_tensor(counts, counts[lo:hi].clone(), group=self.group)
+            if bad is not None:
+                dist.all_gather_into_tensor(bad, bad[lo:hi].clone(), group=self.group)
+        self.ops.plan(counts, plan)
+        self.ops.reroute(ids_local, plan, phys_local)
+
+    def sync(self, slot_bases, slot_bytes: int, plan, relay: bool = True) -> None:
+        """Replica weight sync: the relay rounds (or the direct form), a
+        barrier before each round after the first and after the last."""
+        rounds = range(self.relay_rounds) if relay else (-1,)
+        for i, k in enumerate(rounds):
+            if i > 0:
+                self.barrier()
+            self.ops.sync(slot_bases, slot_bytes, plan, k)
+        self.barrier()
+
+    def grad_reduce(self, master_local, grad_bases, grads_dtype, P: int, plan) -> None:
+        """Replica gradient reduction on the home GPUs, fenced by barriers."""
+        self.barrier()
+        self.ops.grad_reduce(master_local, grad_bases, grads_dtype, P, plan)
+        self.barrier()

@@ -26,7 +26,8 @@ PLAN_FIELDS = ("slot_expert", "slot_quota", "rep_off", "rep_slot", "rep_cum", "r
 # Entry points declared in include/ue.h (checked against the header by the tests).
 EXPORTS = ("ue_plan_sizes", "ue_ctx_create", "ue_ctx_destroy", "ue_ctx_device_error", "ue_load",
            "ue_plan", "ue_plan_ex", "ue_reroute", "ue_rebalance", "ue_rebalance_ex", "ue_dispatch", "ue_rebalance_dispatch", "ue_sync", "ue_sync_delta",
-           "ue_grad_reduce", "ue_status_string", "ue_last_error")
+           "ue_grad_reduce", "ue_load_shard", "ue_reroute_shard", "ue_relay_rounds", "ue_sync_shard",
+           "ue_grad_reduce_shard", "ue_status_string", "ue_last_error")
 
 
 class UeConfig(ctypes.Structure):
@@ -41,6 +42,10 @@ class UePlanBuffers(ctypes.Structure):
 class UeDispatchBuffers(ctypes.Structure):
     _fields_ = [("gates", ctypes.c_void_p), ("slot_off", ctypes.c_void_p), ("src_index", ctypes.c_void_p),
                 ("gates_out", ctypes.c_void_p)]
+
+
+class UeShard(ctypes.Structure):
+    _fields_ = [("G", ctypes.c_int32), ("g", ctypes.c_int32)]
 
 
 class UeError(RuntimeError):
@@ -65,6 +70,7 @@ def lib() -> ctypes.CDLL:
             vp, i64, ci = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
             cfgp, planp = ctypes.POINTER(UeConfig), ctypes.POINTER(UePlanBuffers)
             dispp = ctypes.POINTER(UeDispatchBuffers)
+            shardp, vpp = ctypes.POINTER(UeShard), ctypes.POINTER(ctypes.c_void_p)
             sig = {
                 "ue_plan_sizes": [cfgp, ctypes.POINTER(ctypes.c_int64)],
                 "ue_ctx_create": [ci, ctypes.POINTER(vp)],
@@ -81,6 +87,11 @@ def lib() -> ctypes.CDLL:
                 "ue_sync": [vp, cfgp, vp, i64, planp, vp],
                 "ue_sync_delta": [vp, cfgp, vp, i64, planp, vp, vp],
                 "ue_grad_reduce": [vp, cfgp, vp, vp, ci, i64, planp, vp],
+                "ue_load_shard": [vp, cfgp, shardp, vp, vp, vp, vp],
+                "ue_reroute_shard": [vp, cfgp, shardp, vp, planp, vp, vp],
+                "ue_relay_rounds": [ctypes.c_int32],
+                "ue_sync_shard": [vp, cfgp, shardp, vpp, i64, planp, ctypes.c_int32, vp],
+                "ue_grad_reduce_shard": [vp, cfgp, shardp, vp, vpp, ci, i64, planp, vp],
             }
             for name, args in sig.items():
                 fn = getattr(L, name)
@@ -291,3 +302,53 @@ def ue_grad_reduce(ctx: Context, cfg: Config, master: torch.Tensor, grads: torch
         raise TypeError("replica grads must be float32 or bfloat16")
     _check(lib().ue_grad_reduce(ctx.handle, ctypes.byref(cfg.c()), _ptr(master), _ptr(grads), dt, int(P),
                                 plan.ref(), _stream(stream)), "ue_grad_reduce")
+
+
+# ---- across the GPUs of one NVLink domain ------------------------------------
+
+def _grad_dtype(grads_dtype) -> int:
+    if grads_dtype == torch.bfloat16:
+        return 1
+    if grads_dtype == torch.float32:
+        return 0
+    raise TypeError("replica grads must be float32 or bfloat16")
+
+
+def _peer_table(bases) -> ctypes.Array:
+    """Host array of device pointers from tensors or integer addresses."""
+    ptrs = [b if isinstance(b, int) else b.data_ptr() for b in bases]
+    return (ctypes.c_void_p * len(ptrs))(*ptrs)
+
+
+def ue_relay_rounds(G: int) -> int:
+    return int(lib().ue_relay_rounds(int(G)))
+
+
+def ue_load_shard(ctx: Context, cfg: Config, G: int, g: int, ids_local: torch.Tensor, counts: torch.Tensor,
+                  bad: torch.Tensor | None = None, stream=None) -> None:
+    _check(lib().ue_load_shard(ctx.handle, ctypes.byref(cfg.c()), ctypes.byref(UeShard(G, g)), _ptr(ids_local),
+                               _ptr(counts), _ptr(bad), _stream(stream)), "ue_load_shard")
+
+
+def ue_reroute_shard(ctx: Context, cfg: Config, G: int, g: int, ids_local: torch.Tensor, plan: Plan,
+                     phys_local: torch.Tensor, stream=None) -> None:
+    _check(lib().ue_reroute_shard(ctx.handle, ctypes.byref(cfg.c()), ctypes.byref(UeShard(G, g)), _ptr(ids_local),
+                                  plan.ref(), _ptr(phys_local), _stream(stream)), "ue_reroute_shard")
+
+
+def ue_sync_shard(ctx: Context, cfg: Config, G: int, g: int, slot_bases, slot_bytes: int, plan: Plan,
+                  round: int, stream=None) -> None:
+    """slot_bases: G tensors or device addresses, GPU h's slots as mapped on this GPU."""
+    t = _peer_table(slot_bases)
+    _check(lib().ue_sync_shard(ctx.handle, ctypes.byref(cfg.c()), ctypes.byref(UeShard(G, g)), t, int(slot_bytes),
+                               plan.ref(), int(round), _stream(stream)), "ue_sync_shard")
+
+
+def ue_grad_reduce_shard(ctx: Context, cfg: Config, G: int, g: int, master_local: torch.Tensor, grad_bases,
+                         grads_dtype, P: int, plan: Plan, stream=None) -> None:
+    """grad_bases: G tensors or device addresses (GPU h's replica-gradient rows);
+    grads_dtype: torch.float32 or torch.bfloat16."""
+    t = None if grad_bases is None else _peer_table(grad_bases)
+    _check(lib().ue_grad_reduce_shard(ctx.handle, ctypes.byref(cfg.c()), ctypes.byref(UeShard(G, g)),
+                                      _ptr(master_local), t, _grad_dtype(grads_dtype), int(P), plan.ref(),
+                                      _stream(stream)), "ue_grad_reduce_shard")

@@ -24,7 +24,7 @@ def L():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return set(re.findall(r"^\s*(?:const\s+char\s*\*\s*|ue_status\s+)(ue_\w+)\s*\(", text, flags=re.M))
+    return set(re.findall(r"^\s*(?:const\s+char\s*\*\s*|ue_status\s+|int32_t\s+)(ue_\w+)\s*\(", text, flags=re.M))
 
 
 def test_exports_match_header(L):
@@ -204,3 +204,58 @@ def test_plan_variant_refused(L):
     assert L.ue_rebalance_ex(FAKE_CTX, ctypes.byref(c), ids_p, counts.ctypes.data, None, ctypes.byref(hp.c),
                              phys.ctypes.data, -1, None) == 1
     assert hp.untouched() and (phys == 7).all()
+
+
+def test_relay_rounds(L):
+    assert [L.ue_relay_rounds(G) for G in (1, 2, 3, 4, 5, 8, 9, 64, 72, 128)] == [1, 1, 2, 2, 3, 3, 4, 6, 7, 7]
+    assert L.ue_relay_rounds(0) == -1 and L.ue_relay_rounds(129) == -1
+
+
+def test_shard_refusals(L):
+    hp = _HostPlan()
+    c = ue.UeConfig(16, 4, 1, 8, 64)
+    ids = np.zeros(64 * 8 + 4, np.int32)
+    ids_p = ids.ctypes.data + (-ids.ctypes.data % 16)
+    counts = np.full(64, 7, np.int32)
+    phys = np.full(512, 7, np.int32)
+
+    def load(G, g, ip=ids_p):
+        return L.ue_load_shard(FAKE_CTX, ctypes.byref(c), ctypes.byref(ue.UeShard(G, g)), ip, counts.ctypes.data,
+                               None, None)
+
+    for G, g, msg in ((0, 0, "G=0"), (129, 0, "G=129"), (3, 0, "multiple of G"), (2, 2, "g=2"), (2, -1, "g=-1")):
+        assert load(G, g) == 1 and msg in L.ue_last_error().decode(), (G, g)
+    assert load(2, 1, ids_p + 4) == 1 and "aligned" in L.ue_last_error().decode()
+    assert L.ue_load_shard(FAKE_CTX, ctypes.byref(c), None, ids_p, counts.ctypes.data, None, None) == 1
+    assert L.ue_reroute_shard(FAKE_CTX, ctypes.byref(c), ctypes.byref(ue.UeShard(2, 0)), ids_p, ctypes.byref(hp.c),
+                              None, None) == 1 and "phys_local" in L.ue_last_error().decode()
+
+    w = np.zeros(4096, np.uint8)
+    base = w.ctypes.data + (-w.ctypes.data % 16)
+    ok = (ctypes.c_void_p * 2)(base, base + 1024)
+
+    def sync(tab, rd, nbytes=64, G=2):
+        return L.ue_sync_shard(FAKE_CTX, ctypes.byref(c), ctypes.byref(ue.UeShard(G, 0)), tab, nbytes,
+                               ctypes.byref(hp.c), rd, None)
+
+    assert sync(None, 0) == 1 and "slot_bases" in L.ue_last_error().decode()
+    assert sync((ctypes.c_void_p * 2)(base, base + 8), 0) == 1 and "slot_bases[1]" in L.ue_last_error().decode()
+    assert sync((ctypes.c_void_p * 2)(base, None), 0) == 1
+    assert sync(ok, 0, nbytes=40) == 1 and "slot_bytes" in L.ue_last_error().decode()
+    assert sync(ok, 1) == 1 and "round=1" in L.ue_last_error().decode()       # G = 2: one round
+    assert sync(ok, -2) == 1 and "round=-2" in L.ue_last_error().decode()
+    four = (ctypes.c_void_p * 4)(base, base + 1024, base + 2048, base + 3072)
+    assert sync(four, 2, G=4) == 1 and "round=2" in L.ue_last_error().decode()
+
+    m = np.zeros(64, np.float32)
+
+    def grad(mp, tab, dt=0, P=8):
+        return L.ue_grad_reduce_shard(FAKE_CTX, ctypes.byref(c), ctypes.byref(ue.UeShard(2, 1)), mp, tab, dt, P,
+                                      ctypes.byref(hp.c), None)
+
+    mp = m.ctypes.data + (-m.ctypes.data % 16)
+    assert grad(mp, ok, dt=2) == 1 and "grad_dtype" in L.ue_last_error().decode()
+    assert grad(mp, ok, P=12) == 1 and "P=12" in L.ue_last_error().decode()
+    assert grad(mp + 4, ok) == 1 and "master_local" in L.ue_last_error().decode()
+    assert grad(mp, None) == 1 and "grad_bases" in L.ue_last_error().decode()
+    assert hp.untouched() and (counts == 7).all() and (phys == 7).all() and (w == 0).all()
