@@ -42,17 +42,18 @@ VARIANTS = {"requeue": 1, "spread": 2, "requeue+spread": 3}     # plan variant b
 # dram__bytes_write.sum) next to that launch's algorithmic bytes, per kernel
 # and full-size workload; summarised in profiles/.  The JSON's roofline.traffic
 # scales the measured ratio to the mean launch of the run, and is null when the
-# kernel's source no longer matches the one that was captured.
+# kernel's sources (its file and header, hashed together) no longer match the
+# ones that were captured.
 TRAFFIC = {
     ("grad_reduce", "671B-class"): {
-        "source": "moe_expert_load_ue_b200/csrc/ue_grad_reduce.cu",
-        "sha256": "3503a95d76ce7d9ac8808ca3d9a351d3e71755bfeb60fc4a02b0e73bc6855973",
-        "dram_bytes": 7905546496, "algorithmic_bytes": 7927234560,
+        "sources": ["moe_expert_load_ue_b200/csrc/ue_grad_reduce.cu", "moe_expert_load_ue_b200/csrc/ue_grad.cuh"],
+        "sha256": "c1f443d9b89c58c94a8a2c0f2cfc98dc4a9e957d73ae8be1947f66c895057371",
+        "dram_bytes": 7905483008, "algorithmic_bytes": 7927234560,
         "profile": "profiles/grad_reduce_and_sync_dram_671B-class.md"},
     ("sync", "671B-class"): {
-        "source": "moe_expert_load_ue_b200/csrc/ue_sync.cu",
-        "sha256": "b665e6bdb8798ed602856a77a966653df27c20822157ce0b62ea2de003b35571",
-        "dram_bytes": 4962380288, "algorithmic_bytes": 5020581888,
+        "sources": ["moe_expert_load_ue_b200/csrc/ue_sync.cu", "moe_expert_load_ue_b200/csrc/ue_bulk.cuh"],
+        "sha256": "191ad325243d74d5e0543fed305057763301e296b4f5889e597257146ad53a9b",
+        "dram_bytes": 4961509632, "algorithmic_bytes": 5020581888,
         "profile": "profiles/grad_reduce_and_sync_dram_671B-class.md"},
 }
 
@@ -62,11 +63,14 @@ def traffic_per_launch(kernel: str, workload: str, full_size: bool, mean_alg: fl
     if t is None or not full_size:
         return None
     import hashlib
+    m = hashlib.sha256()
     try:
-        with open(os.path.join(ROOT, t["source"]), "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest() != t["sha256"]:
-                return None
+        for src in t["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                m.update(f.read())
     except OSError:
+        return None
+    if m.hexdigest() != t["sha256"]:
         return None
     return round(t["dram_bytes"] / t["algorithmic_bytes"] * mean_alg)
 
