@@ -216,29 +216,34 @@ NVLINK_GBS = 770.0     # measured peer copy per direction per GPU on this machine's
 
 def nvlink_model(slot_expert, w, G, slot_bytes, gbs):
     """Bytes each GPU sends and receives between GPUs in each relay round and
-    in the direct form, from the plan's slot table (holders of an expert: its
-    home GPU, then the other GPUs with a filled redundant slot of it in
-    increasing id; round k: holder i in [2^k, 2^(k+1)) receives from holder
-    i - 2^k), and the resulting time if every round ran at `gbs` per direction
-    on its busiest GPU."""
+    in the direct form, from the plan's slot table (consumers of an expert: the
+    GPUs other than its home GPU with a filled redundant slot of it, in
+    increasing id; the slot cut into f parts of q = 16*ceil(slot_bytes/(16 f))
+    bytes; round 0: consumer j receives part j from the home; round 1: each
+    consumer receives every other part from its consumer), and the resulting
+    time if every round ran at `gbs` per direction on its busiest GPU."""
     SG = w.S // G
     red = (np.arange(w.S) % (w.H + w.R)) >= w.H
-    rounds = 1
-    while (1 << rounds) < G:
-        rounds += 1
+    rounds = 1 if G <= 2 else 2
     eg_r, in_r = np.zeros((rounds, G)), np.zeros((rounds, G))
     eg_d, in_d = np.zeros(G), np.zeros(G)
     for e in np.unique(slot_expert[red & (slot_expert >= 0)]):
         hg = ((e // w.H) * (w.H + w.R)) // SG
-        others = sorted(set((np.nonzero(red & (slot_expert == e))[0] // SG).tolist()) - {hg})
-        holders = [hg] + others
-        for i in range(1, len(holders)):
-            k = i.bit_length() - 1                   # 2^k <= i < 2^(k+1)
-            src = holders[i - (1 << k)]
-            eg_r[k, src] += slot_bytes
-            in_r[k, holders[i]] += slot_bytes
+        cons = sorted(set((np.nonzero(red & (slot_expert == e))[0] // SG).tolist()) - {hg})
+        f = len(cons)
+        if f == 0:
+            continue
+        q = 16 * -(-slot_bytes // (16 * f))
+        part = [max(0, min(q, slot_bytes - j * q)) for j in range(f)]
+        for j, c in enumerate(cons):
+            eg_r[0, hg] += part[j]
+            in_r[0, c] += part[j]
             eg_d[hg] += slot_bytes
-            in_d[holders[i]] += slot_bytes
+            in_d[c] += slot_bytes
+            for i, d in enumerate(cons):
+                if i != j:
+                    eg_r[1, c] += part[j]
+                    in_r[1, d] += part[j]
     per_round = np.maximum(eg_r.max(axis=1), in_r.max(axis=1))
     return {"relay_us": float(per_round.sum() / (gbs * 1e9) * 1e6),
             "direct_us": float(max(eg_d.max(), in_d.max()) / (gbs * 1e9) * 1e6),

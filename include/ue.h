@@ -258,21 +258,23 @@ ue_status ue_reroute_shard(ue_ctx *ctx, const ue_config *cfg, const ue_shard *sh
                            const int32_t *ids_local, const ue_plan_buffers *plan,
                            int32_t *phys_local, void *stream);
 
-/* Relay rounds needed for G GPUs: max(1, ceil(log2 G)); -1 if G is out of range. */
+/* Relay rounds for G GPUs: 1 when G <= 2, else 2; -1 if G is out of range. */
 int32_t ue_relay_rounds(int32_t G);
 
 /* Step 4 across GPUs with the relay against fan-out overload (news summary,
- * "Comment fonctionne l'équilibrage en 300 microsecondes").  Holders of expert
- * e = [its home GPU, then every other GPU with a filled redundant slot of e,
- * in increasing GPU id].  Relay round k (0 <= k < ue_relay_rounds(G)): the
- * holder at position i, 2^k <= i < 2^(k+1), copies e from the holder at
- * position i - 2^k (the home slot, else that GPU's lowest slot holding e) into
- * every one of its redundant slots of e; round 0 also fills the home GPU's own
- * redundant slots.  round = -1: the direct form, every GPU copies from the home
- * slot (one call instead of the rounds).  This call writes only GPU g's slots
- * (slot_bases[g]) and reads home slots and, from round 1, slots other GPUs
- * filled in earlier rounds.  After all rounds every GPU's slots hold what
- * ue_sync gives.
+ * "Comment fonctionne l'équilibrage en 300 microsecondes"), as a scatter then
+ * an all-gather.  The consumers of expert e are the GPUs other than its home
+ * GPU with a filled redundant slot of e, c_0 < c_1 < ... < c_{f-1}; the slot is
+ * cut into f parts of q = 16 * ceil(slot_bytes / (16 f)) bytes, part j =
+ * [j q, min((j+1) q, slot_bytes)).  Round 0: c_j copies part j from the home
+ * slot, and the home GPU fills its own redundant slots of e; round 1: c_i
+ * copies every other part j from c_j's lowest slot of e.  A received range is
+ * written into every redundant slot of e on the receiving GPU, so the home
+ * sends each byte once.  round = -1: the direct form, every consumer copies
+ * the whole slot from the home slot (one call instead of the rounds).  This
+ * call writes only GPU g's slots (slot_bases[g]) and reads home slots and, in
+ * round 1, parts other GPUs received in round 0.  After all rounds every
+ * GPU's slots hold what ue_sync gives.
  *   slot_bases  [G] host array of device pointers, each GPU's SG slots of
  *               slot_bytes bytes (multiple of 16). */
 ue_status ue_sync_shard(ue_ctx *ctx, const ue_config *cfg, const ue_shard *shard,

@@ -85,7 +85,9 @@ cudaError_t launch_grad_reduce(const Shape &sh, const Launch &ln, float *master,
 size_t grad_smem_bytes(const Shape &sh);
 
 // Calls across G GPUs (GPU g holds ranks [g*N/G, (g+1)*N/G)).  round >= 0 is
-// a relay round, -1 the direct form; relay_rounds(G) = max(1, ceil(log2 G)).
+// a relay round (0: scatter of the parts from the home slot, 1: all-gather
+// among the consumer GPUs), -1 the direct form; relay_rounds(G) = 1 when
+// G <= 2, else 2.
 int relay_rounds(int G);
 cudaError_t launch_sync_shard(const Shape &sh, const Launch &ln, const PeerTable &base, uint8_t *local, int G,
                               int g, int round, int64_t slot_bytes, const PlanDev &plan, int32_t *dev_err,

@@ -5,22 +5,25 @@
 // [g*SG, (g+1)*SG) (SG = S / G), the experts homed on those ranks and the
 // replica-gradient rows of their redundant slots.  Transfers between GPUs use
 // the relay mechanism against fan-out overload (UltraEP news summary,
-// "Comment fonctionne l'équilibrage en 300 microsecondes"), read as a
-// doubling tree over each expert's holder GPUs:
-//     holders of e = [home GPU of e, then every other GPU with a filled
-//                     redundant slot of e, in increasing GPU id];
-// in relay round k the holder at position i, 2^k <= i < 2^(k+1), pulls e from
-// the holder at position i - 2^k (the home slot on the home GPU, else that
-// GPU's lowest slot holding e, filled in an earlier round); round 0 also fills
-// the home GPU's own redundant slots of e.  Round -1 is the direct form: every
-// GPU pulls from the home slot.  So a hot expert's home sends one copy per
-// round instead of one per receiving GPU.
+// "Comment fonctionne l'équilibrage en 300 microsecondes"), read as a scatter
+// then an all-gather: an expert's consumers c_0 < c_1 < ... < c_{f-1} are the
+// GPUs other than its home GPU holding a filled redundant slot of it; its
+// bytes are cut into f parts of q = 16 * ceil(slot_bytes / (16 f)) bytes;
+//   round 0: c_j pulls part j from the home slot (and the home GPU fills its
+//            own redundant slots of the expert);
+//   round 1: c_i pulls every other part j from c_j's lowest slot of it.
+// So the home sends each byte once, not once per consumer: with every peer at
+// full bandwidth through NVSwitch, the busiest GPU's traffic, not the number
+// of hops, sets the time.  Round -1 is the direct form (every consumer pulls
+// the whole slot from the home slot).
 //
 // Design (sm_100a).  Sync: the single-GPU sync kernel's persistent ring of
-// TMA bulk copies, run on each GPU over the experts it receives in the round.
-// The global->shared bulk load reads the source GPU's slot through the
-// caller's peer mapping (no tensor map, no multicast); the shared->global bulk
-// stores write every local slot of the expert, so a tile crosses NVLink once
+// TMA bulk copies, run on each GPU over the byte ranges it receives in the
+// round.  The CTAs flatten (expert, part, 48 KiB tile) into one item list (a
+// prefix over the experts, a binary search per item); the global->shared bulk
+// load reads the source GPU's slot through the caller's peer mapping (no
+// tensor map, no multicast), and the shared->global bulk stores write the
+// range into every local slot of the expert, so a byte crosses NVLink once
 // per receiving GPU however many of its ranks hold the expert.
 // Gradient reduction: the home GPU of each replicated expert pulls every
 // replica's gradient row from the GPU holding it, in replica order, with the
@@ -91,14 +94,22 @@ k_sync_shard(PeerTable base, uint8_t *__restrict__ local, int64_t slot_bytes, in
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm_sync);                 // [stages]
     uint8_t *stage = sm_sync + 128;                                        // [stages][tile]
     const uint8_t **x_base = reinterpret_cast<const uint8_t **>(stage + (size_t)kSyncStages * kSyncTile);  // [G]
-    int32_t *x_src = reinterpret_cast<int32_t *>(x_base + kMaxGpus);      // [E] source slot (global id)
-    int32_t *x_first = x_src + E;                                          // [E] first destination entry
+    int64_t *x_q = reinterpret_cast<int64_t *>(x_base + kMaxGpus);        // [E] part length
+    int32_t *x_first = reinterpret_cast<int32_t *>(x_q + E);               // [E] first replica entry (off + 1)
     int32_t *x_cnt = x_first + E;                                          // [E] destinations on this GPU
-    int32_t *x_slot = x_cnt + E;                                           // [cap] local destination slots
-    int32_t *x_act = x_slot + cap;                                         // [E+1] experts with work; count
+    int32_t *x_j0 = x_cnt + E;                                             // [E] first part index
+    int32_t *x_pn = x_j0 + E;                                              // [E] part indices (before the skip)
+    int32_t *x_skip = x_pn + E;                                            // [E] part left out (-1: none)
+    int32_t *x_pt = x_skip + E;                                            // [E] tiles per full part
+    int32_t *x_home = x_pt + E;                                            // [E] home slot, or -1: parts from consumers
+    int32_t *x_ipre = x_home + E;                                          // [E+1] exclusive prefix of items
+    int32_t *x_slot = x_ipre + E + 1;                                      // [cap] local destination slots
+    int32_t *x_src = x_slot + cap;                                         // [cap] lowest slot of consumer j
 
     for (int i = threadIdx.x; i < G; i += blockDim.x) x_base[i] = static_cast<const uint8_t *>(base.p[i]);
-    // Per replicated expert: this GPU's slots of it, and where this round's copy comes from.
+    // Per replicated expert: this GPU's slots of it, its consumers (the GPUs
+    // other than the home one holding it) and, for this round, which parts of
+    // the slot this GPU receives and from where.
     const int M = clampi(__ldg(info + 3), 0, E);
     for (int m = threadIdx.x; m < M; m += blockDim.x) {
         const int e = clampi(__ldg(rep_experts + m), 0, E - 1);
@@ -106,89 +117,124 @@ k_sync_shard(PeerTable base, uint8_t *__restrict__ local, int64_t slot_bytes, in
         const int end = clampi(__ldg(rep_off + e + 1), off + 1, cap);
         const int home = clampi(__ldg(rep_slot + off), 0, S - 1);
         const int hg = home / SG;
-        GpuSet others;                       // holders other than the home GPU
-        others.clear();
+        GpuSet cons;
+        cons.clear();
         int c = 0;
         for (int p = off + 1; p < end; ++p) {
             const int s = clampi(__ldg(rep_slot + p), 0, S - 1);
             const int gp = s / SG;
-            if (gp != hg) others.add(gp);
+            if (gp != hg) cons.add(gp);
             if (gp == g) x_slot[off + 1 + c++] = s - g * SG;
         }
-        int src = -1;
-        if (c > 0) {
+        const int f = cons.count_below(kMaxGpus);
+        int64_t q = slot_bytes;
+        int j0 = 0, pn = 1, skip = -1, src_home = home;
+        bool active = c > 0;
+        if (active) {
             if (g == hg) {
-                if (round <= 0) src = home;  // the home GPU's own replicas: round 0
-            } else {
-                const int i = 1 + others.count_below(g);   // this GPU's holder position
-                int q = -1;
-                if (round < 0) q = 0;
-                else if (i >= (1 << round) && i < (2 << round)) q = i - (1 << round);
-                if (q == 0) {
-                    src = home;
-                } else if (q > 0) {
-                    const int sg = others.select(q);
-                    int lo = INT_MAX;
+                active = round <= 0;                 // the home GPU's own replicas: round 0 (or direct)
+            } else if (round >= 0) {
+                const int i = cons.count_below(g);   // this GPU's consumer index
+                q = 16 * ((slot_bytes + 16 * (int64_t)f - 1) / (16 * (int64_t)f));
+                if (round == 0) {
+                    j0 = i;                          // scatter: its own part, from the home slot
+                } else {
+                    pn = f;                          // all-gather: every other part, from its consumer
+                    skip = i;
+                    src_home = -1;
+                    for (int j = 0; j < f; ++j) x_src[off + 1 + j] = INT_MAX;
                     for (int p = off + 1; p < end; ++p) {
                         const int s = clampi(__ldg(rep_slot + p), 0, S - 1);
-                        if (s / SG == sg && s < lo) lo = s;
+                        const int gp = s / SG;
+                        if (gp == hg) continue;
+                        const int j = cons.count_below(gp);
+                        if (s < x_src[off + 1 + j]) x_src[off + 1 + j] = s;
                     }
-                    src = lo == INT_MAX ? -1 : lo;
                 }
             }
         }
-        x_src[m] = src;
+        int items = 0;
+        const int pt = (int)((q + kSyncTile - 1) / kSyncTile);
+        if (active)
+            for (int j = j0; j < j0 + pn; ++j) {
+                if (j == skip) continue;
+                const int64_t lo = (int64_t)j * q;
+                const int64_t len = lo < slot_bytes ? (slot_bytes - lo < q ? slot_bytes - lo : q) : 0;
+                items += (int)((len + kSyncTile - 1) / kSyncTile);
+            }
+        x_q[m] = q;
         x_first[m] = off + 1;
-        x_cnt[m] = src >= 0 ? c : 0;
+        x_cnt[m] = c;
+        x_j0[m] = j0;
+        x_pn[m] = pn;
+        x_skip[m] = skip;
+        x_pt[m] = pt;
+        x_home[m] = src_home;
+        x_ipre[m] = items;                           // turned into the exclusive prefix below
     }
     if (threadIdx.x == 0) {
         for (int i = 0; i < kSyncStages; ++i) mbar_init(&bar[i], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
-    if (threadIdx.x < 32) {                  // compact the experts this GPU receives in this round
+    if (threadIdx.x < 32) {                  // exclusive prefix of the items over the experts
         const int lane = threadIdx.x;
-        int n = 0;
+        int run = 0;
         for (int m0 = 0; m0 < M; m0 += 32) {
             const int m = m0 + lane;
-            const bool a = m < M && x_cnt[m] > 0;
-            const unsigned b = __ballot_sync(0xffffffffu, a);
-            if (a) x_act[n + __popc(b & lanemask_lt())] = m;
-            n += __popc(b);
+            const int v = m < M ? x_ipre[m] : 0;
+            int x = v;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, d);
+                if (lane >= d) x += y;
+            }
+            if (m < M) x_ipre[m] = run + x - v;
+            run += __shfl_sync(0xffffffffu, x, 31);
         }
-        if (lane == 0) x_act[E] = n;
+        if (lane == 0) x_ipre[M] = run;
     }
     __syncthreads();
-    const int MA = x_act[E];
-    if (threadIdx.x != 0 || MA == 0) return;
-
-    const int64_t ntiles = (slot_bytes + kSyncTile - 1) / kSyncTile;
-    const int64_t total = (int64_t)MA * ntiles;
-    if ((int64_t)blockIdx.x >= total) return;
-    const int64_t nmy = (total - 1 - blockIdx.x) / gridDim.x + 1;
+    const int total = x_ipre[M];
+    if (threadIdx.x != 0 || total == 0 || (int)blockIdx.x >= total) return;
+    const int64_t nmy = (total - 1 - (int)blockIdx.x) / (int)gridDim.x + 1;
 
     struct Item {
         int m;
         unsigned bytes;
         int64_t offset;
+        const uint8_t *src;
     };
     auto item = [&](int64_t k) {
-        const int64_t i = (int64_t)blockIdx.x + k * gridDim.x;
+        const int idx = (int)blockIdx.x + (int)(k * gridDim.x);
+        int lo = 0, hi = M - 1;                      // last m with x_ipre[m] <= idx
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (x_ipre[mid] <= idx) lo = mid;
+            else hi = mid - 1;
+        }
         Item it;
-        it.m = x_act[(int)(i % MA)];
-        it.offset = (i / MA) * kSyncTile;
-        const int64_t left = slot_bytes - it.offset;
+        it.m = lo;
+        const int l = idx - x_ipre[lo];
+        const int pt = x_pt[lo];
+        const int ord = l / pt;                      // ordinal among the parts received
+        const int sk = x_skip[lo];
+        const int j = x_j0[lo] + ord + (sk >= 0 && x_j0[lo] + ord >= sk ? 1 : 0);
+        const int64_t q = x_q[lo];
+        const int64_t pend = ((int64_t)j + 1) * q < slot_bytes ? ((int64_t)j + 1) * q : slot_bytes;
+        it.offset = (int64_t)j * q + (int64_t)(l - ord * pt) * kSyncTile;
+        const int64_t left = pend - it.offset;
         it.bytes = (unsigned)(left < kSyncTile ? left : kSyncTile);
+        const int src = x_home[lo] >= 0 ? x_home[lo] : x_src[x_first[lo] + j];
+        const int sg = src / SG;
+        it.src = x_base[sg] + (int64_t)(src - sg * SG) * slot_bytes + it.offset;
         return it;
     };
     auto issue_load = [&](int64_t k) {
         const Item it = item(k);
-        const int src = x_src[it.m];
-        const int sg = src / SG;
-        const uint8_t *p = x_base[sg] + (int64_t)(src - sg * SG) * slot_bytes + it.offset;
         const int b = (int)(k % kSyncStages);
         mbar_expect_tx(&bar[b], it.bytes);
-        bulk_load(stage + (size_t)b * kSyncTile, p, it.bytes, &bar[b]);
+        bulk_load(stage + (size_t)b * kSyncTile, it.src, it.bytes, &bar[b]);
     };
 
     for (int64_t k = 0; k < nmy && k < kSyncStages; ++k) issue_load(k);
@@ -298,17 +344,13 @@ k_grad_reduce_shard(float *__restrict__ master, PeerTable grads, int64_t P, int 
 
 }  // namespace
 
-int relay_rounds(int G)
-{
-    int k = 1;
-    while ((1 << k) < G) ++k;
-    return k;
-}
+int relay_rounds(int G) { return G <= 2 ? 1 : 2; }
 
 size_t sync_shard_smem_bytes(const Shape &sh)
 {
-    return 128 + (size_t)kSyncStages * kSyncTile + kMaxGpus * sizeof(void *) +
-           (size_t)(3 * sh.E + sh.E + sh.NR + sh.E + 1) * sizeof(int32_t);
+    const int cap = sh.E + sh.NR;
+    return 128 + (size_t)kSyncStages * kSyncTile + kMaxGpus * sizeof(void *) + (size_t)sh.E * sizeof(int64_t) +
+           (size_t)(8 * sh.E + 1 + 2 * cap) * sizeof(int32_t);
 }
 
 size_t grad_shard_smem_bytes(const Shape &sh)

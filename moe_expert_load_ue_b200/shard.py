@@ -11,7 +11,8 @@ this module issues them in order around the library's sharded calls:
   computes the same plan (placement planning is deterministic) with its
   per-rank offsets for routing expansion;
 - barriers across GPUs that order the relay rounds of the replica weight sync
-  (a GPU pulls in round k only from holders filled before it) and fence the
+  (a GPU pulls in the all-gather round only parts the scatter round brought to
+  the other GPUs) and fence the
   replica gradient reduction (every replica gradient written before the home
   GPUs read them; all reads done before the buffers are reused).
 

@@ -30,12 +30,12 @@ Pinning status (what fixes each function other than itself; the tests under
                 previous plan, the incremental sync leaves exactly the state a
                 full sync gives; slots whose expert is unchanged are untouched;
                 the copied-slot count equals a numpy count.
-  sync_relay    after max(1, ceil(log2 G)) relay rounds (or the one direct round) the
-                state equals the single-GPU sync on tagged bytes, so a pull
-                from a GPU that had not yet received its copy shows; holders
-                per round double; every GPU sends at most one copy of an
-                expert per round; hand-worked schedules
-                (tests/golden/relay_cases.json).
+  sync_relay    after the relay rounds (or the one direct round) the state
+                equals the single-GPU sync on tagged bytes, so a pull from a
+                GPU that had not yet received its part shows; the home sends
+                each byte once (its egress per expert is the slot size, not f
+                times it); relay and direct receive the same bytes per GPU;
+                hand-worked schedules (tests/golden/relay_cases.json).
   grad_reduce   exact closed-form sums on dyadic values; zero gradients
                 leave the master unchanged; numpy float32 reference order.
 
@@ -220,16 +220,17 @@ def sync_delta(W: np.ndarray, nbytes: int, E: int, N: int, R: int, slot_expert: 
 
 
 def relay_rounds(G: int) -> int:
-    """Relay rounds after which every holder of an expert has it: max(1, ceil(log2 G))."""
+    """Relay rounds after which every holder of an expert has it: 1 when G <= 2, else 2."""
     return int(_get().ue_oracle_relay_rounds(G))
 
 
 def sync_relay(W: np.ndarray, nbytes: int, E: int, N: int, R: int, slot_expert: np.ndarray,
                G: int, round: int, dst_gpu: int = -1) -> np.ndarray:
-    """Step 4 over G GPUs: one relay round (round >= 0) or the direct form
-    (round = -1), in place on W viewed as bytes [S][slot_stride], writing only
-    destinations on GPU dst_gpu (all when -1).  Returns the expert copies each
-    GPU sent to other GPUs in this round."""
+    """Step 4 over G GPUs: relay round 0 (scatter of the parts from the home
+    slot) or 1 (all-gather of the parts among the consumer GPUs), or the direct
+    form (round = -1), in place on W viewed as bytes [S][slot_stride], writing
+    only destinations on GPU dst_gpu (all when -1).  Returns the bytes each GPU
+    sent to other GPUs in this round."""
     if not (W.flags.c_contiguous and W.ndim == 2):
         raise OracleError("W must be a C-contiguous [S][stride] array")
     stride = W.shape[1] * W.itemsize

@@ -452,32 +452,31 @@ int ue_oracle_sync_delta(uint8_t *W, int64_t slot_stride, int64_t nbytes,
     return ORC_OK;
 }
 
-/* ---- step 4 across GPUs: relay tree against fan-out overload --------------
+/* ---- step 4 across GPUs: relay against fan-out overload -------------------
  * The news summary ("Comment fonctionne l'équilibrage en 300 microsecondes")
  * streams expert states between GPUs with a relay mechanism against fan-out
  * overload.  Reading taken here: the N ranks are spread over G GPUs, GPU g
  * holding ranks [g*N/G, (g+1)*N/G) and so slots [g*SG, (g+1)*SG), SG = S/G.
- * For an expert e with filled redundant slots, its holder list is
- *     [home GPU of e, then every other GPU holding a filled redundant slot of
- *      e, in increasing GPU id].
- * Relay round k (k = 0, 1, ...): the holder at list position i, 2^k <= i <
- * 2^(k+1), receives e from the holder at position i - 2^k (the home slot on
- * the home GPU, else that GPU's lowest slot holding e, filled in an earlier
- * round), and the received copy fills every redundant slot of e on that GPU.
- * In round 0 the home GPU also fills its own redundant slots of e from the
- * home slot.  After max(1, ceil(log2 G)) rounds every holder has e, and each
- * GPU sends at most one copy of each expert per round.  round = -1 is the direct form:
- * every redundant slot of e is filled from the home slot (the single-GPU sync),
- * so the home GPU sends one copy to every other holder.
+ * For an expert e, its consumers c_0 < c_1 < ... < c_{f-1} are the GPUs other
+ * than its home GPU that hold a filled redundant slot of e.  The expert's
+ * bytes are cut into f parts of q = 16 * ceil(nbytes / (16 f)) bytes, part j
+ * = [j q, min((j+1) q, nbytes)) (trailing parts may be empty).
+ *   round 0: consumer c_j receives part j from the home slot; the home GPU
+ *            fills its own redundant slots of e from the home slot;
+ *   round 1: consumer c_i receives every part j != i from consumer c_j
+ *            (c_j's lowest slot holding e, filled in round 0).
+ * A received range is written into every redundant slot of e on the GPU.  So
+ * the home sends each byte once whatever f is (a scatter, then an all-gather
+ * among the consumers).  Rounds: 1 when G <= 2 (f <= 1), else 2.
+ * round = -1 is the direct form: every redundant slot of e is filled from the
+ * home slot (the single-GPU sync), the home sending nbytes to each consumer.
  * Only destinations on GPU dst_gpu are written (every GPU when dst_gpu = -1).
- * egress[G] (optional) receives, per GPU, the expert copies it sent to other
- * GPUs in this round (for the destinations written).
+ * egress[G] (optional) receives the bytes each GPU sent to other GPUs in this
+ * round (for the destinations written).
  */
 int ue_oracle_relay_rounds(int G)
 {
-    int k = 1;
-    while ((1 << k) < G) ++k;
-    return k;
+    return G <= 2 ? 1 : 2;
 }
 
 int ue_oracle_sync_relay(uint8_t *W, int64_t slot_stride, int64_t nbytes,
@@ -485,57 +484,63 @@ int ue_oracle_sync_relay(uint8_t *W, int64_t slot_stride, int64_t nbytes,
                          int G, int round, int dst_gpu, int64_t *egress)
 {
     if (E < 1 || N < 1 || R < 0 || E % N != 0 || nbytes > slot_stride || nbytes < 0) return ORC_BAD_ARG;
-    if (G < 1 || N % G != 0 || round < -1 || round >= 31 || dst_gpu < -1 || dst_gpu >= G) return ORC_BAD_ARG;
+    if (G < 1 || N % G != 0 || round < -1 || round > 1 || dst_gpu < -1 || dst_gpu >= G) return ORC_BAD_ARG;
     const int H = E / N, HR = H + R, S = N * HR, SG = S / G;
-    int *holder = (int *)malloc(sizeof(int) * (size_t)(G + 1));
-    if (!holder) return ORC_BAD_ARG;
+    int *cons = (int *)malloc(sizeof(int) * (size_t)G);
+    int *first = (int *)malloc(sizeof(int) * (size_t)G);
+    if (!cons || !first) { free(cons); free(first); return ORC_BAD_ARG; }
     if (egress) memset(egress, 0, sizeof(int64_t) * (size_t)G);
     for (int s = 0; s < S; ++s)
-        if (slot_expert[s] >= E) { free(holder); return ORC_BAD_ARG; }
+        if (slot_expert[s] >= E) { free(cons); free(first); return ORC_BAD_ARG; }
     for (int e = 0; e < E; ++e) {
         const int home = (e / H) * HR + (e % H);
         const int hg = home / SG;
-        /* holder list: home GPU, then the other GPUs with a redundant slot of e */
-        int n = 0;
-        holder[n++] = hg;
+        /* consumers in increasing GPU id, with each one's lowest slot of e */
+        int f = 0;
         for (int g = 0; g < G; ++g) {
-            if (g == hg) continue;
-            int has = 0;
-            for (int s = g * SG; s < (g + 1) * SG; ++s)
-                if (s % HR >= H && slot_expert[s] == e) has = 1;
-            if (has) holder[n++] = g;
+            int lo = -1;
+            for (int s = g * SG; s < (g + 1) * SG && lo < 0; ++s)
+                if (s % HR >= H && slot_expert[s] == e) lo = s;
+            if (lo >= 0 && g != hg) { cons[f] = g; first[f] = lo; ++f; }
         }
-        for (int i = 0; i < n; ++i) {
-            const int dst = holder[i];
-            int src_pos;
-            if (round < 0) {
-                src_pos = 0;
-            } else if (i == 0) {
-                if (round != 0) continue;                  /* home's own replicas: round 0 */
-                src_pos = 0;
-            } else {
-                if (i < (1 << round) || i >= (2 << round)) continue;
-                src_pos = i - (1 << round);
+        const int64_t q = f > 0 ? 16 * ((nbytes + 16 * (int64_t)f - 1) / (16 * (int64_t)f)) : 0;
+        /* every GPU holding e receives, in this round, a list of (source slot, byte range) */
+        for (int g = 0; g < G; ++g) {
+            if (dst_gpu >= 0 && g != dst_gpu) continue;
+            int i = -1;                                  /* g's consumer index */
+            for (int j = 0; j < f; ++j) if (cons[j] == g) i = j;
+            if (g != hg && i < 0) continue;
+            for (int j = 0; j < (g == hg ? 1 : f); ++j) {
+                int src;
+                int64_t lo, hi;
+                if (g == hg) {                           /* home GPU: its own replicas */
+                    if (round > 0) break;
+                    src = home; lo = 0; hi = nbytes;
+                } else if (round < 0) {                  /* direct: the whole slot, once */
+                    if (j > 0) break;
+                    src = home; lo = 0; hi = nbytes;
+                } else if (round == 0) {                 /* scatter: its own part from home */
+                    if (j != i) continue;
+                    src = home; lo = j * q; hi = (j + 1) * q;
+                } else {                                 /* all-gather: the other parts */
+                    if (j == i) continue;
+                    src = first[j]; lo = j * q; hi = (j + 1) * q;
+                }
+                if (hi > nbytes) hi = nbytes;
+                if (lo >= hi) continue;
+                int wrote = 0;
+                for (int s = g * SG; s < (g + 1) * SG; ++s) {
+                    if (s % HR < H || slot_expert[s] != e) continue;
+                    memcpy(W + (int64_t)s * slot_stride + lo, W + (int64_t)src * slot_stride + lo, (size_t)(hi - lo));
+                    wrote = 1;
+                }
+                const int sg = src / SG;
+                if (wrote && sg != g && egress) egress[sg] += hi - lo;
             }
-            if (dst_gpu >= 0 && dst != dst_gpu) continue;
-            const int src_gpu = holder[src_pos];
-            int src = home;
-            if (src_pos > 0) {
-                src = -1;
-                for (int s = src_gpu * SG; s < (src_gpu + 1) * SG && src < 0; ++s)
-                    if (s % HR >= H && slot_expert[s] == e) src = s;
-                if (src < 0) { free(holder); return ORC_INVARIANT; }
-            }
-            int wrote = 0;
-            for (int s = dst * SG; s < (dst + 1) * SG; ++s) {
-                if (s % HR < H || slot_expert[s] != e) continue;
-                memcpy(W + (int64_t)s * slot_stride, W + (int64_t)src * slot_stride, (size_t)nbytes);
-                wrote = 1;
-            }
-            if (wrote && src_gpu != dst && egress) egress[src_gpu] += 1;
         }
     }
-    free(holder);
+    free(cons);
+    free(first);
     return ORC_OK;
 }
 

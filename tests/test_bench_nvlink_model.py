@@ -1,6 +1,6 @@
 """The benchmark's NVLink model of the relay: its per-round and direct egress
-per GPU equal the oracle's relay schedule (expert copies sent per GPU) times
-the slot size, on random plans (CPU only)."""
+per GPU equal the bytes the oracle's relay schedule sends from each GPU, on
+random plans (CPU only)."""
 import os
 import sys
 
@@ -24,10 +24,10 @@ def test_model_egress_matches_oracle_schedule(seed):
     p = (rng.permutation(E) + 1.0) ** -1.5
     load = rng.multinomial(50000, p / p.sum()).astype(np.int32)
     se = oracle.plan(load, N, R)["slot_expert"]
-    G = int(rng.choice([g for g in (2, 4, 8) if N % g == 0]))
-    m = bench.nvlink_model(se, w, G, 16, 770.0)
-    W = np.zeros((se.size, 16), np.uint8)
+    G = int(rng.choice([g for g in (2, 4, 8, 16) if N % g == 0]))
+    nb = int(rng.choice([16, 96, 4000]))
+    m = bench.nvlink_model(se, w, G, nb, 770.0)
+    W = np.zeros((se.size, nb), np.uint8)
     for k in range(oracle.relay_rounds(G)):
-        assert np.array_equal(m["relay_egress"][k], oracle.sync_relay(W, 16, E, N, R, se, G, k) * 16.0), k
-    assert np.array_equal(m["direct_egress"], oracle.sync_relay(W, 16, E, N, R, se, G, -1) * 16.0)
-    assert m["relay_max_egress"] <= m["direct_max_egress"]
+        assert np.array_equal(m["relay_egress"][k], oracle.sync_relay(W, nb, E, N, R, se, G, k)), k
+    assert np.array_equal(m["direct_egress"], oracle.sync_relay(W, nb, E, N, R, se, G, -1))
