@@ -367,6 +367,27 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
         // Running occurrence index of each (warp, expert): base + earlier warps.
         for (int w = 0; w < kRerouteWarps; ++w)
             for (int e = threadIdx.x; e < E; e += blockDim.x) s.hist[w * E + e] += s.base[e];
+        // An expert whose occurrences in this CTA, [base, base + tot), all fall
+        // into one replica's range gets its slot and position offset directly:
+        // tab[e] = {soff[slot] - rep_cum, -1 - slot}; it is taken only when that
+        // whole range of positions lies inside the slot's segment and below
+        // T*K, so no per-id check is needed.  Others keep {entry, count}.  The
+        // local grouping index becomes rexp[e] + j (j the occurrence index).
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            const int b = s.base[e], nt = s.tot[e];
+            const int2 t = s.tab[e];
+            if (b >= 0 && nt > 0) {
+                const int k = covering_entry(s.rc + t.x, t.y & 0xffff, b);
+                const int2 q = s.rc[t.x + k];
+                if (q.y >= 0 && q.y < S) {
+                    const int lo = s.soff[q.y], hi = s.soff[q.y + 1];
+                    if (lo >= 0 && hi >= lo && (int64_t)hi <= da.L && b >= q.x &&
+                        (int64_t)b + nt <= (int64_t)q.x + (hi - lo))
+                        s.tab[e] = make_int2(lo - q.x, -1 - q.y);
+                }
+            }
+            s.rexp[e] -= b;
+        }
         __syncthreads();
 
         // Pass 2: every valid id is ranked among the warp's equal ids (lane
@@ -414,19 +435,24 @@ k_reroute(const int32_t *__restrict__ ids, int64_t per_rank, int E, int cap,
                 if (valid) {
                     const int j = wh[id] + before;
                     const int2 t = s.tab[id];
-                    const int2 q = s.rc[t.x + covering_entry(s.rc + t.x, t.y & 0xffff, j)];
-                    out = q.y;
                     int pos = -1;
-                    // Inside the slot's segment whenever the ids are the ones the
-                    // plan was computed from; anything else is reported, not written.
-                    if (out >= 0 && out < S) {
-                        pos = s.soff[out] + (j - q.x);
-                        if (pos < s.soff[out] || pos >= s.soff[out + 1] || (int64_t)pos >= da.L) pos = -1;
+                    if (t.y < 0) {                       // one replica for all of this CTA's ids
+                        out = -1 - t.y;
+                        pos = j + t.x;
+                    } else {
+                        const int2 q = s.rc[t.x + covering_entry(s.rc + t.x, t.y & 0xffff, j)];
+                        out = q.y;
+                        // Inside the slot's segment whenever the ids are the ones the
+                        // plan was computed from; anything else is reported, not written.
+                        if (out >= 0 && out < S) {
+                            pos = s.soff[out] + (j - q.x);
+                            if (pos < s.soff[out] || pos >= s.soff[out + 1] || (int64_t)pos >= da.L) pos = -1;
+                        }
+                        if (pos < 0) atomicOr(da.err, 2);
                     }
-                    if (pos < 0) atomicOr(da.err, 2);
                     if (staged) {
                         s.stage[li] = pos;
-                        s.oli[s.rexp[id] + (j - s.base[id])] = (uint16_t)li;
+                        s.oli[s.rexp[id] + j] = (uint16_t)li;
                     } else if (pos >= 0) {
                         da.src_index[pos] = (int32_t)(lo + li);
                         if (da.gates != nullptr) da.gates_out[pos] = __ldg(da.gates + lo + li);

@@ -67,21 +67,6 @@ struct GpuSet {
         }
         return n;
     }
-    // The q-th member (q >= 1) in increasing order; -1 if there are fewer.
-    __device__ __forceinline__ int select(int q) const
-    {
-#pragma unroll
-        for (int i = 0; i < kMaxGpus / 32; ++i) {
-            const int n = __popc(w[i]);
-            if (q <= n) {
-                uint32_t v = w[i];
-                for (int k = 1; k < q; ++k) v &= v - 1u;
-                return i * 32 + __ffs(v) - 1;
-            }
-            q -= n;
-        }
-        return -1;
-    }
 };
 
 __global__ void __launch_bounds__(kSyncThreads, 1)
