@@ -165,3 +165,70 @@ def test_grad_reduce_shards(ctx, w, G, dtype):
     oracle.grad_reduce(m_host, np.ascontiguousarray(g_host), P, w.E, w.N, w.R, plan.to_host())
     got = master.cpu().numpy()
     assert np.array_equal(got.view(np.uint32), m_host.view(np.uint32))
+
+
+def test_shards_empty_microbatch_and_no_redundant_slots(ctx):
+    # T = 0: the counts rows are written (zeros) and nothing else is touched
+    E, N, R, K = 32, 8, 2, 4
+    cfg = ue.Config(E=E, N=N, R=R, K=K, T=0)
+    counts = torch.full((N, E), -7, dtype=torch.int32, device="cuda")
+    bad = torch.full((N,), -7, dtype=torch.int32, device="cuda")
+    empty = torch.empty((0, K), dtype=torch.int32, device="cuda")
+    for g in range(4):
+        ue.ue_load_shard(ctx, cfg, 4, g, empty, counts, bad)
+    plan = ue.Plan(cfg)
+    ue.ue_plan(ctx, cfg, counts, plan)
+    for g in range(4):
+        ue.ue_reroute_shard(ctx, cfg, 4, g, empty, plan, empty)
+    torch.cuda.synchronize()
+    assert (counts == 0).all().item() and (bad == 0).all().item()
+    # R = 0: no replica anywhere, the sync and the gradient reduction change nothing
+    ids = np.random.default_rng(8).integers(0, 64, size=(8 * 64, 4)).astype(np.int32)
+    cfg0, counts0, _, plan0, phys0 = _rebalance_sharded(ctx, ids, 64, 8, 0, 4)
+    ref = oracle.rebalance(ids, 64, 8, 0)
+    assert np.array_equal(phys0, ref["phys"])
+    W = torch.randint(0, 256, (cfg0.S, 4096), dtype=torch.uint8, device="cuda")
+    W0 = W.clone()
+    bases = [W[h * (cfg0.S // 4)] for h in range(4)]
+    for k in range(ue.ue_relay_rounds(4)):
+        for g in range(4):
+            ue.ue_sync_shard(ctx, cfg0, 4, g, bases, 4096, plan0, k)
+    master = torch.randn((64, 64), device="cuda")
+    m0 = master.clone()
+    for g in range(4):
+        ue.ue_grad_reduce_shard(ctx, cfg0, 4, g, master[g * 16:(g + 1) * 16], None, torch.float32, 64, plan0)
+    torch.cuda.synchronize()
+    assert torch.equal(W, W0) and torch.equal(master, m0)
+
+
+def test_sharded_balancer_on_one_gpu(ctx):
+    """The host sequence (ShardedBalancer with the device calls) for G = 1:
+    rebalance, relay sync and gradient reduction equal the oracle."""
+    from moe_expert_load_ue_b200.shard import DeviceOps, ShardedBalancer
+    w = inputs.CLASS_106B
+    ids = inputs.topk_ids(w, 2)
+    cfg = ue.Config(E=w.E, N=w.N, R=w.R, K=w.K, T=w.T)
+    bal = ShardedBalancer(cfg, DeviceOps(ctx, cfg, 1, 0), G=1, g=0)
+    d_ids = torch.from_numpy(ids).cuda()
+    counts = torch.empty((w.N, w.E), dtype=torch.int32, device="cuda")
+    bad = torch.empty(w.N, dtype=torch.int32, device="cuda")
+    plan = ue.Plan(cfg)
+    phys = torch.empty_like(d_ids)
+    bal.rebalance(d_ids, counts, bad, plan, phys)
+    slot_bytes = 48 * 1024 + 64
+    W = torch.randint(0, 256, (cfg.S, slot_bytes), dtype=torch.uint8, device="cuda")
+    host = W.cpu().numpy()
+    bal.sync([W], slot_bytes, plan)
+    P = 2048 + 16
+    master = torch.randn((w.E, P), device="cuda") * 1e-2
+    grads = torch.randn((w.N * w.R, P), device="cuda") * 1e-3
+    m_host = master.cpu().numpy().copy()
+    bal.grad_reduce(master, [grads], torch.float32, P, plan)
+    torch.cuda.synchronize()
+    ref = oracle.rebalance(ids, w.E, w.N, w.R)
+    assert np.array_equal(counts.cpu().numpy(), ref["counts"])
+    assert np.array_equal(phys.cpu().numpy(), ref["phys"])
+    oracle.sync(host, slot_bytes, w.E, w.N, w.R, ref["plan"]["slot_expert"])
+    assert np.array_equal(W.cpu().numpy(), host)
+    oracle.grad_reduce(m_host, grads.cpu().numpy(), P, w.E, w.N, w.R, ref["plan"])
+    assert np.array_equal(master.cpu().numpy().view(np.uint32), m_host.view(np.uint32))
