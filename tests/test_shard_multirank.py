@@ -70,11 +70,11 @@ class OracleOps:
         phys_local[:] = torch.from_numpy(self.o.reroute(self.ids_full.numpy(), E, plan)[self.g * n:(self.g + 1) * n])
 
     def sync(self, slot_bases, slot_bytes, plan, round):
-        self._stamp(round, 0)
+        self._stamp(round + 1, 0)              # log row 0: the direct form, 1 + k: relay round k
         if self.g == 0:
             time.sleep(0.3)                    # a missing barrier would let the others run ahead
         self.o.sync_relay(self.W.numpy(), slot_bytes, E, N, R, plan["slot_expert"], self.G, round, self.g)
-        self._stamp(round, 1)
+        self._stamp(round + 1, 1)
 
     def grad_reduce(self, master_local, grad_bases, grads_dtype, P_, plan):
         self._stamp(7, 0)
@@ -85,7 +85,7 @@ class OracleOps:
         self._stamp(7, 1)
 
 
-def _worker(rank, world, port, ids_full, W, master, grads, log, t0, q):
+def _worker(rank, world, relay, port, ids_full, W, master, grads, log, t0, q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     sys.path.insert(0, ROOT)
     sys.path.insert(0, os.path.join(ROOT, "tests"))
@@ -102,15 +102,15 @@ def _worker(rank, world, port, ids_full, W, master, grads, log, t0, q):
     bad = torch.full((N,), -1, dtype=torch.int32)
     plan, phys = {}, torch.empty_like(ids_local)
     bal.rebalance(ids_local, counts, bad, plan, phys)
-    bal.sync(None, NB, plan)
+    bal.sync(None, NB, plan, relay=relay)
     EG = E // world
     bal.grad_reduce(master[rank * EG:(rank + 1) * EG], None, torch.float32, P, plan)
     dist.destroy_process_group()
     q.put((rank, counts.numpy(), bad.numpy(), plan["slot_expert"], phys.numpy(), bal.relay_rounds))
 
 
-@pytest.mark.parametrize("world", [2, 4])
-def test_sharded_balancer_on_gloo_ranks(world):
+@pytest.mark.parametrize("world,relay", [(2, True), (4, True), (4, False)])
+def test_sharded_balancer_on_gloo_ranks(world, relay):
     sys.path.insert(0, ROOT)
     import oracle
     ids, W0, m0, g0 = _inputs()
@@ -123,7 +123,7 @@ def test_sharded_balancer_on_gloo_ranks(world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, ids_t, W, master, grads, log, t0, q))
+    procs = [ctx.Process(target=_worker, args=(r, world, relay, port, ids_t, W, master, grads, log, t0, q))
              for r in range(world)]
     for p in procs:
         p.start()
@@ -146,6 +146,7 @@ def test_sharded_balancer_on_gloo_ranks(world):
     oracle.grad_reduce(mref, g0, P, E, N, R, ref["plan"])
     assert np.array_equal(master.numpy(), mref)
     lg = log.numpy()
-    for k in range(1, rounds):
-        assert lg[:, k, 0].min() >= lg[:, k - 1, 1].max(), f"round {k} started before round {k - 1} ended"
-    assert lg[:, 7, 0].min() >= lg[:, rounds - 1, 1].max()
+    rows = list(range(1, rounds + 1)) if relay else [0]
+    for a, b in zip(rows, rows[1:]):
+        assert lg[:, b, 0].min() >= lg[:, a, 1].max(), f"log row {b} started before row {a} ended"
+    assert lg[:, 7, 0].min() >= lg[:, rows[-1], 1].max()   # gradient reduction after the last sync round
