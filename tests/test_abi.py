@@ -259,3 +259,27 @@ def test_shard_refusals(L):
     assert grad(mp + 4, ok) == 1 and "master_local" in L.ue_last_error().decode()
     assert grad(mp, None) == 1 and "grad_bases" in L.ue_last_error().decode()
     assert hp.untouched() and (counts == 7).all() and (phys == 7).all() and (w == 0).all()
+
+
+def test_header_is_plain_c(tmp_path):
+    # the boundary is a C ABI: ue.h compiles as C99 and as C++ without CUDA headers
+    src = tmp_path / "use.c"
+    src.write_text('#include <string.h>\n'
+                   '#include "ue.h"\n'
+                   'int probe(ue_ctx *ctx, const ue_config *cfg, const ue_shard *sh, void *const *bases)\n'
+                   '{\n'
+                   '    ue_plan_buffers plan;\n'
+                   '    ue_dispatch_buffers disp;\n'
+                   '    memset(&plan, 0, sizeof plan);\n'
+                   '    memset(&disp, 0, sizeof disp);\n'
+                   '    (void)disp;\n'
+                   '    return (int)ue_sync_shard(ctx, cfg, sh, bases, 16, &plan, ue_relay_rounds(sh->G) - 1, 0);\n'
+                   '}\n')
+    inc = os.path.join(ROOT, "include")
+    for cc, std in (("gcc", "-std=c99"), ("g++", "-std=c++17")):
+        args = [cc, std, "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", inc, "-c", str(src),
+                "-o", str(tmp_path / f"use_{cc}.o")]
+        if cc == "g++":
+            args[args.index(str(src))] = "-xc++"
+            args.insert(args.index("-xc++") + 1, str(src))
+        subprocess.run(args, check=True, capture_output=True, text=True)
