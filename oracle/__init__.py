@@ -72,29 +72,34 @@ def build(force: bool = False) -> str:
     return _LIB_PATH
 
 
+def _open(path: str) -> ctypes.CDLL:
+    """Load a compiled oracle library and declare its signatures."""
+    lib = ctypes.CDLL(path)
+    vp, i64, ci = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.ue_oracle_load.argtypes = [vp, i64, ci, ci, ci, vp, vp]
+    lib.ue_oracle_expert_load.argtypes = [vp, ci, ci, vp, vp]
+    lib.ue_oracle_plan.argtypes = [ci, ci, ci, vp] + [vp] * 9
+    lib.ue_oracle_plan_ex.argtypes = [ci, ci, ci, vp, ci] + [vp] * 9
+    lib.ue_oracle_reroute.argtypes = [vp, i64, ci, ci, vp, vp, vp, vp, vp]
+    lib.ue_oracle_dispatch.argtypes = [vp, i64, ci, vp, vp, vp, vp]
+    lib.ue_oracle_sync.argtypes = [vp, i64, i64, ci, ci, ci, vp]
+    lib.ue_oracle_sync_delta.argtypes = [vp, i64, i64, ci, ci, ci, vp, vp, vp]
+    lib.ue_oracle_grad_reduce.argtypes = [vp, i64, vp, ci, i64, i64, ci, ci, ci, vp, vp]
+    lib.ue_oracle_relay_rounds.argtypes = [ci]
+    lib.ue_oracle_sync_relay.argtypes = [vp, i64, i64, ci, ci, ci, vp, ci, ci, ci, vp]
+    for f in ("ue_oracle_load", "ue_oracle_expert_load", "ue_oracle_plan", "ue_oracle_plan_ex",
+              "ue_oracle_reroute", "ue_oracle_dispatch", "ue_oracle_sync",
+              "ue_oracle_sync_delta", "ue_oracle_grad_reduce", "ue_oracle_relay_rounds",
+              "ue_oracle_sync_relay"):
+        getattr(lib, f).restype = ctypes.c_int
+    return lib
+
+
 def _get():
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
-            vp, i64, ci = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
-            lib.ue_oracle_load.argtypes = [vp, i64, ci, ci, ci, vp, vp]
-            lib.ue_oracle_expert_load.argtypes = [vp, ci, ci, vp, vp]
-            lib.ue_oracle_plan.argtypes = [ci, ci, ci, vp] + [vp] * 9
-            lib.ue_oracle_plan_ex.argtypes = [ci, ci, ci, vp, ci] + [vp] * 9
-            lib.ue_oracle_reroute.argtypes = [vp, i64, ci, ci, vp, vp, vp, vp, vp]
-            lib.ue_oracle_dispatch.argtypes = [vp, i64, ci, vp, vp, vp, vp]
-            lib.ue_oracle_sync.argtypes = [vp, i64, i64, ci, ci, ci, vp]
-            lib.ue_oracle_sync_delta.argtypes = [vp, i64, i64, ci, ci, ci, vp, vp, vp]
-            lib.ue_oracle_grad_reduce.argtypes = [vp, i64, vp, ci, i64, i64, ci, ci, ci, vp, vp]
-            lib.ue_oracle_relay_rounds.argtypes = [ci]
-            lib.ue_oracle_sync_relay.argtypes = [vp, i64, i64, ci, ci, ci, vp, ci, ci, ci, vp]
-            for f in ("ue_oracle_load", "ue_oracle_expert_load", "ue_oracle_plan", "ue_oracle_plan_ex",
-                      "ue_oracle_reroute", "ue_oracle_dispatch", "ue_oracle_sync",
-                      "ue_oracle_sync_delta", "ue_oracle_grad_reduce", "ue_oracle_relay_rounds",
-                      "ue_oracle_sync_relay"):
-                getattr(lib, f).restype = ctypes.c_int
-            _lib = lib
+            _lib = _open(build())
     return _lib
 
 
