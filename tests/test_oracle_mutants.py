@@ -14,6 +14,7 @@ import pytest
 import oracle
 import test_oracle_dispatch as tdisp
 import test_oracle_plan as tplan
+import test_oracle_plan_variants as tvar
 import test_oracle_steps as tsteps
 from moe_expert_load_ue_b200 import inputs
 
@@ -27,6 +28,15 @@ def _plan_pins():
         tplan.test_plan_invariants_random(seed)
     tplan.test_plan_invariants_synthetic_workloads()
     tplan.test_brute_force_gap_report()
+
+
+def _variant_pins():
+    for case in tvar._cases():
+        tvar.test_variant_hand_cases(case)
+    for seed in range(40):
+        tvar.test_variant_invariants_random(seed)
+    tvar.test_spread_never_raises_the_max()
+    tvar.test_variant_brute_force_gaps()
 
 
 def _reroute_pins():
@@ -74,6 +84,11 @@ MUTANTS = {
                                   "int64_t take = load[e];"),
     "chunk not capped by spare": (_plan_pins, "int64_t c = rem_e[e] < spare ? rem_e[e] : spare;",
                                   "int64_t c = rem_e[e];"),
+    "requeue ties to the higher id": (_variant_pins, "if (rem_e[x] > 0 && (e < 0 || rem_e[x] > rem_e[e])) e = x;",
+                                      "if (rem_e[x] > 0 && (e < 0 || rem_e[x] >= rem_e[e])) e = x;"),
+    "spread ties to the later replica": (_variant_pins, "if (cur[r] < best_load) { best_load = cur[r]; best_a = a; }",
+                                         "if (cur[r] <= best_load) { best_load = cur[r]; best_a = a; }"),
+    "spread never back to the home": (_variant_pins, "int64_t best_load = cur[h];", "int64_t best_load = INT64_MAX;"),
     "inclusive cumulative quotas": (_reroute_pins, "rep_cum[pos] = (int32_t)cum;\n            cum += asg_c[a];",
                                     "cum += asg_c[a];\n            rep_cum[pos] = (int32_t)cum;"),
     "occurrences counted from 1": (_reroute_pins, "int64_t j = occ[e]++;", "int64_t j = ++occ[e];"),
@@ -118,7 +133,7 @@ def _passes(pins):
     return True
 
 
-@pytest.mark.parametrize("pins", [_plan_pins, _reroute_pins, _load_pins, _dispatch_pins, _sync_pins, _grad_pins],
+@pytest.mark.parametrize("pins", [_plan_pins, _variant_pins, _reroute_pins, _load_pins, _dispatch_pins, _sync_pins, _grad_pins],
                          ids=lambda f: f.__name__)
 def test_unchanged_copy_passes(tmp_path, monkeypatch, pins):
     monkeypatch.setattr(oracle, "_lib", _mutant(tmp_path, "int64_t j = occ[e]++;", "int64_t j = occ[e]++;"))
