@@ -23,11 +23,6 @@ def ctx():
     c.close()
 
 
-def _free_gb():
-    free, _ = torch.cuda.mem_get_info()
-    return free / 2**30
-
-
 def run_rebalance(ctx, ids_np, E, N, R, fused=True, plan=None):
     T, K = ids_np.shape
     cfg = ue.Config(E=E, N=N, R=R, K=K, T=T)
@@ -201,47 +196,6 @@ def test_sync_extreme_fanout(ctx):
     assert (np.diff(off) - 1).max() >= 8
 
 
-def _windows(n, width, count, seed):
-    rng = np.random.default_rng(seed)
-    starts = {0, max(0, n - width)}
-    while len(starts) < count:
-        starts.add(int(rng.integers(0, max(1, n - width))) // 16 * 16)
-    return sorted(starts)
-
-
-def test_sync_671b_full_size_sampled(ctx):
-    w = inputs.CLASS_671B
-    slot_bytes = 2 * w.P
-    if _free_gb() < w.S * slot_bytes / 2**30 + 4:
-        pytest.skip("not enough device memory")
-    plan, pl, cfg = _plan_for(ctx, w, 0)
-    W = torch.empty((w.S, slot_bytes), dtype=torch.uint8, device="cuda")
-    W.view(torch.int32).random_(generator=torch.Generator(device="cuda").manual_seed(5))
-    width = 1 << 18
-    starts = _windows(slot_bytes, width, 4, seed=1)
-    win = lambda: np.concatenate([W[:, a:a + width].cpu().numpy() for a in starts], axis=1)
-    before = win()
-    # checksums of whole slots that must stay untouched (home and empty redundant slots)
-    HR = w.H + w.R
-    keep = [s for s in range(w.S) if s % HR < w.H or pl["slot_expert"][s] < 0]
-    sums_before = W[keep].view(torch.int32).sum(dim=1, dtype=torch.int64).cpu()
-    ue.ue_sync(ctx, cfg, W, slot_bytes, plan)
-    torch.cuda.synchronize()
-    assert ctx.device_error() == 0
-    expect = before.copy()
-    oracle.sync(expect, expect.shape[1], w.E, w.N, w.R, pl["slot_expert"])
-    assert np.array_equal(win(), expect)
-    assert torch.equal(W[keep].view(torch.int32).sum(dim=1, dtype=torch.int64).cpu(), sums_before)
-    # every filled redundant slot equals its home slot in full
-    for s in range(w.S):
-        e = pl["slot_expert"][s]
-        if s % HR >= w.H and e >= 0:
-            home = (e // w.H) * HR + e % w.H
-            assert torch.equal(W[s], W[home]), s
-    del W
-    torch.cuda.empty_cache()
-
-
 # ---- grad reduce ----------------------------------------------------------------
 
 def _grad_tolerance_ok(got, expect, master0, grads_abs_sum):
@@ -294,37 +248,6 @@ def test_grad_reduce_ragged_chunks(ctx, P):
     expect = m0.copy()
     oracle.grad_reduce(expect, gh, P, w.E, w.N, w.R, pl)
     assert np.array_equal(master.cpu().numpy(), expect)
-
-
-def test_grad_reduce_671b_full_size_sampled(ctx):
-    w = inputs.CLASS_671B
-    P = w.P
-    need = (w.E * P * 4 + w.N * w.R * P * 2) / 2**30 + 4
-    if _free_gb() < need:
-        pytest.skip("not enough device memory")
-    plan, pl, cfg = _plan_for(ctx, w, 0)
-    gen = torch.Generator(device="cuda").manual_seed(31)
-    master = torch.empty((w.E, P), device="cuda")
-    for e in range(w.E):          # row by row keeps the temporary small
-        master[e].normal_(0.0, 1e-3, generator=gen)
-    grads = torch.empty((w.N * w.R, P), dtype=torch.bfloat16, device="cuda")
-    for r in range(w.N * w.R):
-        grads[r].normal_(0.0, 1e-3, generator=gen)
-    width = 1 << 16
-    starts = _windows(P, width, 4, seed=2)
-    mwin = lambda: np.concatenate([master[:, a:a + width].cpu().numpy() for a in starts], axis=1)
-    gwin = np.concatenate([grads[:, a:a + width].view(torch.int16).cpu().numpy().view(np.uint16)
-                           for a in starts], axis=1)
-    m0 = mwin()
-    ue.ue_grad_reduce(ctx, cfg, master, grads, P, plan)
-    torch.cuda.synchronize()
-    expect = m0.copy()
-    oracle.grad_reduce(expect, gwin, expect.shape[1], w.E, w.N, w.R, pl)
-    got = mwin()
-    assert _grad_tolerance_ok(got, expect, m0, _grad_abs_sum(gwin, pl, w.E, w.N, w.R, True))
-    assert np.array_equal(got, expect)
-    del master, grads
-    torch.cuda.empty_cache()
 
 
 def test_grad_reduce_no_redundant_slots(ctx):
