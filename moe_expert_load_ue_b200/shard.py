@@ -11,8 +11,9 @@ this module issues them in order around the library's sharded calls:
   computes the same plan (placement planning is deterministic) with its
   per-rank offsets for routing expansion;
 - barriers across GPUs that order the relay rounds of the replica weight sync
-  (a GPU pulls in the all-gather round only parts the scatter round brought to
-  the other GPUs) and fence the
+  (no GPU pulls a home slot before its GPU has finished writing it, and a GPU
+  pulls in the all-gather round only parts the scatter round brought to the
+  other GPUs) and fence the
   replica gradient reduction (every replica gradient written before the home
   GPUs read them; all reads done before the buffers are reused).
 
@@ -87,12 +88,13 @@ class ShardedBalancer:
         self.ops.reroute(ids_local, plan, phys_local)
 
     def sync(self, slot_bases, slot_bytes: int, plan, relay: bool = True) -> None:
-        """Replica weight sync: the relay rounds (or the direct form), a
-        barrier before each round after the first and after the last."""
+        """Replica weight sync: the relay rounds (or the direct form), with a
+        barrier before every round and after the last.  The first barrier
+        makes every GPU's home slots final (an optimizer step or any earlier
+        write on another GPU's stream) before any GPU pulls from them."""
         rounds = range(self.relay_rounds) if relay else (-1,)
-        for i, k in enumerate(rounds):
-            if i > 0:
-                self.barrier()
+        for k in rounds:
+            self.barrier()
             self.ops.sync(slot_bases, slot_bytes, plan, k)
         self.barrier()
 

@@ -10,7 +10,10 @@ Checked: every rank ends with the full counts and the same plan; the ranks'
 phys slices, slots and master rows together equal the single-GPU oracle; and
 no rank starts relay round k (or the gradient reduction) before every rank
 has finished round k - 1 (the sync), which a missing barrier would break
-because rank 0 is slowed down on purpose.
+because rank 0 is slowed down on purpose.  Before the sync every rank writes
+new weights into its own home slots (an optimizer step), rank 0 late: the
+replicas must hold the new weights, which a missing barrier before the first
+round would break (a consumer would pull rank 0's old bytes).
 """
 import os
 import socket
@@ -40,7 +43,8 @@ def _inputs():
     W = rng.integers(0, 256, size=(N * (E // N + R), NB), dtype=np.uint8)
     master = (rng.integers(-64, 64, size=(E, P)) / 256.0).astype(np.float32)
     grads = (rng.integers(-64, 64, size=(N * R, P)) / 1024.0).astype(np.float32)
-    return ids, W, master, grads
+    W_new = rng.integers(0, 256, size=W.shape, dtype=np.uint8)     # home slots after an optimizer step
+    return ids, W, master, grads, W_new
 
 
 class OracleOps:
@@ -54,6 +58,17 @@ class OracleOps:
 
     def _stamp(self, k, i):
         self.log[self.g, k, i] = time.monotonic_ns() - self.t0
+
+    def write_home(self, W_new):
+        """This GPU's home slots get new weights (rank 0 late), log row 6."""
+        self._stamp(6, 0)
+        if self.g == 0:
+            time.sleep(0.3)
+        HR, SG = E // N + R, (N * (E // N + R)) // self.G
+        for s in range(self.g * SG, (self.g + 1) * SG):
+            if s % HR < E // N:
+                self.W[s] = W_new[s]
+        self._stamp(6, 1)
 
     def load(self, ids_local, counts, bad):
         c, b = self.o.load(ids_local.numpy(), E, self.NG)
@@ -85,7 +100,7 @@ class OracleOps:
         self._stamp(7, 1)
 
 
-def _worker(rank, world, relay, port, ids_full, W, master, grads, log, t0, q):
+def _worker(rank, world, relay, port, ids_full, W, master, grads, W_new, log, t0, q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     sys.path.insert(0, ROOT)
     sys.path.insert(0, os.path.join(ROOT, "tests"))
@@ -102,6 +117,7 @@ def _worker(rank, world, relay, port, ids_full, W, master, grads, log, t0, q):
     bad = torch.full((N,), -1, dtype=torch.int32)
     plan, phys = {}, torch.empty_like(ids_local)
     bal.rebalance(ids_local, counts, bad, plan, phys)
+    ops.write_home(W_new)
     bal.sync(None, NB, plan, relay=relay)
     EG = E // world
     bal.grad_reduce(master[rank * EG:(rank + 1) * EG], None, torch.float32, P, plan)
@@ -113,8 +129,9 @@ def _worker(rank, world, relay, port, ids_full, W, master, grads, log, t0, q):
 def test_sharded_balancer_on_gloo_ranks(world, relay):
     sys.path.insert(0, ROOT)
     import oracle
-    ids, W0, m0, g0 = _inputs()
+    ids, W0, m0, g0, Wn = _inputs()
     ids_t = torch.from_numpy(ids).share_memory_()
+    W_new = torch.from_numpy(Wn).share_memory_()
     W = torch.from_numpy(W0.copy()).share_memory_()
     master = torch.from_numpy(m0.copy()).share_memory_()
     grads = torch.from_numpy(g0).share_memory_()
@@ -123,7 +140,7 @@ def test_sharded_balancer_on_gloo_ranks(world, relay):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, relay, port, ids_t, W, master, grads, log, t0, q))
+    procs = [ctx.Process(target=_worker, args=(r, world, relay, port, ids_t, W, master, grads, W_new, log, t0, q))
              for r in range(world)]
     for p in procs:
         p.start()
@@ -140,6 +157,8 @@ def test_sharded_balancer_on_gloo_ranks(world, relay):
         assert np.array_equal(se, ref["plan"]["slot_expert"])
     assert np.array_equal(np.concatenate([o[4] for o in out]), ref["phys"])
     Wref = W0.copy()
+    home = (np.arange(Wref.shape[0]) % (E // N + R)) < E // N
+    Wref[home] = Wn[home]
     oracle.sync(Wref, NB, E, N, R, ref["plan"]["slot_expert"])
     assert np.array_equal(W.numpy(), Wref)
     mref = m0.copy()
@@ -147,6 +166,7 @@ def test_sharded_balancer_on_gloo_ranks(world, relay):
     assert np.array_equal(master.numpy(), mref)
     lg = log.numpy()
     rows = list(range(1, rounds + 1)) if relay else [0]
+    assert lg[:, rows[0], 0].min() >= lg[:, 6, 1].max(), "a sync round started before every home slot was written"
     for a, b in zip(rows, rows[1:]):
         assert lg[:, b, 0].min() >= lg[:, a, 1].max(), f"log row {b} started before row {a} ended"
     assert lg[:, 7, 0].min() >= lg[:, rows[-1], 1].max()   # gradient reduction after the last sync round
