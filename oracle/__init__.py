@@ -30,6 +30,12 @@ Pinning status (what fixes each function other than itself; the tests under
                 previous plan, the incremental sync leaves exactly the state a
                 full sync gives; slots whose expert is unchanged are untouched;
                 the copied-slot count equals a numpy count.
+  sync_restore  replay of a stack of layers sharing the redundant slots
+                (forward syncs, backward restores in reverse) on tagged bytes:
+                after each restore every redundant slot the layer's plan fills
+                holds its expert's home bytes and nothing else changed; the
+                copy count equals a numpy count; restoring the plan the slots
+                hold copies nothing; an unknown holder is a full sync.
   sync_relay    after the relay rounds (or the one direct round) the state
                 equals the single-GPU sync on tagged bytes, so a pull from a
                 GPU that had not yet received its part shows; the home sends
@@ -84,12 +90,13 @@ def _open(path: str) -> ctypes.CDLL:
     lib.ue_oracle_dispatch.argtypes = [vp, i64, ci, vp, vp, vp, vp]
     lib.ue_oracle_sync.argtypes = [vp, i64, i64, ci, ci, ci, vp]
     lib.ue_oracle_sync_delta.argtypes = [vp, i64, i64, ci, ci, ci, vp, vp, vp]
+    lib.ue_oracle_sync_restore.argtypes = [vp, i64, i64, ci, ci, ci, vp, vp, vp]
     lib.ue_oracle_grad_reduce.argtypes = [vp, i64, vp, ci, i64, i64, ci, ci, ci, vp, vp]
     lib.ue_oracle_relay_rounds.argtypes = [ci]
     lib.ue_oracle_sync_relay.argtypes = [vp, i64, i64, ci, ci, ci, vp, ci, ci, ci, vp]
     for f in ("ue_oracle_load", "ue_oracle_expert_load", "ue_oracle_plan", "ue_oracle_plan_ex",
               "ue_oracle_reroute", "ue_oracle_dispatch", "ue_oracle_sync",
-              "ue_oracle_sync_delta", "ue_oracle_grad_reduce", "ue_oracle_relay_rounds",
+              "ue_oracle_sync_delta", "ue_oracle_sync_restore", "ue_oracle_grad_reduce", "ue_oracle_relay_rounds",
               "ue_oracle_sync_relay"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
@@ -221,6 +228,23 @@ def sync_delta(W: np.ndarray, nbytes: int, E: int, N: int, R: int, slot_expert: 
     rc = _get().ue_oracle_sync_delta(_p(W), stride, nbytes, E, N, R, _p(_c(slot_expert, np.int32)), _p(prev),
                                      ctypes.byref(n))
     _check(rc, "sync_delta")
+    return int(n.value)
+
+
+def sync_restore(W: np.ndarray, nbytes: int, E: int, N: int, R: int, target_slot_expert: np.ndarray,
+                 held_slot_expert: np.ndarray | None) -> int:
+    """Weight restore in backward, in place on W viewed as bytes [S][slot_stride]:
+    every redundant slot the target plan fills with expert e and that does not
+    hold e already (held_slot_expert[s] != e; all of them when held is None)
+    receives e's home slot.  Returns the number of slots copied."""
+    if not (W.flags.c_contiguous and W.ndim == 2):
+        raise OracleError("W must be a C-contiguous [S][stride] array")
+    stride = W.shape[1] * W.itemsize
+    n = ctypes.c_int64(0)
+    held = None if held_slot_expert is None else _c(held_slot_expert, np.int32)
+    rc = _get().ue_oracle_sync_restore(_p(W), stride, nbytes, E, N, R, _p(_c(target_slot_expert, np.int32)),
+                                       _p(held), ctypes.byref(n))
+    _check(rc, "sync_restore")
     return int(n.value)
 
 

@@ -452,6 +452,42 @@ int ue_oracle_sync_delta(uint8_t *W, int64_t slot_stride, int64_t nbytes,
     return ORC_OK;
 }
 
+/* ---- weight restore in backward ----------------------------------------------
+ * "How dots-infra/ultraep works" (summary paragraph): after planning, weight
+ * sync and routing expansion before expert execution, UltraEP restores
+ * weights and reduces replica gradients during backward.  Reading taken here:
+ * the layers (and microbatches) share the redundant slots, so when backward
+ * reaches a layer its redundant slots hold the replicas of another plan, the
+ * one last synced into them (held_slot_expert), and the expert backward of the
+ * layer needs the layer's own forward replicas back.  So every redundant slot
+ * that the layer's plan fills with expert e (target_slot_expert[s] = e >= 0)
+ * and that does not hold e already receives e's home slot; slots the target
+ * leaves empty, and home slots, are untouched.  held_slot_expert NULL: what
+ * the slots hold is unknown, and every filled redundant slot of the target is
+ * copied.  *copied = the number of slots copied.
+ */
+int ue_oracle_sync_restore(uint8_t *W, int64_t slot_stride, int64_t nbytes, int E, int N, int R,
+                           const int32_t *target_slot_expert, const int32_t *held_slot_expert,
+                           int64_t *copied)
+{
+    if (E < 1 || N < 1 || R < 0 || E % N != 0 || nbytes > slot_stride || nbytes < 0) return ORC_BAD_ARG;
+    const int H = E / N, HR = H + R;
+    int64_t n = 0;
+    for (int r = 0; r < N; ++r)
+        for (int u = 0; u < R; ++u) {
+            const int s = r * HR + H + u;                 /* rank r's u-th redundant slot */
+            const int e = target_slot_expert[s];
+            if (e < 0) continue;                           /* empty under the target: left as it is */
+            if (e >= E) return ORC_BAD_ARG;
+            if (held_slot_expert && held_slot_expert[s] == e) continue;   /* holds e already */
+            const int64_t home_slot = (int64_t)(e / H) * HR + e % H;
+            memcpy(W + (int64_t)s * slot_stride, W + home_slot * slot_stride, (size_t)nbytes);
+            ++n;
+        }
+    if (copied) *copied = n;
+    return ORC_OK;
+}
+
 /* ---- step 4 across GPUs: relay against fan-out overload -------------------
  * The news summary ("Comment fonctionne l'équilibrage en 300 microsecondes")
  * streams expert states between GPUs with a relay mechanism against fan-out

@@ -15,6 +15,7 @@ import oracle
 import test_oracle_dispatch as tdisp
 import test_oracle_plan as tplan
 import test_oracle_plan_variants as tvar
+import test_oracle_restore as trest
 import test_oracle_steps as tsteps
 from moe_expert_load_ue_b200 import inputs
 
@@ -66,6 +67,14 @@ def _sync_pins():
     tsteps.test_sync_delta_same_plan_copies_nothing_and_none_is_full()
 
 
+def _restore_pins():
+    for E, N, R in ((16, 4, 1), (16, 4, 2), (12, 6, 3)):
+        trest.test_restore_layer_stack(E, N, R)
+    trest.test_restore_skips_slots_that_hold_the_expert()
+    trest.test_restore_same_plan_copies_nothing_and_unknown_holder_is_full_sync()
+    trest.test_restore_hand_case()
+
+
 def _grad_pins():
     for bf16 in (False, True):
         tsteps.test_grad_reduce_exact_dyadic(bf16)
@@ -108,6 +117,13 @@ MUTANTS = {
                                         "        memcpy(W + (int64_t)s * slot_stride"),
     "incremental skip inverted": (_sync_pins, "if (prev_slot_expert && prev_slot_expert[s] == e) continue;",
                                   "if (prev_slot_expert && prev_slot_expert[s] != e) continue;"),
+    "restore skip inverted": (_restore_pins, "if (held_slot_expert && held_slot_expert[s] == e) continue;",
+                              "if (held_slot_expert && held_slot_expert[s] != e) continue;"),
+    "restore ignores the holder": (_restore_pins, "if (held_slot_expert && held_slot_expert[s] == e) continue;",
+                                   "if (0) continue;"),
+    "restore from the rank's first home slot": (_restore_pins,
+                                                "const int64_t home_slot = (int64_t)(e / H) * HR + e % H;",
+                                                "const int64_t home_slot = (int64_t)(e / H) * HR;"),
     "last replica's gradient dropped": (_grad_pins, "for (int i = rep_off[e] + 1; i < rep_off[e + 1]; ++i) {",
                                         "for (int i = rep_off[e] + 1; i < rep_off[e + 1] - 1; ++i) {"),
     "bf16 widened into the low half": (_grad_pins, "uint32_t u = (uint32_t)h << 16;", "uint32_t u = (uint32_t)h;"),
@@ -133,7 +149,8 @@ def _passes(pins):
     return True
 
 
-@pytest.mark.parametrize("pins", [_plan_pins, _variant_pins, _reroute_pins, _load_pins, _dispatch_pins, _sync_pins, _grad_pins],
+@pytest.mark.parametrize("pins", [_plan_pins, _variant_pins, _reroute_pins, _load_pins, _dispatch_pins, _sync_pins,
+                                  _restore_pins, _grad_pins],
                          ids=lambda f: f.__name__)
 def test_unchanged_copy_passes(tmp_path, monkeypatch, pins):
     monkeypatch.setattr(oracle, "_lib", _mutant(tmp_path, "int64_t j = occ[e]++;", "int64_t j = occ[e]++;"))
