@@ -48,7 +48,13 @@ typedef enum {
 } ue_status;
 
 /* Opaque per-device context: caches device properties and kernel attributes
- * and owns one device status word for bounded-wait failures. */
+ * and owns a device status word for bounded-wait failures and a 16 MiB device
+ * workspace, both allocated by ue_ctx_create.  The workspace holds the
+ * per-piece histograms that ue_rebalance(_ex) and ue_reroute(_shard) pass
+ * from their load pass to their reroute pass when a CTA's share of a rank's
+ * ids exceeds what the reroute keeps on chip (many ranks or many tokens per
+ * rank); such calls on one context must not overlap on the GPU (issue them on
+ * one stream, or order the streams). */
 typedef struct ue_ctx ue_ctx;
 
 /* Problem shape.  H = E / N and S = N * (H + R) are derived. */
@@ -91,6 +97,20 @@ ue_status ue_ctx_destroy(ue_ctx *ctx);
  * `stream`) and clear it.  Bit 0: a kernel gave up a bounded wait; bit 1:
  * ue_dispatch met ids that do not match the plan. */
 ue_status ue_ctx_device_error(ue_ctx *ctx, int32_t *host_word, void *stream);
+
+/* Bound of every wait inside the weight-sync kernels (ue_sync, ue_sync_delta,
+ * ue_sync_shard): a copy that has not landed limit_ns nanoseconds (GPU global
+ * timer) after the kernel began to wait for it makes the kernel give up - it
+ * sets bit 0 of the status word, waits for its other copies in flight (each
+ * wait again bounded by limit_ns) and returns; that call's slots are then
+ * incomplete, and a copy that never lands leaves the device state undefined.
+ * Default 2 s; limit_ns in [1000, 6e10].  Host only; affects later calls.
+ *   flags  UE_WAIT_STALL_ONCE (diagnostic, for testing the way out): the next
+ *          weight-sync call on this context makes its first CTA, once its
+ *          first copies are in flight, wait once on a barrier that nothing
+ *          completes, so that this wait runs out; the flag then clears. */
+#define UE_WAIT_STALL_ONCE 1
+ue_status ue_ctx_set_wait_limit(ue_ctx *ctx, int64_t limit_ns, int32_t flags);
 
 /* ---- step 1: load computation ----------------------------------------------
  * "Load computation" (csrc/kernels/load_compute.cu in the component list of
@@ -209,6 +229,23 @@ ue_status ue_sync(ue_ctx *ctx, const ue_config *cfg, void *weights, int64_t slot
  * microbatch after an optimizer step). */
 ue_status ue_sync_delta(ue_ctx *ctx, const ue_config *cfg, void *weights, int64_t slot_bytes,
                         const ue_plan_buffers *plan, const int32_t *prev_slot_expert, void *stream);
+
+/* Weight restore in backward ("How dots-infra/ultraep works", summary
+ * paragraph: UltraEP restores weights and reduces replica gradients during
+ * backward).  The layers (and microbatches) share the redundant slots, so when
+ * backward reaches a layer its slots hold the replicas of another plan; this
+ * call brings back the layer's forward replicas before its expert backward:
+ * every filled redundant slot of `plan` (the layer's saved forward plan) whose
+ * expert differs from held_slot_expert[s] receives a byte copy of its expert's
+ * home slot; other slots are untouched.
+ *   held_slot_expert  [S] device memory, read only: the expert each slot holds
+ *                     now (the slot_expert of the plan last synced into it, or
+ *                     built by the caller slot by slot); NULL = unknown, every
+ *                     filled redundant slot of plan is copied.
+ * The same operation as ue_sync_delta with the saved plan as its target; the
+ * weights, slot_bytes and alignment rules are those of ue_sync. */
+ue_status ue_sync_restore(ue_ctx *ctx, const ue_config *cfg, void *weights, int64_t slot_bytes,
+                          const ue_plan_buffers *plan, const int32_t *held_slot_expert, void *stream);
 
 /* ---- step 5: replica gradient reduction ------------------------------------
  * "Replica gradient reduction" (csrc/kernels/grad_reduce.cu; "Expert compute

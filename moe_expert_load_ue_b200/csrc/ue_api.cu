@@ -3,6 +3,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <new>
 
 #include "ue_internal.cuh"
@@ -13,6 +14,7 @@ cudaError_t set_reroute_attributes(size_t max_smem);
 cudaError_t set_plan_attributes(size_t max_smem);
 cudaError_t set_sync_attributes(size_t max_smem);
 cudaError_t set_shard_attributes(size_t max_smem);
+cudaError_t set_reroute_pieces_attributes(size_t max_smem);
 int grad_blocks_per_sm(int grad_dtype);
 int grad_shard_blocks_per_sm(int grad_dtype);
 }  // namespace ue
@@ -24,7 +26,34 @@ struct ue_ctx {
     int grad_blocks[2];    // resident grad-reduce CTAs per SM (fp32, bf16)
     int grad_shard_blocks[2];  // the same for the gradient reduction across GPUs
     int32_t *dev_err;      // device status word for bounded waits
+    int32_t *ws;           // workspace: piece histogram rows of the persistent reroute
+    int rp_blocks;         // resident persistent-reroute CTAs per SM as registers allow
+    int smem_per_sm;       // shared memory of an SM, and the part each resident CTA reserves
+    int smem_reserved;
+    int64_t wait_ns;       // bound of one wait in the weight-sync kernels
+    int stall_once;        // diagnostic: the next weight sync stalls once (UE_WAIT_STALL_ONCE)
 };
+
+namespace {
+// Workspace of a context (16 MiB): kWsHead ints of counters (the persistent
+// reroute's piece counters, kept at 0 between launches), then the piece rows
+// [N][B + 1][E + 1] of one call.
+constexpr int64_t kWsInts = (int64_t)1 << 22;
+constexpr int64_t kWsHead = 64;
+// Pieces of the persistent reroute are whole sub-chunks of its CTA (8192 ids:
+// 16 per thread), so every warp has work; its per-piece table costs about as
+// much as streaming a few thousand ids.
+constexpr int64_t kPieceQuantum = 8192;
+// Pieces per resident CTA aimed at (they are claimed dynamically; more,
+// smaller pieces shorten the tail).
+constexpr int kPiecesPerCta = 16;
+// Largest CTA share of a rank's ids routed by the rank-per-cluster kernel.
+// Measured on B200 over the sweep's shapes: up to 64 Ki ids per share it is
+// faster (its first pass overlaps the planner; the persistent kernel pays a
+// few microseconds more of fixed cost); from 128 Ki ids the persistent kernel
+// is faster, by up to 2x when the quota boundaries crowd into one rank.
+constexpr int64_t kClusterShareMax = 65536;
+}  // namespace
 
 namespace {
 
@@ -113,6 +142,40 @@ ue::Launch launch_of(const ue_ctx *ctx, const ue::Shape &sh)
     return ln;
 }
 
+// The persistent reroute over pieces is used when a CTA's share of a rank's
+// ids in the rank-per-cluster kernel is large (kClusterShareMax): that kernel
+// would read the ids twice, and one CTA per rank would walk all of a rank's
+// quota boundaries alone.  Pieces: about kPiecesPerCta per resident CTA,
+// whole multiples of kPieceQuantum ids, within the workspace and the load
+// kernel's shared memory.
+ue::Pieces pieces_for(const ue_ctx *ctx, const ue::Shape &sh, const ue::Launch &ln)
+{
+    ue::Pieces pc{0, 0, 0, 0};
+    if (sh.per_rank <= 0) return pc;
+    const int64_t share = ((sh.per_rank + ln.cluster - 1) / ln.cluster + 31) / 32 * 32;
+    if (share <= kClusterShareMax) return pc;
+    const size_t rp_smem = ue::reroute_pieces_smem_bytes(sh);
+    if (rp_smem > (size_t)ctx->max_smem) return pc;
+    const int per_sm = std::min<int>(ctx->rp_blocks, ctx->smem_per_sm / (int)(rp_smem + ctx->smem_reserved));
+    const int grid = ctx->sms * std::max(per_sm, 1);
+    // Pieces per rank within the workspace and within the load kernel's
+    // shared memory (each of its CTAs keeps its pieces' counts).
+    const int64_t b_ws = (kWsInts - kWsHead) / ((int64_t)sh.N * (sh.E + 1)) - 1;
+    const int64_t ppc_smem = ((int64_t)ctx->max_smem - (int64_t)ue::load_smem_bytes(sh, 0)) /
+                             ((int64_t)(sh.E + 1) * (int64_t)sizeof(int32_t));
+    const int64_t b_cap = std::min(b_ws, ppc_smem * ln.cluster);
+    if (grid < 1 || b_cap < 1) return pc;
+    int64_t B = ((int64_t)kPiecesPerCta * grid + sh.N - 1) / sh.N;
+    B = std::max<int64_t>(1, std::min(B, b_cap));
+    int64_t zp = ((sh.per_rank + B - 1) / B + kPieceQuantum - 1) / kPieceQuantum * kPieceQuantum;
+    B = (sh.per_rank + zp - 1) / zp;
+    pc.B = (int)B;
+    pc.zp = zp;
+    pc.NP = (int)(sh.N * B);
+    pc.grid = grid;
+    return pc;
+}
+
 // Run fn with ctx's device current, restoring the caller's device.
 template <class F>
 ue_status on_device(const ue_ctx *ctx, F &&fn)
@@ -173,7 +236,12 @@ ue_status ue_ctx_create(int device, ue_ctx **out)
     tmp.device = device;
     tmp.sms = prop.multiProcessorCount;
     tmp.max_smem = (int)prop.sharedMemPerBlockOptin;
+    tmp.smem_per_sm = (int)prop.sharedMemPerMultiprocessor;
+    tmp.smem_reserved = (int)prop.reservedSharedMemPerBlock;
     tmp.dev_err = nullptr;
+    tmp.ws = nullptr;
+    tmp.wait_ns = 2000000000LL;
+    tmp.stall_once = 0;
     ue_status s = on_device(&tmp, [&]() -> ue_status {
         cudaError_t err;
         const size_t m = (size_t)tmp.max_smem;
@@ -186,17 +254,21 @@ ue_status ue_ctx_create(int device, ue_ctx **out)
         if ((err = ue::set_shard_attributes(m)) != cudaSuccess) return cuda_fail(err, "shard attributes");
         tmp.grad_shard_blocks[0] = ue::grad_shard_blocks_per_sm(0);
         tmp.grad_shard_blocks[1] = ue::grad_shard_blocks_per_sm(1);
+        if ((err = ue::set_reroute_pieces_attributes(m)) != cudaSuccess) return cuda_fail(err, "reroute attributes");
+        tmp.rp_blocks = ue::reroute_pieces_blocks_per_sm(0);
         if ((err = cudaMalloc(&tmp.dev_err, sizeof(int32_t))) != cudaSuccess) return cuda_fail(err, "cudaMalloc");
-        if ((err = cudaMemset(tmp.dev_err, 0, sizeof(int32_t))) != cudaSuccess) {
+        if ((err = cudaMemset(tmp.dev_err, 0, sizeof(int32_t))) != cudaSuccess ||
+            (err = cudaMalloc(&tmp.ws, kWsInts * sizeof(int32_t))) != cudaSuccess ||
+            (err = cudaMemset(tmp.ws, 0, kWsHead * sizeof(int32_t))) != cudaSuccess) {
             cudaFree(tmp.dev_err);
-            return cuda_fail(err, "cudaMemset");
+            return cuda_fail(err, "workspace");
         }
         return UE_OK;
     });
     if (s != UE_OK) return s;
     ue_ctx *ctx = new (std::nothrow) ue_ctx(tmp);
     if (!ctx) {
-        on_device(&tmp, [&]() { cudaFree(tmp.dev_err); return UE_OK; });
+        on_device(&tmp, [&]() { cudaFree(tmp.dev_err); cudaFree(tmp.ws); return UE_OK; });
         return fail(UE_ERR_INVALID_ARG, "out of host memory");
     }
     *out = ctx;
@@ -208,10 +280,24 @@ ue_status ue_ctx_destroy(ue_ctx *ctx)
     if (!ctx) return UE_OK;
     ue_status s = on_device(ctx, [&]() -> ue_status {
         cudaError_t e = cudaFree(ctx->dev_err);
+        const cudaError_t e2 = cudaFree(ctx->ws);
+        if (e == cudaSuccess) e = e2;
         return e == cudaSuccess ? UE_OK : cuda_fail(e, "cudaFree");
     });
     delete ctx;
     return s;
+}
+
+ue_status ue_ctx_set_wait_limit(ue_ctx *ctx, int64_t limit_ns, int32_t flags)
+{
+    ue_status s = check_ctx(ctx);
+    if (s != UE_OK) return s;
+    if (limit_ns < 1000 || limit_ns > 60000000000LL)
+        return fail(UE_ERR_INVALID_ARG, "limit_ns=%lld outside [1000, 6e10]", (long long)limit_ns);
+    if (flags & ~UE_WAIT_STALL_ONCE) return fail(UE_ERR_INVALID_ARG, "flags=%d (bit 0: UE_WAIT_STALL_ONCE)", flags);
+    ctx->wait_ns = limit_ns;
+    ctx->stall_once = (flags & UE_WAIT_STALL_ONCE) ? 1 : 0;
+    return UE_OK;
 }
 
 ue_status ue_ctx_device_error(ue_ctx *ctx, int32_t *host_word, void *stream)
@@ -285,8 +371,19 @@ ue_status ue_reroute(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids, cons
         return fail(UE_ERR_INVALID_ARG, "reroute needs %zu bytes of shared memory (> %d)",
                     ue::reroute_smem_bytes(sh, false, 0, false), ctx->max_smem);
     return on_device(ctx, [&]() -> ue_status {
-        cudaError_t e = ue::launch_reroute(sh, launch_of(ctx, sh), ids, ue::to_dev(*plan), phys,
-                                           static_cast<cudaStream_t>(stream), false);
+        const cudaStream_t st = static_cast<cudaStream_t>(stream);
+        const ue::Launch ln = launch_of(ctx, sh);
+        const ue::Pieces pc = pieces_for(ctx, sh, ln);
+        cudaError_t e;
+        if (pc.NP > 0) {
+            // The piece rows first (no counts), then the persistent reroute.
+            if ((e = ue::launch_load(sh, ln, ids, nullptr, nullptr, st, &pc, ctx->ws + kWsHead)) != cudaSuccess)
+                return cuda_fail(e, "load launch");
+            e = ue::launch_reroute_pieces(sh, pc, ids, ue::to_dev(*plan), ctx->ws + kWsHead, ctx->ws, phys, st,
+                                          false);
+        } else {
+            e = ue::launch_reroute(sh, ln, ids, ue::to_dev(*plan), phys, st, false);
+        }
         return e == cudaSuccess ? UE_OK : cuda_fail(e, "reroute launch");
     });
 }
@@ -311,15 +408,17 @@ ue_status ue_rebalance_ex(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids,
         const cudaStream_t st = static_cast<cudaStream_t>(stream);
         const ue::Launch ln = launch_of(ctx, sh);
         const ue::PlanDev pd = ue::to_dev(*plan);
-        cudaError_t e = ue::launch_load(sh, ln, ids, counts, bad, st);
+        const ue::Pieces pc = pieces_for(ctx, sh, ln);
+        cudaError_t e = ue::launch_load(sh, ln, ids, counts, bad, st, &pc, ctx->ws + kWsHead);
         if (e != cudaSuccess) return cuda_fail(e, "load launch");
         // The planner and the reroute kernel use programmatic dependent launch:
         // each may start while its predecessor drains, and waits for it
         // (griddepcontrol.wait) before reading what it wrote.
         if ((e = ue::launch_plan(sh, counts, pd, st, true, variant)) != cudaSuccess)
             return cuda_fail(e, "plan launch");
-        if ((e = ue::launch_reroute(sh, ln, ids, pd, phys, st, true)) != cudaSuccess)
-            return cuda_fail(e, "reroute launch");
+        e = pc.NP > 0 ? ue::launch_reroute_pieces(sh, pc, ids, pd, ctx->ws + kWsHead, ctx->ws, phys, st, true)
+                      : ue::launch_reroute(sh, ln, ids, pd, phys, st, true);
+        if (e != cudaSuccess) return cuda_fail(e, "reroute launch");
         return UE_OK;
     });
 }
@@ -412,8 +511,10 @@ ue_status sync_common(ue_ctx *ctx, const ue_config *cfg, void *weights, int64_t 
         return fail(UE_ERR_INVALID_ARG, "sync needs %zu bytes of shared memory (> %d)", ue::sync_smem_bytes(sh),
                     ctx->max_smem);
     return on_device(ctx, [&]() -> ue_status {
+        const ue::WaitBound wb{(unsigned long long)ctx->wait_ns, ctx->stall_once};
         cudaError_t e = ue::launch_sync(sh, launch_of(ctx, sh), static_cast<uint8_t *>(weights), slot_bytes,
-                                        ue::to_dev(*plan), prev, ctx->dev_err, static_cast<cudaStream_t>(stream));
+                                        ue::to_dev(*plan), prev, ctx->dev_err, static_cast<cudaStream_t>(stream), wb);
+        ctx->stall_once = 0;
         return e == cudaSuccess ? UE_OK : cuda_fail(e, "sync launch");
     });
 }
@@ -429,6 +530,14 @@ ue_status ue_sync_delta(ue_ctx *ctx, const ue_config *cfg, void *weights, int64_
                         const ue_plan_buffers *plan, const int32_t *prev_slot_expert, void *stream)
 {
     return sync_common(ctx, cfg, weights, slot_bytes, plan, prev_slot_expert, stream);
+}
+
+ue_status ue_sync_restore(ue_ctx *ctx, const ue_config *cfg, void *weights, int64_t slot_bytes,
+                          const ue_plan_buffers *plan, const int32_t *held_slot_expert, void *stream)
+{
+    // The incremental sync towards the saved plan: every filled redundant slot
+    // whose expert differs from the one it holds now receives its home slot.
+    return sync_common(ctx, cfg, weights, slot_bytes, plan, held_slot_expert, stream);
 }
 
 ue_status ue_grad_reduce(ue_ctx *ctx, const ue_config *cfg, float *master, const void *grads, int grad_dtype,
@@ -530,8 +639,17 @@ ue_status ue_reroute_shard(ue_ctx *ctx, const ue_config *cfg, const ue_shard *sh
     ue::PlanDev pd = ue::to_dev(*plan);
     pd.rank_off += (int64_t)shard->g * l.N * sh.E;     // this GPU's rows of rank_off
     return on_device(ctx, [&]() -> ue_status {
-        cudaError_t e = ue::launch_reroute(l, launch_of(ctx, l), ids_local, pd, phys_local,
-                                           static_cast<cudaStream_t>(stream), false);
+        const cudaStream_t st = static_cast<cudaStream_t>(stream);
+        const ue::Launch ln = launch_of(ctx, l);
+        const ue::Pieces pc = pieces_for(ctx, l, ln);
+        cudaError_t e;
+        if (pc.NP > 0) {
+            if ((e = ue::launch_load(l, ln, ids_local, nullptr, nullptr, st, &pc, ctx->ws + kWsHead)) != cudaSuccess)
+                return cuda_fail(e, "load launch");
+            e = ue::launch_reroute_pieces(l, pc, ids_local, pd, ctx->ws + kWsHead, ctx->ws, phys_local, st, false);
+        } else {
+            e = ue::launch_reroute(l, ln, ids_local, pd, phys_local, st, false);
+        }
         return e == cudaSuccess ? UE_OK : cuda_fail(e, "reroute launch");
     });
 }
@@ -555,9 +673,11 @@ ue_status ue_sync_shard(ue_ctx *ctx, const ue_config *cfg, const ue_shard *shard
         return fail(UE_ERR_INVALID_ARG, "sync needs %zu bytes of shared memory (> %d)", ue::sync_shard_smem_bytes(sh),
                     ctx->max_smem);
     return on_device(ctx, [&]() -> ue_status {
+        const ue::WaitBound wb{(unsigned long long)ctx->wait_ns, ctx->stall_once};
         cudaError_t e = ue::launch_sync_shard(sh, launch_of(ctx, sh), t, static_cast<uint8_t *>(slot_bases[shard->g]),
                                               shard->G, shard->g, round, slot_bytes, ue::to_dev(*plan), ctx->dev_err,
-                                              static_cast<cudaStream_t>(stream));
+                                              static_cast<cudaStream_t>(stream), wb);
+        ctx->stall_once = 0;
         return e == cudaSuccess ? UE_OK : cuda_fail(e, "sync launch");
     });
 }

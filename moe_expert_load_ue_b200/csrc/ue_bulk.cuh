@@ -12,7 +12,7 @@ namespace {
 constexpr int kSyncThreads = 128;
 constexpr int kSyncStages = 4;
 constexpr int kSyncTile = 48 * 1024;                       // bytes per stage
-constexpr unsigned long long kWaitLimitNs = 2000000000ull; // 2 s per wait
+constexpr unsigned long long kWaitLimitNs = 2000000000ull; // default bound of one wait: 2 s
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p)
 {
@@ -48,6 +48,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity)
         : "r"(smem_addr(bar)), "r"(parity)
         : "memory");
     return ok != 0;
+}
+
+// Waits until the mbarrier completes the given phase or limit_ns passes on the
+// global timer; false if it gave up.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity, unsigned long long limit_ns)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_ns() - t0 > limit_ns) return false;
+    return true;
+}
+
+// The ring's way out after a wait gave up: record the error, then wait (each
+// wait bounded again) for the loads this thread issued into stages it has not
+// consumed - items first .. issued-1 of the ring - so that no copy lands in
+// shared memory after the CTA exits, and drain its bulk stores.  A load that
+// never completes is abandoned after its bound; the device state is then
+// undefined, which the status word reports.
+__device__ __forceinline__ void ring_give_up(int32_t *dev_err, uint64_t *bar, int stages, int64_t first,
+                                             int64_t issued, unsigned long long limit_ns)
+{
+    atomicOr(dev_err, 1);
+    for (int64_t k = first; k < issued; ++k)
+        mbar_wait_bounded(&bar[k % stages], (unsigned)((k / stages) & 1), limit_ns);
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 __device__ __forceinline__ void bulk_load(void *dst_smem, const void *src, unsigned bytes, uint64_t *bar)

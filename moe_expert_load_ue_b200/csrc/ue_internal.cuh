@@ -54,10 +54,26 @@ struct DispatchOut {
     float *gates_out;
 };
 
+// Cut of each rank's ids into B pieces of zp ids for the persistent reroute
+// kernel (NP = N * B pieces; NP = 0: the rank-per-cluster kernel is used).
+// The load kernel writes to the workspace, per rank, B + 1 rows of E + 1 ints
+// (rows [N][B + 1][E + 1]): row b holds the occurrences of each expert (column
+// E: of ids outside [0, E)) in the rank's ids before piece b, row B the rank's
+// totals.
+struct Pieces {
+    int B;          // pieces per rank
+    int64_t zp;     // ids per piece (a multiple of 32; the last piece of a rank may be shorter)
+    int NP;         // N * B, or 0
+    int grid;       // CTAs of the persistent reroute kernel
+};
+
 // Host launchers (one per kernel file).  Each returns cudaGetLastError().
+// With pc (NP > 0) the load kernel also writes the piece rows; counts may then
+// be nullptr (the rows alone, for a reroute without a preceding load).
 cudaError_t launch_load(const Shape &sh, const Launch &ln, const int32_t *ids, int32_t *counts,
-                        int32_t *bad, cudaStream_t st);
-size_t load_smem_bytes(const Shape &sh);
+                        int32_t *bad, cudaStream_t st, const Pieces *pc = nullptr, int32_t *rows = nullptr);
+// Shared memory of the load kernel; ppc = pieces per CTA (0: no piece rows).
+size_t load_smem_bytes(const Shape &sh, int ppc);
 
 // variant: bit 0 re-queues partly placed overflow, bit 1 spreads stuck
 // remainders over the expert's replicas (0 = the stated rule).
@@ -75,9 +91,25 @@ cudaError_t launch_dispatch(const Shape &sh, const Launch &ln, const int32_t *id
 // many gates when the dispatch variant carries them.
 size_t reroute_smem_bytes(const Shape &sh, bool dispatch, int stage_cap, bool gates);
 
+// The persistent reroute over the pieces whose rows the load kernel wrote.
+// ctr: two ints of the workspace, 0 before the launch (the kernel leaves them 0).
+cudaError_t launch_reroute_pieces(const Shape &sh, const Pieces &pc, const int32_t *ids, const PlanDev &plan,
+                                  const int32_t *rows, int32_t *ctr, int32_t *phys, cudaStream_t st, bool pdl);
+size_t reroute_pieces_smem_bytes(const Shape &sh);
+int reroute_pieces_blocks_per_sm(size_t smem);
+cudaError_t set_reroute_pieces_attributes(size_t max_smem);
+
+// Bound of the weight-sync kernels' mbarrier waits (ns on the global timer)
+// and the diagnostic stall (CTA 0 waits once on a barrier nothing completes).
+struct WaitBound {
+    unsigned long long ns;
+    int stall;
+};
+
 // prev_slot_expert: the previous plan's slot_expert for the incremental form, or nullptr.
 cudaError_t launch_sync(const Shape &sh, const Launch &ln, uint8_t *weights, int64_t slot_bytes,
-                        const PlanDev &plan, const int32_t *prev_slot_expert, int32_t *dev_err, cudaStream_t st);
+                        const PlanDev &plan, const int32_t *prev_slot_expert, int32_t *dev_err, cudaStream_t st,
+                        const WaitBound &wb);
 size_t sync_smem_bytes(const Shape &sh);
 
 cudaError_t launch_grad_reduce(const Shape &sh, const Launch &ln, float *master, const void *grads,
@@ -91,7 +123,7 @@ size_t grad_smem_bytes(const Shape &sh);
 int relay_rounds(int G);
 cudaError_t launch_sync_shard(const Shape &sh, const Launch &ln, const PeerTable &base, uint8_t *local, int G,
                               int g, int round, int64_t slot_bytes, const PlanDev &plan, int32_t *dev_err,
-                              cudaStream_t st);
+                              cudaStream_t st, const WaitBound &wb);
 size_t sync_shard_smem_bytes(const Shape &sh);
 cudaError_t launch_grad_reduce_shard(const Shape &sh, const Launch &ln, float *master, const PeerTable &grads,
                                      int G, int g, int grad_dtype, int64_t P, const PlanDev &plan, cudaStream_t st);

@@ -10,8 +10,10 @@
 // shared atomics on a popular expert collide only inside a warp), sums the
 // copies, and the cluster then reduces its CTA histograms over distributed
 // shared memory, each CTA summing a slice of the E columns.  The rank's row
-// of counts is written with plain stores: no global atomics, no pre-zeroing,
-// no workspace.
+// of counts is written with plain stores: no global atomics, no pre-zeroing.
+// For microbatches routed by the persistent reroute kernel (many ranks or
+// many tokens per rank) the kernel also writes the histogram of every piece
+// of a rank's ids to the context's workspace; otherwise it uses none.
 #include <cooperative_groups.h>
 
 #include "ue_internal.cuh"
@@ -30,63 +32,50 @@ __device__ __forceinline__ void count_id(int32_t *h, int id, int E, int &nbad)
     else ++nbad;
 }
 
-__global__ void __launch_bounds__(kLoadWarps * 32)
-k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
-       int32_t *__restrict__ counts, int32_t *__restrict__ bad)
+// The first four int4 vectors of every thread for the range [lo, hi) (its
+// 16-byte aligned body), loaded before the histograms are cleared or reduced.
+struct Head {
+    int4 q[4];
+};
+
+__device__ __forceinline__ Head load_head(const int32_t *__restrict__ ids, int64_t lo, int64_t hi)
 {
-    extern __shared__ __align__(16) int32_t sm_load[];
-    int32_t *hist = sm_load;                     // [kCopies][E] counts
-    int32_t *tot = hist + kCopies * E;           // [E]    CTA counts (read by the cluster)
-    int32_t *sbad = tot + E;                     // [1]
+    const int64_t vlo = min(hi, (lo + 3) / 4 * 4);
+    const int64_t vhi = max(vlo, hi / 4 * 4);
+    const int4 *vec = reinterpret_cast<const int4 *>(ids + vlo);
+    const int64_t nvec = (vhi - vlo) / 4;
+    Head hd;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int64_t v = threadIdx.x + k * (int64_t)blockDim.x;
+        hd.q[k] = v < nvec ? __ldg(vec + v) : make_int4(-1, -1, -1, -1);
+    }
+    return hd;
+}
 
-    // The planner (launched with programmatic dependent launch) may start
-    // now; it waits for this grid's completion before reading counts.
-    pdl_trigger();
-
-    cg::cluster_group cluster = cg::this_cluster();
-    const int C = (int)cluster.num_blocks();
-    const int c = (int)cluster.block_rank();
-    const int r = blockIdx.x / C;
+// Counts the ids of [lo, hi) into this warp's histogram copy h: a ragged head
+// and tail (< 4 ids each) by warp 0, the body as int4 vectors, four in flight
+// per thread (the first four already in hd).
+__device__ __forceinline__ void count_range(const int32_t *__restrict__ ids, int64_t lo, int64_t hi, int E,
+                                            int32_t *h, int &nbad, const Head &hd)
+{
     const int lane = lane_id(), warp = threadIdx.x >> 5;
-
-    // This CTA's share [lo, hi) of rank r's flat id range, 32-id aligned shares.
-    const int64_t share = ((per_rank + C - 1) / C + 31) / 32 * 32;
-    const int64_t base = (int64_t)r * per_rank;
-    const int64_t lo = base + min(per_rank, (int64_t)c * share);
-    const int64_t hi = base + min(per_rank, (int64_t)(c + 1) * share);
-    // int4 body [vlo, vhi) on 16-byte boundaries (ids is 16-byte aligned).
     const int64_t vlo = min(hi, (lo + 3) / 4 * 4);
     const int64_t vhi = max(vlo, hi / 4 * 4);
     const int4 *vec = reinterpret_cast<const int4 *>(ids + vlo);
     const int64_t nvec = (vhi - vlo) / 4;
     const int64_t stride = (int64_t)blockDim.x;
-    // The first four vectors of every thread are in flight while the
-    // histograms are cleared.
-    int4 q0[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int64_t v = threadIdx.x + k * stride;
-        q0[k] = v < nvec ? __ldg(vec + v) : make_int4(-1, -1, -1, -1);
-    }
-    for (int i = threadIdx.x; i < kCopies * E; i += blockDim.x) hist[i] = 0;
-    if (threadIdx.x == 0) *sbad = 0;
-    __syncthreads();
-    int32_t *h = hist + (warp % kCopies) * E;
-    int nbad = 0;
-
-    // Ragged head (< 4 ids) and tail (< 4 ids).
     if (warp == 0) {
         int64_t i = -1;
         if (lane < vlo - lo) i = lo + lane;
         else if (lane >= 4 && lane - 4 < hi - vhi) i = vhi + (lane - 4);
         if (i >= 0) count_id(h, __ldg(ids + i), E, nbad);
     }
-    // Body: every thread walks int4 vectors, four in flight.
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         if (threadIdx.x + k * stride < nvec) {
-            count_id(h, q0[k].x, E, nbad); count_id(h, q0[k].y, E, nbad);
-            count_id(h, q0[k].z, E, nbad); count_id(h, q0[k].w, E, nbad);
+            count_id(h, hd.q[k].x, E, nbad); count_id(h, hd.q[k].y, E, nbad);
+            count_id(h, hd.q[k].z, E, nbad); count_id(h, hd.q[k].w, E, nbad);
         }
     }
     int64_t v = threadIdx.x + 4 * stride;
@@ -104,13 +93,93 @@ k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
         const int4 a = __ldg(vec + v);
         count_id(h, a.x, E, nbad); count_id(h, a.y, E, nbad); count_id(h, a.z, E, nbad); count_id(h, a.w, E, nbad);
     }
-    if (nbad) atomicAdd(sbad, nbad);
+}
+
+// PIECES: the CTA's share is cut into pieces of zp ids (piece b of the rank is
+// [b*zp, (b+1)*zp), pieces c*ppc .. c*ppc+ppc-1 in CTA c of the cluster).
+// Row b of rank r, rows[(r*(B+1) + b)][0..E), receives the occurrences of
+// every expert in the rank's ids before piece b (an exclusive prefix over the
+// pieces), and row B the rank's totals; column E counts the ids outside
+// [0, E) the same way.  The persistent reroute kernel takes each piece's
+// starting occurrence indices and its counts from two consecutive rows.
+template <bool PIECES>
+__global__ void __launch_bounds__(kLoadWarps * 32)
+k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
+       int32_t *__restrict__ counts, int32_t *__restrict__ bad,
+       int32_t *__restrict__ rows, int64_t zp, int B)
+{
+    extern __shared__ __align__(16) int32_t sm_load[];
+    int32_t *hist = sm_load;                     // [kCopies][E] counts
+    int32_t *tot = hist + kCopies * E;           // [E]    CTA counts (read by the cluster)
+    int32_t *sbad = tot + E;                     // [4]    bad ids: CTA total; current piece
+    int32_t *pcnt = sbad + 4;                    // PIECES: [ppc][E + 1] counts of the CTA's pieces
+
+    // The planner (launched with programmatic dependent launch) may start
+    // now; it waits for this grid's completion before reading counts.
+    pdl_trigger();
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const int C = (int)cluster.num_blocks();
+    const int c = (int)cluster.block_rank();
+    const int r = blockIdx.x / C;
+    const int warp = threadIdx.x >> 5;
+
+    // This CTA's share [lo, hi) of rank r's flat id range (32-id aligned
+    // shares, or whole pieces).
+    const int ppc = PIECES ? (B + C - 1) / C : 1;
+    const int64_t share = PIECES ? (int64_t)ppc * zp : ((per_rank + C - 1) / C + 31) / 32 * 32;
+    const int64_t base = (int64_t)r * per_rank;
+    const int64_t lo = base + min(per_rank, (int64_t)c * share);
+    const int64_t hi = base + min(per_rank, (int64_t)(c + 1) * share);
+    const int64_t len = PIECES ? zp : share;
+    int32_t *h = hist + (warp % kCopies) * E;
+    int nbad = 0;
+
+    Head hd = load_head(ids, lo, min(hi, lo + len));
+    for (int i = threadIdx.x; i < kCopies * E; i += blockDim.x) hist[i] = 0;
+    if (PIECES)
+        for (int e = threadIdx.x; e < E; e += blockDim.x) tot[e] = 0;
+    if (threadIdx.x == 0) sbad[0] = sbad[1] = 0;
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int s = 0;
+
+    if constexpr (!PIECES) {
+        count_range(ids, lo, hi, E, h, nbad, hd);
+        if (nbad) atomicAdd(&sbad[1], nbad);
+        __syncthreads();
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            int s = 0;
 #pragma unroll
-        for (int w = 0; w < kCopies; ++w) s += hist[w * E + e];
-        tot[e] = s;
+            for (int w = 0; w < kCopies; ++w) s += hist[w * E + e];
+            tot[e] = s;
+        }
+        if (threadIdx.x == 0) sbad[0] = sbad[1];
+    } else {
+        for (int64_t plo = lo; plo < hi; plo += len) {
+            const int64_t phi = min(hi, plo + len);
+            count_range(ids, plo, phi, E, h, nbad, hd);
+            if (nbad) atomicAdd(&sbad[1], nbad);
+            nbad = 0;
+            // The next piece's first vectors load while this one is reduced.
+            if (phi < hi) hd = load_head(ids, phi, min(hi, phi + len));
+            __syncthreads();
+            int32_t *pc = pcnt + (int)((plo - lo) / zp) * (E + 1);
+            for (int e = threadIdx.x; e < E; e += blockDim.x) {
+                int s = 0;
+#pragma unroll
+                for (int w = 0; w < kCopies; ++w) {
+                    s += hist[w * E + e];
+                    hist[w * E + e] = 0;
+                }
+                tot[e] += s;
+                pc[e] = s;
+            }
+            if (threadIdx.x == 0) {
+                pc[E] = sbad[1];
+                sbad[0] += sbad[1];
+                sbad[1] = 0;
+            }
+            __syncthreads();
+        }
     }
 
     // Cluster reduction over distributed shared memory.
@@ -124,12 +193,28 @@ k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
         int s = 0;
 #pragma unroll
         for (int q = 0; q < kMaxCluster; ++q) s += part[q];
-        counts[(int64_t)r * E + e] = s;
+        if (counts != nullptr) counts[(int64_t)r * E + e] = s;
     }
     if (bad != nullptr && c == 0 && threadIdx.x == 0) {
         int s = 0;
         for (int q = 0; q < C; ++q) s += *cluster.map_shared_rank(sbad, q);
         bad[r] = s;
+    }
+    if constexpr (PIECES) {
+        // The prefix rows of this CTA's pieces: the earlier CTAs' totals
+        // (peers' shared memory), then the pieces in order; the CTA holding
+        // the rank's last piece also writes the totals row B.
+        const int b0 = c * ppc, nq = min(ppc, B - b0);
+        for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+            const int32_t *src = e < E ? tot + e : sbad;
+            int run = 0;
+            for (int q = 0; q < c; ++q) run += *cluster.map_shared_rank(src, q);
+            for (int q = 0; q < nq; ++q) {
+                rows[((int64_t)r * (B + 1) + b0 + q) * (E + 1) + e] = run;
+                run += pcnt[q * (E + 1) + e];
+            }
+            if (nq > 0 && b0 + nq == B) rows[((int64_t)r * (B + 1) + B) * (E + 1) + e] = run;
+        }
     }
     cluster_arrive_relaxed();   // done reading the peers; they may still read this CTA's totals
     cluster_wait();
@@ -137,18 +222,29 @@ k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
 
 }  // namespace
 
-size_t load_smem_bytes(const Shape &sh) { return (size_t)((kCopies + 1) * sh.E + 4) * sizeof(int32_t); }
+size_t load_smem_bytes(const Shape &sh, int ppc)
+{
+    return (size_t)((kCopies + 1) * sh.E + 4 + (size_t)ppc * (sh.E + 1)) * sizeof(int32_t);
+}
 
 cudaError_t launch_load(const Shape &sh, const Launch &ln, const int32_t *ids, int32_t *counts,
-                        int32_t *bad, cudaStream_t st)
+                        int32_t *bad, cudaStream_t st, const Pieces *pc, int32_t *rows)
 {
-    return launch_ex(k_load, (unsigned)(sh.N * ln.cluster), kLoadWarps * 32, load_smem_bytes(sh), st,
-                     (unsigned)ln.cluster, false, ids, sh.per_rank, sh.E, counts, bad);
+    if (pc != nullptr && pc->NP > 0) {
+        const int ppc = (pc->B + ln.cluster - 1) / ln.cluster;
+        return launch_ex(k_load<true>, (unsigned)(sh.N * ln.cluster), kLoadWarps * 32, load_smem_bytes(sh, ppc), st,
+                         (unsigned)ln.cluster, false, ids, sh.per_rank, sh.E, counts, bad, rows, pc->zp, pc->B);
+    }
+    return launch_ex(k_load<false>, (unsigned)(sh.N * ln.cluster), kLoadWarps * 32, load_smem_bytes(sh, 0), st,
+                     (unsigned)ln.cluster, false, ids, sh.per_rank, sh.E, counts, bad, (int32_t *)nullptr,
+                     (int64_t)0, 0);
 }
 
 cudaError_t set_load_attributes(size_t max_smem)
 {
-    return allow_smem(k_load, max_smem);
+    cudaError_t e = allow_smem(k_load<false>, max_smem);
+    if (e == cudaSuccess) e = allow_smem(k_load<true>, max_smem);
+    return e;
 }
 
 }  // namespace ue

@@ -73,10 +73,10 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
 k_sync_shard(PeerTable base, uint8_t *__restrict__ local, int64_t slot_bytes, int E, int S, int SG, int G, int g,
              int round, int cap, const int32_t *__restrict__ rep_off, const int32_t *__restrict__ rep_slot,
              const int32_t *__restrict__ rep_experts, const int32_t *__restrict__ info,
-             int32_t *__restrict__ dev_err)
+             int32_t *__restrict__ dev_err, unsigned long long wait_ns, int stall)
 {
     extern __shared__ __align__(128) uint8_t sm_sync[];
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm_sync);                 // [stages]
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm_sync);                 // [stages + 1]; the last one: see stall
     uint8_t *stage = sm_sync + 128;                                        // [stages][tile]
     const uint8_t **x_base = reinterpret_cast<const uint8_t **>(stage + (size_t)kSyncStages * kSyncTile);  // [G]
     int64_t *x_q = reinterpret_cast<int64_t *>(x_base + kMaxGpus);        // [E] part length
@@ -158,7 +158,7 @@ k_sync_shard(PeerTable base, uint8_t *__restrict__ local, int64_t slot_bytes, in
         x_ipre[m] = items;                           // turned into the exclusive prefix below
     }
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kSyncStages; ++i) mbar_init(&bar[i], 1);
+        for (int i = 0; i <= kSyncStages; ++i) mbar_init(&bar[i], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
@@ -222,19 +222,19 @@ k_sync_shard(PeerTable base, uint8_t *__restrict__ local, int64_t slot_bytes, in
         bulk_load(stage + (size_t)b * kSyncTile, it.src, it.bytes, &bar[b]);
     };
 
-    for (int64_t k = 0; k < nmy && k < kSyncStages; ++k) issue_load(k);
+    int64_t issued = 0;
+    for (; issued < nmy && issued < kSyncStages; ++issued) issue_load(issued);
+    // Diagnostic: CTA 0 waits once, with its first loads in flight, on the
+    // extra barrier, on which nothing ever arrives (see k_sync).
+    if (stall && blockIdx.x == 0 && !mbar_wait_bounded(&bar[kSyncStages], 0, wait_ns)) {
+        ring_give_up(dev_err, bar, kSyncStages, 0, issued, wait_ns);
+        return;
+    }
     for (int64_t k = 0; k < nmy; ++k) {
         const int b = (int)(k % kSyncStages);
-        const unsigned parity = (unsigned)((k / kSyncStages) & 1);
-        if (!mbar_try_wait(&bar[b], parity)) {
-            const unsigned long long t0 = global_ns();
-            while (!mbar_try_wait(&bar[b], parity)) {
-                if (global_ns() - t0 > kWaitLimitNs) {
-                    atomicOr(dev_err, 1);
-                    bulk_wait_all();
-                    return;
-                }
-            }
+        if (!mbar_wait_bounded(&bar[b], (unsigned)((k / kSyncStages) & 1), wait_ns)) {
+            ring_give_up(dev_err, bar, kSyncStages, k + 1, issued, wait_ns);
+            return;
         }
         const Item it = item(k);
         const uint8_t *src = stage + (size_t)b * kSyncTile;
@@ -245,6 +245,7 @@ k_sync_shard(PeerTable base, uint8_t *__restrict__ local, int64_t slot_bytes, in
         if (k >= 1 && k - 1 + kSyncStages < nmy) {
             bulk_wait_read_1();
             issue_load(k - 1 + kSyncStages);
+            ++issued;
         }
     }
     bulk_wait_all();
@@ -345,11 +346,11 @@ size_t grad_shard_smem_bytes(const Shape &sh)
 
 cudaError_t launch_sync_shard(const Shape &sh, const Launch &ln, const PeerTable &base, uint8_t *local, int G,
                               int g, int round, int64_t slot_bytes, const PlanDev &plan, int32_t *dev_err,
-                              cudaStream_t st)
+                              cudaStream_t st, const WaitBound &wb)
 {
     k_sync_shard<<<ln.sms, kSyncThreads, sync_shard_smem_bytes(sh), st>>>(
         base, local, slot_bytes, sh.E, sh.S, sh.S / G, G, g, round, sh.E + sh.NR, plan.rep_off, plan.rep_slot,
-        plan.rep_experts, plan.info, dev_err);
+        plan.rep_experts, plan.info, dev_err, wb.ns, wb.stall);
     return cudaGetLastError();
 }
 

@@ -13,8 +13,10 @@
 // so each home tile is read from HBM once and fanned out to all of its
 // replicas - the one-GPU form of the pages' relay against fan-out overload.
 // Stage reuse waits on cp.async.bulk.wait_group.read.  No multicast anywhere.
-// Every mbarrier wait is bounded by the global timer; on timeout the kernel
-// records an error in the context's status word, drains its stores and exits.
+// Every mbarrier wait is bounded by the global timer (the context's wait
+// limit); on timeout the kernel records an error in the context's status
+// word, waits (bounded again) for the loads it issued into the other stages,
+// drains its stores and exits.
 //
 // Incremental form: given the previous microbatch's slot_expert, a redundant
 // slot that already held its expert is not copied (the expert weights do not
@@ -37,10 +39,10 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
 k_sync(uint8_t *__restrict__ W, int64_t slot_bytes, int E, int S, int cap,
        const int32_t *__restrict__ rep_off, const int32_t *__restrict__ rep_slot,
        const int32_t *__restrict__ rep_experts, const int32_t *__restrict__ info,
-       const int32_t *__restrict__ prev, int32_t *__restrict__ dev_err)
+       const int32_t *__restrict__ prev, int32_t *__restrict__ dev_err, unsigned long long wait_ns, int stall)
 {
     extern __shared__ __align__(128) uint8_t sm_sync[];
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm_sync);                 // [stages]
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm_sync);                 // [stages + 1]; the last one: see stall
     uint8_t *stage = sm_sync + 128;                                        // [stages][tile]
     int32_t *x_home = reinterpret_cast<int32_t *>(stage + (size_t)kSyncStages * kSyncTile);  // [E]
     int32_t *x_first = x_home + E;                                         // [E] first redundant entry
@@ -65,7 +67,7 @@ k_sync(uint8_t *__restrict__ W, int64_t slot_bytes, int E, int S, int cap,
         x_cnt[m] = c;
     }
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kSyncStages; ++i) mbar_init(&bar[i], 1);
+        for (int i = 0; i <= kSyncStages; ++i) mbar_init(&bar[i], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
@@ -108,19 +110,20 @@ k_sync(uint8_t *__restrict__ W, int64_t slot_bytes, int E, int S, int cap,
         bulk_load(stage + (size_t)b * kSyncTile, it.src, it.bytes, &bar[b]);
     };
 
-    for (int64_t k = 0; k < nmy && k < kSyncStages; ++k) issue_load(k);
+    int64_t issued = 0;
+    for (; issued < nmy && issued < kSyncStages; ++issued) issue_load(issued);
+    // Diagnostic: CTA 0 waits once, with its first loads in flight, on the
+    // extra barrier, on which nothing ever arrives: the wait runs out and the
+    // kernel takes its way out (exercised by a test through the context).
+    if (stall && blockIdx.x == 0 && !mbar_wait_bounded(&bar[kSyncStages], 0, wait_ns)) {
+        ring_give_up(dev_err, bar, kSyncStages, 0, issued, wait_ns);
+        return;
+    }
     for (int64_t k = 0; k < nmy; ++k) {
         const int b = (int)(k % kSyncStages);
-        const unsigned parity = (unsigned)((k / kSyncStages) & 1);
-        if (!mbar_try_wait(&bar[b], parity)) {
-            const unsigned long long t0 = global_ns();
-            while (!mbar_try_wait(&bar[b], parity)) {
-                if (global_ns() - t0 > kWaitLimitNs) {
-                    atomicOr(dev_err, 1);
-                    bulk_wait_all();
-                    return;
-                }
-            }
+        if (!mbar_wait_bounded(&bar[b], (unsigned)((k / kSyncStages) & 1), wait_ns)) {
+            ring_give_up(dev_err, bar, kSyncStages, k + 1, issued, wait_ns);
+            return;
         }
         const SyncItem it = item(k);
         const uint8_t *src = stage + (size_t)b * kSyncTile;
@@ -132,6 +135,7 @@ k_sync(uint8_t *__restrict__ W, int64_t slot_bytes, int E, int S, int cap,
         if (k >= 1 && k - 1 + kSyncStages < nmy) {
             bulk_wait_read_1();
             issue_load(k - 1 + kSyncStages);
+            ++issued;
         }
     }
     bulk_wait_all();
@@ -145,11 +149,13 @@ size_t sync_smem_bytes(const Shape &sh)
 }
 
 cudaError_t launch_sync(const Shape &sh, const Launch &ln, uint8_t *weights, int64_t slot_bytes,
-                        const PlanDev &plan, const int32_t *prev_slot_expert, int32_t *dev_err, cudaStream_t st)
+                        const PlanDev &plan, const int32_t *prev_slot_expert, int32_t *dev_err, cudaStream_t st,
+                        const WaitBound &wb)
 {
     k_sync<<<ln.sms, kSyncThreads, sync_smem_bytes(sh), st>>>(weights, slot_bytes, sh.E, sh.S, sh.E + sh.NR,
                                                                plan.rep_off, plan.rep_slot, plan.rep_experts,
-                                                               plan.info, prev_slot_expert, dev_err);
+                                                               plan.info, prev_slot_expert, dev_err, wb.ns,
+                                                               wb.stall);
     return cudaGetLastError();
 }
 

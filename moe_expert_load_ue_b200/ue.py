@@ -19,13 +19,15 @@ LIB_PATH = os.path.join(_HERE, "libue.so")
 
 UE_OK, UE_ERR_INVALID_ARG, UE_ERR_CUDA, UE_ERR_UNSUPPORTED, UE_ERR_DEVICE = range(5)
 UE_PLAN_REQUEUE, UE_PLAN_SPREAD = 1, 2      # plan variant bits (include/ue.h)
+UE_WAIT_STALL_ONCE = 1                      # ue_ctx_set_wait_limit flag (include/ue.h)
 
 PLAN_FIELDS = ("slot_expert", "slot_quota", "rep_off", "rep_slot", "rep_cum", "rep_experts",
                "load", "rank_off", "rank_load_before", "rank_load_after", "info")
 
 # Entry points declared in include/ue.h (checked against the header by the tests).
-EXPORTS = ("ue_plan_sizes", "ue_ctx_create", "ue_ctx_destroy", "ue_ctx_device_error", "ue_load",
-           "ue_plan", "ue_plan_ex", "ue_reroute", "ue_rebalance", "ue_rebalance_ex", "ue_dispatch", "ue_rebalance_dispatch", "ue_sync", "ue_sync_delta",
+EXPORTS = ("ue_plan_sizes", "ue_ctx_create", "ue_ctx_destroy", "ue_ctx_device_error", "ue_ctx_set_wait_limit",
+           "ue_load",
+           "ue_plan", "ue_plan_ex", "ue_reroute", "ue_rebalance", "ue_rebalance_ex", "ue_dispatch", "ue_rebalance_dispatch", "ue_sync", "ue_sync_delta", "ue_sync_restore",
            "ue_grad_reduce", "ue_load_shard", "ue_reroute_shard", "ue_relay_rounds", "ue_sync_shard",
            "ue_grad_reduce_shard", "ue_status_string", "ue_last_error")
 
@@ -76,6 +78,7 @@ def lib() -> ctypes.CDLL:
                 "ue_ctx_create": [ci, ctypes.POINTER(vp)],
                 "ue_ctx_destroy": [vp],
                 "ue_ctx_device_error": [vp, ctypes.POINTER(ctypes.c_int32), vp],
+                "ue_ctx_set_wait_limit": [vp, ctypes.c_int64, ctypes.c_int32],
                 "ue_load": [vp, cfgp, vp, vp, vp, vp],
                 "ue_plan": [vp, cfgp, vp, planp, vp],
                 "ue_plan_ex": [vp, cfgp, vp, planp, ci, vp],
@@ -86,6 +89,7 @@ def lib() -> ctypes.CDLL:
                 "ue_rebalance_dispatch": [vp, cfgp, vp, vp, vp, planp, vp, dispp, vp],
                 "ue_sync": [vp, cfgp, vp, i64, planp, vp],
                 "ue_sync_delta": [vp, cfgp, vp, i64, planp, vp, vp],
+                "ue_sync_restore": [vp, cfgp, vp, i64, planp, vp, vp],
                 "ue_grad_reduce": [vp, cfgp, vp, vp, ci, i64, planp, vp],
                 "ue_load_shard": [vp, cfgp, shardp, vp, vp, vp, vp],
                 "ue_reroute_shard": [vp, cfgp, shardp, vp, planp, vp, vp],
@@ -201,6 +205,9 @@ class Context:
         except Exception:
             pass
 
+    def set_wait_limit(self, limit_ns: int, flags: int = 0) -> None:
+        _check(lib().ue_ctx_set_wait_limit(self._h, int(limit_ns), int(flags)), "ue_ctx_set_wait_limit")
+
     def device_error(self, stream=None) -> int:
         w = ctypes.c_int32(0)
         _check(lib().ue_ctx_device_error(self._h, ctypes.byref(w), _stream(stream)), "ue_ctx_device_error")
@@ -290,6 +297,12 @@ def ue_sync_delta(ctx: Context, cfg: Config, weights: torch.Tensor, slot_bytes: 
                   prev_slot_expert: torch.Tensor | None, stream=None) -> None:
     _check(lib().ue_sync_delta(ctx.handle, ctypes.byref(cfg.c()), _ptr(weights), int(slot_bytes), plan.ref(),
                                _ptr(prev_slot_expert), _stream(stream)), "ue_sync_delta")
+
+
+def ue_sync_restore(ctx: Context, cfg: Config, weights: torch.Tensor, slot_bytes: int, plan: Plan,
+                    held_slot_expert: torch.Tensor | None, stream=None) -> None:
+    _check(lib().ue_sync_restore(ctx.handle, ctypes.byref(cfg.c()), _ptr(weights), int(slot_bytes), plan.ref(),
+                                 _ptr(held_slot_expert), _stream(stream)), "ue_sync_restore")
 
 
 def ue_grad_reduce(ctx: Context, cfg: Config, master: torch.Tensor, grads: torch.Tensor, P: int,

@@ -283,3 +283,8 @@ def test_header_is_plain_c(tmp_path):
             args[args.index(str(src))] = "-xc++"
             args.insert(args.index("-xc++") + 1, str(src))
         subprocess.run(args, check=True, capture_output=True, text=True)
+
+
+def test_set_wait_limit_refuses_without_context(L):
+    assert L.ue_ctx_set_wait_limit(None, 2_000_000_000, 0) == ue.UE_ERR_INVALID_ARG
+    assert "context" in L.ue_last_error().decode()
