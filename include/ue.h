@@ -164,6 +164,28 @@ ue_status ue_plan_ex(ue_ctx *ctx, const ue_config *cfg, const int32_t *counts,
 ue_status ue_reroute(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids,
                      const ue_plan_buffers *plan, int32_t *phys, void *stream);
 
+/* Routing expansion without a context, for callers that cannot allocate
+ * device memory - an engine that reserves its whole device-memory budget in
+ * its own pool at start-up, or a caller in a region of its framework where
+ * allocation is not allowed - and so cannot create a ue_ctx (ue_ctx_create
+ * allocates).  The pages have no counterpart: it is an interface of this
+ * library.  Same arguments and the same phys as ue_reroute, on the current
+ * device; it always takes the reroute over pieces, with its scratch (piece
+ * counters and per-piece occurrence rows) in a 4 MiB device array that the
+ * library holds on every GPU that loads it until the process exits.  It calls
+ * no allocating routine.
+ *   - Limit: 2 * N * (E + 1) + 64 <= 2^20 ints (else UE_ERR_INVALID_ARG,
+ *     phys untouched), plus the limits above.
+ *   - The first call on a device sets that device up (looks up the array's
+ *     device address, sets the kernels' shared-memory limits); make that first
+ *     call before any stream capture.
+ *   - Every call shares the array and leaves its contents behind (each call
+ *     clears the counters it needs at 0 and overwrites the rows it reads):
+ *     calls that overlap on the GPU race - issue them on one stream, or order
+ *     the streams. */
+ue_status ue_reroute_static(const ue_config *cfg, const int32_t *ids, const ue_plan_buffers *plan,
+                            int32_t *phys, void *stream);
+
 /* Steps 1-3 back to back on one stream (three launches). */
 ue_status ue_rebalance(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids,
                        int32_t *counts, int32_t *bad, const ue_plan_buffers *plan,

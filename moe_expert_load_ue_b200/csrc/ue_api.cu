@@ -4,6 +4,7 @@
 #include <cstdio>
 #include <cstring>
 #include <algorithm>
+#include <mutex>
 #include <new>
 
 #include "ue_internal.cuh"
@@ -712,3 +713,119 @@ ue_status ue_grad_reduce_shard(ue_ctx *ctx, const ue_config *cfg, const ue_shard
 }
 
 }  // extern "C"
+
+// ---- routing expansion without a context ------------------------------------------
+//
+// Some callers cannot call cudaMalloc: an engine that reserves its whole
+// device-memory budget in its own pool at start-up (an allocation outside the
+// pool fails or breaks its accounting), or a caller inside a region of its
+// framework where allocation is not allowed.  Such a caller cannot create a
+// ue_ctx, which allocates its status word and workspace.  ue_reroute_static
+// runs the reroute over pieces (the load kernel's piece pass, then the
+// persistent reroute kernel) with its scratch - the piece counters and the rows
+// of occurrences before each piece - in g_scratch, a device array the library
+// holds on every GPU that loads it until the process exits.  The caller passes
+// ids, the plan and phys as for ue_reroute and gets the same phys.
+//
+// In host code g_scratch names a host-side stand-in for the device symbol:
+// the first call on each device, with that device current, asks the runtime
+// for its device address (cudaGetSymbolAddress) and sets the kernels'
+// shared-memory limits; later calls on that device reuse them.
+
+namespace {
+
+constexpr int64_t kStaticScratchInts = (int64_t)1 << 20;   // 4 MiB
+constexpr int64_t kStaticHead = 64;                          // the piece counters, then the rows
+constexpr int kStaticMaxDevices = 64;
+
+static __device__ __align__(256) int32_t g_scratch[kStaticScratchInts];
+
+struct StaticSetup {
+    bool ready;
+    int32_t *scratch;      // g_scratch's address on the device
+    ue_ctx props;          // device properties (sms, shared memory, resident CTAs); no allocations
+};
+StaticSetup g_static[kStaticMaxDevices];
+std::mutex g_static_lock;
+
+}  // namespace
+
+extern "C" ue_status ue_reroute_static(const ue_config *cfg, const int32_t *ids, const ue_plan_buffers *plan,
+                                       int32_t *phys, void *stream)
+{
+    ue::Shape sh{};
+    ue_status s = make_shape(cfg, true, &sh);
+    if (s == UE_OK) s = check_plan(plan);
+    if (s != UE_OK) return s;
+    if (sh.T > 0 && (!ids || !aligned16(ids))) return fail(UE_ERR_INVALID_ARG, "ids must be non-NULL and 16-byte aligned");
+    if (sh.T > 0 && !phys) return fail(UE_ERR_INVALID_ARG, "phys is NULL");
+    // At least two pieces' rows per rank must fit the static scratch.
+    const int64_t row_ints = (int64_t)sh.N * (sh.E + 1);
+    if (kStaticHead + 2 * row_ints > kStaticScratchInts)
+        return fail(UE_ERR_INVALID_ARG,
+                    "N * (E + 1) = %lld exceeds the static scratch (2 * N * (E + 1) + %lld <= %lld ints)",
+                    (long long)row_ints, (long long)kStaticHead, (long long)kStaticScratchInts);
+    if (sh.per_rank == 0) return UE_OK;
+
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kStaticMaxDevices) return fail(UE_ERR_UNSUPPORTED, "device %d beyond %d", dev, kStaticMaxDevices);
+    StaticSetup ds;
+    {
+        std::lock_guard<std::mutex> lock(g_static_lock);
+        StaticSetup &d = g_static[dev];
+        if (!d.ready) {
+            cudaDeviceProp prop;
+            if ((e = cudaGetDeviceProperties(&prop, dev)) != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+            if (prop.major != 10)
+                return fail(UE_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", dev,
+                            prop.major, prop.minor);
+            void *p = nullptr;
+            if ((e = cudaGetSymbolAddress(&p, g_scratch)) != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+            const size_t m = (size_t)prop.sharedMemPerBlockOptin;
+            if ((e = ue::set_load_attributes(m)) != cudaSuccess) return cuda_fail(e, "load attributes");
+            if ((e = ue::set_reroute_pieces_attributes(m)) != cudaSuccess) return cuda_fail(e, "reroute attributes");
+            d.scratch = static_cast<int32_t *>(p);
+            d.props = ue_ctx{};
+            d.props.device = dev;
+            d.props.sms = prop.multiProcessorCount;
+            d.props.max_smem = (int)m;
+            d.props.smem_per_sm = (int)prop.sharedMemPerMultiprocessor;
+            d.props.smem_reserved = (int)prop.reservedSharedMemPerBlock;
+            d.props.rp_blocks = ue::reroute_pieces_blocks_per_sm(0);
+            d.ready = true;
+        }
+        ds = d;
+    }
+
+    // Pieces as for the context's workspace, within the static scratch; this
+    // call takes the persistent reroute whatever the shape.
+    const ue_ctx &px = ds.props;
+    const ue::Launch ln = launch_of(&px, sh);
+    const size_t rp_smem = ue::reroute_pieces_smem_bytes(sh);
+    if (rp_smem > (size_t)px.max_smem) return fail(UE_ERR_INVALID_ARG, "E=%d too large for the reroute's tables", sh.E);
+    const int per_sm = std::min<int>(px.rp_blocks, px.smem_per_sm / (int)(rp_smem + px.smem_reserved));
+    ue::Pieces pc{};
+    pc.grid = px.sms * std::max(per_sm, 1);
+    const int64_t b_ws = (kStaticScratchInts - kStaticHead) / row_ints - 1;
+    const int64_t ppc_smem = ((int64_t)px.max_smem - (int64_t)ue::load_smem_bytes(sh, 0)) /
+                             ((int64_t)(sh.E + 1) * (int64_t)sizeof(int32_t));
+    int64_t B = ((int64_t)kPiecesPerCta * pc.grid + sh.N - 1) / sh.N;
+    B = std::max<int64_t>(1, std::min(B, std::min(b_ws, ppc_smem * ln.cluster)));
+    pc.zp = ((sh.per_rank + B - 1) / B + kPieceQuantum - 1) / kPieceQuantum * kPieceQuantum;
+    pc.B = (int)((sh.per_rank + pc.zp - 1) / pc.zp);
+    pc.NP = sh.N * pc.B;
+
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const ue::PlanDev pd = ue::to_dev(*plan);
+    // The piece counters must start at 0: the reroute kernel leaves them at 0,
+    // but a call that did not complete would not have.
+    if ((e = cudaMemsetAsync(ds.scratch, 0, 2 * sizeof(int32_t), st)) != cudaSuccess) return cuda_fail(e, "counters");
+    if ((e = ue::launch_load(sh, ln, ids, nullptr, nullptr, st, &pc, ds.scratch + kStaticHead)) != cudaSuccess)
+        return cuda_fail(e, "load launch");
+    if ((e = ue::launch_reroute_pieces(sh, pc, ids, pd, ds.scratch + kStaticHead, ds.scratch, phys, st, false)) !=
+        cudaSuccess)
+        return cuda_fail(e, "reroute launch");
+    return UE_OK;
+}

@@ -27,7 +27,7 @@ PLAN_FIELDS = ("slot_expert", "slot_quota", "rep_off", "rep_slot", "rep_cum", "r
 # Entry points declared in include/ue.h (checked against the header by the tests).
 EXPORTS = ("ue_plan_sizes", "ue_ctx_create", "ue_ctx_destroy", "ue_ctx_device_error", "ue_ctx_set_wait_limit",
            "ue_load",
-           "ue_plan", "ue_plan_ex", "ue_reroute", "ue_rebalance", "ue_rebalance_ex", "ue_dispatch", "ue_rebalance_dispatch", "ue_sync", "ue_sync_delta", "ue_sync_restore",
+           "ue_plan", "ue_plan_ex", "ue_reroute", "ue_reroute_static", "ue_rebalance", "ue_rebalance_ex", "ue_dispatch", "ue_rebalance_dispatch", "ue_sync", "ue_sync_delta", "ue_sync_restore",
            "ue_grad_reduce", "ue_load_shard", "ue_reroute_shard", "ue_relay_rounds", "ue_sync_shard",
            "ue_grad_reduce_shard", "ue_status_string", "ue_last_error")
 
@@ -83,6 +83,7 @@ def lib() -> ctypes.CDLL:
                 "ue_plan": [vp, cfgp, vp, planp, vp],
                 "ue_plan_ex": [vp, cfgp, vp, planp, ci, vp],
                 "ue_reroute": [vp, cfgp, vp, planp, vp, vp],
+                "ue_reroute_static": [cfgp, vp, planp, vp, vp],
                 "ue_rebalance": [vp, cfgp, vp, vp, vp, planp, vp, vp],
                 "ue_rebalance_ex": [vp, cfgp, vp, vp, vp, planp, vp, ci, vp],
                 "ue_dispatch": [vp, cfgp, vp, planp, vp, dispp, vp],
@@ -236,6 +237,12 @@ def ue_reroute(ctx: Context, cfg: Config, ids: torch.Tensor, plan: Plan, phys: t
                stream=None) -> None:
     _check(lib().ue_reroute(ctx.handle, ctypes.byref(cfg.c()), _ptr(ids), plan.ref(), _ptr(phys),
                             _stream(stream)), "ue_reroute")
+
+
+def ue_reroute_static(cfg: Config, ids: torch.Tensor, plan: Plan, phys: torch.Tensor, stream=None) -> None:
+    """ue_reroute without a context (no device allocation by the library), on the current device."""
+    _check(lib().ue_reroute_static(ctypes.byref(cfg.c()), _ptr(ids), plan.ref(), _ptr(phys), _stream(stream)),
+           "ue_reroute_static")
 
 
 def ue_rebalance(ctx: Context, cfg: Config, ids: torch.Tensor, counts: torch.Tensor,
