@@ -209,6 +209,27 @@ def measured_peaks() -> tuple[float, str]:
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def workload_of(args, rank):
+    """The bench's workload (rank r of a replicas run draws with base seed r)."""
+    w = inputs.WORKLOADS[args.workload].with_(base_seed=rank)
+    if args.stationary:
+        w = w.with_(repermute=False)
+    if args.expert_shape:
+        rows, cols = (int(x) for x in args.expert_shape.lower().split("x"))
+        w = w.with_(rows=rows, cols=cols)
+    return w
+
+
+def workload_config(w, n_mb, world):
+    """The JSON line's config (the same for both arms)."""
+    return {"workload": w.name, "E": w.E, "N": w.N, "H": w.H, "R": w.R, "K": w.K, "T": w.T,
+            "P": w.P, "slot_bytes": 2 * w.P, "grad_dtype": w.grad_dtype, "zipf_s": w.s,
+            "microbatches_cycled": n_mb, "parallelism": f"replicas x{world}",
+            "popularity": "re-drawn every microbatch" if w.repermute else "stationary",
+            "l2": "inputs larger than L2: every step streams > 1 GB (sync + grad reduce), "
+                  "so each rebalance reads its ids from HBM"}
+
+
 # ---- the GPU arm ------------------------------------------------------------------
 
 NVLINK_GBS = 770.0     # measured peer copy per direction per GPU on this pool's B200s (NVLink 5)
@@ -259,12 +280,7 @@ def run_ours(args, dist: Dist):
     torch.cuda.set_device(dist.local_rank)
     dev = torch.device("cuda", dist.local_rank)
     dist.init("nccl")
-    w = inputs.WORKLOADS[args.workload].with_(base_seed=dist.rank)
-    if args.stationary:
-        w = w.with_(repermute=False)
-    if args.expert_shape:
-        rows, cols = (int(x) for x in args.expert_shape.lower().split("x"))
-        w = w.with_(rows=rows, cols=cols)
+    w = workload_of(args, dist.rank)
     n_mb = args.microbatches or w.microbatches
     cfg = ue.Config(E=w.E, N=w.N, R=w.R, K=w.K, T=w.T)
     ctx = ue.Context(dist.local_rank)
@@ -496,6 +512,43 @@ def run_ours(args, dist: Dist):
                   "gbs": round(delta_bytes / (delta_us * 1e-6) / 1e9, 1) if delta_us > 0 else None}
     del plans2
 
+    # Weight restore in backward over a stack of layers sharing the redundant
+    # slots (the workload's microbatches stand for the layers): forward syncs
+    # the layers in order (incrementally), backward restores them last first,
+    # each from the experts the slots hold then; events around each restore.
+    layer_plans = [ue.Plan(cfg, device=dev) for _ in range(n_mb)]
+    held_np = np.full(w.S, -1, np.int32)
+    with torch.cuda.stream(stream):
+        for li in range(n_mb):
+            ue.ue_rebalance(ctx, cfg, ids_dev[li], counts, bad, layer_plans[li], phys, stream=stream)
+            ue.ue_sync_delta(ctx, cfg, weights, slot_bytes, layer_plans[li],
+                             layer_plans[li - 1]["slot_expert"] if li else None, stream=stream)
+            se = per_mb[li]["slot_expert"]
+            held_np = np.where(red & (se >= 0), se, held_np)
+    held_seq, restore_bytes = [], 0
+    for li in reversed(range(n_mb)):
+        se = per_mb[li]["slot_expert"]
+        held_seq.append(held_np.copy())
+        ch = red & (se >= 0) & (se != held_np)
+        restore_bytes += (len(np.unique(se[ch])) + int(ch.sum())) * slot_bytes
+        held_np = np.where(red & (se >= 0), se, held_np)
+    held_dev = torch.from_numpy(np.stack(held_seq)).to(dev)
+    evr = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_mb)]
+    with torch.cuda.stream(stream):
+        for k, li in enumerate(reversed(range(n_mb))):
+            evr[k][0].record(stream)
+            ue.ue_sync_restore(ctx, cfg, weights, slot_bytes, layer_plans[li], held_dev[k], stream=stream)
+            evr[k][1].record(stream)
+    stream.synchronize()
+    restore_us = float(sum(a.elapsed_time(b) for a, b in evr)) * 1e3
+    sync_delta["restore"] = {
+        "note": "backward of a stack of layers sharing the redundant slots (the microbatches' plans as layers): "
+                "ue_sync_restore, last layer first, from the experts the slots hold",
+        "layers": n_mb, "bytes": int(restore_bytes), "bytes_full_sync": int(delta_full),
+        "us_total": round(restore_us, 1),
+        "gbs": round(restore_bytes / (restore_us * 1e-6) / 1e9, 1) if restore_us > 0 and restore_bytes else None}
+    del layer_plans, held_dev
+
     # The calls across GPUs with G GPUs emulated as parts of this GPU's memory
     # (each GPU's slots, home-expert master rows and replica-gradient rows):
     # the relay rounds and the direct form of the weight sync, and the
@@ -585,34 +638,78 @@ def run_ours(args, dist: Dist):
     vals = dist.max([mean_reb, total_ms, float(seg[:, 1].mean()), float(seg[:, 2].mean())], device=dev)
     mean_reb_max, total_ms_max, sync_us_max, grad_us_max = vals
 
-    # End-to-end through the public API with host buffers: H2D ids, rebalance, D2H phys + plan.
+    # End-to-end through the public API with host buffers: every step copies
+    # its ids from pinned host memory, runs ue_rebalance and copies phys and
+    # every plan array back.  Pipelined over steps on three streams (H2D,
+    # compute, D2H) with two sets of buffers, so one step's D2H overlaps the
+    # next step's H2D; value = time per step from the first H2D to the last
+    # D2H.  latency_us: the same step alone, copies one after another.
     e2e = None
     if not args.no_e2e:
         ids_pinned = [torch.from_numpy(x).pin_memory() for x in ids_host]
-        ids_buf = torch.empty((w.T, w.K), dtype=torch.int32, device=dev)
-        phys_h = torch.empty((w.T, w.K), dtype=torch.int32).pin_memory()
-        plan_h = {k: torch.empty(v.shape, dtype=torch.int32).pin_memory() for k, v in plan.tensors.items()}
         n_e2e = max(8, min(args.steps, 64))
+        nb = 2
+        ids_b = [torch.empty((w.T, w.K), dtype=torch.int32, device=dev) for _ in range(nb)]
+        phys_b = [torch.empty((w.T, w.K), dtype=torch.int32, device=dev) for _ in range(nb)]
+        counts_b = [torch.empty((w.N, w.E), dtype=torch.int32, device=dev) for _ in range(nb)]
+        bad_b = [torch.empty(w.N, dtype=torch.int32, device=dev) for _ in range(nb)]
+        plan_b = [plan, ue.Plan(cfg, device=dev)]
+        phys_h = [torch.empty((w.T, w.K), dtype=torch.int32).pin_memory() for _ in range(nb)]
+        plan_h = [{k: torch.empty(v.shape, dtype=torch.int32).pin_memory() for k, v in plan.tensors.items()}
+                  for _ in range(nb)]
+        s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        in_done = [torch.cuda.Event() for _ in range(nb)]
+        cmp_done = [torch.cuda.Event() for _ in range(nb)]
+        out_done = [torch.cuda.Event() for _ in range(nb)]
+
+        def e2e_step(k):
+            b, mb = k % nb, k % n_mb
+            if k >= nb:
+                s_in.wait_event(out_done[b])            # buffer b's previous step fully copied out
+            with torch.cuda.stream(s_in):
+                ids_b[b].copy_(ids_pinned[mb], non_blocking=True)
+                in_done[b].record(s_in)
+            stream.wait_event(in_done[b])
+            ue.ue_rebalance(ctx, cfg, ids_b[b], counts_b[b], bad_b[b], plan_b[b], phys_b[b], stream=stream)
+            cmp_done[b].record(stream)
+            s_out.wait_event(cmp_done[b])
+            with torch.cuda.stream(s_out):
+                phys_h[b].copy_(phys_b[b], non_blocking=True)
+                for kk, t in plan_b[b].tensors.items():
+                    plan_h[b][kk].copy_(t, non_blocking=True)
+                out_done[b].record(s_out)
+
+        for k in range(args.warmup):
+            e2e_step(k)
+        torch.cuda.synchronize(dev)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(s_in)
+        for k in range(n_e2e):
+            e2e_step(args.warmup + k)
+        t1.record(s_out)
+        torch.cuda.synchronize(dev)
+        e2e_us = dist.max([t0.elapsed_time(t1) * 1e3 / n_e2e], device=dev)[0]
+        # one step alone: copies and rebalance one after another on one stream
         ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_e2e)]
         with torch.cuda.stream(stream):
-            for k in range(args.warmup + n_e2e):
+            for k in range(n_e2e):
                 mb = k % n_mb
-                e = ev2[k - args.warmup] if k >= args.warmup else None
-                if e:
-                    e[0].record(stream)
-                ids_buf.copy_(ids_pinned[mb], non_blocking=True)
-                ue.ue_rebalance(ctx, cfg, ids_buf, counts, bad, plan, phys, stream=stream)
-                phys_h.copy_(phys, non_blocking=True)
-                for kk, t in plan.tensors.items():
-                    plan_h[kk].copy_(t, non_blocking=True)
-                if e:
-                    e[1].record(stream)
-            stream.synchronize()
-        e2e_us = dist.max([statistics.mean(a.elapsed_time(b) * 1e3 for a, b in ev2)], device=dev)[0]
+                ev2[k][0].record(stream)
+                ids_b[0].copy_(ids_pinned[mb], non_blocking=True)
+                ue.ue_rebalance(ctx, cfg, ids_b[0], counts_b[0], bad_b[0], plan_b[0], phys_b[0], stream=stream)
+                phys_h[0].copy_(phys_b[0], non_blocking=True)
+                for kk, t in plan_b[0].tensors.items():
+                    plan_h[0][kk].copy_(t, non_blocking=True)
+                ev2[k][1].record(stream)
+        stream.synchronize()
+        lat_us = dist.max([statistics.mean(a.elapsed_time(b) * 1e3 for a, b in ev2)], device=dev)[0]
         h2d = w.T * w.K * 4
         d2h = w.T * w.K * 4 + plan.nbytes()
         e2e = {"value": round(e2e_us, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "path": "pinned host ids -> ue_rebalance -> pinned host phys + plan, one stream"}
+               "latency_us": round(lat_us, 2),
+               "path": "pinned host ids -> ue_rebalance -> pinned host phys + every plan array; steps pipelined "
+                       "on H2D / compute / D2H streams with two buffer sets (latency_us: one step alone)"}
+        del ids_b, phys_b, plan_b, counts_b, bad_b
 
     peak, peak_kind = measured_peaks()
     dom = "grad_reduce" if seg[:, 2].sum() >= seg[:, 1].sum() else "sync"
@@ -638,12 +735,7 @@ def run_ours(args, dist: Dist):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms_max / args.steps, 4),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "int32",
         "data": "synthetic: seeded Zipf-popularity Gumbel-top-k routing, random bf16 weights and replica grads",
-        "config": {"workload": w.name, "E": w.E, "N": w.N, "H": w.H, "R": w.R, "K": w.K, "T": w.T,
-                   "P": P, "slot_bytes": slot_bytes, "grad_dtype": w.grad_dtype, "zipf_s": w.s,
-                   "microbatches_cycled": n_mb, "parallelism": f"replicas x{dist.world}",
-                   "popularity": "re-drawn every microbatch" if w.repermute else "stationary",
-                   "l2": "inputs larger than L2: every step streams > 1 GB (sync + grad reduce), "
-                         "so each rebalance reads its ids from HBM"},
+        "config": workload_config(w, n_mb, dist.world),
         "breakdown_us": {
             "load": round(float(bd[:, 0].mean()), 2), "plan": round(float(bd[:, 1].mean()), 2),
             "reroute": round(float(bd[:, 2].mean()), 2),
@@ -742,7 +834,7 @@ def run_reference(args, dist: Dist):
     if dist.rank != 0:
         return None
     import oracle
-    w = inputs.WORKLOADS[args.workload]
+    w = workload_of(args, 0)
     n_mb = args.microbatches or w.microbatches
     ids_host = [inputs.topk_ids(w, mb) for mb in range(n_mb)]
     for k in range(args.warmup):
@@ -758,8 +850,7 @@ def run_reference(args, dist: Dist):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(statistics.mean(times) * 1e3, 3),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "int32",
         "data": "synthetic: seeded Zipf-popularity Gumbel-top-k routing",
-        "config": {"workload": w.name, "E": w.E, "N": w.N, "H": w.H, "R": w.R, "K": w.K, "T": w.T,
-                   "microbatches_cycled": n_mb},
+        "config": workload_config(w, n_mb, args.gpus),
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": f"each step one full microbatch (load+plan+reroute), {args.steps} steps"},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -778,6 +869,7 @@ def run_sweep(args, dist: Dist):
     ctx = ue.Context(dist.local_rank)
     stream = torch.cuda.Stream(device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    peak, _ = measured_peaks()
     for w in inputs.sweep(seeds=args.sweep_seeds):
         cfg = ue.Config(E=w.E, N=w.N, R=w.R, K=w.K, T=w.T)
         # Inputs drawn and buffers allocated on the stream the kernels run on,
@@ -821,12 +913,62 @@ def run_sweep(args, dist: Dist):
             variants[name] = {"imbalance_after": round(vi[6] / mean, 4),
                               "rebalance_us_median": round(statistics.median(a.elapsed_time(b) * 1e3 for a, b in vt),
                                                            2)}
+        med = statistics.median(us)
+        alg = 12 * w.L          # ids read by load and reroute, phys written
         print(json.dumps({"sweep_point": w.name, "tokens_per_rank": w.tokens_per_rank, "N": w.N, "zipf_s": w.s,
-                          "seed": w.base_seed, "T": w.T, "rebalance_us_median": round(statistics.median(us), 2),
+                          "seed": w.base_seed, "T": w.T, "rebalance_us_median": round(med, 2),
+                          "rebalance_alg_bytes": alg, "rebalance_gbs": round(alg / (med * 1e-6) / 1e9, 1),
+                          "rebalance_frac": round(alg / (med * 1e-6) / 1e9 / peak, 4),
                           "imbalance_before": round(info[5] / mean, 4), "imbalance_after": round(info[6] / mean, 4),
                           "slots_ran_out": bool(info[2] & 1), "replicated_experts": info[3],
                           "filled_redundant_slots": info[4], "plan_variants": variants}), flush=True)
         del ids, phys, plan, counts, bad
+        torch.cuda.synchronize(dev)
+    del flush
+    # Weight sync and gradient reduction per N at the sweep's expert shape
+    # (3 x 2048 x 1024 bf16 weights, fp32 gradients), on the plan of one
+    # microbatch of 4096 tokens per rank at Zipf 1.2; events around each call,
+    # 10 calls after 3 (every buffer is larger than L2).
+    for n in (8, 32, 64, 128, 256):
+        w = inputs.Workload(f"sweep-sync-n{n}", E=256, K=8, N=n, R=1, tokens_per_rank=4096, s=1.2,
+                            rows=2048, cols=1024, grad_dtype="fp32")
+        cfg = ue.Config(E=w.E, N=w.N, R=w.R, K=w.K, T=w.T)
+        P, slot_bytes = w.P, 2 * w.P
+        with torch.cuda.stream(stream):
+            ids = inputs.topk_ids_device(w, 0, dev)
+            counts = torch.empty((w.N, w.E), dtype=torch.int32, device=dev)
+            plan = ue.Plan(cfg, device=dev)
+            ue.ue_rebalance(ctx, cfg, ids, counts, None, plan, torch.empty_like(ids), stream=stream)
+            weights = torch.empty((w.S, P), dtype=torch.bfloat16, device=dev).normal_(0.0, 0.02)
+            master = torch.empty((w.E, P), dtype=torch.float32, device=dev).normal_(0.0, 1e-3)
+            grads = torch.empty((w.N * w.R, P), dtype=torch.float32, device=dev).normal_(0.0, 1e-3)
+        stream.synchronize()
+        info = plan["info"].cpu().tolist()
+        sync_b = (info[3] + info[4]) * slot_bytes
+        grad_b = info[3] * P * 8 + info[4] * P * 4
+        ts, tg = [], []
+        with torch.cuda.stream(stream):
+            for k in range(13):
+                a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+                a.record(stream)
+                ue.ue_sync(ctx, cfg, weights, slot_bytes, plan, stream=stream)
+                b.record(stream)
+                ue.ue_grad_reduce(ctx, cfg, master, grads, P, plan, stream=stream)
+                c.record(stream)
+                if k >= 3:
+                    ts.append((a, b))
+                    tg.append((b, c))
+        stream.synchronize()
+        su = statistics.median(a.elapsed_time(b) for a, b in ts) * 1e3
+        gu = statistics.median(a.elapsed_time(b) for a, b in tg) * 1e3
+        print(json.dumps({"sweep_sync_grad": w.name, "N": n, "slot_bytes": slot_bytes, "replicated_experts": info[3],
+                          "filled_redundant_slots": info[4], "sync_bytes": sync_b, "sync_us_median": round(su, 1),
+                          "sync_gbs": round(sync_b / (su * 1e-6) / 1e9, 1),
+                          "sync_frac": round(sync_b / (su * 1e-6) / 1e9 / peak, 4),
+                          "grad_reduce_bytes": grad_b, "grad_reduce_us_median": round(gu, 1),
+                          "grad_reduce_gbs": round(grad_b / (gu * 1e-6) / 1e9, 1),
+                          "grad_reduce_frac": round(grad_b / (gu * 1e-6) / 1e9 / peak, 4)}), flush=True)
+        del ids, counts, plan, weights, master, grads
         torch.cuda.synchronize(dev)
     ctx.close()
 

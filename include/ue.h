@@ -98,17 +98,19 @@ ue_status ue_ctx_destroy(ue_ctx *ctx);
  * ue_dispatch met ids that do not match the plan. */
 ue_status ue_ctx_device_error(ue_ctx *ctx, int32_t *host_word, void *stream);
 
-/* Bound of every wait inside the weight-sync kernels (ue_sync, ue_sync_delta,
- * ue_sync_shard): a copy that has not landed limit_ns nanoseconds (GPU global
- * timer) after the kernel began to wait for it makes the kernel give up - it
- * sets bit 0 of the status word, waits for its other copies in flight (each
- * wait again bounded by limit_ns) and returns; that call's slots are then
- * incomplete, and a copy that never lands leaves the device state undefined.
- * Default 2 s; limit_ns in [1000, 6e10].  Host only; affects later calls.
+/* Bound of every wait inside the kernels that stream through rings of bulk
+ * copies - weight sync (ue_sync, ue_sync_delta, ue_sync_restore,
+ * ue_sync_shard) and gradient reduction (ue_grad_reduce): a copy that has not
+ * landed (or a ring slot not released) limit_ns nanoseconds (GPU global timer)
+ * after the kernel began to wait for it makes the kernel give up - it sets bit
+ * 0 of the status word, waits for its other copies in flight (each wait again
+ * bounded by limit_ns) and returns; that call's outputs are then incomplete,
+ * and a copy that never lands leaves the device state undefined.  Default
+ * 2 s; limit_ns in [1000, 6e10].  Host only; affects later calls.
  *   flags  UE_WAIT_STALL_ONCE (diagnostic, for testing the way out): the next
- *          weight-sync call on this context makes its first CTA, once its
- *          first copies are in flight, wait once on a barrier that nothing
- *          completes, so that this wait runs out; the flag then clears. */
+ *          such call on this context makes one party of its first CTA wait
+ *          once on a barrier that nothing completes (after the first copies
+ *          are in flight), so that this wait runs out; the flag then clears. */
 #define UE_WAIT_STALL_ONCE 1
 ue_status ue_ctx_set_wait_limit(ue_ctx *ctx, int64_t limit_ns, int32_t flags);
 

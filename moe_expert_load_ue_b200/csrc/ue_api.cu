@@ -16,6 +16,7 @@ cudaError_t set_plan_attributes(size_t max_smem);
 cudaError_t set_sync_attributes(size_t max_smem);
 cudaError_t set_shard_attributes(size_t max_smem);
 cudaError_t set_reroute_pieces_attributes(size_t max_smem);
+cudaError_t set_grad_bulk_attributes(size_t max_smem);
 int grad_blocks_per_sm(int grad_dtype);
 int grad_shard_blocks_per_sm(int grad_dtype);
 }  // namespace ue
@@ -256,6 +257,7 @@ ue_status ue_ctx_create(int device, ue_ctx **out)
         tmp.grad_shard_blocks[0] = ue::grad_shard_blocks_per_sm(0);
         tmp.grad_shard_blocks[1] = ue::grad_shard_blocks_per_sm(1);
         if ((err = ue::set_reroute_pieces_attributes(m)) != cudaSuccess) return cuda_fail(err, "reroute attributes");
+        if ((err = ue::set_grad_bulk_attributes(m)) != cudaSuccess) return cuda_fail(err, "grad-reduce attributes");
         tmp.rp_blocks = ue::reroute_pieces_blocks_per_sm(0);
         if ((err = cudaMalloc(&tmp.dev_err, sizeof(int32_t))) != cudaSuccess) return cuda_fail(err, "cudaMalloc");
         if ((err = cudaMemset(tmp.dev_err, 0, sizeof(int32_t))) != cudaSuccess ||
@@ -555,10 +557,18 @@ ue_status ue_grad_reduce(ue_ctx *ctx, const ue_config *cfg, float *master, const
         return fail(UE_ERR_INVALID_ARG, "grads must be non-NULL and 16-byte aligned");
     if ((s = check_ctx(ctx)) != UE_OK) return s;
     return on_device(ctx, [&]() -> ue_status {
-        ue::Launch ln = launch_of(ctx, sh);
-        ln.sms = ctx->sms * ctx->grad_blocks[grad_dtype];
-        cudaError_t e = ue::launch_grad_reduce(sh, ln, master, grads, grad_dtype, P, ue::to_dev(*plan),
-                                               static_cast<cudaStream_t>(stream));
+        cudaError_t e;
+        if (ue::grad_bulk_smem_bytes(sh) <= (size_t)ctx->max_smem) {
+            const ue::WaitBound wb{(unsigned long long)ctx->wait_ns, ctx->stall_once};
+            e = ue::launch_grad_reduce_bulk(sh, ctx->sms, master, grads, grad_dtype, P, ue::to_dev(*plan),
+                                            ctx->dev_err, static_cast<cudaStream_t>(stream), wb);
+            ctx->stall_once = 0;
+        } else {
+            ue::Launch ln = launch_of(ctx, sh);
+            ln.sms = ctx->sms * ctx->grad_blocks[grad_dtype];
+            e = ue::launch_grad_reduce(sh, ln, master, grads, grad_dtype, P, ue::to_dev(*plan),
+                                       static_cast<cudaStream_t>(stream));
+        }
         return e == cudaSuccess ? UE_OK : cuda_fail(e, "grad-reduce launch");
     });
 }

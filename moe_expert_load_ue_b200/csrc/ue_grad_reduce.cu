@@ -77,7 +77,267 @@ k_grad_reduce(float *__restrict__ master, const void *__restrict__ grads, int64_
     }
 }
 
+// ---- the same reduction on the Tensor Memory Accelerator's bulk copies ----------
+//
+// One persistent CTA per SM.  A producer lane streams each item's row chunks
+// - the master chunk, then every replica's chunk in replica order - with
+// cp.async.bulk into a ring of shared-memory slots (completion on an mbarrier
+// per slot); eight consumer warps add them, in that order, into registers (the
+// same fp32 round-to-nearest adds as k_grad_reduce, so the result is the same
+// bits) and release each slot on its "empty" mbarrier; the sum goes back to
+// the master row with one bulk store per item from a double-buffered output
+// tile.  A slot holds a master chunk or kGbSlotBytes of replica chunks (one
+// fp32 chunk, two bf16 ones), so the ring holds the same bytes whatever the
+// gradient type.  Every wait is bounded by the global timer; on expiry the kernel
+// records bit 0 in the status word, the producer lets its loads in flight land,
+// and the CTA returns.
+constexpr int kGbConsumers = 256;                 // 8 consumer warps
+constexpr int kGbThreads = kGbConsumers + 32;     // + 1 producer warp
+constexpr int kGbChunk = 8192;                    // elements per item
+constexpr int kGbPer = kGbChunk / kGbConsumers;   // 32 elements per consumer thread
+constexpr int kGbWarpElems = kGbChunk / (kGbConsumers / 32);   // 1024 elements per consumer warp
+constexpr int kGbSlots = 4;
+constexpr int kGbSlotBytes = kGbChunk * 4;        // a master chunk (fp32); a replica chunk fits too
+__device__ __forceinline__ uint32_t gb_smem(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// Waits for the mbarrier phase, at most limit_ns on the global timer.
+__device__ __forceinline__ bool gb_wait(uint64_t *bar, unsigned parity, unsigned long long limit_ns)
+{
+    unsigned ok;
+    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(gb_smem(bar)), "r"(parity) : "memory");
+    if (ok) return true;
+    unsigned long long t0, t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    for (;;) {
+        asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}"
+                     : "=r"(ok) : "r"(gb_smem(bar)), "r"(parity) : "memory");
+        if (ok) return true;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        if (t - t0 > limit_ns) return false;
+    }
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kGbThreads, 1)
+k_grad_reduce_bulk(float *__restrict__ master, const void *__restrict__ grads, int64_t P, int E, int S, int H,
+                   int HR, int R, int cap, const int32_t *__restrict__ rep_off,
+                   const int32_t *__restrict__ rep_slot, const int32_t *__restrict__ rep_experts,
+                   const int32_t *__restrict__ info, int32_t *__restrict__ dev_err, unsigned long long wait_ns,
+                   int stall)
+{
+    extern __shared__ __align__(128) uint8_t sm_gb[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm_gb);           // [kGbSlots]
+    uint64_t *empty = full + kGbSlots;                                // [kGbSlots]
+    uint64_t *never = empty + kGbSlots;                               // diagnostic: nothing arrives on it
+    int32_t *abort_flag = reinterpret_cast<int32_t *>(never + 1);
+    uint8_t *slot = sm_gb + 1024;                                     // [kGbSlots][kGbSlotBytes]
+    float *outb = reinterpret_cast<float *>(slot + kGbSlots * kGbSlotBytes);   // [warps][2][kGbWarpElems]
+    int32_t *x_e = reinterpret_cast<int32_t *>(outb + 2 * kGbChunk);  // [E]
+    int32_t *x_first = x_e + E;                                       // [E]
+    int32_t *x_cnt = x_first + E;                                     // [E]
+    int32_t *x_row = x_cnt + E;                                       // [cap]
+
+    const int M = R > 0 ? clampi(__ldg(info + 3), 0, E) : 0;
+    for (int m = threadIdx.x; m < M; m += blockDim.x) {
+        const int e = clampi(__ldg(rep_experts + m), 0, E - 1);
+        const int off = clampi(__ldg(rep_off + e), 0, cap - 1);
+        const int end = clampi(__ldg(rep_off + e + 1), off + 1, cap);
+        x_e[m] = e;
+        x_first[m] = off + 1;
+        x_cnt[m] = end - off - 1;
+    }
+    for (int p = threadIdx.x; p < cap; p += blockDim.x) {
+        const int sl = clampi(__ldg(rep_slot + p), 0, S - 1);
+        const int u = sl % HR - H;
+        x_row[p] = u >= 0 ? (sl / HR) * R + u : 0;
+    }
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kGbSlots; ++i) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(gb_smem(&full[i])) : "memory");
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(gb_smem(&empty[i])), "r"(kGbConsumers / 32)
+                         : "memory");
+        }
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(gb_smem(never)) : "memory");
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    const int64_t nchunks = (P + kGbChunk - 1) / kGbChunk;
+    const int64_t total = (int64_t)M * nchunks;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int kElem = BF16 ? 2 : 4;
+    constexpr int kRepPerSlot = kGbSlotBytes / (kGbChunk * kElem);   // bf16: two replica chunks per slot
+
+    if (warp == kGbConsumers / 32) {
+        // Producer: one lane walks the segments (master, then replicas) of this
+        // CTA's items in order, one ring slot per segment.
+        if (lane != 0) return;
+        int64_t seg = 0;
+        for (int64_t it = blockIdx.x; it < total; it += gridDim.x) {
+            const int m = (int)(it / nchunks);
+            const int64_t x0 = (it - (int64_t)m * nchunks) * kGbChunk;
+            const int n = (int)min((int64_t)kGbChunk, P - x0);
+            const int cnt = x_cnt[m];
+            const int nseg = 1 + (cnt + kRepPerSlot - 1) / kRepPerSlot;
+            for (int j = 0; j < nseg; ++j, ++seg) {
+                const int b = (int)(seg % kGbSlots);
+                if (seg >= kGbSlots && !gb_wait(&empty[b], (unsigned)(((seg / kGbSlots) - 1) & 1), wait_ns)) {
+                    atomicOr(dev_err, 1);
+                    *reinterpret_cast<volatile int32_t *>(abort_flag) = 1;
+                    // Let the loads already issued into the other slots land.
+                    for (int64_t k = seg - kGbSlots + 1; k < seg; ++k)
+                        gb_wait(&full[k % kGbSlots], (unsigned)((k / kGbSlots) & 1), wait_ns);
+                    return;
+                }
+                // Segment 0: the master chunk; segment j >= 1: replicas
+                // (j - 1) * kRepPerSlot + 1 .. (at most kRepPerSlot, each in
+                // its kGbChunk * kElem bytes of the slot).
+                const int r0 = (j - 1) * kRepPerSlot + 1;
+                const int nr = j == 0 ? 1 : min(kRepPerSlot, cnt - r0 + 1);
+                const unsigned bytes = j == 0 ? (unsigned)n * 4u : (unsigned)n * (unsigned)kElem;
+                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(gb_smem(&full[b])),
+                             "r"(bytes * (unsigned)nr) : "memory");
+                for (int q = 0; q < nr; ++q) {
+                    const void *src = j == 0 ? static_cast<const void *>(master + (int64_t)x_e[m] * P + x0)
+                                             : static_cast<const void *>(
+                                                   static_cast<const uint8_t *>(grads) +
+                                                   ((int64_t)x_row[x_first[m] + r0 - 1 + q] * P + x0) * kElem);
+                    asm volatile(
+                        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                        ::"r"(gb_smem(slot + (size_t)b * kGbSlotBytes + (size_t)q * kGbChunk * kElem)), "l"(src),
+                        "r"(bytes), "r"(gb_smem(&full[b]))
+                        : "memory");
+                }
+            }
+        }
+        // Drain: the consumers wait for the last loads; the producer leaves.
+        return;
+    }
+
+    // Consumers: warp w owns the chunk's elements [w * kGbWarpElems, (w + 1) *
+    // kGbWarpElems), lane l the float4 groups i * 32 + l of them; each warp
+    // writes its part back from its own double-buffered output tile with its
+    // own bulk stores, so no consumer waits on another (only on the ring's
+    // mbarriers, each wait bounded).
+    // Diagnostic: consumer warp 0 of CTA 0 waits once on a barrier nothing
+    // completes; its wait runs out, it leaves, and the producer's wait for it
+    // runs out in turn (the way out exercised by a test through the context).
+    if (stall && blockIdx.x == 0 && warp == 0 && !gb_wait(never, 0, wait_ns)) {
+        if (lane == 0) atomicOr(dev_err, 1);
+        return;
+    }
+    int64_t seg = 0;
+    int ob = 0;
+    float *tile = outb + warp * (2 * kGbWarpElems);
+    for (int64_t it = blockIdx.x; it < total; it += gridDim.x, ob ^= 1) {
+        const int m = (int)(it / nchunks);
+        const int64_t x0 = (it - (int64_t)m * nchunks) * kGbChunk;
+        const int n = (int)min((int64_t)kGbChunk, P - x0);
+        const int cnt = x_cnt[m];
+        const int w0 = warp * kGbWarpElems;                  // this warp's first element of the chunk
+        const int nseg = 1 + (cnt + kRepPerSlot - 1) / kRepPerSlot;
+        float acc[kGbPer];
+        bool ok = true;
+        for (int j = 0; j < nseg; ++j, ++seg) {
+            const int b = (int)(seg % kGbSlots);
+            if (!gb_wait(&full[b], (unsigned)((seg / kGbSlots) & 1), wait_ns)) {
+                ok = false;
+                break;
+            }
+            const uint8_t *src = slot + (size_t)b * kGbSlotBytes;
+            const int nr = j == 0 ? 1 : min(kRepPerSlot, cnt - (j - 1) * kRepPerSlot);
+            for (int q = 0; q < nr; ++q) {                     // replicas in order
+                const uint8_t *sq = src + (size_t)q * kGbChunk * kElem;
+#pragma unroll
+                for (int i = 0; i < kGbPer / 4; ++i) {
+                    const int x = w0 + 4 * (i * 32 + lane);
+                    if (x >= n) continue;
+                    float v[4];
+                    if (j == 0 || !BF16) {
+                        const float4 f = *reinterpret_cast<const float4 *>(sq + (size_t)x * 4);
+                        v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+                    } else {
+                        const uint2 u = *reinterpret_cast<const uint2 *>(sq + (size_t)x * 2);
+                        v[0] = __uint_as_float(u.x << 16);
+                        v[1] = __uint_as_float(u.x & 0xffff0000u);
+                        v[2] = __uint_as_float(u.y << 16);
+                        v[3] = __uint_as_float(u.y & 0xffff0000u);
+                    }
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) acc[4 * i + k] = j == 0 ? v[k] : __fadd_rn(acc[4 * i + k], v[k]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0)
+                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(gb_smem(&empty[b])) : "memory");
+        }
+        if (!ok || *reinterpret_cast<volatile int32_t *>(abort_flag)) {
+            if (lane == 0) {
+                atomicOr(dev_err, 1);
+                asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+            }
+            return;
+        }
+        const int wn = min(kGbWarpElems, n - w0);            // elements of this warp's part (may be <= 0)
+        if (wn <= 0) continue;
+        // This warp's output tile is free once its store of two items ago has read it.
+        float *out = tile + ob * kGbWarpElems;
+        if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < kGbPer / 4; ++i) {
+            const int x = 4 * (i * 32 + lane);
+            if (x < wn) *reinterpret_cast<float4 *>(out + x) = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2],
+                                                                         acc[4 * i + 3]);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+            asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(master +
+                                                                                        (int64_t)x_e[m] * P + x0 + w0),
+                         "r"(gb_smem(out)), "r"((unsigned)wn * 4u)
+                         : "memory");
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        }
+    }
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 }  // namespace
+
+size_t grad_bulk_smem_bytes(const Shape &sh)
+{
+    return 1024 + (size_t)kGbSlots * kGbSlotBytes + 2 * (size_t)kGbChunk * 4 +
+           (size_t)(3 * sh.E + sh.E + sh.NR) * sizeof(int32_t);
+}
+
+cudaError_t launch_grad_reduce_bulk(const Shape &sh, int sms, float *master, const void *grads, int grad_dtype,
+                                    int64_t P, const PlanDev &plan, int32_t *dev_err, cudaStream_t st,
+                                    const WaitBound &wb)
+{
+    const size_t smem = grad_bulk_smem_bytes(sh);
+    const int cap = sh.E + sh.NR;
+    if (grad_dtype == 1)
+        k_grad_reduce_bulk<true><<<sms, kGbThreads, smem, st>>>(master, grads, P, sh.E, sh.S, sh.H, sh.HR, sh.R, cap,
+                                                                plan.rep_off, plan.rep_slot, plan.rep_experts,
+                                                                plan.info, dev_err, wb.ns, wb.stall);
+    else
+        k_grad_reduce_bulk<false><<<sms, kGbThreads, smem, st>>>(master, grads, P, sh.E, sh.S, sh.H, sh.HR, sh.R, cap,
+                                                                 plan.rep_off, plan.rep_slot, plan.rep_experts,
+                                                                 plan.info, dev_err, wb.ns, wb.stall);
+    return cudaGetLastError();
+}
+
+cudaError_t set_grad_bulk_attributes(size_t max_smem)
+{
+    cudaError_t e = allow_smem(k_grad_reduce_bulk<true>, max_smem);
+    if (e == cudaSuccess) e = allow_smem(k_grad_reduce_bulk<false>, max_smem);
+    return e;
+}
 
 int grad_blocks_per_sm(int grad_dtype)
 {

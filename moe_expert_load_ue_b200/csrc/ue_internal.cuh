@@ -106,6 +106,12 @@ struct WaitBound {
     int stall;
 };
 
+// The gradient reduction streamed through a ring of bulk copies (one CTA per
+// SM, sms CTAs); dev_err: bit 0 when a bounded wait gives up.
+cudaError_t launch_grad_reduce_bulk(const Shape &sh, int sms, float *master, const void *grads, int grad_dtype,
+                                    int64_t P, const PlanDev &plan, int32_t *dev_err, cudaStream_t st,
+                                    const WaitBound &wb);
+
 // prev_slot_expert: the previous plan's slot_expert for the incremental form, or nullptr.
 cudaError_t launch_sync(const Shape &sh, const Launch &ln, uint8_t *weights, int64_t slot_bytes,
                         const PlanDev &plan, const int32_t *prev_slot_expert, int32_t *dev_err, cudaStream_t st,
@@ -115,6 +121,7 @@ size_t sync_smem_bytes(const Shape &sh);
 cudaError_t launch_grad_reduce(const Shape &sh, const Launch &ln, float *master, const void *grads,
                                int grad_dtype, int64_t P, const PlanDev &plan, cudaStream_t st);
 size_t grad_smem_bytes(const Shape &sh);
+size_t grad_bulk_smem_bytes(const Shape &sh);
 
 // Calls across G GPUs (GPU g holds ranks [g*N/G, (g+1)*N/G)).  round >= 0 is
 // a relay round (0: scatter of the parts from the home slot, 1: all-gather

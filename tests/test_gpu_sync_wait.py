@@ -1,7 +1,7 @@
-"""The weight-sync kernels' bounded waits: the way out when a wait runs out.
+"""Bounded waits of the bulk-copy rings: the way out when a wait runs out.
 
-Every mbarrier wait of the weight-sync kernels is bounded by the context's
-wait limit.  The diagnostic flag UE_WAIT_STALL_ONCE makes the first CTA of the
+Every mbarrier wait of the weight-sync kernels and of the gradient reduction
+is bounded by the context's wait limit.  The diagnostic flag UE_WAIT_STALL_ONCE makes the first CTA of the
 next sync wait once, with its first copies in flight, on a barrier that nothing
 completes, so that the wait runs out without any fault: the kernel must set bit
 0 of the status word, let its copies in flight land, drain its stores and
@@ -93,3 +93,27 @@ def test_wait_runs_out_then_context_is_usable(ctx, call):
     assert ctx.device_error() == 0
     oracle.sync(expect, slot_bytes, w.E, w.N, w.R, pl["slot_expert"])
     assert np.array_equal(W.cpu().numpy(), expect)
+
+
+def test_grad_reduce_wait_runs_out_then_context_is_usable(ctx):
+    w = inputs.CLASS_671B.with_(tokens_per_rank=256, rows=512, cols=512)
+    cfg, plan, pl = _plan(ctx, w, 2)
+    P = w.P
+    g = torch.Generator(device="cuda").manual_seed(4)
+    master = torch.randn((w.E, P), generator=g, device="cuda")
+    grads = torch.randn((w.N * w.R, P), generator=g, device="cuda").to(torch.bfloat16)
+    ctx.set_wait_limit(LIMIT_NS, ue.UE_WAIT_STALL_ONCE)
+    try:
+        ue.ue_grad_reduce(ctx, cfg, master, grads, P, plan)
+        torch.cuda.synchronize()
+        assert ctx.device_error() & 1, "the stalled wait must report that it gave up"
+    finally:
+        ctx.set_wait_limit(2_000_000_000, 0)
+    master = torch.randn((w.E, P), generator=g, device="cuda")
+    m0 = master.cpu().numpy()
+    ue.ue_grad_reduce(ctx, cfg, master, grads, P, plan)
+    torch.cuda.synchronize()
+    assert ctx.device_error() == 0
+    expect = m0.copy()
+    oracle.grad_reduce(expect, grads.view(torch.int16).cpu().numpy().view(np.uint16), P, w.E, w.N, w.R, pl)
+    assert np.array_equal(master.cpu().numpy(), expect)
