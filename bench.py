@@ -47,13 +47,13 @@ VARIANTS = {"requeue": 1, "spread": 2, "requeue+spread": 3}     # plan variant b
 TRAFFIC = {
     ("grad_reduce", "671B-class"): {
         "sources": ["moe_expert_load_ue_b200/csrc/ue_grad_reduce.cu", "moe_expert_load_ue_b200/csrc/ue_grad.cuh"],
-        "sha256": "c1f443d9b89c58c94a8a2c0f2cfc98dc4a9e957d73ae8be1947f66c895057371",
-        "dram_bytes": 7905483008, "algorithmic_bytes": 7927234560,
+        "sha256": "d86dcac79562c699e8c013a7a24c6fb21e368f71ea703a786ab2d3bbb8125a04",
+        "dram_bytes": 7903631616, "algorithmic_bytes": 7927234560,
         "profile": "profiles/grad_reduce_and_sync_dram_671B-class.md"},
     ("sync", "671B-class"): {
         "sources": ["moe_expert_load_ue_b200/csrc/ue_sync.cu", "moe_expert_load_ue_b200/csrc/ue_bulk.cuh"],
-        "sha256": "191ad325243d74d5e0543fed305057763301e296b4f5889e597257146ad53a9b",
-        "dram_bytes": 4961509632, "algorithmic_bytes": 5020581888,
+        "sha256": "54818e6ae81cee9dea4303af048a3fa945b6e7fc8a5e9eb0ea3c06330eda349d",
+        "dram_bytes": 4962855680, "algorithmic_bytes": 5020581888,
         "profile": "profiles/grad_reduce_and_sync_dram_671B-class.md"},
 }
 
@@ -89,6 +89,8 @@ def parse_args(argv=None):
     ap.add_argument("--sweep", action="store_true",
                     help="rebalance latency and imbalance over the sweep grid (one JSON line per point)")
     ap.add_argument("--sweep-seeds", type=int, default=1)
+    ap.add_argument("--sweep-only", default=None,
+                    help="run only the sweep points TPR:N:S (comma-separated list), without the sync/grad lines")
     ap.add_argument("--stationary", action="store_true",
                     help="keep the expert popularity fixed across microbatches (no re-permutation)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -870,7 +872,12 @@ def run_sweep(args, dist: Dist):
     stream = torch.cuda.Stream(device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     peak, _ = measured_peaks()
+    only = None
+    if args.sweep_only:
+        only = {(int(a), int(b), float(c)) for a, b, c in (x.split(":") for x in args.sweep_only.split(","))}
     for w in inputs.sweep(seeds=args.sweep_seeds):
+        if only is not None and (w.tokens_per_rank, w.N, w.s) not in only:
+            continue
         cfg = ue.Config(E=w.E, N=w.N, R=w.R, K=w.K, T=w.T)
         # Inputs drawn and buffers allocated on the stream the kernels run on,
         # and the device drained before timing: no cross-stream reuse of memory.
@@ -925,6 +932,9 @@ def run_sweep(args, dist: Dist):
         del ids, phys, plan, counts, bad
         torch.cuda.synchronize(dev)
     del flush
+    if only is not None:
+        ctx.close()
+        return
     # Weight sync and gradient reduction per N at the sweep's expert shape
     # (3 x 2048 x 1024 bf16 weights, fp32 gradients), on the plan of one
     # microbatch of 4096 tokens per rank at Zipf 1.2; events around each call,
