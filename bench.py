@@ -95,6 +95,8 @@ def parse_args(argv=None):
                     help="keep the expert popularity fixed across microbatches (no re-permutation)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-across-gpus", action="store_true",
+                    help="with N > 1, skip the sharded calls across the GPUs after the timed region")
     return ap.parse_args(argv)
 
 
@@ -622,6 +624,16 @@ def run_ours(args, dist: Dist):
         },
     }
 
+    # Across real GPUs (torchrun, N > 1): each rank holds one shard of the
+    # resident buffers (its ranks' tokens, slots, home master rows and
+    # replica-gradient rows: views, no new memory), maps the other GPUs' through
+    # CUDA IPC, and runs the sharded calls with NCCL barriers between them;
+    # untimed by the headline, events around each call, max over ranks.
+    across_real = None
+    if dist.world > 1 and not args.no_across_gpus:
+        across_real = across_gpus_real(args, dist, ctx, cfg, w, ids_dev, weights, master, grads, gdt, per_mb,
+                                       slot_bytes, red, n_mb)
+
     # Launch floor: one tiny kernel bracketed by events on the same stream.
     tiny = torch.zeros(1, device=dev)
     floor = []
@@ -763,6 +775,7 @@ def run_ours(args, dist: Dist):
         "frac_of_8000_gbs": {"sync": round(sync_gbs / 8000, 4), "grad_reduce": round(grad_gbs / 8000, 4)},
         "sync_delta": sync_delta,
         "across_gpus_emulated": across_gpus,
+        "across_gpus": across_real,
         "plan_variants": plan_variants,
         "imbalance": {
             "before": round(float(np.mean([p["max_before"] / (p["L"] / w.N) for p in per_mb])), 4),
@@ -784,6 +797,74 @@ def run_ours(args, dist: Dist):
     dist.barrier()
     dist.close()
     return result
+
+
+def across_gpus_real(args, dist, ctx, cfg, w, ids_dev, weights, master, grads, gdt, per_mb, slot_bytes, red, n_mb):
+    """The sharded load/plan/reroute, weight sync (relay rounds and direct form)
+    and home-GPU gradient reduction on the job's GPUs, each rank one GPU."""
+    import torch
+
+    from moe_expert_load_ue_b200 import ue
+    from moe_expert_load_ue_b200.peer import PeerBuffers
+    from moe_expert_load_ue_b200.shard import DeviceOps, ShardedBalancer
+    G, g = dist.world, dist.rank
+    if w.N % G:
+        return {"skipped": f"N={w.N} is not a multiple of {G} GPUs"}
+    try:
+        SG, EG, RG, TG = w.S // G, w.E // G, (w.N // G) * w.R, w.T // G
+        dev = weights.device
+        bal = ShardedBalancer(cfg, DeviceOps(ctx, cfg, G, g), G=G, g=g, device=dev)
+        pw = PeerBuffers(weights[g * SG:(g + 1) * SG])
+        pg = PeerBuffers(grads[g * RG:(g + 1) * RG])
+        counts = torch.empty((w.N, w.E), dtype=torch.int32, device=dev)
+        plan = ue.Plan(cfg, device=dev)
+        phys_l = torch.empty((TG, w.K), dtype=torch.int32, device=dev)
+        n_sh = min(n_mb, 4)
+        st = torch.cuda.current_stream(dev)
+        evs = []
+        for k in range(-1, n_sh):                    # one untimed pass first
+            mb = max(k, 0)
+            bal.rebalance(ids_dev[mb][g * TG:(g + 1) * TG], counts, None, plan, phys_l)
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            e[0].record(st)
+            bal.sync(pw.ptrs, slot_bytes, plan, relay=True)
+            e[1].record(st)
+            bal.sync(pw.ptrs, slot_bytes, plan, relay=False)
+            e[2].record(st)
+            bal.grad_reduce(master[g * EG:(g + 1) * EG], pg.ptrs, gdt, w.P, plan)
+            e[3].record(st)
+            if k >= 0:
+                evs.append(e)
+        torch.cuda.synchronize(dev)
+        t = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(3)] for e in evs]) * 1e3
+        tmax = dist.max(list(t.sum(axis=0)), device=dev)
+        bal.barrier()
+        torch.cuda.synchronize(dev)
+        pw.close()
+        pg.close()
+        sync_b = cross_b = grad_b = 0
+        gsize = 2 if w.grad_dtype == "bf16" else 4
+        for mb in range(n_sh):
+            se = per_mb[mb]["slot_expert"]
+            for e_ in np.unique(se[red & (se >= 0)]):
+                gpus = set((np.nonzero(red & (se == e_))[0] // SG).tolist())
+                hg = ((e_ // w.H) * (w.H + w.R)) // SG
+                sync_b += len(gpus) * slot_bytes
+                cross_b += len(gpus - {hg}) * slot_bytes
+            sync_b += int((red & (se >= 0)).sum()) * slot_bytes
+            grad_b += per_mb[mb]["M"] * w.P * 8 + per_mb[mb]["filled"] * w.P * gsize
+        return {"G": G, "microbatches": n_sh, "relay_rounds": ue.ue_relay_rounds(G),
+                "sync_alg_bytes_mean": int(sync_b / n_sh), "nvlink_bytes_mean": int(cross_b / n_sh),
+                "sync_relay_us": round(tmax[0] / n_sh, 1), "sync_direct_us": round(tmax[1] / n_sh, 1),
+                "grad_reduce_us": round(tmax[2] / n_sh, 1),
+                "sync_relay_gbs": round(sync_b / (tmax[0] * 1e-6) / 1e9, 1),
+                "sync_direct_gbs": round(sync_b / (tmax[1] * 1e-6) / 1e9, 1),
+                "grad_reduce_gbs": round(grad_b / (tmax[2] * 1e-6) / 1e9, 1),
+                "nvlink_gbs_relay": round(cross_b / (tmax[0] * 1e-6) / 1e9, 1),
+                "note": "each rank one GPU holding its shard; peer tables by CUDA IPC; NCCL barriers between "
+                        "relay rounds; GB/s = all GPUs' algorithmic sync / grad bytes / the slowest rank's time"}
+    except Exception as exc:      # reported in the line; the replicas' numbers stand
+        return {"error": repr(exc)[:300]}
 
 
 # ---- the CPU oracle, timed on the host cores ------------------------------------

@@ -20,7 +20,11 @@ this module issues them in order around the library's sharded calls:
 The device steps go through `ops` (`DeviceOps`: the C ABI on this GPU); the
 exchanges through the process group.  With the NCCL backend a barrier is an
 all-reduce of one element on the current stream, so the kernels after it on
-that stream start only once every GPU has reached it.
+that stream start only once every GPU has reached it.  With a host-side group
+(gloo; `host_staged=True`) each barrier first waits for this process's stream,
+then meets the others on the host, and the counts rows travel through host
+memory.  The peer tables of the sync and gradient calls come from
+`peer.PeerBuffers` (CUDA IPC).
 """
 from __future__ import annotations
 
@@ -57,8 +61,8 @@ class ShardedBalancer:
     and rank unless given)."""
 
     def __init__(self, cfg: ue.Config, ops, G: int | None = None, g: int | None = None, group=None,
-                 device: str | torch.device = "cuda"):
-        self.cfg, self.ops, self.group = cfg, ops, group
+                 device: str | torch.device = "cuda", host_staged: bool = False):
+        self.cfg, self.ops, self.group, self.host_staged = cfg, ops, group, host_staged
         self.G = G if G is not None else (dist.get_world_size(group) if dist.is_initialized() else 1)
         self.g = g if g is not None else (dist.get_rank(group) if dist.is_initialized() else 0)
         if cfg.N % self.G != 0:
@@ -72,7 +76,12 @@ class ShardedBalancer:
 
     def barrier(self) -> None:
         if self.G > 1:
-            dist.all_reduce(self._token, group=self.group)
+            if self.host_staged:
+                if self._token.is_cuda:
+                    torch.cuda.current_stream(self._token.device).synchronize()
+                dist.barrier(group=self.group)
+            else:
+                dist.all_reduce(self._token, group=self.group)
 
     def rebalance(self, ids_local, counts, bad, plan, phys_local) -> None:
         """Load computation for this GPU's ranks, all-gather of the counts
@@ -81,9 +90,15 @@ class ShardedBalancer:
         self.ops.load(ids_local, counts, bad)
         if self.G > 1:
             lo, hi = self.g * self.NG, (self.g + 1) * self.NG
-            dist.all_gather_into_tensor(counts, counts[lo:hi].clone(), group=self.group)
-            if bad is not None:
-                dist.all_gather_into_tensor(bad, bad[lo:hi].clone(), group=self.group)
+            for t in (counts, bad):
+                if t is None:
+                    continue
+                if self.host_staged:
+                    full = torch.empty(t.shape, dtype=t.dtype)
+                    dist.all_gather_into_tensor(full, t[lo:hi].cpu(), group=self.group)
+                    t.copy_(full)
+                else:
+                    dist.all_gather_into_tensor(t, t[lo:hi].clone(), group=self.group)
         self.ops.plan(counts, plan)
         self.ops.reroute(ids_local, plan, phys_local)
 
