@@ -17,16 +17,12 @@ cudaError_t set_sync_attributes(size_t max_smem);
 cudaError_t set_shard_attributes(size_t max_smem);
 cudaError_t set_reroute_pieces_attributes(size_t max_smem);
 cudaError_t set_grad_bulk_attributes(size_t max_smem);
-int grad_blocks_per_sm(int grad_dtype);
-int grad_shard_blocks_per_sm(int grad_dtype);
 }  // namespace ue
 
 struct ue_ctx {
     int device;
     int sms;
     int max_smem;          // opt-in dynamic shared memory per block
-    int grad_blocks[2];    // resident grad-reduce CTAs per SM (fp32, bf16)
-    int grad_shard_blocks[2];  // the same for the gradient reduction across GPUs
     int32_t *dev_err;      // device status word for bounded waits
     int32_t *ws;           // workspace: piece histogram rows of the persistent reroute
     int rp_blocks;         // resident persistent-reroute CTAs per SM as registers allow
@@ -251,11 +247,7 @@ ue_status ue_ctx_create(int device, ue_ctx **out)
         if ((err = ue::set_reroute_attributes(m)) != cudaSuccess) return cuda_fail(err, "reroute attributes");
         if ((err = ue::set_plan_attributes(m)) != cudaSuccess) return cuda_fail(err, "plan attributes");
         if ((err = ue::set_sync_attributes(m)) != cudaSuccess) return cuda_fail(err, "sync attributes");
-        tmp.grad_blocks[0] = ue::grad_blocks_per_sm(0);
-        tmp.grad_blocks[1] = ue::grad_blocks_per_sm(1);
         if ((err = ue::set_shard_attributes(m)) != cudaSuccess) return cuda_fail(err, "shard attributes");
-        tmp.grad_shard_blocks[0] = ue::grad_shard_blocks_per_sm(0);
-        tmp.grad_shard_blocks[1] = ue::grad_shard_blocks_per_sm(1);
         if ((err = ue::set_reroute_pieces_attributes(m)) != cudaSuccess) return cuda_fail(err, "reroute attributes");
         if ((err = ue::set_grad_bulk_attributes(m)) != cudaSuccess) return cuda_fail(err, "grad-reduce attributes");
         tmp.rp_blocks = ue::reroute_pieces_blocks_per_sm(0);
@@ -564,8 +556,7 @@ ue_status ue_grad_reduce(ue_ctx *ctx, const ue_config *cfg, float *master, const
                                             ctx->dev_err, static_cast<cudaStream_t>(stream), wb);
             ctx->stall_once = 0;
         } else {
-            ue::Launch ln = launch_of(ctx, sh);
-            ln.sms = ctx->sms * ctx->grad_blocks[grad_dtype];
+            const ue::Launch ln = launch_of(ctx, sh);
             e = ue::launch_grad_reduce(sh, ln, master, grads, grad_dtype, P, ue::to_dev(*plan),
                                        static_cast<cudaStream_t>(stream));
         }
@@ -714,8 +705,7 @@ ue_status ue_grad_reduce_shard(ue_ctx *ctx, const ue_config *cfg, const ue_shard
     }
     if ((s = check_ctx(ctx)) != UE_OK) return s;
     return on_device(ctx, [&]() -> ue_status {
-        ue::Launch ln = launch_of(ctx, sh);
-        ln.sms = ctx->sms * ctx->grad_shard_blocks[grad_dtype];
+        const ue::Launch ln = launch_of(ctx, sh);
         cudaError_t e = ue::launch_grad_reduce_shard(sh, ln, master_local, t, shard->G, shard->g, grad_dtype, P,
                                                      ue::to_dev(*plan), static_cast<cudaStream_t>(stream));
         return e == cudaSuccess ? UE_OK : cuda_fail(e, "grad-reduce launch");

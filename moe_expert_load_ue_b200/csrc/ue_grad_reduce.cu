@@ -339,13 +339,15 @@ cudaError_t set_grad_bulk_attributes(size_t max_smem)
     return e;
 }
 
-int grad_blocks_per_sm(int grad_dtype)
+// Resident CTAs per SM of the vector kernel with the shared memory one launch
+// uses (its tables grow with E and N*R).
+int grad_blocks_per_sm(int grad_dtype, size_t smem)
 {
     int n = 0;
     const cudaError_t e =
         grad_dtype == 1
-            ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_grad_reduce<true>, kGradThreads, 32 * 1024)
-            : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_grad_reduce<false>, kGradThreads, 32 * 1024);
+            ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_grad_reduce<true>, kGradThreads, smem)
+            : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_grad_reduce<false>, kGradThreads, smem);
     return (e == cudaSuccess && n > 0) ? n : 1;
 }
 
@@ -354,8 +356,8 @@ size_t grad_smem_bytes(const Shape &sh) { return (size_t)(3 * sh.E + sh.E + sh.N
 cudaError_t launch_grad_reduce(const Shape &sh, const Launch &ln, float *master, const void *grads,
                                int grad_dtype, int64_t P, const PlanDev &plan, cudaStream_t st)
 {
-    const dim3 grid((unsigned)ln.sms);   // resident CTAs: SMs x blocks per SM
     const size_t smem = grad_smem_bytes(sh);
+    const dim3 grid((unsigned)(ln.sms * grad_blocks_per_sm(grad_dtype, smem)));   // one wave of resident CTAs
     const int cap = sh.E + sh.NR;
     if (grad_dtype == 1)
         k_grad_reduce<true><<<grid, kGradThreads, smem, st>>>(master, grads, P, sh.E, sh.S, sh.H, sh.HR, sh.R, cap,

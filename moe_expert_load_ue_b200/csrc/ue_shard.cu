@@ -354,29 +354,33 @@ cudaError_t launch_sync_shard(const Shape &sh, const Launch &ln, const PeerTable
     return cudaGetLastError();
 }
 
+int grad_shard_blocks_per_sm(int grad_dtype, size_t smem);
+
 cudaError_t launch_grad_reduce_shard(const Shape &sh, const Launch &ln, float *master, const PeerTable &grads,
                                      int G, int g, int grad_dtype, int64_t P, const PlanDev &plan, cudaStream_t st)
 {
     const size_t smem = grad_shard_smem_bytes(sh);
     const int cap = sh.E + sh.NR, NG = sh.N / G;
+    const unsigned grid = (unsigned)(ln.sms * grad_shard_blocks_per_sm(grad_dtype, smem));
     if (grad_dtype == 1)
-        k_grad_reduce_shard<true><<<ln.sms, kGradThreads, smem, st>>>(master, grads, P, sh.E, sh.S, sh.H, sh.HR,
+        k_grad_reduce_shard<true><<<grid, kGradThreads, smem, st>>>(master, grads, P, sh.E, sh.S, sh.H, sh.HR,
                                                                       sh.R, NG, G, g, cap, plan.rep_off,
                                                                       plan.rep_slot, plan.rep_experts, plan.info);
     else
-        k_grad_reduce_shard<false><<<ln.sms, kGradThreads, smem, st>>>(master, grads, P, sh.E, sh.S, sh.H, sh.HR,
+        k_grad_reduce_shard<false><<<grid, kGradThreads, smem, st>>>(master, grads, P, sh.E, sh.S, sh.H, sh.HR,
                                                                        sh.R, NG, G, g, cap, plan.rep_off,
                                                                        plan.rep_slot, plan.rep_experts, plan.info);
     return cudaGetLastError();
 }
 
-int grad_shard_blocks_per_sm(int grad_dtype)
+// Resident CTAs per SM with the shared memory one launch uses.
+int grad_shard_blocks_per_sm(int grad_dtype, size_t smem)
 {
     int n = 0;
     const cudaError_t e =
         grad_dtype == 1
-            ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_grad_reduce_shard<true>, kGradThreads, 32 * 1024)
-            : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_grad_reduce_shard<false>, kGradThreads, 32 * 1024);
+            ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_grad_reduce_shard<true>, kGradThreads, smem)
+            : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_grad_reduce_shard<false>, kGradThreads, smem);
     return (e == cudaSuccess && n > 0) ? n : 1;
 }
 
