@@ -705,6 +705,14 @@ ue_status ue_grad_reduce_shard(ue_ctx *ctx, const ue_config *cfg, const ue_shard
     }
     if ((s = check_ctx(ctx)) != UE_OK) return s;
     return on_device(ctx, [&]() -> ue_status {
+        if (ue::grad_bulk_smem_bytes(sh) <= (size_t)ctx->max_smem) {
+            const ue::WaitBound wb{(unsigned long long)ctx->wait_ns, ctx->stall_once};
+            cudaError_t e = ue::launch_grad_reduce_bulk_shard(sh, ctx->sms, master_local, t, shard->G, shard->g,
+                                                              grad_dtype, P, ue::to_dev(*plan), ctx->dev_err,
+                                                              static_cast<cudaStream_t>(stream), wb);
+            ctx->stall_once = 0;
+            return e == cudaSuccess ? UE_OK : cuda_fail(e, "grad-reduce launch");
+        }
         const ue::Launch ln = launch_of(ctx, sh);
         cudaError_t e = ue::launch_grad_reduce_shard(sh, ln, master_local, t, shard->G, shard->g, grad_dtype, P,
                                                      ue::to_dev(*plan), static_cast<cudaStream_t>(stream));

@@ -120,10 +120,14 @@ __device__ __forceinline__ bool gb_wait(uint64_t *bar, unsigned parity, unsigned
     }
 }
 
-template <bool BF16>
+// SHARD: the same reduction across G GPUs on GPU g: only the experts homed on
+// GPU g (master holds their rows, e - g * E/G), each replica's chunk pulled
+// from the GPU holding its gradient row through the peer table (GPU h =
+// rank / (N/G), local row (rank - h * N/G) * R + u) with plain bulk loads.
+template <bool BF16, bool SHARD>
 __global__ void __launch_bounds__(kGbThreads, 1)
-k_grad_reduce_bulk(float *__restrict__ master, const void *__restrict__ grads, int64_t P, int E, int S, int H,
-                   int HR, int R, int cap, const int32_t *__restrict__ rep_off,
+k_grad_reduce_bulk(float *__restrict__ master, const void *__restrict__ grads, PeerTable peers, int G, int g,
+                   int64_t P, int E, int S, int H, int HR, int R, int cap, const int32_t *__restrict__ rep_off,
                    const int32_t *__restrict__ rep_slot, const int32_t *__restrict__ rep_experts,
                    const int32_t *__restrict__ info, int32_t *__restrict__ dev_err, unsigned long long wait_ns,
                    int stall)
@@ -138,21 +142,45 @@ k_grad_reduce_bulk(float *__restrict__ master, const void *__restrict__ grads, i
     int32_t *x_e = reinterpret_cast<int32_t *>(outb + 2 * kGbChunk);  // [E]
     int32_t *x_first = x_e + E;                                       // [E]
     int32_t *x_cnt = x_first + E;                                     // [E]
-    int32_t *x_row = x_cnt + E;                                       // [cap]
+    int32_t *x_row = x_cnt + E;                                       // [cap] replica row (SHARD: gpu << 16 | local row)
+    int32_t *x_act = x_row + cap;                                     // [E + 1] SHARD: experts with work; count
+    const uint8_t **x_base = reinterpret_cast<const uint8_t **>(
+        (reinterpret_cast<uintptr_t>(x_act + E + 1) + 7) & ~static_cast<uintptr_t>(7));   // [kMaxGpus] SHARD
 
     const int M = R > 0 ? clampi(__ldg(info + 3), 0, E) : 0;
+    const int EG = SHARD ? E / G : E, NG = SHARD ? (S / HR) / G : 1;
     for (int m = threadIdx.x; m < M; m += blockDim.x) {
         const int e = clampi(__ldg(rep_experts + m), 0, E - 1);
         const int off = clampi(__ldg(rep_off + e), 0, cap - 1);
         const int end = clampi(__ldg(rep_off + e + 1), off + 1, cap);
-        x_e[m] = e;
+        x_e[m] = SHARD ? e - g * EG : e;
         x_first[m] = off + 1;
-        x_cnt[m] = end - off - 1;
+        x_cnt[m] = (!SHARD || e / EG == g) ? end - off - 1 : 0;     // across GPUs: reduced on its home GPU
     }
     for (int p = threadIdx.x; p < cap; p += blockDim.x) {
         const int sl = clampi(__ldg(rep_slot + p), 0, S - 1);
-        const int u = sl % HR - H;
-        x_row[p] = u >= 0 ? (sl / HR) * R + u : 0;
+        const int r = sl / HR, u = sl % HR - H;
+        if constexpr (SHARD) {
+            const int h = r / NG;
+            x_row[p] = u >= 0 ? (h << 16) | ((r - h * NG) * R + u) : 0;
+        } else {
+            x_row[p] = u >= 0 ? r * R + u : 0;
+        }
+    }
+    if constexpr (SHARD) {
+        for (int h = threadIdx.x; h < G; h += blockDim.x) x_base[h] = static_cast<const uint8_t *>(peers.p[h]);
+        __syncthreads();
+        if (threadIdx.x < 32) {                  // the experts homed here that have replicas
+            int n = 0;
+            for (int m0 = 0; m0 < M; m0 += 32) {
+                const int m = m0 + threadIdx.x;
+                const bool a = m < M && x_cnt[m] > 0;
+                const unsigned bal = __ballot_sync(0xffffffffu, a);
+                if (a) x_act[n + __popc(bal & lanemask_lt())] = m;
+                n += __popc(bal);
+            }
+            if (threadIdx.x == 0) x_act[E] = n;
+        }
     }
     if (threadIdx.x == 0) {
         for (int i = 0; i < kGbSlots; ++i) {
@@ -167,7 +195,9 @@ k_grad_reduce_bulk(float *__restrict__ master, const void *__restrict__ grads, i
     __syncthreads();
 
     const int64_t nchunks = (P + kGbChunk - 1) / kGbChunk;
-    const int64_t total = (int64_t)M * nchunks;
+    const int MA = SHARD ? x_act[E] : M;                  // work groups: SHARD lists them in x_act
+    const int64_t total = (int64_t)MA * nchunks;
+    auto group = [&](int64_t it) { return SHARD ? x_act[(int)(it / nchunks)] : (int)(it / nchunks); };
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int kElem = BF16 ? 2 : 4;
     constexpr int kRepPerSlot = kGbSlotBytes / (kGbChunk * kElem);   // bf16: two replica chunks per slot
@@ -178,8 +208,8 @@ k_grad_reduce_bulk(float *__restrict__ master, const void *__restrict__ grads, i
         if (lane != 0) return;
         int64_t seg = 0;
         for (int64_t it = blockIdx.x; it < total; it += gridDim.x) {
-            const int m = (int)(it / nchunks);
-            const int64_t x0 = (it - (int64_t)m * nchunks) * kGbChunk;
+            const int m = group(it);
+            const int64_t x0 = (it % nchunks) * kGbChunk;
             const int n = (int)min((int64_t)kGbChunk, P - x0);
             const int cnt = x_cnt[m];
             const int nseg = 1 + (cnt + kRepPerSlot - 1) / kRepPerSlot;
@@ -202,10 +232,15 @@ k_grad_reduce_bulk(float *__restrict__ master, const void *__restrict__ grads, i
                 asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(gb_smem(&full[b])),
                              "r"(bytes * (unsigned)nr) : "memory");
                 for (int q = 0; q < nr; ++q) {
-                    const void *src = j == 0 ? static_cast<const void *>(master + (int64_t)x_e[m] * P + x0)
-                                             : static_cast<const void *>(
-                                                   static_cast<const uint8_t *>(grads) +
-                                                   ((int64_t)x_row[x_first[m] + r0 - 1 + q] * P + x0) * kElem);
+                    const void *src;
+                    if (j == 0) {
+                        src = master + (int64_t)x_e[m] * P + x0;
+                    } else {
+                        const int loc = x_row[x_first[m] + r0 - 1 + q];
+                        const uint8_t *gb = SHARD ? x_base[loc >> 16] : static_cast<const uint8_t *>(grads);
+                        const int64_t row = SHARD ? (loc & 0xffff) : loc;
+                        src = gb + (row * P + x0) * kElem;
+                    }
                     asm volatile(
                         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                         ::"r"(gb_smem(slot + (size_t)b * kGbSlotBytes + (size_t)q * kGbChunk * kElem)), "l"(src),
@@ -234,8 +269,8 @@ k_grad_reduce_bulk(float *__restrict__ master, const void *__restrict__ grads, i
     int ob = 0;
     float *tile = outb + warp * (2 * kGbWarpElems);
     for (int64_t it = blockIdx.x; it < total; it += gridDim.x, ob ^= 1) {
-        const int m = (int)(it / nchunks);
-        const int64_t x0 = (it - (int64_t)m * nchunks) * kGbChunk;
+        const int m = group(it);
+        const int64_t x0 = (it % nchunks) * kGbChunk;
         const int n = (int)min((int64_t)kGbChunk, P - x0);
         const int cnt = x_cnt[m];
         const int w0 = warp * kGbWarpElems;                  // this warp's first element of the chunk
@@ -312,30 +347,51 @@ k_grad_reduce_bulk(float *__restrict__ master, const void *__restrict__ grads, i
 size_t grad_bulk_smem_bytes(const Shape &sh)
 {
     return 1024 + (size_t)kGbSlots * kGbSlotBytes + 2 * (size_t)kGbChunk * 4 +
-           (size_t)(3 * sh.E + sh.E + sh.NR) * sizeof(int32_t);
+           (size_t)(5 * sh.E + sh.NR + 1) * sizeof(int32_t) + 8 + (size_t)kMaxGpus * sizeof(void *);
 }
+
+namespace {
+template <bool SHARD>
+cudaError_t launch_bulk(const Shape &sh, int sms, float *master, const void *grads, const PeerTable &peers, int G,
+                        int g, int grad_dtype, int64_t P, const PlanDev &plan, int32_t *dev_err, cudaStream_t st,
+                        const WaitBound &wb)
+{
+    const size_t smem = grad_bulk_smem_bytes(sh);
+    const int cap = sh.E + sh.NR;
+    if (grad_dtype == 1)
+        k_grad_reduce_bulk<true, SHARD><<<sms, kGbThreads, smem, st>>>(
+            master, grads, peers, G, g, P, sh.E, sh.S, sh.H, sh.HR, sh.R, cap, plan.rep_off, plan.rep_slot,
+            plan.rep_experts, plan.info, dev_err, wb.ns, wb.stall);
+    else
+        k_grad_reduce_bulk<false, SHARD><<<sms, kGbThreads, smem, st>>>(
+            master, grads, peers, G, g, P, sh.E, sh.S, sh.H, sh.HR, sh.R, cap, plan.rep_off, plan.rep_slot,
+            plan.rep_experts, plan.info, dev_err, wb.ns, wb.stall);
+    return cudaGetLastError();
+}
+}  // namespace
 
 cudaError_t launch_grad_reduce_bulk(const Shape &sh, int sms, float *master, const void *grads, int grad_dtype,
                                     int64_t P, const PlanDev &plan, int32_t *dev_err, cudaStream_t st,
                                     const WaitBound &wb)
 {
-    const size_t smem = grad_bulk_smem_bytes(sh);
-    const int cap = sh.E + sh.NR;
-    if (grad_dtype == 1)
-        k_grad_reduce_bulk<true><<<sms, kGbThreads, smem, st>>>(master, grads, P, sh.E, sh.S, sh.H, sh.HR, sh.R, cap,
-                                                                plan.rep_off, plan.rep_slot, plan.rep_experts,
-                                                                plan.info, dev_err, wb.ns, wb.stall);
-    else
-        k_grad_reduce_bulk<false><<<sms, kGbThreads, smem, st>>>(master, grads, P, sh.E, sh.S, sh.H, sh.HR, sh.R, cap,
-                                                                 plan.rep_off, plan.rep_slot, plan.rep_experts,
-                                                                 plan.info, dev_err, wb.ns, wb.stall);
-    return cudaGetLastError();
+    PeerTable none;
+    none.p[0] = nullptr;
+    return launch_bulk<false>(sh, sms, master, grads, none, 1, 0, grad_dtype, P, plan, dev_err, st, wb);
+}
+
+cudaError_t launch_grad_reduce_bulk_shard(const Shape &sh, int sms, float *master, const PeerTable &grads, int G,
+                                          int g, int grad_dtype, int64_t P, const PlanDev &plan, int32_t *dev_err,
+                                          cudaStream_t st, const WaitBound &wb)
+{
+    return launch_bulk<true>(sh, sms, master, nullptr, grads, G, g, grad_dtype, P, plan, dev_err, st, wb);
 }
 
 cudaError_t set_grad_bulk_attributes(size_t max_smem)
 {
-    cudaError_t e = allow_smem(k_grad_reduce_bulk<true>, max_smem);
-    if (e == cudaSuccess) e = allow_smem(k_grad_reduce_bulk<false>, max_smem);
+    cudaError_t e = allow_smem(k_grad_reduce_bulk<true, false>, max_smem);
+    if (e == cudaSuccess) e = allow_smem(k_grad_reduce_bulk<false, false>, max_smem);
+    if (e == cudaSuccess) e = allow_smem(k_grad_reduce_bulk<true, true>, max_smem);
+    if (e == cudaSuccess) e = allow_smem(k_grad_reduce_bulk<false, true>, max_smem);
     return e;
 }
 

@@ -111,6 +111,11 @@ struct WaitBound {
 cudaError_t launch_grad_reduce_bulk(const Shape &sh, int sms, float *master, const void *grads, int grad_dtype,
                                     int64_t P, const PlanDev &plan, int32_t *dev_err, cudaStream_t st,
                                     const WaitBound &wb);
+// The same across G GPUs on GPU g: its home experts' master rows, replica
+// gradient rows pulled through the peer table (plain bulk loads).
+cudaError_t launch_grad_reduce_bulk_shard(const Shape &sh, int sms, float *master, const PeerTable &grads, int G,
+                                          int g, int grad_dtype, int64_t P, const PlanDev &plan, int32_t *dev_err,
+                                          cudaStream_t st, const WaitBound &wb);
 
 // prev_slot_expert: the previous plan's slot_expert for the incremental form, or nullptr.
 cudaError_t launch_sync(const Shape &sh, const Launch &ln, uint8_t *weights, int64_t slot_bytes,
