@@ -154,3 +154,14 @@ def test_pieces_plan_variants(ctx):
         for f in oracle.PLAN_FIELDS:
             assert np.array_equal(pl[f], ref["plan"][f]), (v, f)
         assert np.array_equal(phys.cpu().numpy(), ref["phys"]), v
+
+
+@pytest.mark.parametrize("E,N,R,tpr,s", [
+    (1024, 1024, 1, 16384, 1.2),     # the largest E and N: the workspace caps the pieces per rank
+    (1024, 8, 4, 131072, 0.8),       # 128 home experts per rank, four redundant slots each
+])
+def test_pieces_widest_shapes(ctx, E, N, R, tpr, s):
+    w = inputs.Workload(f"pieces-wide-{E}-{N}", E=E, K=8, N=N, R=R, tokens_per_rank=tpr, s=s, base_seed=11)
+    ids_d = inputs.topk_ids_device(w, 0, "cuda")
+    torch.cuda.synchronize()
+    _check(ctx, ids_d.cpu().numpy(), w.E, w.N, w.R)
