@@ -149,12 +149,20 @@ def plan_sizes(cfg: Config) -> dict:
 
 
 class Plan:
-    """Device buffers of one placement plan (int32 torch tensors)."""
+    """Device buffers of one placement plan: the 11 int32 arrays of
+    ue_plan_buffers as views of one contiguous buffer (each view 16-byte
+    aligned), so that the whole plan moves to or from the host in one copy
+    (`buffer`)."""
 
     def __init__(self, cfg: Config, device="cuda"):
         self.cfg = cfg
-        self.tensors = {f: torch.empty(n, dtype=torch.int32, device=device)
-                        for f, n in plan_sizes(cfg).items()}
+        sizes = plan_sizes(cfg)
+        offs, o = {}, 0
+        for f in PLAN_FIELDS:
+            offs[f] = o
+            o += (sizes[f] + 3) // 4 * 4
+        self.buffer = torch.empty(o, dtype=torch.int32, device=device)
+        self.tensors = {f: self.buffer[offs[f]:offs[f] + sizes[f]] for f in PLAN_FIELDS}
         self.tensors["rank_off"] = self.tensors["rank_off"].view(cfg.N, cfg.E)
         self._c = UePlanBuffers(*[self.tensors[f].data_ptr() for f in PLAN_FIELDS])
 
@@ -168,7 +176,8 @@ class Plan:
         return {k: v.cpu().numpy() for k, v in self.tensors.items()}
 
     def nbytes(self) -> int:
-        return sum(t.numel() * 4 for t in self.tensors.values())
+        """Bytes of the whole plan buffer (the 11 arrays and their alignment padding)."""
+        return self.buffer.numel() * 4
 
 
 def _stream(stream) -> int:
