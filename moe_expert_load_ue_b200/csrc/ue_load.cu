@@ -26,10 +26,33 @@ namespace {
 constexpr int kLoadWarps = 16;
 constexpr int kCopies = 16;      // shared-memory histogram copies per CTA (one per warp)
 
-__device__ __forceinline__ void count_id(int32_t *h, int id, int E, int &nbad)
+#ifndef UE_LOAD_BUILTIN_ATOMIC
+using HistRef = uint32_t;        // shared-state-space address of a histogram copy
+__device__ __forceinline__ HistRef hist_ref(int32_t *h) { return (uint32_t)__cvta_generic_to_shared(h); }
+#else
+using HistRef = int32_t *;
+__device__ __forceinline__ HistRef hist_ref(int32_t *h) { return h; }
+#endif
+
+// One id into a histogram copy of E + 1 bins at shared address h: an id
+// outside [0, E) lands in bin E, so that the count is one unsigned min, one
+// address and one shared reduction, with no branch.
+#ifndef UE_LOAD_BUILTIN_ATOMIC
+__device__ __forceinline__ void count_id(HistRef h, int id, int E)
 {
-    if ((unsigned)id < (unsigned)E) smem_add(h + id, 1);
-    else ++nbad;
+    const uint32_t bin = min((uint32_t)id, (uint32_t)E);
+    asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(h + 4u * bin) : "memory");
+}
+#else
+__device__ __forceinline__ void count_id(int32_t *h, int id, int E)
+{
+    atomicAdd(h + min((uint32_t)id, (uint32_t)E), 1);
+}
+#endif
+
+__device__ __forceinline__ void count4(HistRef h, int4 q, int E)
+{
+    count_id(h, q.x, E); count_id(h, q.y, E); count_id(h, q.z, E); count_id(h, q.w, E);
 }
 
 // The first four int4 vectors of every thread for the range [lo, hi) (its
@@ -57,51 +80,44 @@ __device__ __forceinline__ Head load_head(const int32_t *__restrict__ ids, int64
 // and tail (< 4 ids each) by warp 0, the body as int4 vectors, four in flight
 // per thread (the first four already in hd).
 __device__ __forceinline__ void count_range(const int32_t *__restrict__ ids, int64_t lo, int64_t hi, int E,
-                                            int32_t *h, int &nbad, const Head &hd)
+                                            HistRef h, const Head &hd)
 {
     const int lane = lane_id(), warp = threadIdx.x >> 5;
     const int64_t vlo = min(hi, (lo + 3) / 4 * 4);
     const int64_t vhi = max(vlo, hi / 4 * 4);
     const int4 *vec = reinterpret_cast<const int4 *>(ids + vlo);
-    const int64_t nvec = (vhi - vlo) / 4;
-    const int64_t stride = (int64_t)blockDim.x;
+    const int nvec = (int)((vhi - vlo) / 4);
+    const int stride = (int)blockDim.x;
     if (warp == 0) {
         int64_t i = -1;
         if (lane < vlo - lo) i = lo + lane;
         else if (lane >= 4 && lane - 4 < hi - vhi) i = vhi + (lane - 4);
-        if (i >= 0) count_id(h, __ldg(ids + i), E, nbad);
+        if (i >= 0) count_id(h, __ldg(ids + i), E);
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        if (threadIdx.x + k * stride < nvec) {
-            count_id(h, hd.q[k].x, E, nbad); count_id(h, hd.q[k].y, E, nbad);
-            count_id(h, hd.q[k].z, E, nbad); count_id(h, hd.q[k].w, E, nbad);
-        }
-    }
-    int64_t v = threadIdx.x + 4 * stride;
+    for (int k = 0; k < 4; ++k)
+        if ((int)threadIdx.x + k * stride < nvec) count4(h, hd.q[k], E);
+    int v = (int)threadIdx.x + 4 * stride;
     for (; v + 3 * stride < nvec; v += 4 * stride) {
         int4 q[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) q[k] = __ldg(vec + v + k * stride);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            count_id(h, q[k].x, E, nbad); count_id(h, q[k].y, E, nbad);
-            count_id(h, q[k].z, E, nbad); count_id(h, q[k].w, E, nbad);
-        }
+        for (int k = 0; k < 4; ++k) count4(h, q[k], E);
     }
-    for (; v < nvec; v += stride) {
-        const int4 a = __ldg(vec + v);
-        count_id(h, a.x, E, nbad); count_id(h, a.y, E, nbad); count_id(h, a.z, E, nbad); count_id(h, a.w, E, nbad);
-    }
+    for (; v < nvec; v += stride) count4(h, __ldg(vec + v), E);
 }
 
+// Every histogram row below has E + 1 columns: the E experts, then the ids
+// outside [0, E).
+//
 // PIECES: the CTA's share is cut into pieces of zp ids (piece b of the rank is
 // [b*zp, (b+1)*zp), pieces c*ppc .. c*ppc+ppc-1 in CTA c of the cluster).
-// Row b of rank r, rows[(r*(B+1) + b)][0..E), receives the occurrences of
+// Row b of rank r, rows[(r*(B+1) + b)][0..E], receives the occurrences of
 // every expert in the rank's ids before piece b (an exclusive prefix over the
-// pieces), and row B the rank's totals; column E counts the ids outside
-// [0, E) the same way.  The persistent reroute kernel takes each piece's
-// starting occurrence indices and its counts from two consecutive rows.
+// pieces), and row B the rank's totals.  The persistent reroute kernel takes
+// each piece's starting occurrence indices and its counts from two
+// consecutive rows.
 template <bool PIECES>
 __global__ void __launch_bounds__(kLoadWarps * 32)
 k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
@@ -109,10 +125,10 @@ k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
        int32_t *__restrict__ rows, int64_t zp, int B)
 {
     extern __shared__ __align__(16) int32_t sm_load[];
-    int32_t *hist = sm_load;                     // [kCopies][E] counts
-    int32_t *tot = hist + kCopies * E;           // [E]    CTA counts (read by the cluster)
-    int32_t *sbad = tot + E;                     // [4]    bad ids: CTA total; current piece
-    int32_t *pcnt = sbad + 4;                    // PIECES: [ppc][E + 1] counts of the CTA's pieces
+    const int E1 = E + 1;
+    int32_t *hist = sm_load;                     // [kCopies][E1] counts
+    int32_t *tot = hist + kCopies * E1;          // [E1]  CTA counts (read by the cluster)
+    int32_t *pcnt = tot + E1;                    // PIECES: [ppc][E1] counts of the CTA's pieces
 
     // The planner (launched with programmatic dependent launch) may start
     // now; it waits for this grid's completion before reading counts.
@@ -132,60 +148,50 @@ k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
     const int64_t lo = base + min(per_rank, (int64_t)c * share);
     const int64_t hi = base + min(per_rank, (int64_t)(c + 1) * share);
     const int64_t len = PIECES ? zp : share;
-    int32_t *h = hist + (warp % kCopies) * E;
-    int nbad = 0;
+    const HistRef h = hist_ref(hist + (warp % kCopies) * E1);
 
     Head hd = load_head(ids, lo, min(hi, lo + len));
-    for (int i = threadIdx.x; i < kCopies * E; i += blockDim.x) hist[i] = 0;
+    for (int i = threadIdx.x; i < kCopies * E1; i += blockDim.x) hist[i] = 0;
     if (PIECES)
-        for (int e = threadIdx.x; e < E; e += blockDim.x) tot[e] = 0;
-    if (threadIdx.x == 0) sbad[0] = sbad[1] = 0;
+        for (int e = threadIdx.x; e < E1; e += blockDim.x) tot[e] = 0;
     __syncthreads();
 
     if constexpr (!PIECES) {
-        count_range(ids, lo, hi, E, h, nbad, hd);
-        if (nbad) atomicAdd(&sbad[1], nbad);
+        count_range(ids, lo, hi, E, h, hd);
         __syncthreads();
-        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        for (int e = threadIdx.x; e < E1; e += blockDim.x) {
             int s = 0;
 #pragma unroll
-            for (int w = 0; w < kCopies; ++w) s += hist[w * E + e];
+            for (int w = 0; w < kCopies; ++w) s += hist[w * E1 + e];
             tot[e] = s;
         }
-        if (threadIdx.x == 0) sbad[0] = sbad[1];
     } else {
         for (int64_t plo = lo; plo < hi; plo += len) {
             const int64_t phi = min(hi, plo + len);
-            count_range(ids, plo, phi, E, h, nbad, hd);
-            if (nbad) atomicAdd(&sbad[1], nbad);
-            nbad = 0;
+            count_range(ids, plo, phi, E, h, hd);
             // The next piece's first vectors load while this one is reduced.
             if (phi < hi) hd = load_head(ids, phi, min(hi, phi + len));
             __syncthreads();
-            int32_t *pc = pcnt + (int)((plo - lo) / zp) * (E + 1);
-            for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            int32_t *pc = pcnt + (int)((plo - lo) / zp) * E1;
+            for (int e = threadIdx.x; e < E1; e += blockDim.x) {
                 int s = 0;
 #pragma unroll
                 for (int w = 0; w < kCopies; ++w) {
-                    s += hist[w * E + e];
-                    hist[w * E + e] = 0;
+                    s += hist[w * E1 + e];
+                    hist[w * E1 + e] = 0;
                 }
                 tot[e] += s;
                 pc[e] = s;
-            }
-            if (threadIdx.x == 0) {
-                pc[E] = sbad[1];
-                sbad[0] += sbad[1];
-                sbad[1] = 0;
             }
             __syncthreads();
         }
     }
 
-    // Cluster reduction over distributed shared memory.
+    // Cluster reduction over distributed shared memory; column E is the
+    // rank's count of ids outside [0, E).
     cluster.sync();
-    const int cols = (E + C - 1) / C;
-    const int e0 = c * cols, e1 = min(E, e0 + cols);
+    const int cols = (E1 + C - 1) / C;
+    const int e0 = c * cols, e1 = min(E1, e0 + cols);
     for (int e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
         int part[kMaxCluster];
 #pragma unroll
@@ -193,27 +199,25 @@ k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
         int s = 0;
 #pragma unroll
         for (int q = 0; q < kMaxCluster; ++q) s += part[q];
-        if (counts != nullptr) counts[(int64_t)r * E + e] = s;
-    }
-    if (bad != nullptr && c == 0 && threadIdx.x == 0) {
-        int s = 0;
-        for (int q = 0; q < C; ++q) s += *cluster.map_shared_rank(sbad, q);
-        bad[r] = s;
+        if (e < E) {
+            if (counts != nullptr) counts[(int64_t)r * E + e] = s;
+        } else if (bad != nullptr) {
+            bad[r] = s;
+        }
     }
     if constexpr (PIECES) {
         // The prefix rows of this CTA's pieces: the earlier CTAs' totals
         // (peers' shared memory), then the pieces in order; the CTA holding
         // the rank's last piece also writes the totals row B.
         const int b0 = c * ppc, nq = min(ppc, B - b0);
-        for (int e = threadIdx.x; e <= E; e += blockDim.x) {
-            const int32_t *src = e < E ? tot + e : sbad;
+        for (int e = threadIdx.x; e < E1; e += blockDim.x) {
             int run = 0;
-            for (int q = 0; q < c; ++q) run += *cluster.map_shared_rank(src, q);
+            for (int q = 0; q < c; ++q) run += cluster.map_shared_rank(tot, q)[e];
             for (int q = 0; q < nq; ++q) {
-                rows[((int64_t)r * (B + 1) + b0 + q) * (E + 1) + e] = run;
-                run += pcnt[q * (E + 1) + e];
+                rows[((int64_t)r * (B + 1) + b0 + q) * E1 + e] = run;
+                run += pcnt[q * E1 + e];
             }
-            if (nq > 0 && b0 + nq == B) rows[((int64_t)r * (B + 1) + B) * (E + 1) + e] = run;
+            if (nq > 0 && b0 + nq == B) rows[((int64_t)r * (B + 1) + B) * E1 + e] = run;
         }
     }
     cluster_arrive_relaxed();   // done reading the peers; they may still read this CTA's totals
@@ -224,7 +228,7 @@ k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
 
 size_t load_smem_bytes(const Shape &sh, int ppc)
 {
-    return (size_t)((kCopies + 1) * sh.E + 4 + (size_t)ppc * (sh.E + 1)) * sizeof(int32_t);
+    return (size_t)((kCopies + 1) + (size_t)ppc) * (sh.E + 1) * sizeof(int32_t);
 }
 
 cudaError_t launch_load(const Shape &sh, const Launch &ln, const int32_t *ids, int32_t *counts,
