@@ -47,13 +47,13 @@ VARIANTS = {"requeue": 1, "spread": 2, "requeue+spread": 3}     # plan variant b
 TRAFFIC = {
     ("grad_reduce", "671B-class"): {
         "sources": ["moe_expert_load_ue_b200/csrc/ue_grad_reduce.cu", "moe_expert_load_ue_b200/csrc/ue_grad.cuh"],
-        "sha256": "d86dcac79562c699e8c013a7a24c6fb21e368f71ea703a786ab2d3bbb8125a04",
-        "dram_bytes": 7903631616, "algorithmic_bytes": 7927234560,
+        "sha256": "84d2f94dab75115c86e4fb4eaed56f4b7ab6abc45c4dc9ee2dc5fe468a45f3f0",
+        "dram_bytes": 7903708416, "algorithmic_bytes": 7927234560,
         "profile": "profiles/grad_reduce_and_sync_dram_671B-class.md"},
     ("sync", "671B-class"): {
         "sources": ["moe_expert_load_ue_b200/csrc/ue_sync.cu", "moe_expert_load_ue_b200/csrc/ue_bulk.cuh"],
         "sha256": "54818e6ae81cee9dea4303af048a3fa945b6e7fc8a5e9eb0ea3c06330eda349d",
-        "dram_bytes": 4962855680, "algorithmic_bytes": 5020581888,
+        "dram_bytes": 4962007296, "algorithmic_bytes": 5020581888,
         "profile": "profiles/grad_reduce_and_sync_dram_671B-class.md"},
 }
 
