@@ -286,6 +286,62 @@ __device__ __forceinline__ void greedy_chunks(const PlanSmem &s, int N, int R, i
     }
 }
 
+// The two sorts of the planner as ranks (keys are unique; larger first):
+// order[rank] of the M1 overflow keys s.key[0..M1), and for the K eligible
+// ranks s.key2[0..K) their sorted position, rsorted[rank], and the sum of the
+// spares (high words) of the keys above, rsum[rank] (rsum[K]: the total).  A
+// group of g consecutive lanes shares one key, each lane comparing it with
+// every g-th key of its array, four loads in flight; the group then adds its
+// lanes' counts.  Both arrays are ranked in the same pass over the block.
+__device__ __forceinline__ void rank_keys(const PlanSmem &s, int M1, int K)
+{
+    const int n = M1 + K, nt = blockDim.x;
+    int g = 1;
+    while (g < 32 && 2 * g * n <= nt) g *= 2;
+    const int groups = nt / g, sub = threadIdx.x & (g - 1);
+    const int off2 = (int)(s.key2 - s.key);
+    for (int i0 = 0; i0 < n; i0 += groups) {       // the same trip count in every thread
+        const int i = i0 + (int)threadIdx.x / g;
+        const bool valid = i < n, first = i < M1;
+        const int base = first ? 0 : off2, na = first ? M1 : K;
+        const unsigned long long mine = valid ? s.key[base + (first ? i : i - M1)] : 0ull;
+        int rank = 0;
+        unsigned above = 0;                        // (overflow keys: unused)
+        if (valid) {
+            int k = sub;
+            for (; k + 3 * g < na; k += 4 * g) {
+                unsigned long long o[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) o[u] = s.key[base + k + u * g];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    rank += o[u] > mine ? 1 : 0;
+                    above += o[u] > mine ? (unsigned)(o[u] >> 32) : 0u;
+                }
+            }
+            for (; k < na; k += g) {
+                const unsigned long long o = s.key[base + k];
+                rank += o > mine ? 1 : 0;
+                above += o > mine ? (unsigned)(o >> 32) : 0u;
+            }
+        }
+        for (int x = 1; x < g; x <<= 1) {
+            rank += __shfl_xor_sync(0xffffffffu, rank, x);
+            above += __shfl_xor_sync(0xffffffffu, above, x);
+        }
+        if (valid && sub == 0) {
+            const int id = (int)(0xffffffffu - (unsigned)(mine & 0xffffffffu));
+            if (first) {
+                s.order[rank] = id;
+            } else {
+                s.rsorted[rank] = id;
+                s.rsum[rank] = (int)above;
+                if (rank == K - 1) s.rsum[K] = (int)(above + (unsigned)(mine >> 32));
+            }
+        }
+    }
+}
+
 // R = 1: walk the eligible ranks in sorted order (exclusive spare prefix
 // s.rsum over K ranks); run by warp 0.  Expert m of the overflow order takes
 // the sorted positions [cut[m], cut[m+1]) (recorded in s.afirst / s.acnt);
@@ -297,9 +353,9 @@ __device__ __forceinline__ void greedy_sorted(const PlanSmem &s, int K, int M1)
 {
     const int lane = lane_id();
     int p = 0, stop_pos = M1, stop_rem = 0;
-    int rsum_p = 0;                                   // s.rsum[p]
+    unsigned rsum_p = 0;                              // s.rsum[p]
     int wbase = 1;                                    // window: lane holds s.rsum[wbase + lane]
-    int wv = wbase + lane <= K ? s.rsum[wbase + lane] : INT_MAX;
+    unsigned wv = wbase + lane <= K ? (unsigned)s.rsum[wbase + lane] : UINT_MAX;
     for (int m0 = 0; m0 < M1 && stop_pos == M1; m0 += 32) {
         const int idx = m0 + lane;
         const int e_l = idx < M1 ? s.order[idx] : 0;
@@ -309,32 +365,34 @@ __device__ __forceinline__ void greedy_sorted(const PlanSmem &s, int K, int M1)
         int j = 0;
         for (; j < cnt; ++j) {
             const int rem = __shfl_sync(0xffffffffu, o_l, j);
-            const long long target = (long long)rsum_p + rem;   // smallest q > p with rsum[q] >= target
-            int q = -1, rsum_q = 0;
-            while (wbase <= K) {
-                const bool cand = wbase + lane > p && wbase + lane <= K;
-                const unsigned b = __ballot_sync(0xffffffffu, cand && (long long)wv >= target);
-                if (b) {
-                    const int src = __ffs(b) - 1;
-                    q = wbase + src;
-                    rsum_q = __shfl_sync(0xffffffffu, wv, src);
-                    break;
-                }
-                wbase += 32;                          // the whole window is below the target
-                wv = wbase + lane <= K ? s.rsum[wbase + lane] : INT_MAX;
+            // The cut ends at the smallest q > p with rsum[q] >= target.  The
+            // prefix is strictly increasing (spares > 0) and rem > 0, so that q
+            // is the first position of the window at or above the target and
+            // rsum[q] is the window's smallest value at or above it: one
+            // redux.sync on the critical path; the position by a ballot beside
+            // it.  Values stay below 2^32: a spare sum and an overflow are each
+            // below 2^31.
+            const unsigned target = rsum_p + (unsigned)rem;
+            unsigned rq = __reduce_min_sync(0xffffffffu, wv >= target ? wv : UINT_MAX);
+            while (rq == UINT_MAX && wbase + 32 <= K) {   // the whole window is below the target
+                wbase += 32;
+                wv = wbase + lane <= K ? (unsigned)s.rsum[wbase + lane] : UINT_MAX;
+                rq = __reduce_min_sync(0xffffffffu, wv >= target ? wv : UINT_MAX);
             }
-            const int end = q < 0 ? K : q;
-            my_first = lane == j ? p : my_first;
-            my_end = lane == j ? end : my_end;
-            if (q < 0) {                              // every remaining rank used: the rest stays home
+            if (rq == UINT_MAX) {                     // every remaining rank used: the rest stays home
+                my_first = lane == j ? p : my_first;
+                my_end = lane == j ? K : my_end;
                 stop_pos = m0 + j;
-                stop_rem = rem - (s.rsum[K] - rsum_p);
+                stop_rem = rem - (s.rsum[K] - (int)rsum_p);
                 p = K;
                 ++j;
                 break;
             }
+            const int q = wbase + __popc(__ballot_sync(0xffffffffu, wv < target));
+            my_first = lane == j ? p : my_first;
+            my_end = lane == j ? q : my_end;
             p = q;
-            rsum_p = rsum_q;
+            rsum_p = rq;
         }
         if (lane < j) {
             s.afirst[e_l] = my_first;
@@ -682,28 +740,7 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, int variant, Pla
     if (eligible) s.key2[pk0 >> 16] = ((unsigned long long)(unsigned)my_spare << 32) | (0xffffffffu - (unsigned)tid);
     if (tid == 0 && K == 0) s.rsum[0] = 0;        // no eligible rank: an empty prefix
     __syncthreads();
-    if (tid < M1) {
-        const unsigned long long mine = s.key[tid];
-        int rank = 0;
-#pragma unroll 8
-        for (int k = 0; k < M1; ++k) rank += s.key[k] > mine ? 1 : 0;
-        s.order[rank] = (int)(0xffffffffu - (unsigned)(mine & 0xffffffffu));
-    }
-    if (tid < K) {
-        // Sorted position of this rank and the spares of the ranks before it.
-        const unsigned long long mine = s.key2[tid];
-        int rank = 0, before_sp = 0;
-#pragma unroll 8
-        for (int k = 0; k < K; ++k) {
-            const unsigned long long o = s.key2[k];
-            const bool gt = o > mine;
-            rank += gt ? 1 : 0;
-            before_sp += gt ? (int)(o >> 32) : 0;
-        }
-        s.rsorted[rank] = (int)(0xffffffffu - (unsigned)(mine & 0xffffffffu));
-        s.rsum[rank] = before_sp;
-        if (rank == K - 1) s.rsum[K] = before_sp + (int)(mine >> 32);
-    }
+    rank_keys(s, M1, K);
     __syncthreads();
 
     const bool requeue = kVariants && (variant & 1) != 0, spread = kVariants && (variant & 2) != 0;
