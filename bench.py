@@ -714,13 +714,36 @@ def run_ours(args, dist: Dist):
                 ev2[k][1].record(stream)
         stream.synchronize()
         lat_us = dist.max([statistics.mean(a.elapsed_time(b) * 1e3 for a, b in ev2)], device=dev)[0]
+        # The host link's own floor for these bytes: the same copies, H2D and
+        # D2H at once on the two copy streams, with no kernel between them.
+        go = torch.cuda.Event()
+        link = []
+        for k in range(n_e2e + 3):
+            a, b1, b2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            go.record(stream)
+            a.record(stream)
+            s_in.wait_event(go)
+            s_out.wait_event(go)
+            with torch.cuda.stream(s_in):
+                ids_b[0].copy_(ids_pinned[k % n_mb], non_blocking=True)
+                b1.record(s_in)
+            with torch.cuda.stream(s_out):
+                phys_h[1].copy_(phys_b[1], non_blocking=True)
+                plan_h[1].copy_(plan_b[1].buffer, non_blocking=True)
+                b2.record(s_out)
+            torch.cuda.synchronize(dev)
+            if k >= 3:
+                link.append(max(a.elapsed_time(b1), a.elapsed_time(b2)) * 1e3)
+        link_us = dist.max([statistics.median(link)], device=dev)[0]
         h2d = w.T * w.K * 4
         d2h = w.T * w.K * 4 + plan.nbytes()
         e2e = {"value": round(e2e_us, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "latency_us": round(lat_us, 2),
+               "link_floor_us": round(link_us, 2), "link_frac": round(link_us / e2e_us, 3) if e2e_us > 0 else None,
                "path": "pinned host ids -> ue_rebalance -> pinned host phys + the plan (its 11 arrays in one "
                        "buffer, one copy); steps pipelined on H2D / compute / D2H streams with two buffer sets "
-                       "(latency_us: one step alone)"}
+                       "(latency_us: one step alone; link_floor_us: the same H2D and D2H bytes copied at once "
+                       "with no kernel, the host link's bound for this leg)"}
         del ids_b, phys_b, plan_b, counts_b, bad_b
 
     peak, peak_kind = measured_peaks()
@@ -997,6 +1020,7 @@ def run_sweep(args, dist: Dist):
             stream.synchronize()
             vi = plan["info"].cpu().tolist()
             variants[name] = {"imbalance_after": round(vi[6] / mean, 4),
+                              "gap_bound": round(vi[6] / vi[0] - 1.0, 4) if vi[0] > 0 else None,
                               "rebalance_us_median": round(statistics.median(a.elapsed_time(b) * 1e3 for a, b in vt),
                                                            2)}
         med = statistics.median(us)
@@ -1006,6 +1030,9 @@ def run_sweep(args, dist: Dist):
                           "rebalance_alg_bytes": alg, "rebalance_gbs": round(alg / (med * 1e-6) / 1e9, 1),
                           "rebalance_frac": round(alg / (med * 1e-6) / 1e9 / peak, 4),
                           "imbalance_before": round(info[5] / mean, 4), "imbalance_after": round(info[6] / mean, 4),
+                          # max rank load after / Q - 1: Q = ceil(L / N) bounds every plan's busiest
+                          # rank from below, so this bounds the plan's gap to the optimum from above
+                          "gap_bound": round(info[6] / info[0] - 1.0, 4) if info[0] > 0 else None,
                           "slots_ran_out": bool(info[2] & 1), "replicated_experts": info[3],
                           "filled_redundant_slots": info[4], "plan_variants": variants}), flush=True)
         del ids, phys, plan, counts, bad
