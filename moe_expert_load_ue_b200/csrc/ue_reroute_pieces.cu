@@ -150,8 +150,18 @@ k_reroute_pieces(const int32_t *__restrict__ ids, int per_rank, int E, int cap, 
     // The rows a piece's table needs - rank_off[r][e], rows(r, b)[e] and
     // rows(r, b + 1)[e] - copied asynchronously into f[3][E] (each thread its
     // experts), so that they arrive while the previous piece streams.
+    // Claim p routes piece b = B - 1 - p / Nr of rank r = p % Nr: the load pass
+    // walks every rank's pieces first to last, so the pieces it read last (the
+    // ones still in L2) are routed first.
+    const int Nr = NP / B;
+    auto piece_of = [&](int p, int &r, int &b) {
+        const int q = p / Nr;
+        r = p - q * Nr;
+        b = B - 1 - q;
+    };
     auto fetch_issue = [&](int p) {
-        const int r = p / B, b = p - (p / B) * B;
+        int r, b;
+        piece_of(p, r, b);
         const int32_t *row = rows + ((size_t)r * (B + 1) + b) * stride_row;
         for (int e = threadIdx.x; e < E; e += kRpThreads) {
             cp_async<1>(s.f + e, rank_off + (size_t)r * E + e);
@@ -191,7 +201,8 @@ k_reroute_pieces(const int32_t *__restrict__ ids, int per_rank, int E, int cap, 
         }
     };
     auto piece_range = [&](int p, int &lo, int &hi) {
-        const int r = p / B, b = p - (p / B) * B;
+        int r, b;
+        piece_of(p, r, b);
         lo = (int)r * per_rank + (int)b * zp;
         hi = min(lo + zp, (int)(r + 1) * per_rank);
     };
