@@ -30,14 +30,18 @@ struct ue_ctx {
     int smem_reserved;
     int64_t wait_ns;       // bound of one wait in the weight-sync kernels
     int stall_once;        // diagnostic: the next weight sync stalls once (UE_WAIT_STALL_ONCE)
+    bool lv_dirty;         // a load grid may have added into the load vector without its planner
 };
 
 namespace {
-// Workspace of a context (16 MiB): kWsHead ints of counters (the persistent
-// reroute's piece counters, kept at 0 between launches), then the piece rows
-// [N][B + 1][E + 1] of one call.
+// Workspace of a context (16 MiB): 64 ints of counters (the persistent
+// reroute's piece counters, kept at 0 between launches), the expert load
+// vector of a fused rebalance (kMaxE ints, zeros between calls: the load grid
+// adds into it, its planner reads it and writes the zeros back), then the
+// piece rows [N][B + 1][E + 1] of one call from kWsHead on.
 constexpr int64_t kWsInts = (int64_t)1 << 22;
-constexpr int64_t kWsHead = 64;
+constexpr int64_t kWsLoadVec = 64;
+constexpr int64_t kWsHead = kWsLoadVec + ue::kMaxE;
 // Pieces of the persistent reroute are whole sub-chunks of its CTA (8192 ids:
 // 16 per thread), so every warp has work; its per-piece table costs about as
 // much as streaming a few thousand ids.
@@ -187,6 +191,19 @@ ue_status on_device(const ue_ctx *ctx, F &&fn)
     return s;
 }
 
+// The context's load vector for a fused load + plan on stream st, cleared
+// first when an earlier call queued a load grid without its planner; nullptr
+// if that clear could not be queued.
+int32_t *load_vector(ue_ctx *ctx, cudaStream_t st)
+{
+    int32_t *lv = ctx->ws + kWsLoadVec;
+    if (ctx->lv_dirty) {
+        if (cudaMemsetAsync(lv, 0, ue::kMaxE * sizeof(int32_t), st) != cudaSuccess) return nullptr;
+        ctx->lv_dirty = false;
+    }
+    return lv;
+}
+
 }  // namespace
 
 extern "C" {
@@ -240,6 +257,7 @@ ue_status ue_ctx_create(int device, ue_ctx **out)
     tmp.ws = nullptr;
     tmp.wait_ns = 2000000000LL;
     tmp.stall_once = 0;
+    tmp.lv_dirty = false;
     ue_status s = on_device(&tmp, [&]() -> ue_status {
         cudaError_t err;
         const size_t m = (size_t)tmp.max_smem;
@@ -404,13 +422,17 @@ ue_status ue_rebalance_ex(ue_ctx *ctx, const ue_config *cfg, const int32_t *ids,
         const ue::Launch ln = launch_of(ctx, sh);
         const ue::PlanDev pd = ue::to_dev(*plan);
         const ue::Pieces pc = pieces_for(ctx, sh, ln);
-        cudaError_t e = ue::launch_load(sh, ln, ids, counts, bad, st, &pc, ctx->ws + kWsHead);
+        int32_t *lv = load_vector(ctx, st);
+        if (lv == nullptr) return cuda_fail(cudaGetLastError(), "load vector reset");
+        cudaError_t e = ue::launch_load(sh, ln, ids, counts, bad, st, &pc, ctx->ws + kWsHead, lv);
         if (e != cudaSuccess) return cuda_fail(e, "load launch");
         // The planner and the reroute kernel use programmatic dependent launch:
         // each may start while its predecessor drains, and waits for it
         // (griddepcontrol.wait) before reading what it wrote.
-        if ((e = ue::launch_plan(sh, counts, pd, st, true, variant)) != cudaSuccess)
+        if ((e = ue::launch_plan(sh, counts, pd, st, true, variant, lv)) != cudaSuccess) {
+            ctx->lv_dirty = true;
             return cuda_fail(e, "plan launch");
+        }
         e = pc.NP > 0 ? ue::launch_reroute_pieces(sh, pc, ids, pd, ctx->ws + kWsHead, ctx->ws, phys, st, true)
                       : ue::launch_reroute(sh, ln, ids, pd, phys, st, true);
         if (e != cudaSuccess) return cuda_fail(e, "reroute launch");
@@ -481,9 +503,14 @@ ue_status ue_rebalance_dispatch(ue_ctx *ctx, const ue_config *cfg, const int32_t
         const cudaStream_t st = static_cast<cudaStream_t>(stream);
         const ue::Launch ln = launch_of(ctx, sh);
         const ue::PlanDev pd = ue::to_dev(*plan);
-        cudaError_t e = ue::launch_load(sh, ln, ids, counts, bad, st);
+        int32_t *lv = load_vector(ctx, st);
+        if (lv == nullptr) return cuda_fail(cudaGetLastError(), "load vector reset");
+        cudaError_t e = ue::launch_load(sh, ln, ids, counts, bad, st, nullptr, nullptr, lv);
         if (e != cudaSuccess) return cuda_fail(e, "load launch");
-        if ((e = ue::launch_plan(sh, counts, pd, st, true, 0)) != cudaSuccess) return cuda_fail(e, "plan launch");
+        if ((e = ue::launch_plan(sh, counts, pd, st, true, 0, lv)) != cudaSuccess) {
+            ctx->lv_dirty = true;
+            return cuda_fail(e, "plan launch");
+        }
         if ((e = ue::launch_dispatch(sh, ln, ids, pd, phys, out, ctx->dev_err, st, true)) != cudaSuccess)
             return cuda_fail(e, "dispatch launch");
         return UE_OK;

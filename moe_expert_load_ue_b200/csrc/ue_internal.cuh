@@ -69,16 +69,21 @@ struct Pieces {
 
 // Host launchers (one per kernel file).  Each returns cudaGetLastError().
 // With pc (NP > 0) the load kernel also writes the piece rows; counts may then
-// be nullptr (the rows alone, for a reroute without a preceding load).
+// be nullptr (the rows alone, for a reroute without a preceding load).  With
+// lv it also adds every rank's counts into lv[0..E) (which must hold zeros):
+// the expert loads, for a planner launched with the same lv right after it.
 cudaError_t launch_load(const Shape &sh, const Launch &ln, const int32_t *ids, int32_t *counts,
-                        int32_t *bad, cudaStream_t st, const Pieces *pc = nullptr, int32_t *rows = nullptr);
+                        int32_t *bad, cudaStream_t st, const Pieces *pc = nullptr, int32_t *rows = nullptr,
+                        int32_t *lv = nullptr);
 // Shared memory of the load kernel; ppc = pieces per CTA (0: no piece rows).
 size_t load_smem_bytes(const Shape &sh, int ppc);
 
 // variant: bit 0 re-queues partly placed overflow, bit 1 spreads stuck
-// remainders over the expert's replicas (0 = the stated rule).
+// remainders over the expert's replicas (0 = the stated rule).  lv: the expert
+// loads summed by the preceding load grid (launch_load with lv), read instead
+// of summing counts and set back to zeros; nullptr: the loads from counts.
 cudaError_t launch_plan(const Shape &sh, const int32_t *counts, const PlanDev &plan, cudaStream_t st,
-                        bool pdl, int variant);
+                        bool pdl, int variant, int32_t *lv = nullptr);
 size_t plan_smem_bytes(const Shape &sh);
 int plan_cluster(const Shape &sh);
 

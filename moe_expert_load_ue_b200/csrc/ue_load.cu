@@ -122,7 +122,7 @@ template <bool PIECES>
 __global__ void __launch_bounds__(kLoadWarps * 32)
 k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
        int32_t *__restrict__ counts, int32_t *__restrict__ bad,
-       int32_t *__restrict__ rows, int64_t zp, int B)
+       int32_t *__restrict__ rows, int64_t zp, int B, int32_t *__restrict__ lv)
 {
     extern __shared__ __align__(16) int32_t sm_load[];
     const int E1 = E + 1;
@@ -201,6 +201,7 @@ k_load(const int32_t *__restrict__ ids, int64_t per_rank, int E,
         for (int q = 0; q < kMaxCluster; ++q) s += part[q];
         if (e < E) {
             if (counts != nullptr) counts[(int64_t)r * E + e] = s;
+            if (lv != nullptr && s != 0) atomicAdd(lv + e, s);
         } else if (bad != nullptr) {
             bad[r] = s;
         }
@@ -232,16 +233,16 @@ size_t load_smem_bytes(const Shape &sh, int ppc)
 }
 
 cudaError_t launch_load(const Shape &sh, const Launch &ln, const int32_t *ids, int32_t *counts,
-                        int32_t *bad, cudaStream_t st, const Pieces *pc, int32_t *rows)
+                        int32_t *bad, cudaStream_t st, const Pieces *pc, int32_t *rows, int32_t *lv)
 {
     if (pc != nullptr && pc->NP > 0) {
         const int ppc = (pc->B + ln.cluster - 1) / ln.cluster;
         return launch_ex(k_load<true>, (unsigned)(sh.N * ln.cluster), kLoadWarps * 32, load_smem_bytes(sh, ppc), st,
-                         (unsigned)ln.cluster, false, ids, sh.per_rank, sh.E, counts, bad, rows, pc->zp, pc->B);
+                         (unsigned)ln.cluster, false, ids, sh.per_rank, sh.E, counts, bad, rows, pc->zp, pc->B, lv);
     }
     return launch_ex(k_load<false>, (unsigned)(sh.N * ln.cluster), kLoadWarps * 32, load_smem_bytes(sh, 0), st,
                      (unsigned)ln.cluster, false, ids, sh.per_rank, sh.E, counts, bad, (int32_t *)nullptr,
-                     (int64_t)0, 0);
+                     (int64_t)0, 0, lv);
 }
 
 cudaError_t set_load_attributes(size_t max_smem)

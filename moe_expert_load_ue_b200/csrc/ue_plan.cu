@@ -648,7 +648,7 @@ __device__ __forceinline__ void spread_stuck(const PlanSmem &s, int ns, int Q, i
 // the default planner carries none of the variants' code.
 template <int NRL, bool kVariants>
 __global__ void __launch_bounds__(kPlanMaxThreads, 1)
-k_plan(const int32_t *__restrict__ counts, int E, int N, int R, int variant, PlanDev plan)
+k_plan(const int32_t *__restrict__ counts, int E, int N, int R, int variant, PlanDev plan, int32_t *lv)
 {
     extern __shared__ __align__(16) int32_t sm_plan[];
     const int H = E / N, HR = H + R, S = N * HR, NR = N * R, cap = E + NR;
@@ -670,9 +670,13 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, int variant, Pla
     pdl_trigger();
     pdl_wait();
 
-    if (C == 1 || c != 0) slice_sums(counts, E, r0, r1, s.sload);
+    // direct: the load grid summed the expert loads into lv, which CTA 0 reads
+    // (and sets back to zeros) without waiting for the slices, whose partial
+    // vectors then serve rank_off alone.
+    const bool direct = lv != nullptr && c == 0;
+    if (!direct && (C == 1 || c != 0)) slice_sums(counts, E, r0, r1, s.sload);
     cluster_arrive();          // #1: this slice's partial loads are ready
-    cluster_wait();
+    if (!direct) cluster_wait();
     if (c != 0) {
         // Off the critical path: rank_off for this slice (the slices of the
         // lower peers give its start), then stay resident until every CTA has
@@ -686,7 +690,10 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, int variant, Pla
     const bool ve = e < E;
     int ld = 0;
     if (ve) {
-        if (C == 1) {
+        if (direct) {
+            ld = __ldcg(lv + e);
+            lv[e] = 0;
+        } else if (C == 1) {
             ld = s.sload[e];
         } else {
             int part[kMaxCluster];
@@ -697,7 +704,7 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, int variant, Pla
         }
         plan.load[e] = ld;
     }
-    cluster_arrive_relaxed();  // #2: done reading the peers; CTA 0 holds nothing they read
+    if (!direct) cluster_arrive_relaxed();  // #2: done reading the peers; CTA 0 holds nothing they read
 
     // ---- the plan (CTA 0; blockDim >= max(E, N)) ---------------------------------
     int L;
@@ -934,6 +941,10 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, int variant, Pla
         }
     }
     if (C == 1) slice_rank_off(cluster, counts, E, r0, r1, 0, 0, s.sload, plan.rank_off);
+    if (direct) {              // the barrier phases CTA 0 skipped above
+        cluster_wait();        // #1
+        cluster_arrive_relaxed();   // #2
+    }
     cluster_wait();
 }
 
@@ -963,15 +974,15 @@ int plan_cluster(const Shape &sh)
 }
 
 cudaError_t launch_plan(const Shape &sh, const int32_t *counts, const PlanDev &plan, cudaStream_t st, bool pdl,
-                        int variant)
+                        int variant, int32_t *lv)
 {
     const unsigned C = (unsigned)plan_cluster(sh);
     const unsigned threads = (unsigned)plan_threads(sh);
     const int nrl = (sh.N + 31) / 32;
     const size_t smem = plan_smem_bytes(sh);
 #define UE_PLAN_LAUNCH(V)                                                                                       \
-    (variant ? launch_ex(k_plan<V, true>, C, threads, smem, st, C, pdl, counts, sh.E, sh.N, sh.R, variant, plan)  \
-             : launch_ex(k_plan<V, false>, C, threads, smem, st, C, pdl, counts, sh.E, sh.N, sh.R, 0, plan))
+    (variant ? launch_ex(k_plan<V, true>, C, threads, smem, st, C, pdl, counts, sh.E, sh.N, sh.R, variant, plan, lv) \
+             : launch_ex(k_plan<V, false>, C, threads, smem, st, C, pdl, counts, sh.E, sh.N, sh.R, 0, plan, lv))
     if (nrl <= 1) return UE_PLAN_LAUNCH(1);
     if (nrl <= 2) return UE_PLAN_LAUNCH(2);
     if (nrl <= 4) return UE_PLAN_LAUNCH(4);
