@@ -58,19 +58,56 @@ TRAFFIC = {
 }
 
 
-def traffic_per_launch(kernel: str, workload: str, full_size: bool, mean_alg: float):
-    t = TRAFFIC.get((kernel, workload))
-    if t is None or not full_size:
-        return None
+# Each ncu summary under profiles/ with the kernel sources it was captured on
+# (the files hashed together, in this order); the JSON line's "profiles" object
+# reports each as "current" or "stale" (the code changed since the capture).
+PROFILES = {
+    "profiles/launch_list_671B-class.md": {
+        "sources": ["moe_expert_load_ue_b200/csrc/ue_load.cu", "moe_expert_load_ue_b200/csrc/ue_plan.cu", "moe_expert_load_ue_b200/csrc/ue_reroute.cu", "moe_expert_load_ue_b200/csrc/ue_sync.cu", "moe_expert_load_ue_b200/csrc/ue_bulk.cuh", "moe_expert_load_ue_b200/csrc/ue_grad_reduce.cu", "moe_expert_load_ue_b200/csrc/ue_grad.cuh"],
+        "sha256": "77a2c6f8676dfacc48cb324c401daacc1f950615179c85de6faa55638c30c17f"},
+    "profiles/hot_path_kernels_full_set_671B-class_small_experts.md": {
+        "sources": ["moe_expert_load_ue_b200/csrc/ue_load.cu", "moe_expert_load_ue_b200/csrc/ue_plan.cu", "moe_expert_load_ue_b200/csrc/ue_reroute.cu"],
+        "sha256": "df7ac359c9235188a5ea2619b5425cd59cc7178c8b5deca009dec6dc8697ef95"},
+    "profiles/grad_reduce_and_sync_dram_671B-class.md": {
+        "sources": ["moe_expert_load_ue_b200/csrc/ue_grad_reduce.cu", "moe_expert_load_ue_b200/csrc/ue_grad.cuh", "moe_expert_load_ue_b200/csrc/ue_sync.cu", "moe_expert_load_ue_b200/csrc/ue_bulk.cuh"],
+        "sha256": "da0a296cfaa1768c8d038f549d9e7908a3badbd34d0fd5f91ef33d3b903ee0aa"},
+    "profiles/grad_reduce_bulk_full_set_671B-class_small_experts.md": {
+        "sources": ["moe_expert_load_ue_b200/csrc/ue_grad_reduce.cu", "moe_expert_load_ue_b200/csrc/ue_grad.cuh"],
+        "sha256": "84d2f94dab75115c86e4fb4eaed56f4b7ab6abc45c4dc9ee2dc5fe468a45f3f0"},
+    "profiles/reroute_pieces_full_set_sweep_256x32768.md": {
+        "sources": ["moe_expert_load_ue_b200/csrc/ue_reroute_pieces.cu"],
+        "sha256": "b7a569b8c061375205de5e91ce6748c7d57b75a3bdcb83db7cd7753fbcc90e82"},
+    "profiles/dispatch_layout_671B-class_small_experts.md": {
+        "sources": ["moe_expert_load_ue_b200/csrc/ue_reroute.cu"],
+        "sha256": "6f1fe8f23d9a123d558ba2f6db0ed74b3e6aca91013f82ffdb93c6b289aa27e5"},
+    "profiles/sync_and_grad_across_gpus_dram_671B-class_emulated.md": {
+        "sources": ["moe_expert_load_ue_b200/csrc/ue_shard.cu", "moe_expert_load_ue_b200/csrc/ue_bulk.cuh", "moe_expert_load_ue_b200/csrc/ue_grad_reduce.cu", "moe_expert_load_ue_b200/csrc/ue_grad.cuh"],
+        "sha256": "01ca9e26e079f67826811838b5e22f8b2f5dac0d3bbaf00ec47deba039fd9997"},
+}
+
+
+def _sources_hash(sources) -> str | None:
     import hashlib
     m = hashlib.sha256()
     try:
-        for src in t["sources"]:
+        for src in sources:
             with open(os.path.join(ROOT, src), "rb") as f:
                 m.update(f.read())
     except OSError:
         return None
-    if m.hexdigest() != t["sha256"]:
+    return m.hexdigest()
+
+
+def profile_status() -> dict:
+    return {os.path.basename(p): ("current" if _sources_hash(t["sources"]) == t["sha256"] else "stale")
+            for p, t in PROFILES.items()}
+
+
+def traffic_per_launch(kernel: str, workload: str, full_size: bool, mean_alg: float):
+    t = TRAFFIC.get((kernel, workload))
+    if t is None or not full_size:
+        return None
+    if _sources_hash(t["sources"]) != t["sha256"]:
         return None
     return round(t["dram_bytes"] / t["algorithmic_bytes"] * mean_alg)
 
@@ -813,6 +850,7 @@ def run_ours(args, dist: Dist):
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clk,
         "job_microbatches_per_s": round(dist.world * args.steps / (total_ms_max * 1e-3), 2),
+        "profiles": profile_status(),
     }
     ctx.close()
     dist.barrier()
