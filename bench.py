@@ -64,10 +64,10 @@ TRAFFIC = {
 PROFILES = {
     "profiles/launch_list_671B-class.md": {
         "sources": ["moe_expert_load_ue_b200/csrc/ue_load.cu", "moe_expert_load_ue_b200/csrc/ue_plan.cu", "moe_expert_load_ue_b200/csrc/ue_reroute.cu", "moe_expert_load_ue_b200/csrc/ue_sync.cu", "moe_expert_load_ue_b200/csrc/ue_bulk.cuh", "moe_expert_load_ue_b200/csrc/ue_grad_reduce.cu", "moe_expert_load_ue_b200/csrc/ue_grad.cuh"],
-        "sha256": "77a2c6f8676dfacc48cb324c401daacc1f950615179c85de6faa55638c30c17f"},
+        "sha256": "417c54ca7f02435589460382a4235d6445668c6023fbcacacac10004777f857b"},
     "profiles/hot_path_kernels_full_set_671B-class_small_experts.md": {
         "sources": ["moe_expert_load_ue_b200/csrc/ue_load.cu", "moe_expert_load_ue_b200/csrc/ue_plan.cu", "moe_expert_load_ue_b200/csrc/ue_reroute.cu"],
-        "sha256": "df7ac359c9235188a5ea2619b5425cd59cc7178c8b5deca009dec6dc8697ef95"},
+        "sha256": "caa9633e08bb050a0799afa0639e93a75877c5f103a75e30e08838f134977225"},
     "profiles/grad_reduce_and_sync_dram_671B-class.md": {
         "sources": ["moe_expert_load_ue_b200/csrc/ue_grad_reduce.cu", "moe_expert_load_ue_b200/csrc/ue_grad.cuh", "moe_expert_load_ue_b200/csrc/ue_sync.cu", "moe_expert_load_ue_b200/csrc/ue_bulk.cuh"],
         "sha256": "da0a296cfaa1768c8d038f549d9e7908a3badbd34d0fd5f91ef33d3b903ee0aa"},

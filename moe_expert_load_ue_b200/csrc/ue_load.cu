@@ -26,29 +26,17 @@ namespace {
 constexpr int kLoadWarps = 16;
 constexpr int kCopies = 16;      // shared-memory histogram copies per CTA (one per warp)
 
-#ifndef UE_LOAD_BUILTIN_ATOMIC
 using HistRef = uint32_t;        // shared-state-space address of a histogram copy
 __device__ __forceinline__ HistRef hist_ref(int32_t *h) { return (uint32_t)__cvta_generic_to_shared(h); }
-#else
-using HistRef = int32_t *;
-__device__ __forceinline__ HistRef hist_ref(int32_t *h) { return h; }
-#endif
 
 // One id into a histogram copy of E + 1 bins at shared address h: an id
 // outside [0, E) lands in bin E, so that the count is one unsigned min, one
 // address and one shared reduction, with no branch.
-#ifndef UE_LOAD_BUILTIN_ATOMIC
 __device__ __forceinline__ void count_id(HistRef h, int id, int E)
 {
     const uint32_t bin = min((uint32_t)id, (uint32_t)E);
     asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(h + 4u * bin) : "memory");
 }
-#else
-__device__ __forceinline__ void count_id(int32_t *h, int id, int E)
-{
-    atomicAdd(h + min((uint32_t)id, (uint32_t)E), 1);
-}
-#endif
 
 __device__ __forceinline__ void count4(HistRef h, int4 q, int E)
 {
