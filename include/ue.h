@@ -53,8 +53,11 @@ typedef enum {
  * per-piece histograms that ue_rebalance(_ex) and ue_reroute(_shard) pass
  * from their load pass to their reroute pass when a CTA's share of a rank's
  * ids exceeds what the reroute keeps on chip (many ranks or many tokens per
- * rank); such calls on one context must not overlap on the GPU (issue them on
- * one stream, or order the streams). */
+ * rank), and the expert loads that the load pass of ue_rebalance,
+ * ue_rebalance_ex and ue_rebalance_dispatch sums for their planner (zeros
+ * between calls: the planner writes them back); such calls on one context
+ * must not overlap on the GPU (issue them on one stream, or order the
+ * streams).  Capturing them in a CUDA graph and replaying it is fine. */
 typedef struct ue_ctx ue_ctx;
 
 /* Problem shape.  H = E / N and S = N * (H + R) are derived. */
