@@ -897,69 +897,93 @@ def run_ours(args, dist: Dist):
 def across_gpus_real(args, dist, ctx, cfg, w, ids_dev, weights, master, grads, gdt, per_mb, slot_bytes, red, n_mb):
     """The sharded load/plan/reroute, weight sync (relay rounds and direct form)
     and home-GPU gradient reduction on the job's GPUs, each rank one GPU."""
+    if w.N % dist.world:
+        return {"skipped": f"N={w.N} is not a multiple of {dist.world} GPUs"}
+    return run_isolated(dist, lambda grp: _across_gpus(grp, dist, ctx, cfg, w, ids_dev, weights, master, grads,
+                                                       gdt, per_mb, slot_bytes, red, n_mb))
+
+
+def run_isolated(dist, fn, timeout_s: float = 60.0) -> dict:
+    """fn(group) on a gloo group of its own with a short timeout: a failure on
+    some ranks ends, on every rank, as an exception within the timeout (the
+    others' waits in that group run out), reported as {"error": ...}; the
+    job's main group is never left waiting.  Every rank calls it."""
+    import datetime
+    grp = dist.pg.new_group(backend="gloo", timeout=datetime.timedelta(seconds=timeout_s))
+    try:
+        return fn(grp)
+    except Exception as exc:      # reported in the line; the replicas' numbers stand
+        return {"error": repr(exc)[:300]}
+    finally:
+        try:
+            dist.pg.destroy_process_group(grp)
+        except Exception:
+            pass
+
+
+def _across_gpus(grp, dist, ctx, cfg, w, ids_dev, weights, master, grads, gdt, per_mb, slot_bytes, red, n_mb):
     import torch
 
     from moe_expert_load_ue_b200 import ue
     from moe_expert_load_ue_b200.peer import PeerBuffers
     from moe_expert_load_ue_b200.shard import DeviceOps, ShardedBalancer
     G, g = dist.world, dist.rank
-    if w.N % G:
-        return {"skipped": f"N={w.N} is not a multiple of {G} GPUs"}
-    try:
-        SG, EG, RG, TG = w.S // G, w.E // G, (w.N // G) * w.R, w.T // G
-        dev = weights.device
-        bal = ShardedBalancer(cfg, DeviceOps(ctx, cfg, G, g), G=G, g=g, device=dev)
-        pw = PeerBuffers(weights[g * SG:(g + 1) * SG])
-        pg = PeerBuffers(grads[g * RG:(g + 1) * RG])
-        counts = torch.empty((w.N, w.E), dtype=torch.int32, device=dev)
-        plan = ue.Plan(cfg, device=dev)
-        phys_l = torch.empty((TG, w.K), dtype=torch.int32, device=dev)
-        n_sh = min(n_mb, 4)
-        st = torch.cuda.current_stream(dev)
-        evs = []
-        for k in range(-1, n_sh):                    # one untimed pass first
-            mb = max(k, 0)
-            bal.rebalance(ids_dev[mb][g * TG:(g + 1) * TG], counts, None, plan, phys_l)
-            e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-            e[0].record(st)
-            bal.sync(pw.ptrs, slot_bytes, plan, relay=True)
-            e[1].record(st)
-            bal.sync(pw.ptrs, slot_bytes, plan, relay=False)
-            e[2].record(st)
-            bal.grad_reduce(master[g * EG:(g + 1) * EG], pg.ptrs, gdt, w.P, plan)
-            e[3].record(st)
-            if k >= 0:
-                evs.append(e)
-        torch.cuda.synchronize(dev)
-        t = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(3)] for e in evs]) * 1e3
-        tmax = dist.max(list(t.sum(axis=0)), device=dev)
-        bal.barrier()
-        torch.cuda.synchronize(dev)
-        pw.close()
-        pg.close()
-        sync_b = cross_b = grad_b = 0
-        gsize = 2 if w.grad_dtype == "bf16" else 4
-        for mb in range(n_sh):
-            se = per_mb[mb]["slot_expert"]
-            for e_ in np.unique(se[red & (se >= 0)]):
-                gpus = set((np.nonzero(red & (se == e_))[0] // SG).tolist())
-                hg = ((e_ // w.H) * (w.H + w.R)) // SG
-                sync_b += len(gpus) * slot_bytes
-                cross_b += len(gpus - {hg}) * slot_bytes
-            sync_b += int((red & (se >= 0)).sum()) * slot_bytes
-            grad_b += per_mb[mb]["M"] * w.P * 8 + per_mb[mb]["filled"] * w.P * gsize
-        return {"G": G, "microbatches": n_sh, "relay_rounds": ue.ue_relay_rounds(G),
-                "sync_alg_bytes_mean": int(sync_b / n_sh), "nvlink_bytes_mean": int(cross_b / n_sh),
-                "sync_relay_us": round(tmax[0] / n_sh, 1), "sync_direct_us": round(tmax[1] / n_sh, 1),
-                "grad_reduce_us": round(tmax[2] / n_sh, 1),
-                "sync_relay_gbs": round(sync_b / (tmax[0] * 1e-6) / 1e9, 1),
-                "sync_direct_gbs": round(sync_b / (tmax[1] * 1e-6) / 1e9, 1),
-                "grad_reduce_gbs": round(grad_b / (tmax[2] * 1e-6) / 1e9, 1),
-                "nvlink_gbs_relay": round(cross_b / (tmax[0] * 1e-6) / 1e9, 1),
-                "note": "each rank one GPU holding its shard; peer tables by CUDA IPC; NCCL barriers between "
-                        "relay rounds; GB/s = all GPUs' algorithmic sync / grad bytes / the slowest rank's time"}
-    except Exception as exc:      # reported in the line; the replicas' numbers stand
-        return {"error": repr(exc)[:300]}
+    # Barriers are host-staged (stream synchronize, then a gloo barrier).
+    SG, EG, RG, TG = w.S // G, w.E // G, (w.N // G) * w.R, w.T // G
+    dev = weights.device
+    bal = ShardedBalancer(cfg, DeviceOps(ctx, cfg, G, g), G=G, g=g, group=grp, device=dev, host_staged=True)
+    pw = PeerBuffers(weights[g * SG:(g + 1) * SG], group=grp)
+    pg = PeerBuffers(grads[g * RG:(g + 1) * RG], group=grp)
+    counts = torch.empty((w.N, w.E), dtype=torch.int32, device=dev)
+    plan = ue.Plan(cfg, device=dev)
+    phys_l = torch.empty((TG, w.K), dtype=torch.int32, device=dev)
+    n_sh = min(n_mb, 4)
+    st = torch.cuda.current_stream(dev)
+    evs = []
+    for k in range(-1, n_sh):                    # one untimed pass first
+        mb = max(k, 0)
+        bal.rebalance(ids_dev[mb][g * TG:(g + 1) * TG], counts, None, plan, phys_l)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        e[0].record(st)
+        bal.sync(pw.ptrs, slot_bytes, plan, relay=True)
+        e[1].record(st)
+        bal.sync(pw.ptrs, slot_bytes, plan, relay=False)
+        e[2].record(st)
+        bal.grad_reduce(master[g * EG:(g + 1) * EG], pg.ptrs, gdt, w.P, plan)
+        e[3].record(st)
+        if k >= 0:
+            evs.append(e)
+    torch.cuda.synchronize(dev)
+    t = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(3)] for e in evs]) * 1e3
+    tt = torch.tensor(list(t.sum(axis=0)), dtype=torch.float64)
+    dist.pg.all_reduce(tt, op=dist.pg.ReduceOp.MAX, group=grp)
+    tmax = tt.tolist()
+    bal.barrier()
+    torch.cuda.synchronize(dev)
+    pw.close()
+    pg.close()
+    sync_b = cross_b = grad_b = 0
+    gsize = 2 if w.grad_dtype == "bf16" else 4
+    for mb in range(n_sh):
+        se = per_mb[mb]["slot_expert"]
+        for e_ in np.unique(se[red & (se >= 0)]):
+            gpus = set((np.nonzero(red & (se == e_))[0] // SG).tolist())
+            hg = ((e_ // w.H) * (w.H + w.R)) // SG
+            sync_b += len(gpus) * slot_bytes
+            cross_b += len(gpus - {hg}) * slot_bytes
+        sync_b += int((red & (se >= 0)).sum()) * slot_bytes
+        grad_b += per_mb[mb]["M"] * w.P * 8 + per_mb[mb]["filled"] * w.P * gsize
+    return {"G": G, "microbatches": n_sh, "relay_rounds": ue.ue_relay_rounds(G),
+            "sync_alg_bytes_mean": int(sync_b / n_sh), "nvlink_bytes_mean": int(cross_b / n_sh),
+            "sync_relay_us": round(tmax[0] / n_sh, 1), "sync_direct_us": round(tmax[1] / n_sh, 1),
+            "grad_reduce_us": round(tmax[2] / n_sh, 1),
+            "sync_relay_gbs": round(sync_b / (tmax[0] * 1e-6) / 1e9, 1),
+            "sync_direct_gbs": round(sync_b / (tmax[1] * 1e-6) / 1e9, 1),
+            "grad_reduce_gbs": round(grad_b / (tmax[2] * 1e-6) / 1e9, 1),
+            "nvlink_gbs_relay": round(cross_b / (tmax[0] * 1e-6) / 1e9, 1),
+            "note": "each rank one GPU holding its shard; peer tables by CUDA IPC; host-staged barriers "
+                    "(stream synchronize + gloo) between relay rounds, inside the times; GB/s = all GPUs' "
+                    "algorithmic sync / grad bytes / the slowest rank's time"}
 
 
 # ---- the CPU oracle, timed on the host cores ------------------------------------
