@@ -675,7 +675,9 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, int variant, Pla
     // vectors then serve rank_off alone.
     const bool direct = lv != nullptr && c == 0;
     if (!direct && (C == 1 || c != 0)) slice_sums(counts, E, r0, r1, s.sload);
-    cluster_arrive();          // #1: this slice's partial loads are ready
+    // #1: this slice's partial loads are ready (CTA 0 of a cluster publishes none).
+    if (c == 0 && C > 1) cluster_arrive_relaxed();
+    else cluster_arrive();
     if (!direct) cluster_wait();
     if (c != 0) {
         // Off the critical path: rank_off for this slice (the slices of the
