@@ -110,7 +110,12 @@ k_sync(uint8_t *__restrict__ W, int64_t slot_bytes, int E, int S, int cap,
         bulk_load(stage + (size_t)b * kSyncTile, it.src, it.bytes, &bar[b]);
     };
 
-    int64_t issued = 0;
+    // Store groups left reading shared memory before a stage is refilled: with
+    // many tiles, kSyncStages - 1 (more writes in flight, the next load issued
+    // one tile ahead); a CTA with few tiles keeps its loads ahead instead (its
+    // ring would otherwise wait on each load while filling).
+    const int keep = nmy >= 16 ? kSyncStages - 1 : 1;
+    int64_t issued = 0;      // tiles whose load was issued; tile i goes to stage i % kSyncStages
     for (; issued < nmy && issued < kSyncStages; ++issued) issue_load(issued);
     // Diagnostic: CTA 0 waits once, with its first loads in flight, on the
     // extra barrier, on which nothing ever arrives: the wait runs out and the
@@ -131,11 +136,15 @@ k_sync(uint8_t *__restrict__ W, int64_t slot_bytes, int E, int S, int cap,
         for (int j = 0; j < cnt; ++j)
             bulk_store(W + (int64_t)x_slot[first + j] * slot_bytes + it.offset, src, it.bytes);
         bulk_commit();
-        // Refill the previous stage once its stores have read it.
-        if (k >= 1 && k - 1 + kSyncStages < nmy) {
-            bulk_wait_read_1();
-            issue_load(k - 1 + kSyncStages);
-            ++issued;
+        // Stages are refilled oldest first, each once its stores have read it
+        // (tile issued - kSyncStages is the oldest not yet refilled), leaving
+        // up to `keep` store groups still reading.
+        if (issued < nmy && k + 1 - (issued - kSyncStages) > keep) {
+            bulk_wait_read_n(keep);
+            while (issued < nmy && k + 1 - (issued - kSyncStages) > keep) {
+                issue_load(issued);
+                ++issued;
+            }
         }
     }
     bulk_wait_all();
