@@ -690,34 +690,6 @@ def run_ours(args, dist: Dist):
     launch_floor_us = statistics.median(floor)
     del busy
 
-    # HBM by read/write mix on this GPU, for the kernels' mixes: write-only
-    # (cudaMemsetAsync of 2 GiB) and a 1:1 device copy of 2 GiB (bytes read +
-    # written); weight sync writes four bytes per byte it reads.
-    hbm_mix = None
-    try:
-        nb = 2 << 30
-        xa = torch.empty(nb, dtype=torch.uint8, device=dev)
-        xb = torch.empty(nb, dtype=torch.uint8, device=dev)
-
-        def _t(fn):
-            ts = []
-            for k in range(8):
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                fn()
-                b.record(stream)
-                stream.synchronize()
-                if k >= 3:
-                    ts.append(a.elapsed_time(b) * 1e-3)
-            return statistics.median(ts)
-        with torch.cuda.stream(stream):
-            xa.fill_(1)
-            t_w = _t(lambda: xb.zero_())
-            t_c = _t(lambda: xb.copy_(xa))
-        hbm_mix = {"write_only_memset_gbs": round(nb / t_w / 1e9, 1), "copy_rw_gbs": round(2 * nb / t_c / 1e9, 1)}
-        del xa, xb
-    except torch.cuda.OutOfMemoryError:
-        hbm_mix = {"skipped": "no room for 4 GiB beside the workload"}
 
     # Max over ranks (timings) / sums (work).
     mean_reb = float(rebalance_us.mean())
@@ -866,7 +838,6 @@ def run_ours(args, dist: Dist):
         "sync_gbs": round(sync_gbs, 1), "sync_frac": round(sync_gbs / peak, 4),
         "grad_reduce_gbs": round(grad_gbs, 1), "grad_reduce_frac": round(grad_gbs / peak, 4),
         "frac_of_8000_gbs": {"sync": round(sync_gbs / 8000, 4), "grad_reduce": round(grad_gbs / 8000, 4)},
-        "hbm_mix": hbm_mix,
         "sync_delta": sync_delta,
         "across_gpus_emulated": across_gpus,
         "across_gpus": across_real,
