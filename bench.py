@@ -48,12 +48,12 @@ TRAFFIC = {
     ("grad_reduce", "671B-class"): {
         "sources": ["moe_expert_load_ue_b200/csrc/ue_grad_reduce.cu", "moe_expert_load_ue_b200/csrc/ue_grad.cuh"],
         "sha256": "84d2f94dab75115c86e4fb4eaed56f4b7ab6abc45c4dc9ee2dc5fe468a45f3f0",
-        "dram_bytes": 7903708416, "algorithmic_bytes": 7927234560,
+        "dram_bytes": 7903370496, "algorithmic_bytes": 7927234560,
         "profile": "profiles/grad_reduce_and_sync_dram_671B-class.md"},
     ("sync", "671B-class"): {
         "sources": ["moe_expert_load_ue_b200/csrc/ue_sync.cu", "moe_expert_load_ue_b200/csrc/ue_bulk.cuh"],
-        "sha256": "54818e6ae81cee9dea4303af048a3fa945b6e7fc8a5e9eb0ea3c06330eda349d",
-        "dram_bytes": 4962007296, "algorithmic_bytes": 5020581888,
+        "sha256": "30d277eb08f295b207de478b8bbae039ddf6a66e4e350f56fe563415d7bd29e1",
+        "dram_bytes": 4962409728, "algorithmic_bytes": 5020581888,
         "profile": "profiles/grad_reduce_and_sync_dram_671B-class.md"},
 }
 
@@ -64,13 +64,13 @@ TRAFFIC = {
 PROFILES = {
     "profiles/launch_list_671B-class.md": {
         "sources": ["moe_expert_load_ue_b200/csrc/ue_load.cu", "moe_expert_load_ue_b200/csrc/ue_plan.cu", "moe_expert_load_ue_b200/csrc/ue_reroute.cu", "moe_expert_load_ue_b200/csrc/ue_sync.cu", "moe_expert_load_ue_b200/csrc/ue_bulk.cuh", "moe_expert_load_ue_b200/csrc/ue_grad_reduce.cu", "moe_expert_load_ue_b200/csrc/ue_grad.cuh"],
-        "sha256": "417c54ca7f02435589460382a4235d6445668c6023fbcacacac10004777f857b"},
+        "sha256": "b0eb639e81619a6bb130e16f5938f1036862f27ae7789977d67789423e54a5c1"},
     "profiles/hot_path_kernels_full_set_671B-class_small_experts.md": {
         "sources": ["moe_expert_load_ue_b200/csrc/ue_load.cu", "moe_expert_load_ue_b200/csrc/ue_plan.cu", "moe_expert_load_ue_b200/csrc/ue_reroute.cu"],
-        "sha256": "caa9633e08bb050a0799afa0639e93a75877c5f103a75e30e08838f134977225"},
+        "sha256": "f41fc7ca9c2de9498af540ee5b21ce6e356def837c50ee0c81e65d0857c72178"},
     "profiles/grad_reduce_and_sync_dram_671B-class.md": {
         "sources": ["moe_expert_load_ue_b200/csrc/ue_grad_reduce.cu", "moe_expert_load_ue_b200/csrc/ue_grad.cuh", "moe_expert_load_ue_b200/csrc/ue_sync.cu", "moe_expert_load_ue_b200/csrc/ue_bulk.cuh"],
-        "sha256": "da0a296cfaa1768c8d038f549d9e7908a3badbd34d0fd5f91ef33d3b903ee0aa"},
+        "sha256": "b9abe4d9121c77eacef6677e75661787b8ba03244a94c6be4cc03dd3806bd751"},
     "profiles/grad_reduce_bulk_full_set_671B-class_small_experts.md": {
         "sources": ["moe_expert_load_ue_b200/csrc/ue_grad_reduce.cu", "moe_expert_load_ue_b200/csrc/ue_grad.cuh"],
         "sha256": "84d2f94dab75115c86e4fb4eaed56f4b7ab6abc45c4dc9ee2dc5fe468a45f3f0"},
@@ -82,7 +82,7 @@ PROFILES = {
         "sha256": "6f1fe8f23d9a123d558ba2f6db0ed74b3e6aca91013f82ffdb93c6b289aa27e5"},
     "profiles/sync_and_grad_across_gpus_dram_671B-class_emulated.md": {
         "sources": ["moe_expert_load_ue_b200/csrc/ue_shard.cu", "moe_expert_load_ue_b200/csrc/ue_bulk.cuh", "moe_expert_load_ue_b200/csrc/ue_grad_reduce.cu", "moe_expert_load_ue_b200/csrc/ue_grad.cuh"],
-        "sha256": "01ca9e26e079f67826811838b5e22f8b2f5dac0d3bbaf00ec47deba039fd9997"},
+        "sha256": "9c1747afaab1a7b76e1cb389c15d37ca9033c2971500ae78c90356b73e392cd6"},
 }
 
 
