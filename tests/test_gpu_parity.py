@@ -188,6 +188,21 @@ def test_sync_ragged_tiles(ctx, slot_bytes):
     _check_sync_full(ctx, inputs.CLASS_671B.with_(tokens_per_rank=256), slot_bytes, mb=3)
 
 
+def test_sync_store_depth_switch(ctx):
+    # The sync's CTAs leave three store groups in flight when they stream 16 or
+    # more tiles of 48 KiB, one otherwise: a slot size that gives about half the
+    # CTAs 16 tiles and the others 15 runs both in one launch.
+    w = inputs.TINY
+    _, pl, _ = _plan_for(ctx, w, 0)
+    M = int(pl["info"][3])
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    ntiles = -(-(15 * sms + sms // 2) // M)
+    slot_bytes = ntiles * 48 * 1024 - 48            # a ragged last tile
+    total = M * ntiles
+    assert total // sms == 15 and total % sms > 0
+    _check_sync_full(ctx, w, slot_bytes)
+
+
 def test_sync_extreme_fanout(ctx):
     # the hot expert fans out to many replicas: each of its tiles is read once, written ~10 times
     w = inputs.EXTREME
