@@ -644,6 +644,62 @@ __device__ __forceinline__ void spread_stuck(const PlanSmem &s, int ns, int Q, i
     }
 }
 
+// The plan's slot table, and (loads) the rank loads before / after with their
+// maxima (info[5], info[6]), from CTA 0's final plan state read over DSMEM:
+// the part of a cluster's output its helper CTAs write while CTA 0 writes the
+// replica lists.  Helper hc of nh takes every nh-th run of blockDim.x slots.
+__device__ __forceinline__ void plan_tail(cg::cluster_group &cluster, const PlanSmem &s, const PlanDev &plan, int hc,
+                                          int nh, int N, int R, int H, int HR, int S, bool loads)
+{
+    const int32_t *qh = cluster.map_shared_rank(s.qh, 0);
+    const int32_t *sasg = cluster.map_shared_rank(s.sasg, 0);
+    const int32_t *ae = cluster.map_shared_rank(s.ae, 0);
+    const int32_t *ac = cluster.map_shared_rank(s.ac, 0);
+    for (int sl = hc * (int)blockDim.x + (int)threadIdx.x; sl < S; sl += nh * (int)blockDim.x) {
+        const int r = sl / HR, u = sl % HR;
+        int se, sq;
+        if (u < H) {
+            se = r * H + u;
+            sq = qh[se];
+        } else {
+            const int a = sasg[r * R + (u - H)];
+            se = a >= 0 ? ae[a] : -1;
+            sq = a >= 0 ? ac[a] : 0;
+        }
+        plan.slot_expert[sl] = se;
+        plan.slot_quota[sl] = sq;
+    }
+    if (!loads) return;
+    const int32_t *spare = cluster.map_shared_rank(s.spare, 0);
+    const int32_t *extra = cluster.map_shared_rank(s.extra, 0);
+    const int32_t *before = cluster.map_shared_rank(s.before, 0);
+    const int Q = cluster.map_shared_rank(s.misc, 0)[4];
+    const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int mb = 0, ma = 0;
+    for (int r = threadIdx.x; r < N; r += blockDim.x) {
+        const int b = before[r], after = Q - spare[r] + extra[r];
+        plan.rank_load_before[r] = b;
+        plan.rank_load_after[r] = after;
+        mb = max(mb, b);
+        ma = max(ma, after);
+    }
+    mb = __reduce_max_sync(0xffffffffu, mb);
+    ma = __reduce_max_sync(0xffffffffu, ma);
+    if (lane_id() == 0) {
+        s.ws[warp] = mb;
+        s.ws[32 + warp] = ma;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        mb = __reduce_max_sync(0xffffffffu, lane_id() < nw ? s.ws[lane_id()] : 0);
+        ma = __reduce_max_sync(0xffffffffu, lane_id() < nw ? s.ws[32 + lane_id()] : 0);
+        if (threadIdx.x == 0) {
+            plan.info[5] = mb;
+            plan.info[6] = ma;
+        }
+    }
+}
+
 // kVariants = false compiles the stated rule alone (variant is ignored), so
 // the default planner carries none of the variants' code.
 template <int NRL, bool kVariants>
@@ -685,6 +741,9 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, int variant, Pla
         // read this CTA's partial vector.
         slice_rank_off(cluster, counts, E, r0, r1, c, 1, s.sload, plan.rank_off);
         cluster_arrive_relaxed();   // #2: done reading the lower peers
+        cluster_wait();             // #2: CTA 0's plan state is final (it arrived with release)
+        plan_tail(cluster, s, plan, c - 1, C - 1, N, R, H, HR, S, c == 1);
+        cluster_arrive_relaxed();   // #3: done reading CTA 0
         cluster_wait();
         return;
     }
@@ -706,13 +765,14 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, int variant, Pla
         }
         plan.load[e] = ld;
     }
-    if (!direct) cluster_arrive_relaxed();  // #2: done reading the peers; CTA 0 holds nothing they read
+    if (!direct && C == 1) cluster_arrive_relaxed();  // #2 (a cluster of one)
 
     // ---- the plan (CTA 0; blockDim >= max(E, N)) ---------------------------------
     int L;
     const int pre = block_excl_scan(ld, s.ws, &L);
     const int Q = L == 0 ? 0 : (L - 1) / N + 1;
     if (ve) s.pre[e] = pre;
+    if (tid == 0) s.misc[4] = Q;                  // for the rank loads (plan_tail)
     for (int r = tid; r < N; r += nt) s.extra[r] = 0;
     for (int i = tid; i < NR; i += nt) s.sasg[i] = -1;
     __syncthreads();
@@ -846,6 +906,12 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, int variant, Pla
         }
     }
     __syncthreads();
+    if (C > 1) {
+        // #2: the plan state the helpers read (qh, sasg, ae, ac, spare, extra,
+        // before, Q) is final; they write the slot table and the rank loads.
+        if (direct) cluster_wait();     // #1, skipped above
+        cluster_arrive();
+    }
 
     // Replica lists (CSR) and the replicated-expert list from one packed scan:
     // the low 16 bits count replica entries, the high bits replicated experts.
@@ -895,59 +961,35 @@ k_plan(const int32_t *__restrict__ counts, int E, int N, int R, int variant, Pla
     }
     for (int p = M + tid; p < E; p += nt) plan.rep_experts[p] = -1;
 
-    // Slot table.
-    for (int sl = tid; sl < S; sl += nt) {
-        const int r = sl / HR, u = sl % HR;
-        int se, sq;
-        if (u < H) {
-            se = r * H + u;
-            sq = s.qh[se];
-        } else {
-            const int a = s.sasg[r * R + (u - H)];
-            se = a >= 0 ? s.ae[a] : -1;
-            sq = a >= 0 ? s.ac[a] : 0;
-        }
-        plan.slot_expert[sl] = se;
-        plan.slot_quota[sl] = sq;
-    }
-
-    // Rank loads before / after and their maxima.
-    int mb = 0, ma = 0;
-    for (int r = tid; r < N; r += nt) {
-        const int after = Q - s.spare[r] + s.extra[r];
-        plan.rank_load_before[r] = s.before[r];
-        plan.rank_load_after[r] = after;
-        mb = max(mb, s.before[r]);
-        ma = max(ma, after);
-    }
-    mb = __reduce_max_sync(0xffffffffu, mb);
-    ma = __reduce_max_sync(0xffffffffu, ma);
-    if (lane_id() == 0) {
-        s.ws[warp] = mb;
-        s.ws[32 + warp] = ma;
-    }
-    __syncthreads();
-    if (warp == 0) {
-        const int nw = nt >> 5;
-        mb = __reduce_max_sync(0xffffffffu, lane_id() < nw ? s.ws[lane_id()] : 0);
-        ma = __reduce_max_sync(0xffffffffu, lane_id() < nw ? s.ws[32 + lane_id()] : 0);
+    if (C == 1) {
+        plan_tail(cluster, s, plan, 0, 1, N, R, H, HR, S, true);
         if (tid == 0) {
             plan.info[0] = Q;
             plan.info[1] = L;
             plan.info[2] = flags;
             plan.info[3] = M;
             plan.info[4] = n_asg;
-            plan.info[5] = mb;
-            plan.info[6] = ma;
             plan.info[7] = 0;
         }
+        slice_rank_off(cluster, counts, E, r0, r1, 0, 0, s.sload, plan.rank_off);
+        if (direct) {          // the barrier phases CTA 0 skipped above
+            cluster_wait();    // #1
+            cluster_arrive_relaxed();   // #2
+        }
+        cluster_wait();        // #2
+        return;
     }
-    if (C == 1) slice_rank_off(cluster, counts, E, r0, r1, 0, 0, s.sload, plan.rank_off);
-    if (direct) {              // the barrier phases CTA 0 skipped above
-        cluster_wait();        // #1
-        cluster_arrive_relaxed();   // #2
+    if (tid == 0) {            // info[5], info[6]: the rank loads' maxima, by helper CTA 1
+        plan.info[0] = Q;
+        plan.info[1] = L;
+        plan.info[2] = flags;
+        plan.info[3] = M;
+        plan.info[4] = n_asg;
+        plan.info[7] = 0;
     }
-    cluster_wait();
+    cluster_wait();                // #2
+    cluster_arrive_relaxed();      // #3
+    cluster_wait();                // #3: the helpers have read this CTA's plan state
 }
 
 }  // namespace
