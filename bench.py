@@ -64,10 +64,10 @@ TRAFFIC = {
 PROFILES = {
     "profiles/launch_list_671B-class.md": {
         "sources": ["moe_expert_load_ue_b200/csrc/ue_load.cu", "moe_expert_load_ue_b200/csrc/ue_plan.cu", "moe_expert_load_ue_b200/csrc/ue_reroute.cu", "moe_expert_load_ue_b200/csrc/ue_sync.cu", "moe_expert_load_ue_b200/csrc/ue_bulk.cuh", "moe_expert_load_ue_b200/csrc/ue_grad_reduce.cu", "moe_expert_load_ue_b200/csrc/ue_grad.cuh"],
-        "sha256": "b0eb639e81619a6bb130e16f5938f1036862f27ae7789977d67789423e54a5c1"},
+        "sha256": "e57c3082f70b10a83401255ec6446612178b7df6601eab8bc36b02c21d589931"},
     "profiles/hot_path_kernels_full_set_671B-class_small_experts.md": {
         "sources": ["moe_expert_load_ue_b200/csrc/ue_load.cu", "moe_expert_load_ue_b200/csrc/ue_plan.cu", "moe_expert_load_ue_b200/csrc/ue_reroute.cu"],
-        "sha256": "f41fc7ca9c2de9498af540ee5b21ce6e356def837c50ee0c81e65d0857c72178"},
+        "sha256": "03db1fa3cdc407f27b2380446dc7ffad9df87b426c73b4fe5146d8092f7f3170"},
     "profiles/grad_reduce_and_sync_dram_671B-class.md": {
         "sources": ["moe_expert_load_ue_b200/csrc/ue_grad_reduce.cu", "moe_expert_load_ue_b200/csrc/ue_grad.cuh", "moe_expert_load_ue_b200/csrc/ue_sync.cu", "moe_expert_load_ue_b200/csrc/ue_bulk.cuh"],
         "sha256": "b9abe4d9121c77eacef6677e75661787b8ba03244a94c6be4cc03dd3806bd751"},
